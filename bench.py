@@ -1,0 +1,411 @@
+#!/usr/bin/env python3
+"""Throughput of the DSA hot path on B200.
+
+One step = one whole DSA prefill forward (lightning indexer + deterministic top-k, in
+row chunks, then sparse GQA attention) over the 128K-token long-video workload
+(L=131072, Hq=32, Hkv=4, d=128, H_I=64, d_I=128, k=2048).  The decode workload (16
+sequences x 262144 cached tokens) is measured in the same run and reported under
+"decode".  Inputs are synthetic and seeded (workloads.generators) and larger than L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent replica;
+the path has no cross-rank exchange, so only the timing uses the process group.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import generators as gen  # noqa: E402
+
+PREFILL_CHUNK = 8192
+METRIC = "DSA prefill tokens/s at 128K ctx (indexer + top-k + sparse attention)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_rate(wl, n_rows: int, seed: int):
+    """Times the fp64 oracle on ``n_rows`` random query rows; returns (tokens/s, seconds,
+    threads, rows).  The whole-workload time is estimated as mean row time x rows."""
+    from oracle import dsa_oracle as orc  # the CPU baseline leg is the one bench use of the oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    rng = np.random.default_rng(seed)
+    rows = sorted(int(r) for r in rng.integers(0, wl.Tq, size=n_rows))
+    D = orc.Decoded(wl)
+    t0 = time.perf_counter()
+    for r in rows:
+        orc.forward_row(D, r)
+    dt = time.perf_counter() - t0
+    est_total = dt / len(rows) * wl.Tq
+    return wl.Tq / est_total, dt, threads, rows
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    wl = gen.video_prefill_128k()
+    for _ in range(args.warmup):
+        oracle_rate(wl, 2, seed=100)
+    vals, secs, thr = [], 0.0, 1
+    for s in range(args.steps):
+        v, dt, thr, _ = oracle_rate(wl, 6, seed=s)
+        vals.append(v)
+        secs += dt
+    value = statistics.mean(vals)
+    sample = f"{args.steps} steps x 6 random query rows of the 131072-row workload; whole-workload time " \
+             f"extrapolated as mean row time x 131072"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 131072 / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "video_prefill_128k", "seq_len": 131072, "batch": 1,
+                                            "Hq": 32, "Hkv": 4, "d": 128, "H_I": 64, "d_I": 128, "topk": 2048},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU helpers
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def bf16_dev(bits, device):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def run_prefill(args, rank, world, device, dist):
+    import torch
+    import lightning_indexer_b200 as dsa
+
+    wl = gen.video_prefill_128k()
+    L = wl.Tq
+    cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+    k = wl.topk
+    ld = (L + 3) // 4 * 4
+    chunk = PREFILL_CHUNK
+    scores = torch.empty((chunk, ld), dtype=torch.float32, device=device)
+    idx = torch.empty((L, k), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    chunks = [(r0, min(L, r0 + chunk)) for r0 in range(0, L, chunk)]
+
+    def step(ev=None):
+        for ci, (r0, r1) in enumerate(chunks):
+            if ev is not None:
+                ev[ci][0].record(stream)
+            dsa.index(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, r0, r1, scores=scores[: r1 - r0])
+            if ev is not None:
+                ev[ci][1].record(stream)
+            dsa.topk(scores[: r1 - r0], cu, cu, k, r0, r1, indices=idx[r0:r1])
+            if ev is not None:
+                ev[ci][2].record(stream)
+        out = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu)
+        if ev is not None:
+            ev[-1][0].record(stream)
+        return out
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    evs = [[[E(), E(), E()] for _ in chunks] + [[E()]] for _ in range(args.steps)]
+    start, stop = E(), E()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+    if dist is not None:
+        dist.barrier()
+    ms = start.elapsed_time(stop)
+    t_idx = t_topk = t_attn = 0.0
+    for s in range(args.steps):
+        for ci in range(len(chunks)):
+            e0, e1, e2 = evs[s][ci]
+            t_idx += e0.elapsed_time(e1)
+            t_topk += e1.elapsed_time(e2)
+        t_attn += evs[s][len(chunks) - 1][2].elapsed_time(evs[s][-1][0])
+    if dist is not None:
+        x = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms = float(x.item())
+    ms_step = ms / args.steps
+    value = world * L / (ms_step / 1e3)
+
+    pairs = wl.causal_pairs()
+    sel_pairs = wl.selected_pairs()
+    idx_flops = pairs * wl.H_I * wl.d_I * 2
+    attn_flops = sel_pairs * wl.Hq * wl.d * 4
+    n_idx_launch = len(chunks) * args.steps
+    res = {
+        "value": value, "ms_per_step": ms_step, "clocks": clk.summary(),
+        "breakdown_ms_per_step": {"indexer": t_idx / args.steps, "topk": t_topk / args.steps,
+                                  "sparse_attn": t_attn / args.steps},
+        "idx_flops_per_launch": idx_flops / len(chunks), "idx_ms_per_launch": t_idx / n_idx_launch,
+        "launches_per_step": 2 * len(chunks) + 1,
+        "flops_per_step": idx_flops + attn_flops, "idx_flops": idx_flops, "attn_flops": attn_flops,
+        "scores_bytes_per_step": pairs * 4,
+        "gather_bytes_per_step": sel_pairs * wl.Hkv * wl.d * 2 * 2,
+    }
+
+    if not args.no_e2e:
+        # end to end through the public API from pinned host buffers
+        host = {n: torch.from_numpy(np.ascontiguousarray(getattr(wl, n)).view(np.int16)).view(torch.bfloat16)
+                .pin_memory() for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+        cu_h = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).pin_memory()
+        o_h = torch.empty(tuple(wl.Q.shape), dtype=torch.bfloat16).pin_memory()
+        ws = torch.empty(dsa.prefill_workspace_bytes(chunk, L), dtype=torch.uint8, device=device)
+        dev_in = {n: torch.empty_like(v, device=device) for n, v in host.items()}
+        cu_d = torch.empty_like(cu_h, device=device)
+        outs = (idx, torch.empty_like(dev_in["Q"]), torch.empty((L, wl.Hq), dtype=torch.float32, device=device))
+        h2d = sum(v.numel() * v.element_size() for v in host.values()) + cu_h.numel() * 4
+        d2h = o_h.numel() * 2
+
+        def e2e_step():
+            for n, v in host.items():
+                dev_in[n].copy_(v, non_blocking=True)
+            cu_d.copy_(cu_h, non_blocking=True)
+            _, O, _ = dsa.prefill(dev_in["q_idx"], dev_in["k_idx"], dev_in["w"], dev_in["Q"], dev_in["K"],
+                                  dev_in["V"], cu_d, cu_d, L, L, k, chunk_rows=chunk, workspace=ws, out=outs)
+            o_h.copy_(O, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        a, b = E(), E()
+        if dist is not None:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = a.elapsed_time(b) / args.steps
+        if dist is not None:
+            x = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+            dist.all_reduce(x, op=dist.ReduceOp.MAX)
+            e2e_ms = float(x.item())
+        res["e2e"] = {"value": world * L / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del host, dev_in, ws
+    del t, scores, idx
+    torch.cuda.empty_cache()
+    return wl, res
+
+
+def run_decode(args, device, dist):
+    import torch
+    import lightning_indexer_b200 as dsa
+
+    wl = gen.decode_256k()
+    B, N, k = wl.B, wl.meta["N"], wl.topk
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+    cu_q = torch.arange(B + 1, dtype=torch.int32, device=device)
+    cu_k = torch.from_numpy(wl.cu_seqlens_k.astype(np.int32)).to(device)
+    ld = (N + 3) // 4 * 4
+    scores = torch.empty((B, ld), dtype=torch.float32, device=device)
+    idx = torch.empty((B, k), dtype=torch.int32, device=device)
+    ws = torch.empty(dsa.decode_attn_workspace_bytes(B, wl.Hq, wl.d, k), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, 1, N, 0, B, scores=scores)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.topk(scores, cu_q, cu_k, k, 0, B, indices=idx)
+        if ev is not None:
+            ev[2].record(stream)
+        dsa.sparse_attn_decode(t["Q"], t["K"], t["V"], idx, cu_k, workspace=ws)
+        if ev is not None:
+            ev[3].record(stream)
+
+    steps = max(args.steps, 20)
+    for _ in range(max(args.warmup, 5)):
+        step()
+    torch.cuda.synchronize(device)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    evs = [[E(), E(), E(), E()] for _ in range(steps)]
+    for s in range(steps):
+        step(evs[s])
+    torch.cuda.synchronize(device)
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
+                     e[0].elapsed_time(e[3])] for e in evs])
+    us = per.mean(axis=0) * 1e3
+    idx_bytes = B * N * wl.d_I * 2 + B * wl.H_I * wl.d_I * 2 + B * wl.H_I * 2
+    attn_bytes = B * k * wl.Hkv * wl.d * 2 * 2 + B * wl.Hq * wl.d * 2 * 2 + B * k * 4
+    del t, scores, idx, ws
+    torch.cuda.empty_cache()
+    return {"us_per_step": float(us[3]), "us_per_token": float(us[3]) / B,
+            "breakdown_us": {"indexer": float(us[0]), "topk": float(us[1]), "sparse_attn": float(us[2])},
+            "idx_bytes": idx_bytes, "attn_bytes": attn_bytes, "steps": steps,
+            "launches_per_step": 4}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        if world > 1:
+            import torch.distributed as dist_mod
+            dist_mod.init_process_group("gloo")
+            dist_mod.destroy_process_group()
+        run_reference(args, rank)
+        return
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
+    import lightning_indexer_b200 as dsa  # noqa: F401  (fails loudly if the library is missing)
+
+    peaks, peak_src = measured_peaks()
+    wl, res = run_prefill(args, rank, world, device, dist)
+    dec = None if args.no_decode else run_decode(args, device, dist)
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        v, dt, thr, rows = oracle_rate(wl, 24, seed=7)
+        cpu = {"value": v, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "sample": f"24 random query rows of the 131072-row workload ({dt:.1f} s of CPU work); "
+                         f"whole-workload time extrapolated as mean row time x 131072"}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak_tf = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    achieved = res["idx_flops_per_launch"] / (res["idx_ms_per_launch"] / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "video_prefill_128k", "seq_len": wl.Tq, "batch": 1, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "d": wl.d, "H_I": wl.H_I, "d_I": wl.d_I, "topk": wl.topk, "chunk_rows": PREFILL_CHUNK,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (q_idx 2 GiB, Q 1 GiB), no flush"},
+        "roofline": {"kernel": "indexer (tcgen05)", "bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"},
+        "clocks": res["clocks"],
+        "gpu_launches": res["launches_per_step"] * args.steps,
+        "breakdown_ms_per_step": res["breakdown_ms_per_step"],
+        "total_tflops_per_s": res["flops_per_step"] / (res["ms_per_step"] / 1e3) / 1e12,
+    }
+    if "e2e" in res:
+        line["e2e"] = res["e2e"]
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if dec is not None:
+        hbm = peaks.get("hbm_gbs")
+        dec_bytes = dec["idx_bytes"] + dec["attn_bytes"]
+        line["decode"] = {
+            "metric": "DSA decode us/step at 256K ctx (16 sequences, one token each)",
+            "workload": "decode_256k", "value": dec["us_per_step"], "unit": "us/step",
+            "us_per_token": dec["us_per_token"], "breakdown_us": dec["breakdown_us"],
+            "roofline": {"kernel": "whole decode step", "bound": "hbm",
+                         "achieved": dec_bytes / (dec["us_per_step"] / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": dec_bytes / (dec["us_per_step"] / 1e6) / 1e9 / hbm},
+            "indexer_roofline": {"bound": "hbm", "achieved": dec["idx_bytes"] / (dec["breakdown_us"]["indexer"] / 1e6) / 1e9,
+                                 "peak": hbm, "unit": "GB/s"},
+            "gpu_launches": dec["launches_per_step"] * dec["steps"],
+        }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

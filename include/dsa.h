@@ -1,0 +1,233 @@
+/*
+ * dsa.h -- C ABI of libdsa_b200: DeepSeek Sparse Attention (DSA) adapted to a GQA
+ * decoder, for NVIDIA B200 (sm_100a).
+ *
+ * The method (Keye-VL-2.0 technical-report summary, mqxn.cn/news/1966, section 1):
+ * a lightweight "Lightning Indexer" with one MQA-shared indexer key per position scores
+ * every visible context position for each query token; each token keeps its top-k
+ * (k = 2048 in the report) positions; GQA attention then runs only over those
+ * positions, so attention cost falls from O(L^2) to O(L*k).  The indexer is trained in a
+ * dense warm-up stage by a KL divergence to the full attention distribution, then the
+ * whole model trains through sparse attention (same section).  Section 8 of the same
+ * summary asks for a deterministic top-k and a DSA-specific decode path.
+ *
+ * Shared conventions for every call below
+ * ---------------------------------------
+ * - Pointers named as device data are caller-owned device pointers.  The library never
+ *   allocates device memory, never synchronises the device, and keeps no pointer after
+ *   the work it enqueued has completed.  Scratch memory, where a call needs it, is a
+ *   caller-provided workspace whose size the matching *_workspace_size() call returns.
+ * - Tensors are dense, row-major (last index fastest).  "bf16" is the 16-bit bfloat16
+ *   bit pattern.  Every base pointer must be 16-byte aligned.
+ * - Varlen packing: B sequences are concatenated along the token axis.
+ *   cu_seqlens_q / cu_seqlens_k are device int32 arrays [B+1] of offsets (0 first,
+ *   non-decreasing).  Query row r belongs to the sequence b with
+ *   cu_seqlens_q[b] <= r < cu_seqlens_q[b+1]; its sequence-local index is
+ *   i = r - cu_seqlens_q[b]; Lq = cu_seqlens_q[b+1]-cu_seqlens_q[b], Lk likewise.
+ * - Causality is bottom-right aligned: query i sees the sequence-local key positions
+ *   0 .. vis-1 with vis = clamp(i + Lk - Lq + 1, 0, Lk).  Prefill uses Lq == Lk (query i
+ *   sees keys 0..i); decode uses Lq == 1 (the query sees its whole cache).
+ * - Key positions in `indices` are sequence-local (0-based within the sequence); -1 marks
+ *   an unused slot.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call only
+ *   enqueues work on it and returns; errors of that work surface through the stream.
+ * - Return value: DSA_OK, or a negative dsa_status.  Argument errors are detected on the
+ *   host before anything is enqueued.  DSA_ERR_CUDA reports a failed launch.
+ * - Device-side waits (pipeline barriers inside kernels) are bounded: a wait that runs
+ *   out records DSA_ERR_TIMEOUT in a device status word that dsa_get_device_status()
+ *   reads, and the kernel returns instead of hanging.
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = -1, /* a null pointer, bad size, misaligned pointer, bad ld */
+  DSA_ERR_UNSUPPORTED = -2, /* a valid shape this build has no kernel for */
+  DSA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than *_workspace_size() */
+  DSA_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+  DSA_ERR_TIMEOUT = -5      /* a bounded device-side wait ran out (device status word) */
+} dsa_status;
+
+/* Human-readable name of a dsa_status value.  Never returns NULL. */
+DSA_API const char* dsa_status_string(int status);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+DSA_API int dsa_version(void);
+
+/* Reads and clears the device status word on the current device.  Synchronises the
+ * device first (a debugging helper, not for hot paths).  *status_out receives DSA_OK or
+ * DSA_ERR_TIMEOUT; *detail_out (may be NULL) receives a kernel-specific code of where
+ * the wait ran out.  Returns DSA_ERR_CUDA if the synchronisation itself failed. */
+DSA_API int dsa_get_device_status(int* status_out, int* detail_out);
+
+/* ---------------------------------------------------------------------------------
+ * (1) Lightning indexer scores.  Source: report summary section 1 (an MQA-shared
+ * scout scans all positions).  For every query row r in [row_begin, row_end):
+ *     scores[(r-row_begin)*ld_scores + s] = sum_j w[r,j] * max(0, q_idx[r,j,:] . k_idx[k0+s,:])
+ * for s in [0, vis(r)), where k0 = cu_seqlens_k[b].  Products are bf16 x bf16 with fp32
+ * accumulation (tensor cores); ReLU, the w-weighting and the head sum are fp32.
+ *   q_idx  device bf16 [total_q, H_I, d_I]   indexer queries
+ *   k_idx  device bf16 [total_k, d_I]        indexer keys (one per position, shared)
+ *   w      device bf16 [total_q, H_I]        per-token indexer head weights
+ *   total_q, total_k  host: rows of q_idx/w and of k_idx (cu_seqlens_q[B], cu_seqlens_k[B])
+ *   max_seqlen_q  host int >= every Lq (used only to size the launch)
+ *   scores device fp32 [row_end-row_begin, ld_scores]; only columns s < vis(r) are
+ *          written, the rest is left untouched.  ld_scores >= the longest Lk and a
+ *          multiple of 4.
+ * Supported: (H_I, d_I) in {(64,128), (32,128), (16,128), (4,32), (8,64)}.
+ * ------------------------------------------------------------------------------- */
+DSA_API int dsa_index(const void* q_idx, const void* k_idx, const void* w,
+                      const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                      int64_t total_q, int64_t total_k, int max_seqlen_q, int max_seqlen_k,
+                      int H_I, int d_I, int64_t row_begin, int64_t row_end, float* scores,
+                      int64_t ld_scores, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (2) Deterministic top-k.  Source: report summary section 1 (each token keeps its 2048
+ * most relevant positions) and section 8 (the selection must be deterministic so that
+ * training and inference select the same set).  For each row r in [row_begin, row_end)
+ * the selected set is the k largest scores[(r-row_begin)*ld_scores + s], s < vis(r),
+ * where equal scores are ranked by the lower position and +0.0 equals -0.0.  If
+ * vis(r) <= k every visible position is selected.  Output:
+ *   indices device int32 [row_end-row_begin, k]: the selected positions in ascending
+ *           order, then -1 in the unused slots.  Bit-for-bit reproducible.
+ * Supported: 1 <= k <= 4096.  No workspace.
+ * ------------------------------------------------------------------------------- */
+DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_seqlens_q,
+                     const int32_t* cu_seqlens_k, int batch, int64_t row_begin, int64_t row_end,
+                     int k, int32_t* indices, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (3) Sparse GQA attention, prefill/varlen.  Source: report summary section 1 (attention
+ * only over the selected positions, O(L*k); GQA adapted to DSA: the one selected set of a
+ * token is shared by all its query heads).  For row r, head h, KV head g = h/(Hq/Hkv),
+ * set S = {indices[r,:] >= 0}:
+ *     O[r,h,:]  = sum_{s in S} softmax_s(scale * Q[r,h,:].K[k0+s,g,:]) V[k0+s,g,:]
+ *     lse[r,h]  = natural log of sum_{s in S} exp(scale * Q[r,h,:].K[k0+s,g,:])
+ * An empty set gives O = 0 and lse = -inf.
+ *   Q  device bf16 [total_q, Hq, d];  K, V device bf16 [total_k, Hkv, d]
+ *   indices device int32 [total_q, k] (as produced by dsa_topk)
+ *   O  device bf16 [total_q, Hq, d];  lse device fp32 [total_q, Hq] (may be NULL)
+ * Supported: d in {64, 128}; Hq/Hkv in {4, 8}; k a multiple of 16, <= 4096.
+ * ------------------------------------------------------------------------------- */
+DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
+                                    const int32_t* indices, const int32_t* cu_seqlens_q,
+                                    const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                    int Hq, int Hkv, int d, int k, float scale, void* O,
+                                    float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (4) Sparse GQA attention, decode.  Source: report summary section 8 (a decode path
+ * specific to DSA).  Same arithmetic as (3) for one query row per sequence (Lq == 1), with
+ * the k selected keys split over several thread blocks and their partial softmax states
+ * merged by log-sum-exp.
+ *   Q device bf16 [batch, Hq, d]; K, V device bf16 [total_k, Hkv, d] (sequence b's cache
+ *   is rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1); indices device int32 [batch, k];
+ *   O device bf16 [batch, Hq, d]; lse device fp32 [batch, Hq] (may be NULL).
+ *   workspace: device scratch of dsa_sparse_attn_decode_workspace_size() bytes.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_sparse_attn_decode_workspace_size(int batch, int Hq, int d, int k);
+DSA_API int dsa_sparse_attn_decode(const void* Q, const void* K, const void* V,
+                                   const int32_t* indices, const int32_t* cu_seqlens_k, int batch,
+                                   int Hq, int Hkv, int d, int k, float scale, void* O, float* lse,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (5) Whole DSA forward for prefill: (1) then (2) over row chunks of at most
+ * `chunk_rows` query rows (bounding the fp32 score scratch), then (3).
+ *   max_seqlen_q / max_seqlen_k: host ints >= every Lq / Lk.
+ *   indices device int32 [total_q, k] receives the selected sets.
+ *   workspace: dsa_prefill_workspace_size(chunk_rows, max_seqlen_k) bytes.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k);
+DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, const void* Q,
+                        const void* K, const void* V, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                        int64_t total_k, int max_seqlen_q,
+                        int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I, int k,
+                        float scale, int64_t chunk_rows, int32_t* indices, void* O, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (6) Whole DSA decode step: (1) with one query row per sequence over its cache, (2),
+ * then (4).  q_idx device bf16 [batch, H_I, d_I]; w device bf16 [batch, H_I]; k_idx
+ * device bf16 [total_k, d_I]; Q/K/V/O as in (4); indices device int32 [batch, k].
+ *   workspace: dsa_decode_workspace_size(batch, max_seqlen_k, Hq, d, k) bytes.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_decode_workspace_size(int batch, int max_seqlen_k, int Hq, int d, int k);
+DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, const void* Q,
+                       const void* K, const void* V, const int32_t* cu_seqlens_k, int batch,
+                       int64_t total_k, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I, int k,
+                       float scale, int32_t* indices, void* O, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (7) Sparse attention backward.  Source: report summary section 1, sparse-adaptation
+ * stage (the whole model trains through sparse attention); QbitAI launch article
+ * (news.chathome.org): varlen DSA training kernels.  For the fixed sets in `indices` and
+ * the forward's O and lse:
+ *     P[s] = exp(scale*Q[r,h].K[s,g] - lse[r,h]),  D = dO[r,h].O[r,h]
+ *     dS[s] = P[s] * (dO[r,h].V[s,g] - D)
+ *     dQ[r,h] = scale * sum_s dS[s] K[s,g]
+ *     dK[s,g] += scale * dS[s] Q[r,h],   dV[s,g] += P[s] dO[r,h]   (over all r, h)
+ *   dQ device bf16 [total_q, Hq, d]; dK, dV device bf16 [total_k, Hkv, d].
+ *   dK/dV are accumulated in fp32 in the workspace (float atomics: the summation order,
+ *   and so the last bits, can vary between runs) and rounded to bf16 once at the end.
+ *   workspace: dsa_sparse_attn_bwd_workspace_size(total_q, total_k, Hq, Hkv, d) bytes.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_sparse_attn_bwd_workspace_size(int64_t total_q, int64_t total_k, int Hq,
+                                                  int Hkv, int d);
+DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void* V,
+                                        const void* O, const void* dO, const float* lse,
+                                        const int32_t* indices, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                        int64_t total_k, int Hq, int Hkv, int d, int k,
+                                        float scale, void* dQ, void* dK, void* dV,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (8) Indexer KL loss (dense warm-up).  Source: report summary section 1 (the indexer is
+ * trained to match the full attention distribution by minimising a KL divergence, with
+ * dense attention kept).  For each query row t with visible keys s < vis(t):
+ *     p[t,s] = (1/Hq) sum_h softmax_s(scale * Q[t,h].K[s,g(h)])   (target, a constant)
+ *     q[t,s] = softmax_s(I[t,s]),  I = the indexer score of (1)
+ *     kl[t]  = sum_s p log(p/q)  (0 log 0 = 0);   *loss = (1/total_q) sum_t kl[t]
+ * and the gradients of *loss:
+ *     dw[t,j]       = sum_s g[t,s] max(0, x[t,j,s])
+ *     dq_idx[t,j,:] = w[t,j] sum_s g[t,s] [x[t,j,s] > 0] k_idx[s,:]
+ *     dk_idx[s,:]   = sum_t sum_j g[t,s] w[t,j] [x[t,j,s] > 0] q_idx[t,j,:]
+ * with g = (q - p)/total_q and x[t,j,s] = q_idx[t,j].k_idx[s].
+ *   loss device fp32 [1]; kl device fp32 [total_q]; dq_idx bf16 [total_q,H_I,d_I];
+ *   dk_idx bf16 [total_k, d_I]; dw bf16 [total_q, H_I].
+ *   workspace: dsa_indexer_kl_loss_workspace_size(...) bytes.
+ * Supported: the (H_I, d_I) pairs of (1); d in {64, 128}; Hq/Hkv in {4, 8}; Lq == Lk.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_indexer_kl_loss_workspace_size(int64_t total_q, int64_t total_k,
+                                                  int max_seqlen_k, int Hq, int H_I, int d_I,
+                                                  int64_t chunk_rows);
+DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx, const void* k_idx,
+                                const void* w, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                int64_t total_k, int max_seqlen_q, int max_seqlen_k, int Hq,
+                                int Hkv, int d, int H_I, int d_I, float scale, int64_t chunk_rows,
+                                float* loss, float* kl, void* dq_idx, void* dk_idx, void* dw,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_B200_H */

@@ -1,0 +1,244 @@
+// C ABI of libdsa_b200 (declared in include/dsa.h): argument checks, launch selection,
+// and the chunked prefill / decode pipelines.  Every check happens on the host before
+// anything is enqueued; the library never allocates and never synchronises.
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace dsa {
+__global__ void iota_kernel(int* dst, int n, int step) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i <= n) dst[i] = i * step;
+}
+}  // namespace dsa
+
+namespace dsa_host {
+
+// kernels implemented in the sibling translation units of this unity build
+int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
+                   int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k,
+                   int H_I, int d_I, long long row_begin, long long row_end, float* scores, long long ld,
+                   cudaStream_t stream);
+int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
+                long long row_begin, long long row_end, int k, int* indices, cudaStream_t stream);
+int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                               const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
+                               float scale, void* O, float* lse, cudaStream_t stream);
+size_t decode_workspace_bytes(int batch, int Hq, int d, int k);
+int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_k,
+                              int batch, int Hq, int Hkv, int d, int k, float scale, void* O, float* lse,
+                              void* ws, cudaStream_t stream);
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_pitch_bytes,
+                      uint32_t box_rows, uint32_t box_cols, int swizzle_bytes) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return DSA_ERR_CUDA;
+  if (rows == 0) rows = 1;  // an empty operand is never read; keep the descriptor valid
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_pitch_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_INVALID_ARG;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+int last_launch_status() { return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static bool index_shape_supported(int H_I, int d_I) {
+  return (H_I == 64 && d_I == 128) || (H_I == 32 && d_I == 128) || (H_I == 16 && d_I == 128) ||
+         (H_I == 8 && d_I == 64) || (H_I == 4 && d_I == 32);
+}
+
+static bool attn_shape_supported(int Hq, int Hkv, int d) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return false;
+  const int G = Hq / Hkv;
+  return (d == 64 || d == 128) && (G == 4 || G == 8);
+}
+
+}  // namespace dsa_host
+
+using namespace dsa_host;
+
+extern "C" {
+
+DSA_API const char* dsa_status_string(int status) {
+  switch (status) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    default: return "DSA_ERR_UNKNOWN";
+  }
+}
+
+DSA_API int dsa_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+DSA_API int dsa_get_device_status(int* status_out, int* detail_out) {
+  if (!status_out) return DSA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+  int st = 0, det = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&st, dsa::g_status, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&det, dsa::g_status_detail, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(dsa::g_status_detail, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  *status_out = st;
+  if (detail_out) *detail_out = det;
+  return DSA_OK;
+}
+
+DSA_API int dsa_index(const void* q_idx, const void* k_idx, const void* w, const int32_t* cu_seqlens_q,
+                      const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                      int max_seqlen_k, int H_I, int d_I, int64_t row_begin, int64_t row_end, float* scores,
+                      int64_t ld_scores, void* stream) {
+  if (!q_idx || !k_idx || !w || !cu_seqlens_q || !cu_seqlens_k || !scores) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return DSA_ERR_INVALID_ARG;
+  if (row_begin < 0 || row_end < row_begin || row_end > total_q) return DSA_ERR_INVALID_ARG;
+  if (ld_scores < max_seqlen_k || (ld_scores % 4) != 0) return DSA_ERR_INVALID_ARG;
+  if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  if (!index_shape_supported(H_I, d_I)) return DSA_ERR_UNSUPPORTED;
+  if (row_end == row_begin) return DSA_OK;
+  return indexer_launch(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                        max_seqlen_k, H_I, d_I, row_begin, row_end, scores, ld_scores,
+                        static_cast<cudaStream_t>(stream));
+}
+
+DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_seqlens_q,
+                     const int32_t* cu_seqlens_k, int batch, int64_t row_begin, int64_t row_end, int k,
+                     int32_t* indices, void* stream) {
+  if (!scores || !cu_seqlens_q || !cu_seqlens_k || !indices) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || (ld_scores % 4) != 0 || ld_scores <= 0) return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARG;
+  if (k < 1) return DSA_ERR_INVALID_ARG;
+  if (k > 4096) return DSA_ERR_UNSUPPORTED;
+  return topk_launch(scores, ld_scores, cu_seqlens_q, cu_seqlens_k, batch, row_begin, row_end, k, indices,
+                     static_cast<cudaStream_t>(stream));
+}
+
+DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V, const int32_t* indices,
+                                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                                    int64_t total_q, int Hq, int Hkv, int d, int k, float scale, void* O,
+                                    float* lse, void* stream) {
+  if (!Q || !K || !V || !indices || !cu_seqlens_q || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(indices))
+    return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0) return DSA_OK;
+  return sparse_attn_prefill_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k,
+                                    scale, O, lse, static_cast<cudaStream_t>(stream));
+}
+
+DSA_API size_t dsa_sparse_attn_decode_workspace_size(int batch, int Hq, int d, int k) {
+  if (batch < 1 || Hq < 1 || d < 1 || k < 1) return 0;
+  return decode_workspace_bytes(batch, Hq, d, k);
+}
+
+DSA_API int dsa_sparse_attn_decode(const void* Q, const void* K, const void* V, const int32_t* indices,
+                                   const int32_t* cu_seqlens_k, int batch, int Hq, int Hkv, int d, int k,
+                                   float scale, void* O, float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!Q || !K || !V || !indices || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(batch, Hq, d, k))
+    return DSA_ERR_WORKSPACE;
+  return sparse_attn_decode_launch(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale, O, lse, workspace,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k) {
+  if (chunk_rows < 1 || max_seqlen_k < 0) return 0;
+  const size_t ld = round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
+  return round_up((size_t)chunk_rows * ld * sizeof(float), 256);
+}
+
+DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, const void* Q, const void* K,
+                        const void* V, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                        int64_t total_q, int64_t total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv,
+                        int d, int H_I, int d_I, int k, float scale, int64_t chunk_rows, int32_t* indices,
+                        void* O, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!indices || !O || chunk_rows < 1) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || !index_shape_supported(H_I, d_I) || k % 16 != 0 || k > 4096)
+    return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < dsa_prefill_workspace_size(chunk_rows, max_seqlen_k))
+    return DSA_ERR_WORKSPACE;
+  const int64_t ld = (int64_t)round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
+  float* scores = static_cast<float*>(workspace);
+  for (int64_t r0 = 0; r0 < total_q; r0 += chunk_rows) {
+    const int64_t r1 = r0 + chunk_rows < total_q ? r0 + chunk_rows : total_q;
+    int st = dsa_index(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                       max_seqlen_k, H_I, d_I, r0, r1, scores, ld, stream);
+    if (st != DSA_OK) return st;
+    st = dsa_topk(scores, ld, cu_seqlens_q, cu_seqlens_k, batch, r0, r1, k, indices + r0 * k, stream);
+    if (st != DSA_OK) return st;
+  }
+  return dsa_sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k, scale,
+                                 O, lse, stream);
+}
+
+DSA_API size_t dsa_decode_workspace_size(int batch, int max_seqlen_k, int Hq, int d, int k) {
+  if (batch < 1 || max_seqlen_k < 0 || Hq < 1 || d < 1 || k < 1) return 0;
+  const size_t ld = round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
+  return round_up((size_t)(batch + 1) * sizeof(int), 256) + round_up((size_t)batch * ld * sizeof(float), 256) +
+         round_up(decode_workspace_bytes(batch, Hq, d, k), 256);
+}
+
+DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, const void* Q, const void* K,
+                       const void* V, const int32_t* cu_seqlens_k, int batch, int64_t total_k, int max_seqlen_k,
+                       int Hq, int Hkv, int d, int H_I, int d_I, int k, float scale, int32_t* indices, void* O,
+                       float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!indices || !O || batch < 1) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || !index_shape_supported(H_I, d_I) || k % 16 != 0 || k > 4096)
+    return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < dsa_decode_workspace_size(batch, max_seqlen_k, Hq, d, k))
+    return DSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* cu_q = reinterpret_cast<int*>(ws);
+  ws += round_up((size_t)(batch + 1) * sizeof(int), 256);
+  const int64_t ld = (int64_t)round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
+  float* scores = reinterpret_cast<float*>(ws);
+  ws += round_up((size_t)batch * ld * sizeof(float), 256);
+  dsa::iota_kernel<<<(batch + 1 + 255) / 256, 256, 0, s>>>(cu_q, batch, 1);
+  if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
+  int st = dsa_index(q_idx, k_idx, w, cu_q, cu_seqlens_k, batch, batch, total_k, 1, max_seqlen_k, H_I, d_I, 0, batch,
+                     scores, ld, stream);
+  if (st != DSA_OK) return st;
+  st = dsa_topk(scores, ld, cu_q, cu_seqlens_k, batch, 0, batch, k, indices, stream);
+  if (st != DSA_OK) return st;
+  return dsa_sparse_attn_decode(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale, O, lse, ws,
+                                workspace_bytes - (size_t)(ws - static_cast<uint8_t*>(workspace)), stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,7 @@
+// Unity build of libdsa_b200: every kernel and the C ABI in one translation unit, so the
+// device status word is shared without relocatable device code.
+#include "api.cu"
+#include "indexer.cu"
+#include "topk.cu"
+#include "sparse_attn.cu"
+#include "train_stubs.cu"

@@ -1,0 +1,426 @@
+// Sparse GQA attention over the top-k selected positions (sm_100a).
+//
+// Source: Keye-VL-2.0 report summary (mqxn.cn/news/1966), section 1: attention runs only
+// over the positions the indexer selected (O(L*k) instead of O(L^2)), and DSA is adapted
+// to GQA: one selected set per token, shared by every query head of that token.
+// Section 8 of the same summary: a decode path specific to DSA.
+//
+// One warp owns one (query row, KV head g, key split).  The G = Hq/Hkv query heads of the
+// group share every gathered K/V row.  The work is a gather (k rows of K and V per token
+// and group) followed by two tiny products (G x d by d x 16 per 16 keys), so it is bound
+// by the gather bandwidth, not by the tensor pipe.  The products use warp-level MMA
+// in swap-AB form (M = 16 keys, N = 8 heads, so no M padding is wasted):
+//   S^T[16 keys x 8 heads]  = K_chunk[16 x d] . Q_g^T[d x 8]
+//   O^T[d x 8 heads]       += V_chunk^T[d x 16] . P^T[16 x 8]
+// P^T goes from the accumulator layout to the B-operand layout with movmatrix.trans.
+// Online softmax in the log2 domain; K/V rows stream through a 3-stage cp.async ring per
+// warp (16-byte zero-filling copies for the -1 slots).
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace dsa {
+
+struct SAParams {
+  const uint16_t* Q;  // [rows, Hq, D]
+  const uint16_t* K;  // [total_k, Hkv, D]
+  const uint16_t* V;
+  const int* indices;  // [rows, k]
+  const int* cu_q;     // null for decode (row b is sequence b)
+  const int* cu_k;
+  int batch;
+  long long rows;
+  int Hq, Hkv, G, k;
+  int nsplit;  // key splits per (row, group); 1 = write final O/LSE
+  float scale_log2;
+  uint16_t* O;  // [rows, Hq, D] (nsplit == 1)
+  float* lse;   // [rows, Hq] or null
+  float* part_o;  // [rows, nsplit, Hq, D] (nsplit > 1)
+  float* part_ml; // [rows, nsplit, Hq, 4]: max (log2 domain), exact sum, sum of bf16-rounded weights
+};
+
+constexpr int SA_WARPS = 8;
+constexpr int SA_STAGES = 3;
+constexpr int SA_CHUNK = 16;
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// byte offset of 16-byte segment `seg` of row `row` in a [rows][D] bf16 tile, XOR-swizzled
+// so that 8 consecutive rows at one logical segment fall in distinct bank groups
+template <int D>
+__device__ __forceinline__ uint32_t tile_off(int row, int seg) {
+  return (uint32_t)(row * (D * 2) + ((seg ^ (row & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAParams p) {
+  constexpr int SEGS = D / 8;                          // 16-byte segments per row
+  constexpr int TILE_BYTES = SA_CHUNK * D * 2;         // one K or V chunk
+  constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  constexpr int MT = D / 16;                           // m-tiles of O^T, k-steps of S^T
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint8_t* my = smem + warp * SA_STAGES * STAGE_BYTES;
+  const uint32_t my_s = smem_u32(my);
+
+  const long long task = (long long)blockIdx.x * SA_WARPS + warp;
+  const long long per_row = (long long)p.Hkv * p.nsplit;
+  const long long row = task / per_row;
+  if (row >= p.rows) return;
+  const int rem = (int)(task % per_row);
+  const int split = rem / p.Hkv;
+  const int g = rem % p.Hkv;
+  int kbase = 0;
+  if (p.cu_q) {
+    int lo = 0, hi = p.batch;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
+    }
+    kbase = p.cu_k[lo];
+  } else {
+    kbase = p.cu_k[row];
+  }
+  const int keys_per_split = p.k / p.nsplit;
+  const int* idx = p.indices + row * p.k + split * keys_per_split;
+  const int nchunks = keys_per_split / SA_CHUNK;
+  const uint16_t* Kg = p.K + (size_t)g * D;
+  const uint16_t* Vg = p.V + (size_t)g * D;
+  const size_t kv_row_stride = (size_t)p.Hkv * D;
+
+  // Q_g^T as the B operand: b[kk][0..1] for k-step kk (head n = lane/4, d pair (lane%4)*2)
+  uint32_t qb[MT][2];
+  {
+    const int head = lane / 4;
+    const bool hv = head < p.G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(p.Q + ((size_t)row * p.Hq + g * p.G + (hv ? head : 0)) * D);
+#pragma unroll
+    for (int kk = 0; kk < MT; ++kk) {
+      qb[kk][0] = hv ? __ldg(qrow + kk * 8 + (lane % 4)) : 0u;
+      qb[kk][1] = hv ? __ldg(qrow + kk * 8 + 4 + (lane % 4)) : 0u;
+    }
+  }
+
+  // issue the gather of chunk c into stage st
+  auto issue = [&](int c, int st) {
+    const int my_idx = __ldg(idx + c * SA_CHUNK + (lane & 15));
+    const uint32_t kdst = my_s + st * STAGE_BYTES;
+    const uint32_t vdst = kdst + TILE_BYTES;
+#pragma unroll
+    for (int j = 0; j < SA_CHUNK * SEGS / 32; ++j) {
+      const int e = j * 32 + lane;
+      const int r = e / SEGS, seg = e % SEGS;
+      const int s = __shfl_sync(0xffffffffu, my_idx, r);
+      const bool valid = s >= 0;
+      const size_t off = valid ? (size_t)(kbase + s) * kv_row_stride + seg * 8 : 0;
+      cp_async_16(kdst + tile_off<D>(r, seg), Kg + off, valid);
+      cp_async_16(vdst + tile_off<D>(r, seg), Vg + off, valid);
+    }
+  };
+
+  float acc[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 domain) of heads h0, h1
+  float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums (for the LSE)
+  float r0 = 0.f, r1 = 0.f;              // same, of the bf16-rounded weights that multiply V
+
+#pragma unroll
+  for (int st = 0; st < SA_STAGES - 1; ++st) {
+    if (st < nchunks) issue(st, st);
+    cp_async_commit();
+  }
+
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c % SA_STAGES;
+    {
+      const int cn = c + SA_STAGES - 1;
+      if (cn < nchunks) issue(cn, cn % SA_STAGES);
+      cp_async_commit();
+    }
+    cp_async_wait<SA_STAGES - 1>();
+    __syncwarp();
+    const uint32_t kt = my_s + st * STAGE_BYTES;
+    const uint32_t vt = kt + TILE_BYTES;
+
+    // ---- S^T = K_chunk . Q^T
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < MT; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(kt + tile_off<D>(lane & 15, kk * 2 + (lane >> 4)), a0, a1, a2, a3);
+      mma_bf16_16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+    }
+    // keys of this lane: r0 = lane/4, r1 = lane/4 + 8; heads h0 = 2*(lane%4), h1 = h0 + 1
+    const int myi = __ldg(idx + c * SA_CHUNK + (lane & 15));
+    const bool v0 = __shfl_sync(0xffffffffu, myi, lane / 4) >= 0;
+    const bool v1 = __shfl_sync(0xffffffffu, myi, lane / 4 + 8) >= 0;
+    const float x00 = v0 ? s[0] * p.scale_log2 : -INFINITY;  // (r0, h0)
+    const float x01 = v0 ? s[1] * p.scale_log2 : -INFINITY;  // (r0, h1)
+    const float x10 = v1 ? s[2] * p.scale_log2 : -INFINITY;  // (r1, h0)
+    const float x11 = v1 ? s[3] * p.scale_log2 : -INFINITY;  // (r1, h1)
+    float cm0 = fmaxf(x00, x10), cm1 = fmaxf(x01, x11);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, o));
+      cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, o));
+    }
+    const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
+    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
+    m0 = mn0;
+    m1 = mn1;
+    const float p00 = exp2f(x00 - mu0), p01 = exp2f(x01 - mu1);
+    const float p10 = exp2f(x10 - mu0), p11 = exp2f(x11 - mu1);
+    l0 = l0 * al0 + p00 + p10;
+    l1 = l1 * al1 + p01 + p11;
+    // O is normalised by the sum of the weights exactly as they enter the PV product
+    const uint32_t pk0 = pack_bf16x2(p00, p01), pk1 = pack_bf16x2(p10, p11);
+    r0 = r0 * al0 + __uint_as_float(pk0 << 16) + __uint_as_float(pk1 << 16);
+    r1 = r1 * al1 + __uint_as_float(pk0 & 0xFFFF0000u) + __uint_as_float(pk1 & 0xFFFF0000u);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      acc[mt][0] *= al0;
+      acc[mt][1] *= al1;
+      acc[mt][2] *= al0;
+      acc[mt][3] *= al1;
+    }
+    // ---- O^T += V^T . P^T
+    const uint32_t pb0 = movmatrix_trans(pk0);  // keys 0-7
+    const uint32_t pb1 = movmatrix_trans(pk1);  // keys 8-15
+    const int vrow = (lane & 7) + ((lane >> 4) << 3);
+    const int vseg_off = (lane >> 3) & 1;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4_trans(vt + tile_off<D>(vrow, mt * 2 + vseg_off), a0, a1, a2, a3);
+      mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
+    }
+    __syncwarp();  // stage st is refilled by the next iteration's issue
+  }
+  cp_async_wait<0>();
+
+  // ---- finish: reduce the sums over the lanes holding the same heads
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    r0 += __shfl_xor_sync(0xffffffffu, r0, o);
+    r1 += __shfl_xor_sync(0xffffffffu, r1, o);
+  }
+  const int h0 = 2 * (lane % 4), h1 = h0 + 1;
+  if (p.nsplit == 1) {
+    const float inv0 = r0 > 0.f ? 1.f / r0 : 0.f, inv1 = r1 > 0.f ? 1.f / r1 : 0.f;
+    uint16_t* orow = p.O + ((size_t)row * p.Hq + g * p.G) * D;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int d0 = mt * 16 + lane / 4;
+      if (h0 < p.G) {
+        orow[h0 * D + d0] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][0] * inv0));
+        orow[h0 * D + d0 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][2] * inv0));
+      }
+      if (h1 < p.G) {
+        orow[h1 * D + d0] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][1] * inv1));
+        orow[h1 * D + d0 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[mt][3] * inv1));
+      }
+    }
+    if (p.lse && lane < 4) {
+      const float ln2 = 0.69314718055994531f;
+      if (h0 < p.G) p.lse[row * p.Hq + g * p.G + h0] = l0 > 0.f ? (m0 + log2f(l0)) * ln2 : -INFINITY;
+      if (h1 < p.G) p.lse[row * p.Hq + g * p.G + h1] = l1 > 0.f ? (m1 + log2f(l1)) * ln2 : -INFINITY;
+    }
+  } else {
+    float* po = p.part_o + (((size_t)row * p.nsplit + split) * p.Hq + g * p.G) * D;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int d0 = mt * 16 + lane / 4;
+      if (h0 < p.G) {
+        po[h0 * D + d0] = acc[mt][0];
+        po[h0 * D + d0 + 8] = acc[mt][2];
+      }
+      if (h1 < p.G) {
+        po[h1 * D + d0] = acc[mt][1];
+        po[h1 * D + d0 + 8] = acc[mt][3];
+      }
+    }
+    if (lane < 4) {
+      float* pml = p.part_ml + (((size_t)row * p.nsplit + split) * p.Hq + g * p.G) * 4;
+      if (h0 < p.G) { pml[h0 * 4] = m0; pml[h0 * 4 + 1] = l0; pml[h0 * 4 + 2] = r0; }
+      if (h1 < p.G) { pml[h1 * 4] = m1; pml[h1 * 4 + 1] = l1; pml[h1 * 4 + 2] = r1; }
+    }
+  }
+}
+
+// Merges the per-split partial softmax states of decode: one warp per (row, head).
+template <int D>
+__global__ void decode_combine_kernel(const float* part_o, const float* part_ml, int rows, int Hq, int nsplit,
+                                      uint16_t* O, float* lse) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (gw >= rows * Hq) return;
+  const int row = gw / Hq, h = gw % Hq;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part_ml[(((size_t)row * nsplit + s) * Hq + h) * 4]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  float L = 0.f, R = 0.f;
+  float o[D / 32];
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) o[j] = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const size_t base = ((size_t)row * nsplit + s) * Hq + h;
+    const float m = part_ml[base * 4], l = part_ml[base * 4 + 1], rr = part_ml[base * 4 + 2];
+    const float f = (m == -INFINITY) ? 0.f : exp2f(m - Mu);
+    L += l * f;
+    R += rr * f;
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) o[j] += f * part_o[base * D + j * 32 + lane];
+  }
+  const float inv = R > 0.f ? 1.f / R : 0.f;
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j)
+    O[((size_t)row * Hq + h) * D + j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o[j] * inv));
+  if (lse && lane == 0) lse[(size_t)row * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace dsa
+
+namespace dsa_host {
+
+static int sa_launch_common(dsa::SAParams& p, int d, cudaStream_t stream) {
+  const long long tasks = p.rows * p.Hkv * p.nsplit;
+  const long long blocks = (tasks + dsa::SA_WARPS - 1) / dsa::SA_WARPS;
+  if (blocks <= 0) return DSA_OK;
+  const int smem = dsa::SA_WARPS * dsa::SA_STAGES * 2 * dsa::SA_CHUNK * d * 2;
+  if (d == 128) {
+    static bool done = false;
+    if (!done) {
+      if (cudaFuncSetAttribute(dsa::sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return DSA_ERR_CUDA;
+      done = true;
+    }
+    dsa::sparse_attn_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
+  } else {
+    static bool done = false;
+    if (!done) {
+      if (cudaFuncSetAttribute(dsa::sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return DSA_ERR_CUDA;
+      done = true;
+    }
+    dsa::sparse_attn_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
+  }
+  return last_launch_status();
+}
+
+int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                               const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
+                               float scale, void* O, float* lse, cudaStream_t stream) {
+  dsa::SAParams p{};
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.V = static_cast<const uint16_t*>(V);
+  p.indices = indices;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.rows = total_q;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.k = k;
+  p.nsplit = 1;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.O = static_cast<uint16_t*>(O);
+  p.lse = lse;
+  return sa_launch_common(p, d, stream);
+}
+
+int decode_nsplit(int k) {
+  int ns = k / 128;  // 128 keys per split
+  if (ns < 1) ns = 1;
+  while (ns > 1 && (k % (ns * dsa::SA_CHUNK)) != 0) --ns;
+  return ns;
+}
+
+size_t decode_workspace_bytes(int batch, int Hq, int d, int k) {
+  const int ns = decode_nsplit(k);
+  return (size_t)batch * ns * Hq * ((size_t)d + 4) * sizeof(float) + 256;
+}
+
+int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_k,
+                              int batch, int Hq, int Hkv, int d, int k, float scale, void* O, float* lse,
+                              void* ws, cudaStream_t stream) {
+  dsa::SAParams p{};
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.V = static_cast<const uint16_t*>(V);
+  p.indices = indices;
+  p.cu_q = nullptr;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.rows = batch;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.k = k;
+  p.nsplit = decode_nsplit(k);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.O = static_cast<uint16_t*>(O);
+  p.lse = lse;
+  if (p.nsplit == 1) return sa_launch_common(p, d, stream);
+  p.part_o = static_cast<float*>(ws);
+  p.part_ml = p.part_o + (size_t)batch * p.nsplit * Hq * d;
+  int st = sa_launch_common(p, d, stream);
+  if (st != DSA_OK) return st;
+  const int warps = batch * Hq;
+  const int threads = 256;
+  const int blocks = (warps * 32 + threads - 1) / threads;
+  if (d == 128)
+    dsa::decode_combine_kernel<128><<<blocks, threads, 0, stream>>>(p.part_o, p.part_ml, batch, Hq, p.nsplit,
+                                                                   p.O, lse);
+  else
+    dsa::decode_combine_kernel<64><<<blocks, threads, 0, stream>>>(p.part_o, p.part_ml, batch, Hq, p.nsplit,
+                                                                  p.O, lse);
+  return last_launch_status();
+}
+
+}  // namespace dsa_host

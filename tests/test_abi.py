@@ -1,0 +1,74 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point that
+include/dsa.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lightning_indexer_b200 import _lib
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "dsa.h")
+
+
+def declared_functions():
+    text = open(HDR).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"DSA_API\s+[\w\s\*]+?\b(dsa_\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_status_strings_and_version():
+    lib = _lib.load()
+    assert lib.dsa_status_string(0) == b"DSA_OK"
+    assert lib.dsa_status_string(-3) == b"DSA_ERR_WORKSPACE"
+    assert lib.dsa_status_string(12345) == b"DSA_ERR_UNKNOWN"
+    assert lib.dsa_version() >= 10000
+
+
+def test_host_side_argument_errors():
+    lib = _lib.load()
+    fake = 1 << 20  # never dereferenced: every call below fails its host checks first
+    mis = fake + 2  # misaligned
+    # null pointer
+    assert lib.dsa_index(None, fake, fake, fake, fake, 1, 8, 8, 8, 8, 64, 128, 0, 8, fake, 8, None) == -1
+    # misaligned operand
+    assert lib.dsa_index(mis, fake, fake, fake, fake, 1, 8, 8, 8, 8, 64, 128, 0, 8, fake, 8, None) == -1
+    # row range outside [0, total_q]
+    assert lib.dsa_index(fake, fake, fake, fake, fake, 1, 8, 8, 8, 8, 64, 128, 0, 9, fake, 8, None) == -1
+    # ld not a multiple of 4 / smaller than max_seqlen_k
+    assert lib.dsa_index(fake, fake, fake, fake, fake, 1, 8, 8, 8, 8, 64, 128, 0, 8, fake, 6, None) == -1
+    assert lib.dsa_index(fake, fake, fake, fake, fake, 1, 8, 8, 8, 16, 64, 128, 0, 8, fake, 8, None) == -1
+    # unsupported indexer shape
+    assert lib.dsa_index(fake, fake, fake, fake, fake, 1, 8, 8, 8, 8, 48, 128, 0, 8, fake, 8, None) == -2
+    # top-k bounds
+    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 0, fake, None) == -1
+    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 5000, fake, None) == -2
+    # attention shapes
+    assert lib.dsa_sparse_attn_prefill(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 96, 64, 0.1, fake,
+                                       None, None) == -2
+    assert lib.dsa_sparse_attn_prefill(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 128, 40, 0.1, fake,
+                                       None, None) == -2
+    assert lib.dsa_sparse_attn_prefill(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 128, 64, -1.0, fake,
+                                       None, None) == -1
+    # workspace too small
+    need = lib.dsa_sparse_attn_decode_workspace_size(16, 32, 128, 2048)
+    assert need > 0
+    assert lib.dsa_sparse_attn_decode(fake, fake, fake, fake, fake, 16, 32, 4, 128, 2048, 0.1, fake, None,
+                                      fake, need - 1, None) == -3
+    assert lib.dsa_prefill_workspace_size(8192, 131072) >= 8192 * 131072 * 4
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.load()

@@ -1,0 +1,227 @@
+"""GPU parity of the forward hot path (indexer, top-k, sparse attention, prefill and
+decode pipelines) against the fp64 oracle, through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import lightning_indexer_b200 as dsa
+from oracle import dsa_oracle as orc
+from workloads import generators as gen
+
+from dsa_testutil import bf16_dev, set_mismatch_ok, to_device
+
+pytestmark = pytest.mark.gpu
+
+ATTN_ATOL = 1e-2  # max-abs on O: bf16 I/O, fp32 accumulation, unit-variance inputs
+LSE_ATOL = 2e-3   # fp32 softmax statistics vs fp64
+
+
+def _oracle_scores(D, r):
+    b, i, Lq, Lk = D.seq_of_row(r)
+    k0 = int(D.cu_k[b])
+    n = orc.visible_keys(i, Lq, Lk)
+    return orc.indexer_scores_row(D.rows("q_idx", r), D.rows("w", r), D.rows("k_idx", slice(k0, k0 + n)))
+
+
+# ------------------------------------------------------------------------- indexer
+
+def test_indexer_integer_bit_exact():
+    wl = gen.tiny_integer_1k()
+    t = to_device(wl)
+    s = dsa.index(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"]).cpu().numpy()
+    D = orc.Decoded(wl)
+    for r in range(wl.Tq):
+        ref = _oracle_scores(D, r)
+        assert np.array_equal(s[r, :ref.size].astype(np.float64), ref), r
+
+
+@pytest.mark.parametrize("H_I,d_I", [(64, 128), (32, 128), (16, 128), (8, 64), (4, 32)])
+def test_indexer_gaussian_varlen_chunks(H_I, d_I):
+    # three sequences with ragged tails (not multiples of the 128-key tile or token block)
+    wl = gen.make_prefill([300, 1, 777], 8, 2, 64, H_I, d_I, 64, seed=21)
+    t = to_device(wl)
+    D = orc.Decoded(wl)
+    for (r0, r1) in [(0, wl.Tq), (5, 301), (301, wl.Tq)]:
+        s = dsa.index(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"],
+                      row_begin=r0, row_end=r1).cpu().numpy()
+        for r in range(r0, r1):
+            ref = _oracle_scores(D, r)
+            got = s[r - r0, :ref.size].astype(np.float64)
+            tol = 2e-5 * np.abs(ref).max() + 1e-6
+            assert np.max(np.abs(got - ref)) <= tol, (r, np.max(np.abs(got - ref)), tol)
+            # columns past the visible range are never written
+            assert np.all(np.isneginf(s[r - r0, ref.size:min(ref.size + 200, s.shape[1])]))
+
+
+def test_indexer_decode_shape():
+    wl = gen.make_decode(3, 5000, 32, 4, 128, 64, 128, 256, seed=22, layout="video")
+    t = to_device(wl)
+    s = dsa.index(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], 1, t["max_k"]).cpu().numpy()
+    D = orc.Decoded(wl)
+    for r in range(3):
+        ref = _oracle_scores(D, r)
+        tol = 2e-5 * np.abs(ref).max() + 1e-6
+        assert np.max(np.abs(s[r, :5000] - ref)) <= tol
+
+
+# ------------------------------------------------------------------------- top-k
+
+def _topk_case(rows_vis, k, seed, ties=False):
+    rng = np.random.default_rng(seed)
+    B = len(rows_vis)
+    cu_q = np.arange(B + 1, dtype=np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(rows_vis)]).astype(np.int32)
+    ld = (max(rows_vis) + 3) // 4 * 4
+    sc = np.full((B, ld), np.nan, np.float32)
+    for b, n in enumerate(rows_vis):
+        if ties:
+            v = rng.integers(-6, 7, size=n).astype(np.float32) * np.float32(0.5)
+            v[rng.random(n) < 0.05] = -0.0
+        else:
+            v = rng.standard_normal(n).astype(np.float32)
+        sc[b, :n] = v
+    return sc, cu_q, cu_k
+
+
+@pytest.mark.parametrize("ties", [False, True])
+@pytest.mark.parametrize("k", [1, 16, 128, 2048])
+def test_topk_bit_exact(k, ties):
+    vis = [1, 5, 127, 128, 129, 2047, 2048, 2049, 5000, 33333]
+    sc, cu_q, cu_k = _topk_case(vis, k, seed=k + 7 * ties, ties=ties)
+    idx = dsa.topk(torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                   k).cpu().numpy()
+    for b, n in enumerate(vis):
+        ref = orc.topk_row(sc[b, :n].astype(np.float64), k)
+        assert np.array_equal(idx[b], ref), (b, n)
+
+
+def test_topk_long_rows_decode_length():
+    vis = [262144, 262143, 131072]
+    sc, cu_q, cu_k = _topk_case(vis, 2048, seed=3, ties=True)
+    idx = dsa.topk(torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                   2048).cpu().numpy()
+    for b, n in enumerate(vis):
+        assert np.array_equal(idx[b], orc.topk_row(sc[b, :n].astype(np.float64), 2048))
+
+
+def test_topk_deterministic_repeat():
+    sc, cu_q, cu_k = _topk_case([70000] * 4, 2048, seed=9, ties=True)
+    args = (torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(), 2048)
+    a = dsa.topk(*args)
+    b = dsa.topk(*args)
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------------- sparse attention
+
+def _oracle_sets(D, k):
+    wl = D.wl
+    return np.stack([orc.forward_row(D, r, k)["idx"] for r in range(wl.Tq)])
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 4, 128), (8, 2, 64), (16, 4, 64)])
+def test_sparse_attention_prefill_given_sets(Hq, Hkv, d):
+    wl = gen.make_prefill([200, 57, 400], Hq, Hkv, d, 4, 32, 64, seed=31)
+    D = orc.Decoded(wl)
+    idx = _oracle_sets(D, 64)
+    t = to_device(wl)
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx.astype(np.int32)).cuda(),
+                                     t["cu_q"], t["cu_k"])
+    O = O.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    for r in range(wl.Tq):
+        b, i, Lq, Lk = D.seq_of_row(r)
+        sel = idx[r][idx[r] >= 0] + int(D.cu_k[b])
+        Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL, r
+        assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL, r
+
+
+def test_sparse_attention_empty_and_padded_sets():
+    wl = gen.make_prefill([40], 8, 2, 64, 4, 32, 32, seed=32)
+    D = orc.Decoded(wl)
+    idx = np.full((40, 32), -1, np.int32)
+    idx[1, :5] = [0, 1, 7, 20, 39]
+    idx[2, 3] = 11  # a single selected key in the middle of the padding
+    t = to_device(wl)
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"])
+    O = O.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    assert np.all(O[0] == 0) and np.all(np.isneginf(lse[0]))
+    for r in (1, 2):
+        sel = idx[r][idx[r] >= 0]
+        Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL
+        assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL
+
+
+def test_sparse_attention_decode_given_sets():
+    wl = gen.make_decode(5, 3000, 32, 4, 128, 64, 128, 2048, seed=33, layout="video")
+    D = orc.Decoded(wl)
+    idx = _oracle_sets(D, 2048)
+    t = to_device(wl)
+    O, lse = dsa.sparse_attn_decode(t["Q"], t["K"], t["V"], torch.from_numpy(idx.astype(np.int32)).cuda(),
+                                    t["cu_k"])
+    O = O.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    for r in range(5):
+        sel = idx[r][idx[r] >= 0] + int(D.cu_k[r])
+        Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL
+        assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL
+
+
+# ------------------------------------------------------------------------- pipelines
+
+def test_prefill_pipeline_integer_bit_exact_sets():
+    wl = gen.tiny_integer_1k()
+    t = to_device(wl)
+    idx, O, lse = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_q"], t["cu_k"],
+                              t["max_q"], t["max_k"], wl.topk, chunk_rows=300)
+    idx = idx.cpu().numpy()
+    O = O.float().cpu().numpy()
+    D = orc.Decoded(wl)
+    ref = orc.forward(D)
+    assert np.array_equal(idx, ref["idx"])
+    assert np.max(np.abs(O - ref["O"])) <= ATTN_ATOL
+    assert np.max(np.abs(lse.cpu().numpy() - ref["lse"])) <= LSE_ATOL
+
+
+def test_prefill_pipeline_gaussian_varlen():
+    wl = gen.make_prefill([1500, 700, 2300], 32, 4, 128, 64, 128, 512, seed=41, layout="video")
+    t = to_device(wl)
+    idx, O, lse = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_q"], t["cu_k"],
+                              t["max_q"], t["max_k"], wl.topk, chunk_rows=1024)
+    idx, O = idx.cpu().numpy(), O.float().cpu().numpy()
+    D = orc.Decoded(wl)
+    rows = orc.sample_rows(wl.Tq, seed=5, n_first=32, n_last=32, n_mid=96) + [1499, 1500, 2199, 2200]
+    swaps = 0
+    for r in rows:
+        ref = orc.forward_row(D, r)
+        ok, nsw = set_mismatch_ok(idx[r], ref["idx"], ref["scores"])
+        assert ok, r
+        swaps += nsw
+        if nsw == 0:
+            assert np.array_equal(idx[r], ref["idx"])
+            assert np.max(np.abs(O[r] - ref["O"])) <= ATTN_ATOL, r
+
+
+def test_decode_pipeline():
+    wl = gen.make_decode(4, 20000, 32, 4, 128, 64, 128, 2048, seed=42, layout="video")
+    t = to_device(wl)
+    idx, O, lse = dsa.decode(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_k"], t["max_k"],
+                             wl.topk)
+    idx, O = idx.cpu().numpy(), O.float().cpu().numpy()
+    D = orc.Decoded(wl)
+    for r in range(4):
+        ref = orc.forward_row(D, r)
+        ok, nsw = set_mismatch_ok(idx[r], ref["idx"], ref["scores"])
+        assert ok, r
+        if nsw == 0:
+            assert np.max(np.abs(O[r] - ref["O"])) <= ATTN_ATOL
+
+
+def test_no_device_timeouts_recorded():
+    assert dsa.device_status() == (0, 0)
