@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode"],
+                    help="run one kernel on a small case (for profiler captures) instead of the bench")
+    ap.add_argument("--case-len", type=int, default=16384, help="sequence length of the --case workload")
     return ap.parse_args()
 
 
@@ -331,8 +334,46 @@ def run_decode(args, device, dist):
             "launches_per_step": 4}
 
 
+def run_case(args):
+    """One kernel, steps+warmup launches, on a small video-layout case (profiling aid)."""
+    import torch
+    import lightning_indexer_b200 as dsa
+    device = torch.device("cuda", 0)
+    L = args.case_len
+    if args.case == "decode":
+        wl = gen.make_decode(16, L, 32, 4, 128, 64, 128, 2048, seed=3, layout="video")
+    else:
+        wl = gen.make_prefill([L], 32, 4, 128, 64, 128, 2048, seed=2, layout="video")
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+    cu_q = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+    cu_k = torch.from_numpy(wl.cu_seqlens_k.astype(np.int32)).to(device)
+    Tq, Lk = wl.Tq, int(wl.seqlens_k.max())
+    scores = dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk)
+    idx = dsa.topk(scores, cu_q, cu_k, wl.topk)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(args.warmup + args.steps):
+        if it == args.warmup:
+            a.record()
+        if args.case in ("indexer", "decode"):
+            dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, scores=scores)
+        if args.case in ("topk", "decode"):
+            dsa.topk(scores, cu_q, cu_k, wl.topk, indices=idx)
+        if args.case == "sparse_attn":
+            dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu_q, cu_k)
+        if args.case == "decode":
+            dsa.sparse_attn_decode(t["Q"], t["K"], t["V"], idx, cu_k)
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "len": L, "ms_per_iter": a.elapsed_time(b) / max(1, args.steps),
+                      "causal_pairs": wl.causal_pairs(), "selected_pairs": wl.selected_pairs()}))
+
+
 def main():
     args = parse()
+    if args.case:
+        run_case(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
