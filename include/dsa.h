@@ -147,6 +147,26 @@ DSA_API int dsa_sparse_attn_decode(const void* Q, const void* K, const void* V,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * (4b) Decode attention without any caller workspace.  The paper has no counterpart: this
+ * is a library convenience for callers that cannot allocate device memory where they run
+ * decode (a host that owns a preallocated pool and offers plugins no allocator, or a
+ * latency-critical loop that must not call cudaMalloc) and have no scratch buffer to pass.
+ * Same inputs, outputs and arithmetic as (4); the split-K scratch lives in a fixed 8 MiB
+ * device array inside the library, held on every GPU that loads the library until exit.
+ *   - Returns DSA_ERR_WORKSPACE when (4) would need more than 8 MiB of scratch, i.e. when
+ *     dsa_sparse_attn_decode_workspace_size(batch, Hq, d, k) > 8388608 (at d = 128 and
+ *     k = 2048 that allows batch * Hq <= 992).
+ *   - The first call on a device looks up the array's device address with that device
+ *     current (a one-time set-up); make that first call before any stream capture.
+ *   - All calls on a device share the one array; calls that can overlap on the GPU race
+ *     and must be ordered by the caller.  Nothing in it needs clearing between calls.
+ * ------------------------------------------------------------------------------- */
+DSA_API int dsa_sparse_attn_decode_noalloc(const void* Q, const void* K, const void* V,
+                                           const int32_t* indices, const int32_t* cu_seqlens_k,
+                                           int batch, int Hq, int Hkv, int d, int k, float scale,
+                                           void* O, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * (5) Whole DSA forward for prefill: (1) then (2) over row chunks of at most
  * `chunk_rows` query rows (bounding the fp32 score scratch), then (3).
  *   max_seqlen_q / max_seqlen_k: host ints >= every Lq / Lk.

@@ -5,3 +5,4 @@
 #include "topk.cu"
 #include "sparse_attn.cu"
 #include "train_stubs.cu"
+#include "decode_noalloc.cu"
