@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-train", action="store_true")
     ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode"],
                     help="run one kernel on a small case (for profiler captures) instead of the bench")
     ap.add_argument("--case-len", type=int, default=16384, help="sequence length of the --case workload")
@@ -369,6 +370,55 @@ def run_case(args):
                       "causal_pairs": wl.causal_pairs(), "selected_pairs": wl.selected_pairs()}))
 
 
+def run_train(args, device):
+    """Training step on the varlen 64K workload: DSA forward (indexer + top-k + sparse
+    attention), sparse-attention backward, and the indexer KL loss with its gradients."""
+    import torch
+    import lightning_indexer_b200 as dsa
+
+    wl = gen.train_varlen_64k()
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V", "dO")}
+    cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+    mq, k = int(wl.seqlens_q.max()), wl.topk
+    chunk = 8192
+    ws = torch.empty(dsa.prefill_workspace_bytes(chunk, mq), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        idx, O, lse = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], cu, cu, mq, mq, k,
+                                  chunk_rows=chunk, workspace=ws)
+        if ev:
+            ev[1].record(stream)
+        dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse, idx, cu, cu)
+        if ev:
+            ev[2].record(stream)
+        dsa.indexer_kl_loss(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], cu, cu, mq, mq, chunk_rows=chunk)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize(device)
+    n = max(2, min(args.steps, 3))
+    evs = [[E(), E(), E(), E()] for _ in range(n)]
+    for i in range(n):
+        step(evs[i])
+    torch.cuda.synchronize(device)
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
+                     e[0].elapsed_time(e[3])] for e in evs]).mean(axis=0)
+    pairs, sel = wl.causal_pairs(), wl.selected_pairs()
+    flops = (pairs * (2 * wl.H_I * wl.d_I * 3 + 2 * wl.Hq * wl.d) + sel * wl.Hq * wl.d * 12)
+    del t, ws
+    torch.cuda.empty_cache()
+    return {"workload": "train_varlen_64k", "seqlens": wl.meta["seqlens"], "ms_per_step": float(per[3]),
+            "breakdown_ms": {"forward": float(per[0]), "sparse_attn_bwd": float(per[1]),
+                             "indexer_kl_loss": float(per[2])},
+            "algorithmic_tflop": flops / 1e12, "tflops_per_s": flops / (per[3] / 1e3) / 1e12}
+
+
 def main():
     args = parse()
     if args.case:
@@ -397,6 +447,7 @@ def main():
     peaks, peak_src = measured_peaks()
     wl, res = run_prefill(args, rank, world, device, dist)
     dec = None if args.no_decode else run_decode(args, device, dist)
+    train = None if args.no_train else run_train(args, device)
     cpu = None
     if rank == 0 and not args.no_cpu:
         v, dt, thr, rows = oracle_rate(wl, 24, seed=7)
@@ -445,6 +496,14 @@ def main():
                                  "peak": hbm, "unit": "GB/s"},
             "gpu_launches": dec["launches_per_step"] * dec["steps"],
         }
+    if train is not None:
+        pk = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        train["roofline"] = {"bound": "tensor", "achieved": train["tflops_per_s"], "peak": pk, "unit": "TFLOP/s",
+                             "frac": train["tflops_per_s"] / pk,
+                             "counting": "indexer fwd + dq/dk backward (3 x 2*H_I*d_I per causal pair), dense "
+                                         "target logits (2*Hq*d per causal pair), sparse attention fwd+bwd "
+                                         "(12*Hq*d per selected pair)"}
+        line["train"] = train
     print(json.dumps(line), flush=True)
 
 

@@ -234,7 +234,9 @@ DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void
  *   loss device fp32 [1]; kl device fp32 [total_q]; dq_idx bf16 [total_q,H_I,d_I];
  *   dk_idx bf16 [total_k, d_I]; dw bf16 [total_q, H_I].
  *   workspace: dsa_indexer_kl_loss_workspace_size(...) bytes.
- * Supported: the (H_I, d_I) pairs of (1); d in {64, 128}; Hq/Hkv in {4, 8}; Lq == Lk.
+ * Supported: H_I in {16, 32, 64} with d_I = 128; d in {64, 128}; Hq/Hkv in {4, 8}; Hkv <= 8;
+ * self-attention packing (Lq == Lk per sequence).  dk_idx is accumulated in fp32 in the
+ * workspace by one thread block per key tile (no atomics: bit-reproducible).
  * ------------------------------------------------------------------------------- */
 DSA_API size_t dsa_indexer_kl_loss_workspace_size(int64_t total_q, int64_t total_k,
                                                   int max_seqlen_k, int Hq, int H_I, int d_I,

@@ -30,6 +30,20 @@ int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const
                               int batch, int Hq, int Hkv, int d, int k, float scale, void* O, float* lse,
                               void* ws, cudaStream_t stream);
 
+size_t sparse_attn_bwd_workspace_bytes(long long total_k, int Hkv, int d);
+int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                           const float* lse, const int* indices, const int* cu_q, const int* cu_k, int batch,
+                           long long total_q, long long total_k, int Hq, int Hkv, int d, int k, float scale,
+                           void* dQ, void* dK, void* dV, void* ws, cudaStream_t stream);
+
+struct KLWorkspace;
+size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int d_I, long long chunk_rows);
+int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
+                           const int* cu_q, const int* cu_k, int batch, long long T, long long Tk,
+                           int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I,
+                           float scale, long long chunk_rows, float* loss, float* kl, void* dq, void* dk, void* dw,
+                           void* ws, cudaStream_t s);
+
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 static std::once_flag g_encode_once;
 
@@ -239,6 +253,62 @@ DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, cons
   if (st != DSA_OK) return st;
   return dsa_sparse_attn_decode(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale, O, lse, ws,
                                 workspace_bytes - (size_t)(ws - static_cast<uint8_t*>(workspace)), stream);
+}
+
+DSA_API size_t dsa_sparse_attn_bwd_workspace_size(int64_t total_q, int64_t total_k, int Hq, int Hkv, int d) {
+  (void)total_q;
+  (void)Hq;
+  if (total_k < 0 || Hkv < 1 || d < 1) return 0;
+  return sparse_attn_bwd_workspace_bytes(total_k, Hkv, d);
+}
+
+DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                        const float* lse, const int32_t* indices, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
+                                        int Hq, int Hkv, int d, int k, float scale, void* dQ, void* dK, void* dV,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !O || !dO || !lse || !indices || !cu_seqlens_q || !cu_seqlens_k || !dQ || !dK || !dV)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
+      !aligned16(dK) || !aligned16(dV))
+    return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < sparse_attn_bwd_workspace_bytes(total_k, Hkv, d))
+    return DSA_ERR_WORKSPACE;
+  return sparse_attn_bwd_launch(Q, K, V, O, dO, lse, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                Hq, Hkv, d, k, scale, dQ, dK, dV, workspace, static_cast<cudaStream_t>(stream));
+}
+
+DSA_API size_t dsa_indexer_kl_loss_workspace_size(int64_t total_q, int64_t total_k, int max_seqlen_k, int Hq,
+                                                  int H_I, int d_I, int64_t chunk_rows) {
+  (void)H_I;
+  if (total_q < 0 || total_k < 0 || max_seqlen_k < 0 || Hq < 1 || d_I < 1 || chunk_rows < 1) return 0;
+  return kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, d_I, chunk_rows);
+}
+
+DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                int64_t total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I,
+                                int d_I, float scale, int64_t chunk_rows, float* loss, float* kl, void* dq_idx,
+                                void* dk_idx, void* dw, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !q_idx || !k_idx || !w || !cu_seqlens_q || !cu_seqlens_k || !loss || !kl || !dq_idx || !dk_idx ||
+      !dw)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) ||
+      !aligned16(dq_idx) || !aligned16(dk_idx) || !aligned16(dw))
+    return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || chunk_rows < 1 || !(scale > 0.f) || max_seqlen_k < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || Hkv > 8) return DSA_ERR_UNSUPPORTED;
+  if (!((H_I == 64 || H_I == 32 || H_I == 16) && d_I == 128)) return DSA_ERR_UNSUPPORTED;
+  if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, d_I, chunk_rows))
+    return DSA_ERR_WORKSPACE;
+  return indexer_kl_loss_launch(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                max_seqlen_q, max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, loss, kl, dq_idx,
+                                dk_idx, dw, workspace, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -4,5 +4,6 @@
 #include "indexer.cu"
 #include "topk.cu"
 #include "sparse_attn.cu"
-#include "train_stubs.cu"
+#include "sparse_attn_bwd.cu"
+#include "kl_loss.cu"
 #include "decode_noalloc.cu"

@@ -1,0 +1,92 @@
+"""GPU parity of the training rows: sparse-attention backward and the indexer KL loss
+(with its gradients), through the C ABI, against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import lightning_indexer_b200 as dsa
+from oracle import dsa_oracle as orc
+from workloads import generators as gen
+
+from dsa_testutil import to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _rel_err(got, ref):
+    return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,k", [(8, 2, 64, 32), (32, 4, 128, 64), (16, 4, 64, 48)])
+def test_sparse_attention_backward(Hq, Hkv, d, k):
+    wl = gen.make_prefill([150, 33, 211], Hq, Hkv, d, 4, 32, k, seed=51, with_dO=True, layout="video")
+    D = orc.Decoded(wl)
+    ref_f = orc.forward(D, k=k)
+    ref = orc.sparse_attention_backward(D, ref_f["idx"], ref_f["O"], ref_f["lse"], D.full("dO"))
+    t = to_device(wl)
+    idx = torch.from_numpy(ref_f["idx"].astype(np.int32)).cuda()
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, t["cu_q"], t["cu_k"])
+    dQ, dK, dV = dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse, idx, t["cu_q"], t["cu_k"])
+    dQ, dK, dV = (x.float().cpu().numpy() for x in (dQ, dK, dV))
+    # bf16 weights inside the products and bf16 outputs: ~2^-8 relative per element
+    assert _rel_err(dQ, ref["dQ"]) <= 1.5e-2
+    assert _rel_err(dK, ref["dK"]) <= 1.5e-2
+    assert _rel_err(dV, ref["dV"]) <= 1.5e-2
+    # the identities that hold at any size
+    assert np.max(np.abs(dK.reshape(-1, Hkv, d).sum(0))) <= 2e-2 * np.max(np.abs(ref["dK"])) * np.sqrt(wl.Tk)
+    grp = D.full("dO").reshape(wl.Tq, Hkv, Hq // Hkv, d).sum(axis=(0, 2))
+    np.testing.assert_allclose(dV.sum(0), grp, rtol=2e-2, atol=2e-2 * np.abs(grp).max())
+
+
+def test_sparse_attention_backward_padded_sets():
+    wl = gen.make_prefill([40], 8, 2, 64, 4, 32, 32, seed=52, with_dO=True)
+    D = orc.Decoded(wl)
+    idx = np.full((40, 32), -1, np.int64)
+    for r in range(40):
+        n = min(r + 1, 32 if r % 3 else 5)
+        idx[r, :n] = np.sort(np.random.default_rng(r).choice(r + 1, size=n, replace=False))
+    O, lse = [], []
+    for r in range(40):
+        sel = idx[r][idx[r] >= 0]
+        o, l = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        O.append(o)
+        lse.append(l)
+    ref = orc.sparse_attention_backward(D, idx, np.stack(O), np.stack(lse), D.full("dO"))
+    t = to_device(wl)
+    tidx = torch.from_numpy(idx.astype(np.int32)).cuda()
+    Og, lg = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], tidx, t["cu_q"], t["cu_k"])
+    dQ, dK, dV = dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], Og, t["dO"], lg, tidx, t["cu_q"], t["cu_k"])
+    assert _rel_err(dQ.float().cpu().numpy(), ref["dQ"]) <= 1.5e-2
+    assert _rel_err(dK.float().cpu().numpy(), ref["dK"]) <= 1.5e-2
+    assert _rel_err(dV.float().cpu().numpy(), ref["dV"]) <= 1.5e-2
+
+
+@pytest.mark.parametrize("H_I,Hq,Hkv,d", [(16, 8, 2, 64), (64, 32, 4, 128), (32, 16, 4, 128)])
+def test_indexer_kl_loss(H_I, Hq, Hkv, d):
+    wl = gen.make_prefill([260, 1, 129, 75], Hq, Hkv, d, H_I, 128, 64, seed=53, layout="video")
+    D = orc.Decoded(wl)
+    ref = orc.indexer_kl_loss(D)
+    t = to_device(wl)
+    for chunk in (wl.Tq, 100):
+        loss, kl, dq, dk, dw = dsa.indexer_kl_loss(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], t["cu_q"],
+                                                   t["cu_k"], t["max_q"], t["max_k"], chunk_rows=chunk)
+        kl = kl.cpu().numpy()
+        assert abs(loss.item() - ref["loss"]) <= 1e-4 * abs(ref["loss"]) + 1e-6
+        assert np.max(np.abs(kl - ref["kl"])) <= 1e-4 * np.max(np.abs(ref["kl"])) + 1e-6
+        assert _rel_err(dq.float().cpu().numpy(), ref["dq_idx"]) <= 1.5e-2
+        assert _rel_err(dk.float().cpu().numpy(), ref["dk_idx"]) <= 1.5e-2
+        assert _rel_err(dw.float().cpu().numpy(), ref["dw"]) <= 1.5e-2
+
+
+def test_indexer_kl_gradient_homogeneity_identity():
+    # I is positively homogeneous of degree 1 in k_idx, in w and in q_idx, so
+    # sum_s k.dk = sum_{t,j} w.dw = sum_{t,j} q.dq = sum_{t,s} g I  (any size)
+    wl = gen.make_prefill([500, 300], 16, 4, 64, 64, 128, 64, seed=54)
+    t = to_device(wl)
+    loss, kl, dq, dk, dw = dsa.indexer_kl_loss(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], t["cu_q"],
+                                               t["cu_k"], t["max_q"], t["max_k"])
+    a = float((t["k_idx"].float() * dk.float()).sum())
+    b = float((t["w"].float() * dw.float()).sum())
+    c = float((t["q_idx"].float() * dq.float()).sum())
+    scale = max(abs(a), abs(b), abs(c), 1e-30)
+    assert abs(a - b) <= 3e-2 * scale and abs(a - c) <= 3e-2 * scale
