@@ -68,6 +68,10 @@ DSA_API const char* dsa_status_string(int status);
 /* Library ABI version (major*10000 + minor*100 + patch). */
 DSA_API int dsa_version(void);
 
+/* The cudaError_t code behind the most recent DSA_ERR_CUDA returned on this host thread
+ * (0 if none), and, if message is not NULL, its text (a static string). */
+DSA_API int dsa_last_cuda_error(const char** message);
+
 /* Reads and clears the device status word on the current device.  Synchronises the
  * device first (a debugging helper, not for hot paths).  *status_out receives DSA_OK or
  * DSA_ERR_TIMEOUT; *detail_out (may be NULL) receives a kernel-specific code of where

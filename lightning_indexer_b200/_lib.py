@@ -15,6 +15,7 @@ c_int, c_i64, c_f32, c_size, c_vp = ctypes.c_int, ctypes.c_int64, ctypes.c_float
 SIGNATURES = {
     "dsa_status_string": (ctypes.c_char_p, [c_int]),
     "dsa_version": (c_int, []),
+    "dsa_last_cuda_error": (c_int, [ctypes.POINTER(ctypes.c_char_p)]),
     "dsa_get_device_status": (c_int, [ctypes.POINTER(c_int), ctypes.POINTER(c_int)]),
     "dsa_index": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int,
                           c_i64, c_i64, c_vp, c_i64, c_vp]),
@@ -64,6 +65,10 @@ def load() -> ctypes.CDLL:
 class DSAError(RuntimeError):
     def __init__(self, name: str, status: int):
         msg = load().dsa_status_string(status).decode()
+        if status == -4:
+            text = ctypes.c_char_p()
+            code = load().dsa_last_cuda_error(ctypes.byref(text))
+            msg += f" [cuda error {code}: {text.value.decode() if text.value else ''}]"
         super().__init__(f"{name} failed: {msg} ({status})")
         self.status = status
 

@@ -21,7 +21,7 @@ int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const in
                    int H_I, int d_I, long long row_begin, long long row_end, float* scores, long long ld,
                    cudaStream_t stream);
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
-                long long row_begin, long long row_end, int k, int* indices, cudaStream_t stream);
+                long long row_begin, long long row_end, int k, int* indices, int max_vis, cudaStream_t stream);
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
                                const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
                                float scale, void* O, float* lse, cudaStream_t stream);
@@ -78,7 +78,19 @@ int sm_count() {
   return n;
 }
 
-int last_launch_status() { return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+static thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return DSA_ERR_CUDA;
+}
+
+int last_launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return DSA_OK;
+  g_last_cuda_error = (int)e;
+  return DSA_ERR_CUDA;
+}
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -115,14 +127,20 @@ DSA_API const char* dsa_status_string(int status) {
 
 DSA_API int dsa_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
+DSA_API int dsa_last_cuda_error(const char** message) {
+  const int e = g_last_cuda_error;
+  if (message) *message = cudaGetErrorString((cudaError_t)e);
+  return e;
+}
+
 DSA_API int dsa_get_device_status(int* status_out, int* detail_out) {
   if (!status_out) return DSA_ERR_INVALID_ARG;
-  if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+  if (const cudaError_t e_ = cudaDeviceSynchronize(); e_ != cudaSuccess) return cuda_fail(e_);
   int st = 0, det = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&st, dsa::g_status, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
-  if (cudaMemcpyFromSymbol(&det, dsa::g_status_detail, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
-  if (cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
-  if (cudaMemcpyToSymbol(dsa::g_status_detail, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (const cudaError_t e_ = cudaMemcpyFromSymbol(&st, dsa::g_status, sizeof(int)); e_ != cudaSuccess) return cuda_fail(e_);
+  if (const cudaError_t e_ = cudaMemcpyFromSymbol(&det, dsa::g_status_detail, sizeof(int)); e_ != cudaSuccess) return cuda_fail(e_);
+  if (const cudaError_t e_ = cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof(int)); e_ != cudaSuccess) return cuda_fail(e_);
+  if (const cudaError_t e_ = cudaMemcpyToSymbol(dsa::g_status_detail, &zero, sizeof(int)); e_ != cudaSuccess) return cuda_fail(e_);
   *status_out = st;
   if (detail_out) *detail_out = det;
   return DSA_OK;
@@ -153,7 +171,9 @@ DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_s
   if (batch < 1 || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARG;
   if (k < 1) return DSA_ERR_INVALID_ARG;
   if (k > 4096) return DSA_ERR_UNSUPPORTED;
-  return topk_launch(scores, ld_scores, cu_seqlens_q, cu_seqlens_k, batch, row_begin, row_end, k, indices,
+  // the row length is bounded by ld_scores (>= the longest visible range)
+  const int max_vis = ld_scores > 0x7FFFFFFF ? 0x7FFFFFFF : (int)ld_scores;
+  return topk_launch(scores, ld_scores, cu_seqlens_q, cu_seqlens_k, batch, row_begin, row_end, k, indices, max_vis,
                      static_cast<cudaStream_t>(stream));
 }
 

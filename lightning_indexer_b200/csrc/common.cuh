@@ -164,6 +164,19 @@ __device__ __forceinline__ void tmem_ld_x32_sync(uint32_t taddr, float* v) {
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns, load and wait in one statement.
+__device__ __forceinline__ void tmem_ld_x16_sync(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored as rows of
 // `swizzle_bytes` (128 or 64) bytes with the matching TMA swizzle; 8-row groups are
 // 8*swizzle_bytes apart.  Fields: start address >> 4 (bits 0-13), leading byte offset
@@ -214,6 +227,7 @@ int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_
                       uint64_t row_pitch_bytes, uint32_t box_rows, uint32_t box_cols, int swizzle_bytes);
 
 int sm_count();
-int last_launch_status();  // DSA_ERR_CUDA if the last launch failed, else DSA_OK
+int last_launch_status();    // DSA_ERR_CUDA if the last launch failed, else DSA_OK
+int cuda_fail(cudaError_t e);  // records e for dsa_last_cuda_error(); returns DSA_ERR_CUDA
 
 }  // namespace dsa_host

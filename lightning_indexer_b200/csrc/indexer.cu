@@ -262,6 +262,13 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_ST
       }
       named_bar_sync(1, C::EPI_THREADS);
       const int dvis = it.Lk - it.Lq + 1;  // vis(i) = clamp(i + dvis, 0, Lk)
+      // this thread's weights for the whole item (reused by every key tile): keeping them in
+      // registers leaves the shared-memory pipe to the tensor core's operand reads
+      float wr[H_I >= 32 ? C::CPT : 1];
+      if constexpr (H_I >= 32) {
+#pragma unroll
+        for (int c = 0; c < C::CPT; ++c) wr[c] = w_s[col0 + c];
+      }
       for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
         if (!(ok = mbar_wait(&acc_full[ab], abph, abort_flag, 6))) break;
         tc_fence_after();
@@ -269,26 +276,18 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_ST
         const uint32_t tbase = tmem_base + lane_off + ab * C::N + col0;
         float* out_row0 = p.scores + (it.t0 - p.row_begin) * p.ld + s;
         if constexpr (H_I >= 32) {
-#pragma unroll 1
+#pragma unroll
           for (int c = 0; c < C::CPT; c += H_I) {
             const int tok = (col0 + c) / H_I;
             float acc = 0.f;
 #pragma unroll
-            for (int h0 = 0; h0 < H_I; h0 += 32) {
-              float v[32];
-              tmem_ld_x32_sync(tbase + c + h0, v);
-              const float4* wv = reinterpret_cast<const float4*>(w_s + tok * H_I + h0);
+            for (int h0 = 0; h0 < H_I; h0 += 16) {
+              float v[16];
+              tmem_ld_x16_sync(tbase + c + h0, v);
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 ww = wv[q];
-                acc = fmaf(ww.x, fmaxf(v[4 * q + 0], 0.f), acc);
-                acc = fmaf(ww.y, fmaxf(v[4 * q + 1], 0.f), acc);
-                acc = fmaf(ww.z, fmaxf(v[4 * q + 2], 0.f), acc);
-                acc = fmaf(ww.w, fmaxf(v[4 * q + 3], 0.f), acc);
-              }
+              for (int q = 0; q < 16; ++q) acc = fmaf(wr[c + h0 + q], fmaxf(v[q], 0.f), acc);
             }
-            const int i_tok = it.i0 + tok;
-            const int vis = min(max(i_tok + dvis, 0), it.Lk);
+            const int vis = min(max(it.i0 + tok + dvis, 0), it.Lk);
             if (tok < it.ntok && s < vis) out_row0[(long long)tok * p.ld] = acc;
           }
         } else {
@@ -338,8 +337,7 @@ static int launch_indexer(const void* q_idx, const void* k_idx, const void* w, c
   static bool attr_done = false;
   const int smem = std::max(C::SMEM_BYTES, 120 * 1024);  // one CTA per SM (TMEM ownership)
   if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return DSA_ERR_CUDA;
+    if (const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
     attr_done = true;
   }
   CUtensorMap tk, tq;

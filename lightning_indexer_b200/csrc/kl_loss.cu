@@ -607,8 +607,7 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
     const int smem = 2 * 64 * D_I * 2;
     static bool done = false;
     if (!done) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return DSA_ERR_CUDA;
+      if (const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
       done = true;
     }
     kern<<<(unsigned)(r1 - r0), H_I / 16 * 32, smem, s>>>(
@@ -621,8 +620,7 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
     const int smem = 2 * H_I * D_I * 2 + 2 * H_I * 4 + 2 * 128 * 4;
     static bool done = false;
     if (!done) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return DSA_ERR_CUDA;
+      if (const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
       done = true;
     }
     const int tiles = (max_seqlen_k + 127) / 128;
@@ -642,7 +640,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
   KLWorkspace W = kl_workspace_layout(ws, T, Tk, max_seqlen_k, Hq, d_I, chunk_rows);
   const long long ld = ((long long)(max_seqlen_k > 0 ? max_seqlen_k : 1) + 3) / 4 * 4;
   const float scale_log2 = scale * 1.4426950408889634f;
-  if (cudaMemsetAsync(W.dk_acc, 0, (size_t)Tk * d_I * 4, s) != cudaSuccess) return DSA_ERR_CUDA;
+  if (const cudaError_t e_ = cudaMemsetAsync(W.dk_acc, 0, (size_t)Tk * d_I * 4, s); e_ != cudaSuccess) return cuda_fail(e_);
   // 1. dense LSE
   {
     const long long tasks = T * Hkv;
@@ -651,18 +649,22 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     if (blocks > 0) {
       if (d == 128) {
         static bool done = false;
-        if (!done && cudaFuncSetAttribute(dsa::dense_lse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          smem) != cudaSuccess)
-          return DSA_ERR_CUDA;
+        if (!done) {
+          const cudaError_t e_ = cudaFuncSetAttribute(dsa::dense_lse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          smem);
+          if (e_ != cudaSuccess) return cuda_fail(e_);
+        }
         done = true;
         dsa::dense_lse_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, s>>>(
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, T, Hq, Hkv,
             scale_log2, W.lse_att);
       } else {
         static bool done = false;
-        if (!done && cudaFuncSetAttribute(dsa::dense_lse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          smem) != cudaSuccess)
-          return DSA_ERR_CUDA;
+        if (!done) {
+          const cudaError_t e_ = cudaFuncSetAttribute(dsa::dense_lse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          smem);
+          if (e_ != cudaSuccess) return cuda_fail(e_);
+        }
         done = true;
         dsa::dense_lse_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, s>>>(
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, T, Hq, Hkv,
@@ -683,18 +685,22 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
       const int smem = Hkv * dsa::SA_STAGES * dsa::SA_CHUNK * d * 2;
       if (d == 128) {
         static bool done = false;
-        if (!done && cudaFuncSetAttribute(dsa::kl_target_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          8 * dsa::SA_STAGES * dsa::SA_CHUNK * 128 * 2) != cudaSuccess)
-          return DSA_ERR_CUDA;
+        if (!done) {
+          const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          8 * dsa::SA_STAGES * dsa::SA_CHUNK * 128 * 2);
+          if (e_ != cudaSuccess) return cuda_fail(e_);
+        }
         done = true;
         dsa::kl_target_kernel<128><<<(unsigned)(r1 - r0), 32 * Hkv, smem, s>>>(
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, r0, Hq, Hkv,
             scale_log2, W.lse_att, W.lseI, W.scores, ld, inv_T, kl);
       } else {
         static bool done = false;
-        if (!done && cudaFuncSetAttribute(dsa::kl_target_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          8 * dsa::SA_STAGES * dsa::SA_CHUNK * 64 * 2) != cudaSuccess)
-          return DSA_ERR_CUDA;
+        if (!done) {
+          const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          8 * dsa::SA_STAGES * dsa::SA_CHUNK * 64 * 2);
+          if (e_ != cudaSuccess) return cuda_fail(e_);
+        }
         done = true;
         dsa::kl_target_kernel<64><<<(unsigned)(r1 - r0), 32 * Hkv, smem, s>>>(
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, r0, Hq, Hkv,

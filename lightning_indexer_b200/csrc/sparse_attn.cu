@@ -332,18 +332,18 @@ static int sa_launch_common(dsa::SAParams& p, int d, cudaStream_t stream) {
   if (d == 128) {
     static bool done = false;
     if (!done) {
-      if (cudaFuncSetAttribute(dsa::sparse_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-          cudaSuccess)
-        return DSA_ERR_CUDA;
+      const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<128>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e_ != cudaSuccess) return cuda_fail(e_);
       done = true;
     }
     dsa::sparse_attn_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
   } else {
     static bool done = false;
     if (!done) {
-      if (cudaFuncSetAttribute(dsa::sparse_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-          cudaSuccess)
-        return DSA_ERR_CUDA;
+      const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<64>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e_ != cudaSuccess) return cuda_fail(e_);
       done = true;
     }
     dsa::sparse_attn_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);

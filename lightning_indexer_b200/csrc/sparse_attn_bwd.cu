@@ -263,7 +263,7 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
   const size_t half = sparse_attn_bwd_workspace_bytes(total_k, Hkv, d) / 2;
   float* dk_acc = static_cast<float*>(ws);
   float* dv_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + half);
-  if (cudaMemsetAsync(ws, 0, 2 * half, stream) != cudaSuccess) return DSA_ERR_CUDA;
+  if (const cudaError_t e_ = cudaMemsetAsync(ws, 0, 2 * half, stream); e_ != cudaSuccess) return cuda_fail(e_);
   dsa::SABwdParams p{};
   p.Q = static_cast<const uint16_t*>(Q);
   p.K = static_cast<const uint16_t*>(K);
@@ -292,18 +292,16 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
     if (d == 128) {
       static bool done = false;
       if (!done) {
-        if (cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem) != cudaSuccess)
-          return DSA_ERR_CUDA;
+        if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem); e_ != cudaSuccess) return cuda_fail(e_);
         done = true;
       }
       dsa::sparse_attn_bwd_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
     } else {
       static bool done = false;
       if (!done) {
-        if (cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem) != cudaSuccess)
-          return DSA_ERR_CUDA;
+        if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem); e_ != cudaSuccess) return cuda_fail(e_);
         done = true;
       }
       dsa::sparse_attn_bwd_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);

@@ -7,14 +7,30 @@
 // Selection rule: the k largest scores among the visible positions; equal scores are
 // ranked by the lower position (+0.0 == -0.0).  Output: ascending positions, -1 padded.
 //
-// Method (one thread block per row, no global atomics, no data-dependent ordering):
-//   1. three radix-histogram passes (11 + 11 + 10 bits of the order-preserving uint32
-//      key) find the exact k-th largest key K* and how many of the ties at K* to take;
-//   2. one ordered compaction pass: position s is selected if key(s) > K*, or
-//      key(s) == K* and fewer than `remaining` ties precede it.  Its output slot is
-//      (#keys > K* before s) + min(#ties before s, remaining), so the output is the
-//      ascending position list and is bit-for-bit reproducible.
+// Method.  A row is split over a cluster of C thread blocks (C = 1, 2, 4 or 8), each
+// owning a contiguous segment.  Scores map to order-preserving uint32 keys.
+//   1. A lower bound T on the k-th largest key is estimated from a fixed strided sample
+//      of the row (the same 1024 positions in every block, so no communication), with a
+//      safety margin.  One global pass compacts the keys >= T of each segment, in
+//      position order, into a shared-memory candidate list.  The cluster checks that at
+//      least k keys passed and that every block's list fit; the estimate only decides
+//      how much is read, never what is selected.
+//   2. Otherwise (an unlucky sample, or a row with huge ties): an exact histogram of the
+//      top 11 key bits (summed over the cluster through distributed shared memory) gives
+//      the threshold bin b1; the keys with bin >= b1 become the candidates if they fit,
+//      else every later step re-reads the segment from global memory.
+//   3. Radix levels (11 + 11 + 10 bits) over the candidates give the exact k-th key K*
+//      and how many ties at K* to take (`remaining`).
+//   4. Ordered output: position s is selected if key > K*, or key == K* and fewer than
+//      `remaining` ties precede it in the row.  Each block learns from the lower-ranked
+//      blocks how many keys > K* and ties come before its segment, so its slots are
+//      (#keys > K* before s) + min(#ties before s, remaining): ascending and
+//      bit-reproducible.  No global atomics are used anywhere.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace dsa {
 
@@ -28,6 +44,9 @@ struct TopkParams {
   int k;
   int* indices;
 };
+
+constexpr int TOPK_THREADS = 1024;
+constexpr int TOPK_CAP = 11264;  // candidates kept in shared memory per block
 
 template <int BLOCK>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -57,8 +76,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
   return before;
 }
 
-// Finds the bin holding the `remaining`-th largest element of the histogram: the bin b
-// with (#elements in bins > b) < remaining <= (#elements in bins >= b).
+// The bin b with (#elements in bins > b) < remaining <= (#elements in bins >= b).
 template <int BLOCK, int NBINS>
 __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t remaining, uint32_t* warp_sums,
                                          uint32_t* scratch, uint32_t* out_bin, uint32_t* out_above) {
@@ -83,15 +101,31 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, uint32_t remainin
   __syncthreads();
 }
 
-template <int BLOCK>
-__global__ void __launch_bounds__(BLOCK) topk_kernel(const TopkParams p) {
-  __shared__ uint32_t hist[2048];
-  __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t s_total, s_bin, s_above;
+template <int C>
+__device__ __forceinline__ void cluster_sync_all() {
+  if constexpr (C > 1) cg::this_cluster().sync();
+  else __syncthreads();
+}
 
-  const long long row = p.row_begin + blockIdx.x;
-  // sequence of this row (cu_q is small; binary search)
-  int lo = 0, hi = p.batch;  // find b with cu_q[b] <= row < cu_q[b+1]
+struct TopkSmem {
+  uint32_t cand_key[TOPK_CAP];
+  int cand_pos[TOPK_CAP];
+  uint32_t hist[2][2048];  // per level parity (remote blocks read them)
+  uint32_t ghist[2048];    // cluster-wide sum
+  uint32_t warp_sums[32];
+  uint32_t total, bin, above;
+  uint32_t flag;     // this block's candidates overflow TOPK_CAP
+  uint32_t counts[2];  // (#keys > K*, #ties) of this block's segment
+};
+
+template <int C>
+__global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) {
+  constexpr int B = TOPK_THREADS;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  const int rank = (C > 1) ? (int)cg::this_cluster().block_rank() : 0;
+  const long long row = p.row_begin + blockIdx.x / C;
+  int lo = 0, hi = p.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) / 2;
     if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
@@ -102,107 +136,347 @@ __global__ void __launch_bounds__(BLOCK) topk_kernel(const TopkParams p) {
   const int Lk = p.cu_k[b + 1] - p.cu_k[b];
   const int vis = min(max(i + Lk - Lq + 1, 0), Lk);
   const int k = p.k;
-  int* out = p.indices + (long long)blockIdx.x * k;
-  const float* src = p.scores + (long long)blockIdx.x * p.ld;
+  int* out = p.indices + (row - p.row_begin) * k;
+  const float* src = p.scores + (row - p.row_begin) * p.ld;
 
-  if (vis <= k) {
-    for (int j = threadIdx.x; j < k; j += BLOCK) out[j] = j < vis ? j : -1;
+  if (vis <= k) {  // uniform over the cluster: no cluster barrier is reached by anyone
+    if (rank == 0)
+      for (int j = threadIdx.x; j < k; j += B) out[j] = j < vis ? j : -1;
     return;
   }
+  // this block's segment [s_lo, s_hi), 4-aligned starts
+  const int seg = ((vis + C - 1) / C + 3) & ~3;
+  const int s_lo = min(rank * seg, vis), s_hi = min(s_lo + seg, vis);
 
-  const int nvec = vis / 4;  // float4 groups; the ragged tail is handled one by one
-  const float4* src4 = reinterpret_cast<const float4*>(src);
-
-  uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
-  // ---------------------------------------------------------------- radix passes
-#pragma unroll 1
-  for (int level = 0; level < 3; ++level) {
-    const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
-    const uint32_t bmask = level == 2 ? 1023u : 2047u;
-    for (int j = threadIdx.x; j < 2048; j += BLOCK) hist[j] = 0;
-    __syncthreads();
-#pragma unroll 4
-    for (int v = threadIdx.x; v < nvec; v += BLOCK) {
-      const float4 x = __ldg(src4 + v);
-      const uint32_t k0 = float_order_key(x.x), k1 = float_order_key(x.y);
-      const uint32_t k2 = float_order_key(x.z), k3 = float_order_key(x.w);
-      if ((k0 & pmask) == prefix) atomicAdd(&hist[(k0 >> shift) & bmask], 1u);
-      if ((k1 & pmask) == prefix) atomicAdd(&hist[(k1 >> shift) & bmask], 1u);
-      if ((k2 & pmask) == prefix) atomicAdd(&hist[(k2 >> shift) & bmask], 1u);
-      if ((k3 & pmask) == prefix) atomicAdd(&hist[(k3 >> shift) & bmask], 1u);
+  auto reduce_hist = [&](int par, int nbins) -> const uint32_t* {
+    if constexpr (C == 1) {
+      return S.hist[par];
+    } else {
+      auto cl = cg::this_cluster();
+      for (int j = threadIdx.x; j < nbins; j += B) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int r = 0; r < C; ++r) t += cl.map_shared_rank(&S.hist[par][0], r)[j];
+        S.ghist[j] = t;
+      }
+      __syncthreads();
+      return S.ghist;
     }
-    for (int s = nvec * 4 + threadIdx.x; s < vis; s += BLOCK) {
-      const uint32_t kk = float_order_key(__ldg(src + s));
-      if ((kk & pmask) == prefix) atomicAdd(&hist[(kk >> shift) & bmask], 1u);
-    }
-    __syncthreads();
-    if (level < 2)
-      find_bin<BLOCK, 2048>(hist, remaining, warp_sums, &s_total, &s_bin, &s_above);
-    else
-      find_bin<BLOCK, 1024>(hist, remaining, warp_sums, &s_total, &s_bin, &s_above);
-    prefix |= s_bin << shift;
-    pmask |= bmask << shift;
-    remaining -= s_above;
-    __syncthreads();
-  }
-  const uint32_t kstar = prefix;  // exact key of the k-th largest score
-  const uint32_t n_gt_total = (uint32_t)k - remaining;
-
-  // ---------------------------------------------------------------- ordered compaction
-  constexpr int ITEMS = 4;
-  uint32_t base_gt = 0, base_tie = 0;
-#pragma unroll 1
-  for (int start = 0; start < vis; start += BLOCK * ITEMS) {
-    const int s0 = start + threadIdx.x * ITEMS;
-    uint32_t key[ITEMS];
-    if (s0 + ITEMS <= vis) {
-      const float4 x = __ldg(src4 + s0 / 4);
-      key[0] = float_order_key(x.x);
-      key[1] = float_order_key(x.y);
-      key[2] = float_order_key(x.z);
-      key[3] = float_order_key(x.w);
+  };
+  constexpr int ITEMS = 16;  // contiguous elements per thread per tile (4 x float4 in flight)
+  // loads ITEMS keys of positions [s0, s0 + ITEMS) clipped to the segment (s0 4-aligned)
+  auto load_keys = [&](int s0, uint32_t* key) {
+    if (s0 + ITEMS <= s_hi) {
+      float4 x[ITEMS / 4];
+#pragma unroll
+      for (int u = 0; u < ITEMS / 4; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(src + s0) + u);
+#pragma unroll
+      for (int u = 0; u < ITEMS / 4; ++u) {
+        key[4 * u + 0] = float_order_key(x[u].x);
+        key[4 * u + 1] = float_order_key(x[u].y);
+        key[4 * u + 2] = float_order_key(x[u].z);
+        key[4 * u + 3] = float_order_key(x[u].w);
+      }
     } else {
 #pragma unroll
-      for (int j = 0; j < ITEMS; ++j) key[j] = (s0 + j < vis) ? float_order_key(__ldg(src + s0 + j)) : 0u;
+      for (int j = 0; j < ITEMS; ++j) key[j] = (s0 + j < s_hi) ? float_order_key(__ldg(src + s0 + j)) : 0u;
     }
-    uint32_t n_gt = 0, n_eq = 0;
+  };
+  // ordered compaction of the segment's keys with pred(key) into the candidate list;
+  // returns the count (which may exceed TOPK_CAP: nothing is written past the end)
+  auto compact = [&](auto&& pred) -> uint32_t {
+    uint32_t base = 0;
+    for (int start = s_lo; start < s_hi; start += B * ITEMS) {
+      const int s0 = start + threadIdx.x * ITEMS;
+      uint32_t key[ITEMS];
+      load_keys(s0, key);
+      uint32_t n = 0;
 #pragma unroll
-    for (int j = 0; j < ITEMS; ++j) {
-      const bool valid = s0 + j < vis;
-      n_gt += (valid && key[j] > kstar);
-      n_eq += (valid && key[j] == kstar);
+      for (int j = 0; j < ITEMS; ++j) n += (s0 + j < s_hi && pred(key[j]));
+      uint32_t pos = base + block_excl_scan<B>(n, S.warp_sums, &S.total);
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) {
+        if (s0 + j < s_hi && pred(key[j])) {
+          if (pos < (uint32_t)TOPK_CAP) {
+            S.cand_key[pos] = key[j];
+            S.cand_pos[pos] = s0 + j;
+          }
+          ++pos;
+        }
+      }
+      base += S.total;
+      __syncthreads();  // S.total is rewritten by the next scan
     }
-    const uint32_t packed = (n_gt << 16) | n_eq;  // each field <= BLOCK*ITEMS < 65536
-    const uint32_t excl = block_excl_scan<BLOCK>(packed, warp_sums, &s_total);
-    uint32_t gt_before = base_gt + (excl >> 16);
-    uint32_t eq_before = base_tie + (excl & 0xFFFFu);
+    return base;
+  };
+  // cluster-wide: (sum of counts >= k) and (every count <= TOPK_CAP)
+  auto cluster_ok = [&](uint32_t cnt) -> bool {
+    if (threadIdx.x == 0) S.counts[0] = cnt;
+    cluster_sync_all<C>();
+    uint32_t tot = 0;
+    bool fit = true;
+    if constexpr (C == 1) {
+      tot = S.counts[0];
+      fit = tot <= (uint32_t)TOPK_CAP;
+    } else {
+      auto cl = cg::this_cluster();
 #pragma unroll
-    for (int j = 0; j < ITEMS; ++j) {
-      if (s0 + j >= vis) break;
-      if (key[j] > kstar) {
-        out[gt_before + min(eq_before, remaining)] = s0 + j;
-        ++gt_before;
-      } else if (key[j] == kstar) {
-        if (eq_before < remaining) out[gt_before + eq_before] = s0 + j;
-        ++eq_before;
+      for (int r = 0; r < C; ++r) {
+        const uint32_t c = *cl.map_shared_rank(&S.counts[0], r);
+        tot += c;
+        fit = fit && c <= (uint32_t)TOPK_CAP;
       }
     }
-    const uint32_t tot = s_total;
-    base_gt += tot >> 16;
-    base_tie += tot & 0xFFFFu;
-    __syncthreads();  // s_total is rewritten by the next scan
-    if (base_gt == n_gt_total && base_tie >= remaining) break;  // every selected position found
+    cluster_sync_all<C>();  // counts[0] is rewritten later
+    return fit && tot >= (uint32_t)k;
+  };
+
+  uint32_t remaining = (uint32_t)k;
+  uint32_t prefix = 0, pmask = 0;
+  int first_level = 0;
+  bool in_smem = false;
+  int ncand = 0;
+  const uint32_t* gh = nullptr;
+
+  // ---------------------------------------------------------------- 1. sampled threshold
+  {
+    constexpr int NS = 1024;  // == B: one sample per thread
+    uint32_t T = 0;
+    if (vis > C * (TOPK_CAP / 2)) {
+      // expected sampled keys above the k-th largest, and a margin of ~4 sigma + 8
+      const float m = (float)k * (float)NS / (float)vis;
+      const int r_low = min(NS, (int)ceilf(1.5f * m + 4.f * sqrtf(m) + 8.f));
+      const long long pos = ((2LL * threadIdx.x + 1) * vis) / (2LL * NS);
+      const uint32_t sk = float_order_key(__ldg(src + pos));
+      // the r_low-th largest sampled key, to 22 bits, by two radix levels over the sample
+      uint32_t sp = 0, sm = 0, rem = (uint32_t)r_low;
+#pragma unroll 1
+      for (int lv = 0; lv < 2; ++lv) {
+        const int shift = lv == 0 ? 21 : 10;
+        for (int j = threadIdx.x; j < 2048; j += B) S.ghist[j] = 0;
+        __syncthreads();
+        if ((sk & sm) == sp) atomicAdd(&S.ghist[(sk >> shift) & 2047u], 1u);
+        __syncthreads();
+        find_bin<B, 2048>(S.ghist, rem, S.warp_sums, &S.total, &S.bin, &S.above);
+        sp |= S.bin << shift;
+        sm |= 2047u << shift;
+        rem -= S.above;
+      }
+      T = sp;  // every sampled key in the top r_low is >= T
+    }
+    const uint32_t cnt = compact([&](uint32_t kk) { return kk >= T; });
+    in_smem = cluster_ok(cnt);
+    ncand = in_smem ? (int)cnt : 0;
   }
+
+  if (!in_smem) {
+    // ---------------------------------------------------------------- 2. exact level 1
+    for (int j = threadIdx.x; j < 2048; j += B) S.hist[0][j] = 0;
+    __syncthreads();
+    {
+      const int v_lo = s_lo / 4, v_hi = s_hi / 4;  // whole float4 groups inside the segment
+      const float4* src4 = reinterpret_cast<const float4*>(src);
+      int v = v_lo + threadIdx.x;
+      for (; v + 3 * B < v_hi; v += 4 * B) {
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = __ldg(src4 + v + u * B);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          atomicAdd(&S.hist[0][float_order_key(x[u].x) >> 21], 1u);
+          atomicAdd(&S.hist[0][float_order_key(x[u].y) >> 21], 1u);
+          atomicAdd(&S.hist[0][float_order_key(x[u].z) >> 21], 1u);
+          atomicAdd(&S.hist[0][float_order_key(x[u].w) >> 21], 1u);
+        }
+      }
+      for (; v < v_hi; v += B) {
+        const float4 x = __ldg(src4 + v);
+        atomicAdd(&S.hist[0][float_order_key(x.x) >> 21], 1u);
+        atomicAdd(&S.hist[0][float_order_key(x.y) >> 21], 1u);
+        atomicAdd(&S.hist[0][float_order_key(x.z) >> 21], 1u);
+        atomicAdd(&S.hist[0][float_order_key(x.w) >> 21], 1u);
+      }
+      for (int s = v_hi * 4 + threadIdx.x; s < s_hi; s += B)
+        atomicAdd(&S.hist[0][float_order_key(__ldg(src + s)) >> 21], 1u);
+    }
+    cluster_sync_all<C>();
+    gh = reduce_hist(0, 2048);
+    find_bin<B, 2048>(gh, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    const uint32_t b1 = S.bin;
+    remaining -= S.above;
+    prefix = b1 << 21;
+    pmask = 0xFFE00000u;
+    first_level = 1;
+    const uint32_t cnt = compact([&](uint32_t kk) { return (kk >> 21) >= b1; });
+    // here the count is >= remaining by construction; only the fit matters
+    if (threadIdx.x == 0) S.counts[0] = cnt;
+    cluster_sync_all<C>();
+    in_smem = true;
+    if constexpr (C == 1) {
+      in_smem = S.counts[0] <= (uint32_t)TOPK_CAP;
+    } else {
+      auto cl = cg::this_cluster();
+#pragma unroll
+      for (int r = 0; r < C; ++r) in_smem = in_smem && (*cl.map_shared_rank(&S.counts[0], r) <= (uint32_t)TOPK_CAP);
+    }
+    cluster_sync_all<C>();
+    ncand = in_smem ? (int)cnt : 0;
+  }
+
+  // visits every element of the block's source in position order: f(key, position)
+  auto for_each_key = [&](auto&& f) {
+    if (in_smem) {
+      for (int j = threadIdx.x; j < ncand; j += B) f(S.cand_key[j], S.cand_pos[j]);
+    } else {
+      for (int s = s_lo + threadIdx.x; s < s_hi; s += B) f(float_order_key(__ldg(src + s)), s);
+    }
+  };
+
+  // ---------------------------------------------------------------- levels 2 and 3
+#pragma unroll 1
+  for (int level = first_level; level < 3; ++level) {
+    const int par = level & 1;
+    const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+    const uint32_t bmask = level == 2 ? 1023u : 2047u;
+    for (int j = threadIdx.x; j < 2048; j += B) S.hist[par][j] = 0;
+    __syncthreads();
+    for_each_key([&](uint32_t kk, int) {
+      if ((kk & pmask) == prefix) atomicAdd(&S.hist[par][(kk >> shift) & bmask], 1u);
+    });
+    cluster_sync_all<C>();
+    gh = reduce_hist(par, level == 2 ? 1024 : 2048);
+    if (level < 2)
+      find_bin<B, 2048>(gh, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    else
+      find_bin<B, 1024>(gh, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    prefix |= S.bin << shift;
+    pmask |= bmask << shift;
+    remaining -= S.above;
+  }
+  const uint32_t kstar = prefix;
+
+  // ---------------------------------------------------------------- ordered output
+  // counts of this block, then the counts of all lower-ranked blocks of the cluster
+  uint32_t base_gt = 0, base_tie = 0;
+  if constexpr (C > 1) {
+    uint32_t ngt = 0, neq = 0;
+    for_each_key([&](uint32_t kk, int) {
+      ngt += kk > kstar;
+      neq += kk == kstar;
+    });
+    block_excl_scan<B>(ngt, S.warp_sums, &S.total);
+    const uint32_t tot_gt = S.total;
+    __syncthreads();
+    block_excl_scan<B>(neq, S.warp_sums, &S.total);
+    if (threadIdx.x == 0) {
+      S.counts[0] = tot_gt;
+      S.counts[1] = S.total;
+    }
+    cluster_sync_all<C>();
+    auto cl = cg::this_cluster();
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t* rc = cl.map_shared_rank(&S.counts[0], r);
+      base_gt += rc[0];
+      base_tie += rc[1];
+    }
+  }
+  if (in_smem) {
+    constexpr int IT = 4;
+    for (int start = 0; start < ncand; start += B * IT) {
+      const int j0 = start + threadIdx.x * IT;
+      uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+      for (int j = 0; j < IT; ++j) {
+        if (j0 + j < ncand) {
+          n_gt += S.cand_key[j0 + j] > kstar;
+          n_eq += S.cand_key[j0 + j] == kstar;
+        }
+      }
+      const uint32_t excl = block_excl_scan<B>((n_gt << 16) | n_eq, S.warp_sums, &S.total);
+      uint32_t gt_before = base_gt + (excl >> 16), eq_before = base_tie + (excl & 0xFFFFu);
+#pragma unroll
+      for (int j = 0; j < IT; ++j) {
+        if (j0 + j >= ncand) break;
+        const uint32_t kk = S.cand_key[j0 + j];
+        if (kk > kstar) {
+          out[gt_before + min(eq_before, remaining)] = S.cand_pos[j0 + j];
+          ++gt_before;
+        } else if (kk == kstar) {
+          if (eq_before < remaining) out[gt_before + eq_before] = S.cand_pos[j0 + j];
+          ++eq_before;
+        }
+      }
+      base_gt += S.total >> 16;
+      base_tie += S.total & 0xFFFFu;
+      __syncthreads();
+    }
+  } else {
+    for (int start = s_lo; start < s_hi; start += B * ITEMS) {
+      const int s0 = start + threadIdx.x * ITEMS;
+      uint32_t key[ITEMS];
+      load_keys(s0, key);
+      uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) {
+        n_gt += (s0 + j < s_hi && key[j] > kstar);
+        n_eq += (s0 + j < s_hi && key[j] == kstar);
+      }
+      // per-thread counts <= 16 and block totals <= 16384 fit the packed 16-bit fields
+      const uint32_t excl = block_excl_scan<B>((n_gt << 16) | n_eq, S.warp_sums, &S.total);
+      uint32_t gt_before = base_gt + (excl >> 16), eq_before = base_tie + (excl & 0xFFFFu);
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) {
+        if (s0 + j >= s_hi) break;
+        if (key[j] > kstar) {
+          out[gt_before + min(eq_before, remaining)] = s0 + j;
+          ++gt_before;
+        } else if (key[j] == kstar) {
+          if (eq_before < remaining) out[gt_before + eq_before] = s0 + j;
+          ++eq_before;
+        }
+      }
+      base_gt += S.total >> 16;
+      base_tie += S.total & 0xFFFFu;
+      __syncthreads();
+    }
+  }
+  // no block may leave while another still reads its shared memory
+  if constexpr (C > 1) cg::this_cluster().sync();
 }
 
 }  // namespace dsa
 
 namespace dsa_host {
 
+template <int C>
+static int topk_launch_c(const dsa::TopkParams& p, long long rows, cudaStream_t stream) {
+  const int smem = (int)sizeof(dsa::TopkSmem);
+  static bool done = false;
+  if (!done) {
+    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
+    done = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
+  cfg.blockDim = dim3(dsa::TOPK_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = C > 1 ? 1 : 0;
+  if (const cudaError_t e_ = cudaLaunchKernelEx(&cfg, dsa::topk_kernel<C>, p); e_ != cudaSuccess) return cuda_fail(e_);
+  return last_launch_status();
+}
+
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
-                long long row_begin, long long row_end, int k, int* indices, cudaStream_t stream) {
+                long long row_begin, long long row_end, int k, int* indices, int max_vis, cudaStream_t stream) {
   const long long rows = row_end - row_begin;
   if (rows <= 0) return DSA_OK;
+  if (rows > 0x7FFFFFFFLL / 8) return DSA_ERR_UNSUPPORTED;
   dsa::TopkParams p;
   p.scores = scores;
   p.ld = ld;
@@ -212,9 +486,16 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
   p.row_begin = row_begin;
   p.k = k;
   p.indices = indices;
-  if (rows > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
-  dsa::topk_kernel<1024><<<(unsigned)rows, 1024, 0, stream>>>(p);
-  return last_launch_status();
+  // a cluster per row when the rows are long and few enough blocks would be busy otherwise
+  const int sms = sm_count();
+  int C = 1;
+  while (C < 8 && (long long)rows * C < 2LL * sms && (long long)max_vis > 16384LL * C) C *= 2;
+  switch (C) {
+    case 1: return topk_launch_c<1>(p, rows, stream);
+    case 2: return topk_launch_c<2>(p, rows, stream);
+    case 4: return topk_launch_c<4>(p, rows, stream);
+    default: return topk_launch_c<8>(p, rows, stream);
+  }
 }
 
 }  // namespace dsa_host

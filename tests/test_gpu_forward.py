@@ -106,6 +106,49 @@ def test_topk_long_rows_decode_length():
         assert np.array_equal(idx[b], orc.topk_row(sc[b, :n].astype(np.float64), 2048))
 
 
+@pytest.mark.parametrize("n_rows,n", [(3, 262144), (600, 40000)])
+def test_topk_candidate_overflow_paths(n_rows, n):
+    # few distinct values: the threshold bin holds far more candidates than fit in shared
+    # memory, so the kernel keeps reading the row from global memory; 3 rows use a
+    # cluster of blocks per row, 600 rows one block per row
+    rng = np.random.default_rng(n_rows)
+    vis = [n - (r % 3) for r in range(n_rows)]
+    cu_q = np.arange(n_rows + 1, dtype=np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(vis)]).astype(np.int32)
+    ld = (n + 3) // 4 * 4
+    sc = np.zeros((n_rows, ld), np.float32)
+    for r in range(n_rows):
+        sc[r, :vis[r]] = rng.integers(0, 3, size=vis[r]).astype(np.float32)
+    idx = dsa.topk(torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                   2048).cpu().numpy()
+    for r in range(0, n_rows, max(1, n_rows // 8)):
+        assert np.array_equal(idx[r], orc.topk_row(sc[r, :vis[r]].astype(np.float64), 2048)), r
+
+
+def test_topk_adversarial_rows():
+    # rows built so that a strided sample of the row misjudges the threshold: the largest
+    # values sit exactly on evenly spaced positions, or everywhere except there; the
+    # selected set must still be exact
+    n, k = 131072, 2048
+    rng = np.random.default_rng(11)
+    sc = np.zeros((4, n), np.float32)
+    spots = ((2 * np.arange(1024) + 1) * n) // 2048
+    sc[0] = rng.standard_normal(n).astype(np.float32)
+    sc[0, spots] = 10.0                       # 1024 huge values on the sampled positions
+    sc[1] = rng.standard_normal(n).astype(np.float32) - 5.0
+    sc[1, spots] = 10.0
+    sc[1, np.arange(7, n, 64)] = 3.0          # the rest of the top-k between the samples
+    sc[2] = 1.0
+    sc[2, spots] = -1.0                       # everything ties except the sampled ones
+    sc[3] = -np.arange(n, dtype=np.float32)   # strictly decreasing
+    cu_q = np.arange(5, dtype=np.int32)
+    cu_k = (np.arange(5) * n).astype(np.int32)
+    idx = dsa.topk(torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                   k).cpu().numpy()
+    for r in range(4):
+        assert np.array_equal(idx[r], orc.topk_row(sc[r].astype(np.float64), k)), r
+
+
 def test_topk_deterministic_repeat():
     sc, cu_q, cu_k = _topk_case([70000] * 4, 2048, seed=9, ties=True)
     args = (torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(), 2048)
