@@ -43,6 +43,7 @@ struct TopkParams {
   long long row_begin;
   int k;
   int* indices;
+  int only_marked;  // exact kernel: process only the rows the fast kernel marked with -2
 };
 
 constexpr int TOPK_THREADS = 1024;
@@ -139,6 +140,8 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) 
   int* out = p.indices + (row - p.row_begin) * k;
   const float* src = p.scores + (row - p.row_begin) * p.ld;
 
+  // (uniform over the cluster: every block reads out[0] before any block writes the row)
+  if (p.only_marked && __ldg(out) != -2) return;
   if (vis <= k) {  // uniform over the cluster: no cluster barrier is reached by anyone
     if (rank == 0)
       for (int j = threadIdx.x; j < k; j += B) out[j] = j < vis ? j : -1;
@@ -444,21 +447,285 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) 
   if constexpr (C > 1) cg::this_cluster().sync();
 }
 
+// ======================================================================================
+// Fast path.  512 threads, two blocks per SM.  A sampled lower bound T is taken first (the
+// same 2048 strided positions in every block of the row); one streaming pass then
+// appends the keys >= T of the block's segment to a shared-memory candidate list with
+// warp-level scans only (no block barrier inside the pass, 4 x float4 loads in flight per
+// thread); three radix levels over the candidates give K*; the selected positions are
+// marked in two shared-memory bitmaps (keys > K*, ties at K*) and written in position
+// order with one block scan.  A row the fast path cannot settle (the sampled bound let
+// fewer than k keys through, a candidate list overflowed, or a segment is longer than
+// the bitmaps) gets -2 in its first output slot and is finished by the exact kernel.
+constexpr int FT = 512;
+constexpr int FCAP = 6144;
+constexpr int FWORDS = 4096;  // bitmap words: segments up to 131072 positions
+
+struct FastSmem {
+  uint32_t cand_key[FCAP];
+  int cand_pos[FCAP];
+  uint32_t hist[2][2048];
+  uint32_t ghist[2048];
+  uint32_t gtb[FWORDS];   // positions with key > K*
+  uint32_t tieb[FWORDS];  // positions with key == K*
+  uint32_t warp_sums[32];
+  uint32_t total, bin, above, ncand;
+  uint32_t counts[2];
+};
+
+template <int C>
+__global__ void __launch_bounds__(FT, 2) topk_fast_kernel(const TopkParams p) {
+  constexpr int B = FT;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FastSmem& S = *reinterpret_cast<FastSmem*>(smem_raw);
+  const int rank = (C > 1) ? (int)cg::this_cluster().block_rank() : 0;
+  const int lane = threadIdx.x % 32;
+  const long long row = p.row_begin + blockIdx.x / C;
+  int lo = 0, hi = p.batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int i = (int)(row - p.cu_q[b]);
+  const int Lq = p.cu_q[b + 1] - p.cu_q[b];
+  const int Lk = p.cu_k[b + 1] - p.cu_k[b];
+  const int vis = min(max(i + Lk - Lq + 1, 0), Lk);
+  const int k = p.k;
+  int* out = p.indices + (row - p.row_begin) * k;
+  const float* src = p.scores + (row - p.row_begin) * p.ld;
+  if (vis <= k) {
+    if (rank == 0)
+      for (int j = threadIdx.x; j < k; j += B) out[j] = j < vis ? j : -1;
+    return;
+  }
+  const int seg = ((vis + C - 1) / C + 3) & ~3;
+  if (seg > FWORDS * 32) {  // uniform over the row
+    if (rank == 0 && threadIdx.x == 0) out[0] = -2;
+    return;
+  }
+  const int s_lo = min(rank * seg, vis), s_hi = min(s_lo + seg, vis);
+  const int nwords = (s_hi - s_lo + 31) / 32;
+
+  // ---------------------------------------------------------------- sampled bound T
+  uint32_t T = 0;
+  if (vis > C * (FCAP / 2)) {
+    constexpr int NS = 2048, PER = NS / B;
+    const float m = (float)k * (float)NS / (float)vis;
+    const int r_low = min(NS, (int)ceilf(m + 3.f * sqrtf(m) + 8.f));
+    uint32_t sk[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const long long pos = ((2LL * (threadIdx.x + u * B) + 1) * vis) / (2LL * NS);
+      sk[u] = float_order_key(__ldg(src + pos));
+    }
+    uint32_t sp = 0, sm = 0, rem = (uint32_t)r_low;
+#pragma unroll 1
+    for (int lv = 0; lv < 2; ++lv) {
+      const int shift = lv == 0 ? 21 : 10;
+      for (int j = threadIdx.x; j < 2048; j += B) S.ghist[j] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < PER; ++u)
+        if ((sk[u] & sm) == sp) atomicAdd(&S.ghist[(sk[u] >> shift) & 2047u], 1u);
+      __syncthreads();
+      find_bin<B, 2048>(S.ghist, rem, S.warp_sums, &S.total, &S.bin, &S.above);
+      sp |= S.bin << shift;
+      sm |= 2047u << shift;
+      rem -= S.above;
+    }
+    T = sp;
+  }
+
+  // ---------------------------------------------------------------- streaming filter
+  if (threadIdx.x == 0) S.ncand = 0;
+  for (int w = threadIdx.x; w < nwords; w += B) {
+    S.gtb[w] = 0;
+    S.tieb[w] = 0;
+  }
+  __syncthreads();
+  {
+    constexpr int IT = 16;
+    for (int start = s_lo; start < s_hi; start += B * IT) {
+      const int s0 = start + threadIdx.x * IT;
+      uint32_t key[IT];
+      if (s0 + IT <= s_hi) {
+        float4 x[IT / 4];
+#pragma unroll
+        for (int u = 0; u < IT / 4; ++u) x[u] = __ldg(reinterpret_cast<const float4*>(src + s0) + u);
+#pragma unroll
+        for (int u = 0; u < IT / 4; ++u) {
+          key[4 * u + 0] = float_order_key(x[u].x);
+          key[4 * u + 1] = float_order_key(x[u].y);
+          key[4 * u + 2] = float_order_key(x[u].z);
+          key[4 * u + 3] = float_order_key(x[u].w);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < IT; ++j) key[j] = (s0 + j < s_hi) ? float_order_key(__ldg(src + s0 + j)) : 0u;
+      }
+      uint32_t n = 0;
+#pragma unroll
+      for (int j = 0; j < IT; ++j) n += (s0 + j < s_hi && key[j] >= T);
+      // warp-level exclusive scan and one shared counter bump per warp
+      uint32_t x = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      uint32_t base = 0;
+      if (lane == 31 && x) base = atomicAdd(&S.ncand, x);
+      base = __shfl_sync(0xffffffffu, base, 31);
+      uint32_t pos = base + x - n;
+#pragma unroll
+      for (int j = 0; j < IT; ++j) {
+        if (s0 + j < s_hi && key[j] >= T) {
+          if (pos < (uint32_t)FCAP) {
+            S.cand_key[pos] = key[j];
+            S.cand_pos[pos] = s0 + j;
+          }
+          ++pos;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t cnt = S.ncand;
+  // cluster-wide: enough keys passed, and every list fit
+  if (threadIdx.x == 0) S.counts[0] = cnt;
+  cluster_sync_all<C>();
+  bool ok;
+  {
+    uint32_t tot = 0;
+    bool fit = true;
+    if constexpr (C == 1) {
+      tot = S.counts[0];
+      fit = tot <= (uint32_t)FCAP;
+    } else {
+      auto cl = cg::this_cluster();
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        const uint32_t c = *cl.map_shared_rank(&S.counts[0], r);
+        tot += c;
+        fit = fit && c <= (uint32_t)FCAP;
+      }
+    }
+    ok = fit && tot >= (uint32_t)k;
+  }
+  cluster_sync_all<C>();
+  if (!ok) {
+    if (rank == 0 && threadIdx.x == 0) out[0] = -2;
+    return;
+  }
+  const int ncand = (int)cnt;
+
+  // ---------------------------------------------------------------- radix levels
+  uint32_t remaining = (uint32_t)k, prefix = 0, pmask = 0;
+#pragma unroll 1
+  for (int level = 0; level < 3; ++level) {
+    const int par = level & 1;
+    const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+    const uint32_t bmask = level == 2 ? 1023u : 2047u;
+    for (int j = threadIdx.x; j < 2048; j += B) S.hist[par][j] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < ncand; j += B) {
+      const uint32_t kk = S.cand_key[j];
+      if ((kk & pmask) == prefix) atomicAdd(&S.hist[par][(kk >> shift) & bmask], 1u);
+    }
+    cluster_sync_all<C>();
+    const uint32_t* gh;
+    if constexpr (C == 1) {
+      gh = S.hist[par];
+    } else {
+      auto cl = cg::this_cluster();
+      for (int j = threadIdx.x; j < 2048; j += B) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int r = 0; r < C; ++r) t += cl.map_shared_rank(&S.hist[par][0], r)[j];
+        S.ghist[j] = t;
+      }
+      __syncthreads();
+      gh = S.ghist;
+    }
+    if (level < 2)
+      find_bin<B, 2048>(gh, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    else
+      find_bin<B, 1024>(gh, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    prefix |= S.bin << shift;
+    pmask |= bmask << shift;
+    remaining -= S.above;
+  }
+  const uint32_t kstar = prefix;
+
+  // ---------------------------------------------------------------- mark and write in order
+  for (int j = threadIdx.x; j < ncand; j += B) {
+    const uint32_t kk = S.cand_key[j];
+    if (kk >= kstar) {
+      const int r = S.cand_pos[j] - s_lo;
+      atomicOr(kk > kstar ? &S.gtb[r >> 5] : &S.tieb[r >> 5], 1u << (r & 31));
+    }
+  }
+  __syncthreads();
+  const int wpt = (nwords + B - 1) / B;
+  const int w0 = threadIdx.x * wpt, w1 = min(w0 + wpt, nwords);
+  uint32_t my_gt = 0, my_tie = 0;
+  for (int w = w0; w < w1; ++w) {
+    my_gt += __popc(S.gtb[w]);
+    my_tie += __popc(S.tieb[w]);
+  }
+  uint32_t gt_before = block_excl_scan<B>(my_gt, S.warp_sums, &S.total);
+  const uint32_t tot_gt = S.total;
+  __syncthreads();
+  uint32_t tie_before = block_excl_scan<B>(my_tie, S.warp_sums, &S.total);
+  const uint32_t tot_tie = S.total;
+  if constexpr (C > 1) {
+    if (threadIdx.x == 0) {
+      S.counts[0] = tot_gt;
+      S.counts[1] = tot_tie;
+    }
+    cluster_sync_all<C>();
+    auto cl = cg::this_cluster();
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t* rc = cl.map_shared_rank(&S.counts[0], r);
+      gt_before += rc[0];
+      tie_before += rc[1];
+    }
+  }
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = S.gtb[w] | S.tieb[w];
+    const uint32_t gmask = S.gtb[w];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int pos = s_lo + w * 32 + bit;
+      if (gmask & (1u << bit)) {
+        out[gt_before + min(tie_before, remaining)] = pos;
+        ++gt_before;
+      } else {
+        if (tie_before < remaining) out[gt_before + tie_before] = pos;
+        ++tie_before;
+      }
+    }
+  }
+  if constexpr (C > 1) cg::this_cluster().sync();
+}
+
 }  // namespace dsa
 
 namespace dsa_host {
 
-template <int C>
-static int topk_launch_c(const dsa::TopkParams& p, long long rows, cudaStream_t stream) {
-  const int smem = (int)sizeof(dsa::TopkSmem);
-  static bool done = false;
-  if (!done) {
-    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
-    done = true;
+template <typename Kern>
+static int launch_cluster(Kern kern, const dsa::TopkParams& p, long long rows, int C, int threads, int smem,
+                          bool& attr_done, cudaStream_t stream) {
+  if (!attr_done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    attr_done = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
-  cfg.blockDim = dim3(dsa::TOPK_THREADS, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -468,8 +735,20 @@ static int topk_launch_c(const dsa::TopkParams& p, long long rows, cudaStream_t 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = C > 1 ? 1 : 0;
-  if (const cudaError_t e_ = cudaLaunchKernelEx(&cfg, dsa::topk_kernel<C>, p); e_ != cudaSuccess) return cuda_fail(e_);
+  if (const cudaError_t e_ = cudaLaunchKernelEx(&cfg, kern, p); e_ != cudaSuccess) return cuda_fail(e_);
   return last_launch_status();
+}
+
+template <int C>
+static int topk_launch_c(dsa::TopkParams p, long long rows, cudaStream_t stream) {
+  static bool fast_done = false, exact_done = false;
+  p.only_marked = 0;
+  int st = launch_cluster(dsa::topk_fast_kernel<C>, p, rows, C, dsa::FT, (int)sizeof(dsa::FastSmem), fast_done,
+                          stream);
+  if (st != DSA_OK) return st;
+  p.only_marked = 1;  // rows the fast path left marked
+  return launch_cluster(dsa::topk_kernel<C>, p, rows, C, dsa::TOPK_THREADS, (int)sizeof(dsa::TopkSmem), exact_done,
+                        stream);
 }
 
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
@@ -486,6 +765,7 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
   p.row_begin = row_begin;
   p.k = k;
   p.indices = indices;
+  p.only_marked = 0;
   // a cluster per row when the rows are long and few enough blocks would be busy otherwise
   const int sms = sm_count();
   int C = 1;
