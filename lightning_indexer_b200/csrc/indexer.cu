@@ -45,7 +45,7 @@ struct Item {
   int tile_begin, tile_end;
 };
 
-template <int NTOK>
+template <int NTOK, int TILE_KEYS = 128>
 __device__ __forceinline__ bool decode_item(long long item, const IndexerParams& p, Item& it) {
   const long long blk = item / p.max_splits;
   const int split = (int)(item % p.max_splits);
@@ -72,7 +72,7 @@ __device__ __forceinline__ bool decode_item(long long item, const IndexerParams&
       it.k0 = p.cu_k[b];
       const int last = it.i0 + it.ntok - 1;
       const int vis = min(max(last + it.Lk - it.Lq + 1, 0), it.Lk);
-      const int ntiles = (vis + 127) / 128;
+      const int ntiles = (vis + TILE_KEYS - 1) / TILE_KEYS;
       it.tile_begin = split * p.tiles_per_split;
       it.tile_end = min(ntiles, it.tile_begin + p.tiles_per_split);
       return it.tile_begin < it.tile_end;
@@ -368,6 +368,10 @@ static int launch_indexer(const void* q_idx, const void* k_idx, const void* w, c
   return last_launch_status();
 }
 
+int indexer2_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
+                    long long total_q, long long total_k, int max_seqlen_k, int H_I, int d_I, long long row_begin,
+                    long long row_end, float* scores, long long ld, cudaStream_t stream);
+
 int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                    int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k,
                    int H_I, int d_I, long long row_begin, long long row_end, float* scores, long long ld,
@@ -375,6 +379,10 @@ int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const in
   const long long rows = row_end - row_begin;
   // Few query rows per sequence (decode): one token per block, split the keys finely.
   const bool decode_like = rows <= 2LL * batch;
+  // Many rows: CTA pairs (tcgen05 cta_group::2) for the 128-wide indexer heads.
+  if (!decode_like && d_I == 128 && (H_I == 64 || H_I == 32))
+    return indexer2_launch(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k, H_I, d_I, row_begin,
+                           row_end, scores, ld, stream);
 #define DSA_IDX(HI, DI, NT, EW, AS, BS, TPS)                                                                  \
   return launch_indexer<HI, DI, NT, EW, AS, BS>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k,     \
                                                 max_seqlen_q, max_seqlen_k, row_begin, row_end, scores, ld, \

@@ -1,0 +1,315 @@
+// Lightning-indexer scores on CTA pairs (tcgen05 cta_group::2), sm_100a.
+//
+// Same computation and epilogue as indexer.cu (Keye-VL-2.0 report summary,
+// mqxn.cn/news/1966, section 1: MQA-shared lightning indexer), with the MMA spread over a
+// pair of CTAs in a cluster of 2:
+//   M = 256 keys per tile (128 from each CTA's shared memory),
+//   N = NTOK tokens x H_I heads (each CTA holds the q_idx rows of half of the tokens),
+//   D = 128 keys x N columns in each CTA's tensor memory.
+// Per SM this halves the tensor core's B-operand reads from shared memory (each SM reads
+// its 128 rows of A and N/2 rows of B per MMA instead of 128 + N), which is what the
+// one-CTA kernel is bound by at N = 256.  The even CTA issues the MMAs; both CTAs load their
+// own operand halves with TMA and run their own epilogue over their own 128 keys.
+//   warp 0   TMA producer (both CTAs; completion counted on the even CTA's barriers)
+//   warp 1   MMA issuer (even CTA only) + TMEM allocation (both, cta_group::2)
+//   warps 2+ epilogue (both): tcgen05.ld -> fp32 ReLU/FMA over heads -> stores
+// Releases go back through multicast commits (stage free, accumulator full) to both CTAs
+// and through remote arrivals (accumulator drained) to the even CTA.
+#include "common.cuh"
+
+namespace dsa {
+
+template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES>
+struct Indexer2Cfg {
+  static constexpr int N = NTOK * H_I;  // MMA N over the pair
+  static constexpr int NH = N / 2;      // q_idx rows held by each CTA
+  static_assert(N % 32 == 0 && N >= 32 && N <= 256 && NTOK % 2 == 0, "pair UMMA N");
+  static constexpr int PANEL = D_I >= 64 ? 64 : D_I;
+  static constexpr int SWZ = PANEL * 2;
+  static constexpr int NPANEL = D_I / PANEL;
+  static constexpr int KSTEPS = PANEL / 16;
+  static constexpr int A_BYTES = 128 * D_I * 2;
+  static constexpr int B_BYTES = NH * D_I * 2;
+  static constexpr int TMEM_COLS = (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
+  static constexpr int EPI_THREADS = NUM_EPI_WARPS * 32;
+  static constexpr int THREADS = 64 + EPI_THREADS;
+  static constexpr int COL_PARTS = NUM_EPI_WARPS / 4;
+  static constexpr int CPT = N / COL_PARTS;
+  static_assert(CPT % H_I == 0 && H_I >= 32, "pair kernel epilogue: whole heads of whole tokens per thread");
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + A_STAGES * A_BYTES;
+  static constexpr int OFF_W = OFF_B + B_STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_W + N * 4;
+  static constexpr int NUM_BARS = 2 * A_STAGES + 2 * B_STAGES + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(256, N);
+  static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB per-block shared memory limit");
+};
+
+template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES>
+__global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>::THREADS, 1)
+    indexer2_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                    const IndexerParams p) {
+  using C = Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
+  constexpr int TILE_KEYS = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sB = smem + C::OFF_B;
+  float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* a_full = bars;                                   // even CTA: both halves landed
+  uint64_t* a_empty = bars + A_STAGES;                       // both CTAs: stage free
+  uint64_t* b_full = bars + 2 * A_STAGES;                    // even CTA
+  uint64_t* b_empty = bars + 2 * A_STAGES + B_STAGES;        // both CTAs
+  uint64_t* acc_full = bars + 2 * A_STAGES + 2 * B_STAGES;   // both CTAs
+  uint64_t* acc_empty = acc_full + 2;                        // even CTA: both epilogues drained
+  uint64_t* mma_done = acc_full + 4;                         // even CTA
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();  // 0 = MMA-issuing CTA of the pair
+  const long long pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < A_STAGES; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < B_STAGES; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 2 * NUM_EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc2(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish2();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM of the pair allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int as = 0, bs = 0;
+      uint32_t aph = 0, bph = 0;
+      bool ok = true;
+      for (long long item = pair; item < p.n_items && ok; item += npairs) {
+        Item it;
+        if (!decode_item<NTOK, TILE_KEYS>(item, p, it)) continue;
+        if (!(ok = mbar_wait(&b_empty[bs], bph ^ 1, abort_flag, 11))) break;
+        if (rank == 0) mbar_arrive_expect_tx(&b_full[bs], 2 * C::B_BYTES);
+        const uint32_t bfull = map_to_rank(&b_full[bs], 0);
+        for (int pn = 0; pn < C::NPANEL; ++pn)
+          tma_load_2d_pair(sB + bs * C::B_BYTES + pn * C::NH * C::SWZ, &tmap_q, bfull, pn * C::PANEL,
+                           (int)((it.t0 + rank * (NTOK / 2)) * H_I));
+        if (++bs == B_STAGES) { bs = 0; bph ^= 1; }
+        for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
+          if (!(ok = mbar_wait(&a_empty[as], aph ^ 1, abort_flag, 12))) break;
+          if (rank == 0) mbar_arrive_expect_tx(&a_full[as], 2 * C::A_BYTES);
+          const uint32_t afull = map_to_rank(&a_full[as], 0);
+          for (int pn = 0; pn < C::NPANEL; ++pn)
+            tma_load_2d_pair(sA + as * C::A_BYTES + pn * 128 * C::SWZ, &tmap_k, afull, pn * C::PANEL,
+                             it.k0 + tile * TILE_KEYS + (int)rank * 128);
+          if (++as == A_STAGES) { as = 0; aph ^= 1; }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int i = 0; i < A_STAGES; ++i) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(smem_u32(&a_full[i]), aph ^ (i >= as ? 1u : 0u)) &&
+                 globaltimer_ns() - t0 < 200000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int as = 0, bs = 0, ab = 0;
+      uint32_t aph = 0, bph = 0, abph = 0;
+      bool ok = true;
+      for (long long item = pair; item < p.n_items && ok; item += npairs) {
+        Item it;
+        if (!decode_item<NTOK, TILE_KEYS>(item, p, it)) continue;
+        if (!(ok = mbar_wait(&b_full[bs], bph, abort_flag, 13))) break;
+        const uint32_t b_base = smem_u32(sB + bs * C::B_BYTES);
+        for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
+          if (!(ok = mbar_wait(&acc_empty[ab], abph ^ 1, abort_flag, 14))) break;
+          tc_fence_after();
+          if (!(ok = mbar_wait(&a_full[as], aph, abort_flag, 15))) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + as * C::A_BYTES);
+          const uint32_t d_tmem = tmem_base + ab * C::N;
+#pragma unroll
+          for (int pn = 0; pn < C::NPANEL; ++pn) {
+#pragma unroll
+            for (int kk = 0; kk < C::KSTEPS; ++kk) {
+              const uint64_t adesc = smem_desc_kmajor(a_base + pn * 128 * C::SWZ + kk * 32, C::SWZ);
+              const uint64_t bdesc = smem_desc_kmajor(b_base + pn * C::NH * C::SWZ + kk * 32, C::SWZ);
+              umma2_bf16(d_tmem, adesc, bdesc, C::IDESC, (pn | kk) != 0);
+            }
+          }
+          umma2_commit_mc(&a_empty[as], 0x3);
+          umma2_commit_mc(&acc_full[ab], 0x3);
+          if (++as == A_STAGES) { as = 0; aph ^= 1; }
+          if (++ab == 2) { ab = 0; abph ^= 1; }
+        }
+        if (!ok) break;
+        umma2_commit_mc(&b_empty[bs], 0x3);
+        if (++bs == B_STAGES) { bs = 0; bph ^= 1; }
+      }
+      umma2_commit_mc(mma_done, 0x1);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int ep = warp - 2;
+    const int lane_grp = warp % 4;
+    const int col_part = ep / 4;
+    const int ep_tid = ep * 32 + lane;
+    const int col0 = col_part * C::CPT;
+    const uint32_t lane_off = (uint32_t)(lane_grp * 32) << 16;
+    const uint32_t acc_empty0 = map_to_rank(&acc_empty[0], 0);
+    const uint32_t acc_empty1 = map_to_rank(&acc_empty[1], 0);
+    int ab = 0;
+    uint32_t abph = 0;
+    bool ok = true;
+    float* w_s = sW;
+    for (long long item = pair; item < p.n_items && ok; item += npairs) {
+      Item it;
+      if (!decode_item<NTOK, TILE_KEYS>(item, p, it)) continue;
+      named_bar_sync(1, C::EPI_THREADS);
+      for (int i = ep_tid; i < C::N; i += C::EPI_THREADS) {
+        const int t = i / H_I;
+        w_s[i] = (t < it.ntok) ? bf16_bits_to_f32(p.w[(it.t0 + t) * H_I + (i % H_I)]) : 0.f;
+      }
+      named_bar_sync(1, C::EPI_THREADS);
+      const int dvis = it.Lk - it.Lq + 1;
+      float wr[C::CPT];
+#pragma unroll
+      for (int c = 0; c < C::CPT; ++c) wr[c] = w_s[col0 + c];
+      for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
+        if (!(ok = mbar_wait(&acc_full[ab], abph, abort_flag, 16))) break;
+        tc_fence_after();
+        const int s = tile * TILE_KEYS + (int)rank * 128 + lane_grp * 32 + lane;
+        const uint32_t tbase = tmem_base + lane_off + ab * C::N + col0;
+        float* out_row0 = p.scores + (it.t0 - p.row_begin) * p.ld + s;
+#pragma unroll
+        for (int c = 0; c < C::CPT; c += H_I) {
+          const int tok = (col0 + c) / H_I;
+          float acc = 0.f;
+#pragma unroll
+          for (int h0 = 0; h0 < H_I; h0 += 16) {
+            float v[16];
+            tmem_ld_x16_sync(tbase + c + h0, v);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) acc = fmaf(wr[c + h0 + q], fmaxf(v[q], 0.f), acc);
+          }
+          const int vis = min(max(it.i0 + tok + dvis, 0), it.Lk);
+          if (tok < it.ntok && s < vis) out_row0[(long long)tok * p.ld] = acc;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ab == 0 ? acc_empty0 : acc_empty1);
+        if (++ab == 2) { ab = 0; abph ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA of the pair leaves while the other may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc2(tmem_base, C::TMEM_COLS);
+}
+
+}  // namespace dsa
+
+namespace dsa_host {
+
+template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES>
+static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
+                           int batch, long long total_q, long long total_k, int max_seqlen_k, long long row_begin,
+                           long long row_end, float* scores, long long ld, int tiles_per_split,
+                           cudaStream_t stream) {
+  using C = dsa::Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
+  auto kern = dsa::indexer2_kernel<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
+  static bool attr_done = false;
+  const int smem = std::max(C::SMEM_BYTES, 120 * 1024);
+  if (!attr_done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    attr_done = true;
+  }
+  CUtensorMap tk, tq;
+  int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)total_k, D_I, (uint64_t)D_I * 2, 128, C::PANEL, C::SWZ);
+  if (st != DSA_OK) return st;
+  st = make_tmap_bf16_2d(&tq, q_idx, (uint64_t)total_q * H_I, D_I, (uint64_t)D_I * 2, C::NH, C::PANEL, C::SWZ);
+  if (st != DSA_OK) return st;
+  dsa::IndexerParams p;
+  p.w = static_cast<const uint16_t*>(w);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.row_begin = row_begin;
+  p.row_end = row_end;
+  p.scores = scores;
+  p.ld = ld;
+  p.tiles_per_split = tiles_per_split;
+  const int max_tiles = (max_seqlen_k + 255) / 256;
+  p.max_splits = std::max(1, (max_tiles + tiles_per_split - 1) / tiles_per_split);
+  const long long rows = row_end - row_begin;
+  const long long nblk = (rows + NTOK - 1) / NTOK + batch;
+  p.n_items = nblk * p.max_splits;
+  const long long pairs = std::min<long long>(p.n_items, (long long)(sm_count() / 2));
+  if (pairs <= 0) return DSA_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (const cudaError_t e_ = cudaLaunchKernelEx(&cfg, kern, tk, tq, p); e_ != cudaSuccess) return cuda_fail(e_);
+  return last_launch_status();
+}
+
+// 128K-class prefill shapes on CTA pairs; returns DSA_ERR_UNSUPPORTED for other shapes
+int indexer2_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
+                    long long total_q, long long total_k, int max_seqlen_k, int H_I, int d_I, long long row_begin,
+                    long long row_end, float* scores, long long ld, cudaStream_t stream) {
+  if (H_I == 64 && d_I == 128)
+    return launch_indexer2<64, 128, 4, 8, 4, 2>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k,
+                                                row_begin, row_end, scores, ld, 32, stream);
+  if (H_I == 32 && d_I == 128)
+    return launch_indexer2<32, 128, 8, 8, 4, 2>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k,
+                                                row_begin, row_end, scores, ld, 32, stream);
+  return DSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace dsa_host

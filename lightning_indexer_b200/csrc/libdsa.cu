@@ -2,6 +2,7 @@
 // device status word is shared without relocatable device code.
 #include "api.cu"
 #include "indexer.cu"
+#include "indexer2.cu"
 #include "topk.cu"
 #include "sparse_attn.cu"
 #include "sparse_attn_bwd.cu"
