@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode"],
                     help="run one kernel on a small case (for profiler captures) instead of the bench")
     ap.add_argument("--case-len", type=int, default=16384, help="sequence length of the --case workload")
+    ap.add_argument("--case-chunk", type=int, default=0,
+                    help="indexer case: only the last N query rows (one late prefill chunk)")
     return ap.parse_args()
 
 
@@ -349,25 +351,28 @@ def run_case(args):
     cu_q = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
     cu_k = torch.from_numpy(wl.cu_seqlens_k.astype(np.int32)).to(device)
     Tq, Lk = wl.Tq, int(wl.seqlens_k.max())
-    scores = dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk)
-    idx = dsa.topk(scores, cu_q, cu_k, wl.topk)
+    r0 = Tq - args.case_chunk if (args.case == "indexer" and args.case_chunk > 0) else 0
+    scores = dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, r0, Tq)
+    idx = dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for it in range(args.warmup + args.steps):
         if it == args.warmup:
             a.record()
         if args.case in ("indexer", "decode"):
-            dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, scores=scores)
+            dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, r0, Tq, scores=scores)
         if args.case in ("topk", "decode"):
-            dsa.topk(scores, cu_q, cu_k, wl.topk, indices=idx)
+            dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq, indices=idx)
         if args.case == "sparse_attn":
             dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu_q, cu_k)
         if args.case == "decode":
             dsa.sparse_attn_decode(t["Q"], t["K"], t["V"], idx, cu_k)
     b.record()
     torch.cuda.synchronize()
-    print(json.dumps({"case": args.case, "len": L, "ms_per_iter": a.elapsed_time(b) / max(1, args.steps),
-                      "causal_pairs": wl.causal_pairs(), "selected_pairs": wl.selected_pairs()}))
+    pairs = sum(min(r + 1, Lk) for r in range(r0, Tq)) if wl.kind != "decode" else wl.causal_pairs()
+    ms = a.elapsed_time(b) / max(1, args.steps)
+    print(json.dumps({"case": args.case, "len": L, "rows": [r0, Tq], "ms_per_iter": ms, "causal_pairs_in_rows": pairs,
+                      "indexer_tflops": pairs * wl.H_I * wl.d_I * 2 / (ms / 1e3) / 1e12}))
 
 
 def run_train(args, device):

@@ -25,6 +25,7 @@ namespace dsa {
 
 struct IndexerParams {
   const uint16_t* w;  // [total_q, H_I] bf16
+  long long w_elems;  // total_q * H_I
   const int* cu_q;
   const int* cu_k;
   int batch;
@@ -45,10 +46,12 @@ struct Item {
   int tile_begin, tile_end;
 };
 
+// Work item -> (token block, key-tile range).  Items are numbered split-major
+// (item = split * blocks + block) with blocks heaviest-first, so consecutive item numbers,
+// which go to consecutive CTAs, are all non-empty for the first split of every block and
+// the empty (split beyond a light block's tiles) items bunch up at the end.
 template <int NTOK, int TILE_KEYS = 128>
 __device__ __forceinline__ bool decode_item(long long item, const IndexerParams& p, Item& it) {
-  const long long blk = item / p.max_splits;
-  const int split = (int)(item % p.max_splits);
   // count the blocks in this row chunk; blocks are numbered from the last one (heaviest)
   long long total = 0;
   for (int b = 0; b < p.batch; ++b) {
@@ -56,7 +59,11 @@ __device__ __forceinline__ bool decode_item(long long item, const IndexerParams&
     const long long hi = min((long long)p.cu_q[b + 1], p.row_end);
     if (hi > lo) total += (hi - lo + NTOK - 1) / NTOK;
   }
-  if (blk >= total) return false;
+  if (total == 0) return false;
+  const long long split_ll = item / total;
+  if (split_ll >= p.max_splits) return false;
+  const int split = (int)split_ll;
+  const long long blk = item % total;
   long long r = total - 1 - blk;  // ascending block number
   for (int b = 0; b < p.batch; ++b) {
     const long long lo = max((long long)p.cu_q[b], p.row_begin);
@@ -348,6 +355,7 @@ static int launch_indexer(const void* q_idx, const void* k_idx, const void* w, c
 
   dsa::IndexerParams p;
   p.w = static_cast<const uint16_t*>(w);
+  p.w_elems = total_q * H_I;
   p.cu_q = cu_q;
   p.cu_k = cu_k;
   p.batch = batch;

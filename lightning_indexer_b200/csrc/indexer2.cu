@@ -39,7 +39,7 @@ struct Indexer2Cfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + A_STAGES * A_BYTES;
   static constexpr int OFF_W = OFF_B + B_STAGES * B_BYTES;
-  static constexpr int OFF_BAR = OFF_W + N * 4;
+  static constexpr int OFF_BAR = OFF_W + 2 * N * 2;  // two bf16 weight buffers
   static constexpr int NUM_BARS = 2 * A_STAGES + 2 * B_STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -191,23 +191,47 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
     const uint32_t lane_off = (uint32_t)(lane_grp * 32) << 16;
     const uint32_t acc_empty0 = map_to_rank(&acc_empty[0], 0);
     const uint32_t acc_empty1 = map_to_rank(&acc_empty[1], 0);
+    uint16_t* w_s = reinterpret_cast<uint16_t*>(sW);  // [2][N] bf16, the next item's prefetched
+    // the head weights of an item (bf16, N values = N*2 bytes) go to w_s[buf] with 16-byte
+    // asynchronous copies; rows past the block's valid tokens are copied too (never used)
+    auto prefetch_w = [&](const Item& nx, int buf) {
+      constexpr int CHUNKS = C::N * 2 / 16;
+      if (ep_tid < CHUNKS) {
+        const uint16_t* src = p.w + nx.t0 * H_I + ep_tid * 8;
+        const bool valid = (nx.t0 * H_I + ep_tid * 8 + 8) <= p.w_elems;
+        cp_async_16(smem_u32(w_s + buf * C::N + ep_tid * 8), valid ? src : p.w, valid);
+      }
+      cp_async_commit();
+    };
     int ab = 0;
     uint32_t abph = 0;
     bool ok = true;
-    float* w_s = sW;
-    for (long long item = pair; item < p.n_items && ok; item += npairs) {
-      Item it;
-      if (!decode_item<NTOK, TILE_KEYS>(item, p, it)) continue;
-      named_bar_sync(1, C::EPI_THREADS);
-      for (int i = ep_tid; i < C::N; i += C::EPI_THREADS) {
-        const int t = i / H_I;
-        w_s[i] = (t < it.ntok) ? bf16_bits_to_f32(p.w[(it.t0 + t) * H_I + (i % H_I)]) : 0.f;
-      }
-      named_bar_sync(1, C::EPI_THREADS);
+    int wbuf = 0;
+    long long item = pair;
+    Item it;
+    bool have = false;
+    for (; item < p.n_items; item += npairs)
+      if ((have = decode_item<NTOK, TILE_KEYS>(item, p, it))) break;
+    if (have) prefetch_w(it, 0);
+    while (have && ok) {
+      cp_async_wait<0>();
+      named_bar_sync(1, C::EPI_THREADS);  // this item's weights landed; the other buffer is free
+      // the next item this pair will see, and its weights in flight while this one runs
+      Item nx;
+      bool have_next = false;
+      long long nitem = item + npairs;
+      for (; nitem < p.n_items; nitem += npairs)
+        if ((have_next = decode_item<NTOK, TILE_KEYS>(nitem, p, nx))) break;
+      if (have_next) prefetch_w(nx, wbuf ^ 1);
       const int dvis = it.Lk - it.Lq + 1;
       float wr[C::CPT];
 #pragma unroll
-      for (int c = 0; c < C::CPT; ++c) wr[c] = w_s[col0 + c];
+      for (int c = 0; c < C::CPT; c += 2) {
+        const uint32_t pr = *reinterpret_cast<const uint32_t*>(w_s + wbuf * C::N + col0 + c);
+        const int tk0 = (col0 + c) / H_I, tk1 = (col0 + c + 1) / H_I;
+        wr[c] = tk0 < it.ntok ? __uint_as_float(pr << 16) : 0.f;
+        wr[c + 1] = tk1 < it.ntok ? __uint_as_float(pr & 0xFFFF0000u) : 0.f;
+      }
       for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
         if (!(ok = mbar_wait(&acc_full[ab], abph, abort_flag, 16))) break;
         tc_fence_after();
@@ -233,7 +257,12 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
         if (lane == 0) mbar_arrive_cluster(ab == 0 ? acc_empty0 : acc_empty1);
         if (++ab == 2) { ab = 0; abph ^= 1; }
       }
+      item = nitem;
+      it = nx;
+      have = have_next;
+      wbuf ^= 1;
     }
+    cp_async_wait<0>();
   }
 
   tc_fence_before();
@@ -268,6 +297,7 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
   if (st != DSA_OK) return st;
   dsa::IndexerParams p;
   p.w = static_cast<const uint16_t*>(w);
+  p.w_elems = total_q * H_I;
   p.cu_q = cu_q;
   p.cu_k = cu_k;
   p.batch = batch;
@@ -305,10 +335,10 @@ int indexer2_launch(const void* q_idx, const void* k_idx, const void* w, const i
                     long long row_end, float* scores, long long ld, cudaStream_t stream) {
   if (H_I == 64 && d_I == 128)
     return launch_indexer2<64, 128, 4, 8, 4, 2>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k,
-                                                row_begin, row_end, scores, ld, 32, stream);
+                                                row_begin, row_end, scores, ld, 64, stream);
   if (H_I == 32 && d_I == 128)
     return launch_indexer2<32, 128, 8, 8, 4, 2>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k,
-                                                row_begin, row_end, scores, ld, 32, stream);
+                                                row_begin, row_end, scores, ld, 64, stream);
   return DSA_ERR_UNSUPPORTED;
 }
 
