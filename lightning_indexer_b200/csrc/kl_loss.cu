@@ -26,6 +26,12 @@
 
 namespace dsa {
 
+// tiling of the dense-target kernels: warps per CTA, chunks in flight per warp (the one in
+// use included), keys per chunk
+constexpr int KL_WARPS = 8;
+constexpr int KL_STAGES = 3;
+constexpr int KL_CHUNK = 16;
+
 __device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
@@ -45,17 +51,17 @@ __device__ __forceinline__ int seq_of_row(const int* cu, int batch, long long ro
 // ------------------------------------------------------------------ 1. dense LSE
 // One warp per (row, KV head): streams the row's visible keys (contiguous) in chunks of 16.
 template <int D>
-__global__ void __launch_bounds__(SA_WARPS * 32)
+__global__ void __launch_bounds__(KL_WARPS * 32)
     dense_lse_kernel(const uint16_t* Q, const uint16_t* K, const int* cu_q, const int* cu_k, int batch,
                      long long rows, int Hq, int Hkv, float scale_log2, float* lse_out) {
   constexpr int SEGS = D / 8;
-  constexpr int TILE = SA_CHUNK * D * 2;
+  constexpr int TILE = KL_CHUNK * D * 2;
   constexpr int MT = D / 16;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
-  const uint32_t my_s = smem_u32(smem + warp * SA_STAGES * TILE);
-  const long long task = (long long)blockIdx.x * SA_WARPS + warp;
+  const uint32_t my_s = smem_u32(smem + warp * KL_STAGES * TILE);
+  const long long task = (long long)blockIdx.x * KL_WARPS + warp;
   const long long row = task / Hkv;
   if (row >= rows) return;
   const int g = (int)(task % Hkv);
@@ -77,13 +83,13 @@ __global__ void __launch_bounds__(SA_WARPS * 32)
       qb[kk][1] = hv ? __ldg(q32 + kk * 8 + 4 + tig) : 0u;
     }
   }
-  const int nchunks = (vis + SA_CHUNK - 1) / SA_CHUNK;
+  const int nchunks = (vis + KL_CHUNK - 1) / KL_CHUNK;
   auto issue = [&](int c, int st) {
 #pragma unroll
-    for (int j = 0; j < SA_CHUNK * SEGS / 32; ++j) {
+    for (int j = 0; j < KL_CHUNK * SEGS / 32; ++j) {
       const int e = j * 32 + lane;
       const int r = e / SEGS, seg = e % SEGS;
-      const int s = c * SA_CHUNK + r;
+      const int s = c * KL_CHUNK + r;
       const bool valid = s < vis;
       cp_async_16(my_s + st * TILE + tile_off<D>(r, seg), Kg + (valid ? (size_t)(kbase + s) * stride + seg * 8 : 0),
                   valid);
@@ -91,19 +97,19 @@ __global__ void __launch_bounds__(SA_WARPS * 32)
   };
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 #pragma unroll
-  for (int st = 0; st < SA_STAGES - 1; ++st) {
+  for (int st = 0; st < KL_STAGES - 1; ++st) {
     if (st < nchunks) issue(st, st);
     cp_async_commit();
   }
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
-    const int st = c % SA_STAGES;
+    const int st = c % KL_STAGES;
     {
-      const int cn = c + SA_STAGES - 1;
-      if (cn < nchunks) issue(cn, cn % SA_STAGES);
+      const int cn = c + KL_STAGES - 1;
+      if (cn < nchunks) issue(cn, cn % KL_STAGES);
       cp_async_commit();
     }
-    cp_async_wait<SA_STAGES - 1>();
+    cp_async_wait<KL_STAGES - 1>();
     __syncwarp();
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(SA_WARPS * 32)
       ldmatrix_x4(my_s + st * TILE + tile_off<D>(lane & 15, kk * 2 + (lane >> 4)), a0, a1, a2, a3);
       mma_bf16_16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
     }
-    const bool v0 = c * SA_CHUNK + gid < vis, v1 = c * SA_CHUNK + gid + 8 < vis;
+    const bool v0 = c * KL_CHUNK + gid < vis, v1 = c * KL_CHUNK + gid + 8 < vis;
     const float x00 = v0 ? s[0] * scale_log2 : -INFINITY, x01 = v0 ? s[1] * scale_log2 : -INFINITY;
     const float x10 = v1 ? s[2] * scale_log2 : -INFINITY, x11 = v1 ? s[3] * scale_log2 : -INFINITY;
     float cm0 = fmaxf(x00, x10), cm1 = fmaxf(x01, x11);
@@ -185,14 +191,14 @@ __global__ void __launch_bounds__(256)
                      long long row_begin, int Hq, int Hkv, float scale_log2, const float* lse_att,
                      const float* lseI, float* scores, long long ld, float inv_T, float* kl_out) {
   constexpr int SEGS = D / 8;
-  constexpr int TILE = SA_CHUNK * D * 2;
+  constexpr int TILE = KL_CHUNK * D * 2;
   constexpr int MT = D / 16;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float psum[8][SA_CHUNK];
+  __shared__ float psum[8][KL_CHUNK];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
   const int g = warp;  // blockDim.x == 32 * Hkv
-  const uint32_t my_s = smem_u32(smem + warp * SA_STAGES * TILE);
+  const uint32_t my_s = smem_u32(smem + warp * KL_STAGES * TILE);
   const long long row = row_begin + blockIdx.x;
   const int G = Hq / Hkv;
   const int b = seq_of_row(cu_q, batch, row);
@@ -217,13 +223,13 @@ __global__ void __launch_bounds__(256)
   const int h0 = 2 * tig, h1 = h0 + 1;
   const float L0 = h0 < G ? lse_att[row * Hq + g * G + h0] * 1.4426950408889634f : -INFINITY;
   const float L1 = h1 < G ? lse_att[row * Hq + g * G + h1] * 1.4426950408889634f : -INFINITY;
-  const int nchunks = (vis + SA_CHUNK - 1) / SA_CHUNK;
+  const int nchunks = (vis + KL_CHUNK - 1) / KL_CHUNK;
   auto issue = [&](int c, int st) {
 #pragma unroll
-    for (int j = 0; j < SA_CHUNK * SEGS / 32; ++j) {
+    for (int j = 0; j < KL_CHUNK * SEGS / 32; ++j) {
       const int e = j * 32 + lane;
       const int r = e / SEGS, seg = e % SEGS;
-      const int s = c * SA_CHUNK + r;
+      const int s = c * KL_CHUNK + r;
       const bool valid = s < vis;
       cp_async_16(my_s + st * TILE + tile_off<D>(r, seg), Kg + (valid ? (size_t)(kbase + s) * stride + seg * 8 : 0),
                   valid);
@@ -231,19 +237,19 @@ __global__ void __launch_bounds__(256)
   };
   float kl = 0.f;
 #pragma unroll
-  for (int st = 0; st < SA_STAGES - 1; ++st) {
+  for (int st = 0; st < KL_STAGES - 1; ++st) {
     if (st < nchunks) issue(st, st);
     cp_async_commit();
   }
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
-    const int st = c % SA_STAGES;
+    const int st = c % KL_STAGES;
     {
-      const int cn = c + SA_STAGES - 1;
-      if (cn < nchunks) issue(cn, cn % SA_STAGES);
+      const int cn = c + KL_STAGES - 1;
+      if (cn < nchunks) issue(cn, cn % KL_STAGES);
       cp_async_commit();
     }
-    cp_async_wait<SA_STAGES - 1>();
+    cp_async_wait<KL_STAGES - 1>();
     __syncwarp();
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -264,8 +270,8 @@ __global__ void __launch_bounds__(256)
       psum[g][gid + 8] = e1;
     }
     __syncthreads();
-    if (warp == 0 && lane < SA_CHUNK) {
-      const int sidx = c * SA_CHUNK + lane;
+    if (warp == 0 && lane < KL_CHUNK) {
+      const int sidx = c * KL_CHUNK + lane;
       if (sidx < vis) {
         float pp = 0.f;
         for (int w = 0; w < Hkv; ++w) pp += psum[w][lane];
@@ -644,8 +650,8 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
   // 1. dense LSE
   {
     const long long tasks = T * Hkv;
-    const long long blocks = (tasks + dsa::SA_WARPS - 1) / dsa::SA_WARPS;
-    const int smem = dsa::SA_WARPS * dsa::SA_STAGES * dsa::SA_CHUNK * d * 2;
+    const long long blocks = (tasks + dsa::KL_WARPS - 1) / dsa::KL_WARPS;
+    const int smem = dsa::KL_WARPS * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;
     if (blocks > 0) {
       if (d == 128) {
         static bool done = false;
@@ -655,7 +661,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
           if (e_ != cudaSuccess) return cuda_fail(e_);
         }
         done = true;
-        dsa::dense_lse_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, s>>>(
+        dsa::dense_lse_kernel<128><<<(unsigned)blocks, dsa::KL_WARPS * 32, smem, s>>>(
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, T, Hq, Hkv,
             scale_log2, W.lse_att);
       } else {
@@ -666,7 +672,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
           if (e_ != cudaSuccess) return cuda_fail(e_);
         }
         done = true;
-        dsa::dense_lse_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, s>>>(
+        dsa::dense_lse_kernel<64><<<(unsigned)blocks, dsa::KL_WARPS * 32, smem, s>>>(
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, T, Hq, Hkv,
             scale_log2, W.lse_att);
       }
@@ -682,12 +688,12 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     dsa::row_lse_kernel<<<(unsigned)(r1 - r0), 256, 0, s>>>(W.scores, ld, cu_q, cu_k, batch, r0, W.lseI);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
     {
-      const int smem = Hkv * dsa::SA_STAGES * dsa::SA_CHUNK * d * 2;
+      const int smem = Hkv * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;
       if (d == 128) {
         static bool done = false;
         if (!done) {
           const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          8 * dsa::SA_STAGES * dsa::SA_CHUNK * 128 * 2);
+                                          8 * dsa::KL_STAGES * dsa::KL_CHUNK * 128 * 2);
           if (e_ != cudaSuccess) return cuda_fail(e_);
         }
         done = true;
@@ -698,7 +704,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
         static bool done = false;
         if (!done) {
           const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          8 * dsa::SA_STAGES * dsa::SA_CHUNK * 64 * 2);
+                                          8 * dsa::KL_STAGES * dsa::KL_CHUNK * 64 * 2);
           if (e_ != cudaSuccess) return cuda_fail(e_);
         }
         done = true;

@@ -8,13 +8,25 @@
 // One warp owns one (query row, KV head g, key split).  The G = Hq/Hkv query heads of the
 // group share every gathered K/V row.  The work is a gather (k rows of K and V per token
 // and group) followed by two tiny products (G x d by d x 16 per 16 keys), so it is bound
-// by the gather bandwidth, not by the tensor pipe.  The products use warp-level MMA
-// in swap-AB form (M = 16 keys, N = 8 heads, so no M padding is wasted):
+// by the gather and by the latency of each warp's dependent chain, not by the tensor
+// pipe.  The products use warp-level MMA in swap-AB form (M = 16 keys, N = 8 heads, so no
+// M padding is wasted):
 //   S^T[16 keys x 8 heads]  = K_chunk[16 x d] . Q_g^T[d x 8]
 //   O^T[d x 8 heads]       += V_chunk^T[d x 16] . P^T[16 x 8]
 // P^T goes from the accumulator layout to the B-operand layout with movmatrix.trans.
-// Online softmax in the log2 domain; K/V rows stream through a 3-stage cp.async ring per
-// warp (16-byte zero-filling copies for the -1 slots).
+//
+// Gather: the K and V rows of a 16-key chunk stream into a per-warp ring of shared-memory
+// stages with 16-byte cp.async copies (zero-filling for -1 slots), XOR-swizzled so that
+// ldmatrix reads 8 rows without bank conflicts.  The chunk's slot indices are loaded one
+// chunk ahead of their copies, so the index load never sits on the issue path.  (Bulk
+// 256-byte copies per row, one per lane, were measured slower on B200: the per-copy cost
+// of the bulk-copy unit outweighs the instructions they save.)  Two stages per warp keep
+// shared memory small enough for 12 warps per SM; the warp's chain of dependent MMA,
+// shuffle and exp2 steps, not the memory latency, sets the pace.
+//
+// Online softmax in the log2 domain.  The running max of a head only moves when a chunk
+// exceeds it by more than 8 (so every weight stays below 2^8 and fp32 sums stay exact
+// enough); the accumulator rescale is skipped in the common case where no head moved.
 #include <algorithm>
 
 #include "common.cuh"
@@ -39,10 +51,14 @@ struct SAParams {
   float* part_ml; // [rows, nsplit, Hq, 4]: max (log2 domain), exact sum, sum of bf16-rounded weights
 };
 
-constexpr int SA_WARPS = 8;
-constexpr int SA_STAGES = 3;
+constexpr int SA_WARPS = 4;   // warps per CTA (several CTAs per SM)
+constexpr int SA_STAGES = 2;  // chunks in flight per warp, the one in use included
 constexpr int SA_CHUNK = 16;
 
+template <int D>
+constexpr int sa_smem_bytes(int warps) {
+  return warps * SA_STAGES * 2 * SA_CHUNK * D * 2;
+}
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -72,7 +88,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-
 // byte offset of 16-byte segment `seg` of row `row` in a [rows][D] bf16 tile, XOR-swizzled
 // so that 8 consecutive rows at one logical segment fall in distinct bank groups
 template <int D>
@@ -82,19 +97,19 @@ __device__ __forceinline__ uint32_t tile_off(int row, int seg) {
 
 template <int D>
 __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAParams p) {
-  constexpr int SEGS = D / 8;                          // 16-byte segments per row
-  constexpr int TILE_BYTES = SA_CHUNK * D * 2;         // one K or V chunk
+  constexpr int SEGS = D / 8;                   // 16-byte segments per row
+  constexpr int TILE_BYTES = SA_CHUNK * D * 2;  // one K or V chunk
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  constexpr int MT = D / 16;                           // m-tiles of O^T, k-steps of S^T
+  constexpr int MT = D / 16;                    // m-tiles of O^T, k-steps of S^T
+  static_assert(MT % 2 == 0, "two interleaved S chains");
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  uint8_t* my = smem + warp * SA_STAGES * STAGE_BYTES;
-  const uint32_t my_s = smem_u32(my);
+  const uint32_t my_s = smem_u32(smem + warp * SA_STAGES * STAGE_BYTES);
 
   const long long task = (long long)blockIdx.x * SA_WARPS + warp;
   const long long per_row = (long long)p.Hkv * p.nsplit;
   const long long row = task / per_row;
-  if (row >= p.rows) return;
+  if (row >= p.rows) return;  // warp-uniform; the kernel has no CTA-wide barrier
   const int rem = (int)(task % per_row);
   const int split = rem / p.Hkv;
   const int g = rem % p.Hkv;
@@ -129,9 +144,9 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
     }
   }
 
-  // issue the gather of chunk c into stage st
-  auto issue = [&](int c, int st) {
-    const int my_idx = __ldg(idx + c * SA_CHUNK + (lane & 15));
+  // Issues the gather of one chunk into stage st; lane j < 16 holds the index of slot j
+  // (lanes 16-31 the same).  Returns the chunk's valid-slot mask, the same in every lane.
+  auto issue = [&](int st, int my_idx) -> uint32_t {
     const uint32_t kdst = my_s + st * STAGE_BYTES;
     const uint32_t vdst = kdst + TILE_BYTES;
 #pragma unroll
@@ -144,6 +159,8 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
       cp_async_16(kdst + tile_off<D>(r, seg), Kg + off, valid);
       cp_async_16(vdst + tile_off<D>(r, seg), Vg + off, valid);
     }
+    cp_async_commit();
+    return __ballot_sync(0xffffffffu, my_idx >= 0) & 0xFFFFu;
   };
 
   float acc[MT][4];
@@ -153,67 +170,87 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
   float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums (for the LSE)
   float r0 = 0.f, r1 = 0.f;              // same, of the bf16-rounded weights that multiply V
 
+  // valid-slot masks of the chunks in flight (vmr[0] = the chunk in use next) and the
+  // prefetched slot index of the next chunk to issue
+  const int slot = lane & 15;
+  uint32_t vmr[SA_STAGES - 1];
+  int nxt = nchunks > 0 ? __ldg(idx + slot) : -1;
 #pragma unroll
-  for (int st = 0; st < SA_STAGES - 1; ++st) {
-    if (st < nchunks) issue(st, st);
-    cp_async_commit();
+  for (int c = 0; c < SA_STAGES - 1; ++c) {
+    const int cur = nxt;
+    nxt = c + 1 < nchunks ? __ldg(idx + (c + 1) * SA_CHUNK + slot) : -1;
+    vmr[c] = c < nchunks ? issue(c, cur) : (cp_async_commit(), 0u);
   }
 
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
     const int st = c % SA_STAGES;
+    uint32_t vnew = 0;
     {
       const int cn = c + SA_STAGES - 1;
-      if (cn < nchunks) issue(cn, cn % SA_STAGES);
-      cp_async_commit();
+      if (cn < nchunks) {
+        const int cur = nxt;
+        nxt = cn + 1 < nchunks ? __ldg(idx + (cn + 1) * SA_CHUNK + slot) : -1;
+        vnew = issue(cn % SA_STAGES, cur);
+      } else {
+        cp_async_commit();
+      }
     }
     cp_async_wait<SA_STAGES - 1>();
     __syncwarp();
     const uint32_t kt = my_s + st * STAGE_BYTES;
     const uint32_t vt = kt + TILE_BYTES;
 
-    // ---- S^T = K_chunk . Q^T
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- S^T = K_chunk . Q^T, two interleaved accumulator chains
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int kk = 0; kk < MT; ++kk) {
-      uint32_t a0, a1, a2, a3;
+    for (int kk = 0; kk < MT; kk += 2) {
+      uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
       ldmatrix_x4(kt + tile_off<D>(lane & 15, kk * 2 + (lane >> 4)), a0, a1, a2, a3);
-      mma_bf16_16816(s, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+      ldmatrix_x4(kt + tile_off<D>(lane & 15, (kk + 1) * 2 + (lane >> 4)), e0, e1, e2, e3);
+      mma_bf16_16816(sa, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+      mma_bf16_16816(sb, e0, e1, e2, e3, qb[kk + 1][0], qb[kk + 1][1]);
     }
-    // keys of this lane: r0 = lane/4, r1 = lane/4 + 8; heads h0 = 2*(lane%4), h1 = h0 + 1
-    const int myi = __ldg(idx + c * SA_CHUNK + (lane & 15));
-    const bool v0 = __shfl_sync(0xffffffffu, myi, lane / 4) >= 0;
-    const bool v1 = __shfl_sync(0xffffffffu, myi, lane / 4 + 8) >= 0;
-    const float x00 = v0 ? s[0] * p.scale_log2 : -INFINITY;  // (r0, h0)
-    const float x01 = v0 ? s[1] * p.scale_log2 : -INFINITY;  // (r0, h1)
-    const float x10 = v1 ? s[2] * p.scale_log2 : -INFINITY;  // (r1, h0)
-    const float x11 = v1 ? s[3] * p.scale_log2 : -INFINITY;  // (r1, h1)
+    // keys of this lane: q0 = lane/4, q1 = lane/4 + 8; heads h0 = 2*(lane%4), h1 = h0 + 1
+    const uint32_t vm = vmr[0];
+    const bool v0 = (vm >> (lane >> 2)) & 1u;
+    const bool v1 = (vm >> ((lane >> 2) + 8)) & 1u;
+    const float x00 = v0 ? (sa[0] + sb[0]) * p.scale_log2 : -INFINITY;  // (q0, h0)
+    const float x01 = v0 ? (sa[1] + sb[1]) * p.scale_log2 : -INFINITY;  // (q0, h1)
+    const float x10 = v1 ? (sa[2] + sb[2]) * p.scale_log2 : -INFINITY;  // (q1, h0)
+    const float x11 = v1 ? (sa[3] + sb[3]) * p.scale_log2 : -INFINITY;  // (q1, h1)
     float cm0 = fmaxf(x00, x10), cm1 = fmaxf(x01, x11);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, o));
       cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, o));
     }
-    const float mn0 = fmaxf(m0, cm0), mn1 = fmaxf(m1, cm1);
-    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float al0 = exp2f(m0 - mu0), al1 = exp2f(m1 - mu1);
-    m0 = mn0;
-    m1 = mn1;
+    const bool up0 = cm0 > m0 + 8.f, up1 = cm1 > m1 + 8.f;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+      const float al0 = up0 ? exp2f(m0 - cm0) : 1.f, al1 = up1 ? exp2f(m1 - cm1) : 1.f;
+      if (up0) m0 = cm0;
+      if (up1) m1 = cm1;
+      l0 *= al0;
+      l1 *= al1;
+      r0 *= al0;
+      r1 *= al1;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        acc[mt][0] *= al0;
+        acc[mt][1] *= al1;
+        acc[mt][2] *= al0;
+        acc[mt][3] *= al1;
+      }
+    }
+    const float mu0 = m0 == -INFINITY ? 0.f : m0, mu1 = m1 == -INFINITY ? 0.f : m1;
     const float p00 = exp2f(x00 - mu0), p01 = exp2f(x01 - mu1);
     const float p10 = exp2f(x10 - mu0), p11 = exp2f(x11 - mu1);
-    l0 = l0 * al0 + p00 + p10;
-    l1 = l1 * al1 + p01 + p11;
+    l0 += p00 + p10;
+    l1 += p01 + p11;
     // O is normalised by the sum of the weights exactly as they enter the PV product
     const uint32_t pk0 = pack_bf16x2(p00, p01), pk1 = pack_bf16x2(p10, p11);
-    r0 = r0 * al0 + __uint_as_float(pk0 << 16) + __uint_as_float(pk1 << 16);
-    r1 = r1 * al1 + __uint_as_float(pk0 & 0xFFFF0000u) + __uint_as_float(pk1 & 0xFFFF0000u);
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      acc[mt][0] *= al0;
-      acc[mt][1] *= al1;
-      acc[mt][2] *= al0;
-      acc[mt][3] *= al1;
-    }
+    r0 += __uint_as_float(pk0 << 16) + __uint_as_float(pk1 << 16);
+    r1 += __uint_as_float(pk0 & 0xFFFF0000u) + __uint_as_float(pk1 & 0xFFFF0000u);
     // ---- O^T += V^T . P^T
     const uint32_t pb0 = movmatrix_trans(pk0);  // keys 0-7
     const uint32_t pb1 = movmatrix_trans(pk1);  // keys 8-15
@@ -225,6 +262,9 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
       ldmatrix_x4_trans(vt + tile_off<D>(vrow, mt * 2 + vseg_off), a0, a1, a2, a3);
       mma_bf16_16816(acc[mt], a0, a1, a2, a3, pb0, pb1);
     }
+#pragma unroll
+    for (int j = 0; j + 1 < SA_STAGES - 1; ++j) vmr[j] = vmr[j + 1];
+    vmr[SA_STAGES - 2] = vnew;
     __syncwarp();  // stage st is refilled by the next iteration's issue
   }
   cp_async_wait<0>();
@@ -315,31 +355,25 @@ __global__ void decode_combine_kernel(const float* part_o, const float* part_ml,
 
 namespace dsa_host {
 
+template <int D>
+static int sa_launch_d(const dsa::SAParams& p, long long tasks, cudaStream_t stream) {
+  const long long blocks = (tasks + dsa::SA_WARPS - 1) / dsa::SA_WARPS;
+  const int smem = dsa::sa_smem_bytes<D>(dsa::SA_WARPS);
+  static bool done = false;
+  if (!done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                smem);
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    done = true;
+  }
+  dsa::sparse_attn_kernel<D><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
+  return last_launch_status();
+}
+
 static int sa_launch_common(dsa::SAParams& p, int d, cudaStream_t stream) {
   const long long tasks = p.rows * p.Hkv * p.nsplit;
-  const long long blocks = (tasks + dsa::SA_WARPS - 1) / dsa::SA_WARPS;
-  if (blocks <= 0) return DSA_OK;
-  const int smem = dsa::SA_WARPS * dsa::SA_STAGES * 2 * dsa::SA_CHUNK * d * 2;
-  if (d == 128) {
-    static bool done = false;
-    if (!done) {
-      const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<128>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e_ != cudaSuccess) return cuda_fail(e_);
-      done = true;
-    }
-    dsa::sparse_attn_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
-  } else {
-    static bool done = false;
-    if (!done) {
-      const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<64>,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e_ != cudaSuccess) return cuda_fail(e_);
-      done = true;
-    }
-    dsa::sparse_attn_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
-  }
-  return last_launch_status();
+  if (tasks <= 0) return DSA_OK;
+  return d == 128 ? sa_launch_d<128>(p, tasks, stream) : sa_launch_d<64>(p, tasks, stream);
 }
 
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,

@@ -18,6 +18,11 @@
 
 namespace dsa {
 
+// warps per CTA, chunks in flight per warp (the one in use included), keys per chunk
+constexpr int BWD_WARPS = 8;
+constexpr int BWD_STAGES = 3;
+constexpr int BWD_CHUNK = 16;
+
 struct SABwdParams {
   const uint16_t* Q;
   const uint16_t* K;
@@ -42,18 +47,18 @@ __device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_bwd_kernel(const SABwdParams p) {
+__global__ void __launch_bounds__(BWD_WARPS * 32) sparse_attn_bwd_kernel(const SABwdParams p) {
   constexpr int SEGS = D / 8;
-  constexpr int TILE_BYTES = SA_CHUNK * D * 2;
+  constexpr int TILE_BYTES = BWD_CHUNK * D * 2;
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   constexpr int MT = D / 16;  // k-steps over d, and m-tiles of dQ^T
   constexpr int NT = D / 8;   // n-tiles of dK / dV rows
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
-  const uint32_t my_s = smem_u32(smem + warp * SA_STAGES * STAGE_BYTES);
+  const uint32_t my_s = smem_u32(smem + warp * BWD_STAGES * STAGE_BYTES);
 
-  const long long task = (long long)blockIdx.x * SA_WARPS + warp;
+  const long long task = (long long)blockIdx.x * BWD_WARPS + warp;
   const long long row = task / p.Hkv;
   if (row >= p.rows) return;
   const int g = (int)(task % p.Hkv);
@@ -64,7 +69,7 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_bwd_kernel(const SA
   }
   const int kbase = p.cu_k[lo];
   const int* idx = p.indices + row * p.k;
-  const int nchunks = p.k / SA_CHUNK;
+  const int nchunks = p.k / BWD_CHUNK;
   const size_t kv_row_stride = (size_t)p.Hkv * D;
   const uint16_t* Kg = p.K + (size_t)g * D;
   const uint16_t* Vg = p.V + (size_t)g * D;
@@ -114,11 +119,11 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_bwd_kernel(const SA
   const bool live0 = L0 > -INFINITY, live1 = L1 > -INFINITY;
 
   auto issue = [&](int c, int st) {
-    const int my_idx = __ldg(idx + c * SA_CHUNK + (lane & 15));
+    const int my_idx = __ldg(idx + c * BWD_CHUNK + (lane & 15));
     const uint32_t kdst = my_s + st * STAGE_BYTES;
     const uint32_t vdst = kdst + TILE_BYTES;
 #pragma unroll
-    for (int j = 0; j < SA_CHUNK * SEGS / 32; ++j) {
+    for (int j = 0; j < BWD_CHUNK * SEGS / 32; ++j) {
       const int e = j * 32 + lane;
       const int r = e / SEGS, seg = e % SEGS;
       const int s = __shfl_sync(0xffffffffu, my_idx, r);
@@ -134,19 +139,19 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_bwd_kernel(const SA
   for (int mt = 0; mt < MT; ++mt) dq[mt][0] = dq[mt][1] = dq[mt][2] = dq[mt][3] = 0.f;
 
 #pragma unroll
-  for (int st = 0; st < SA_STAGES - 1; ++st) {
+  for (int st = 0; st < BWD_STAGES - 1; ++st) {
     if (st < nchunks) issue(st, st);
     cp_async_commit();
   }
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
-    const int st = c % SA_STAGES;
+    const int st = c % BWD_STAGES;
     {
-      const int cn = c + SA_STAGES - 1;
-      if (cn < nchunks) issue(cn, cn % SA_STAGES);
+      const int cn = c + BWD_STAGES - 1;
+      if (cn < nchunks) issue(cn, cn % BWD_STAGES);
       cp_async_commit();
     }
-    cp_async_wait<SA_STAGES - 1>();
+    cp_async_wait<BWD_STAGES - 1>();
     __syncwarp();
     const uint32_t kt = my_s + st * STAGE_BYTES;
     const uint32_t vt = kt + TILE_BYTES;
@@ -160,7 +165,7 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_bwd_kernel(const SA
       ldmatrix_x4(vt + tile_off<D>(lane & 15, kk * 2 + (lane >> 4)), a0, a1, a2, a3);
       mma_bf16_16816(dp, a0, a1, a2, a3, ob[kk][0], ob[kk][1]);
     }
-    const int myi = __ldg(idx + c * SA_CHUNK + (lane & 15));
+    const int myi = __ldg(idx + c * BWD_CHUNK + (lane & 15));
     const int sA = __shfl_sync(0xffffffffu, myi, gid);      // key of accumulator row gid
     const int sB = __shfl_sync(0xffffffffu, myi, gid + 8);  // key of row gid + 8
     const bool v0 = sA >= 0, v1 = sB >= 0;
@@ -286,8 +291,8 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
   p.dK_acc = dk_acc;
   p.dV_acc = dv_acc;
   const long long tasks = total_q * Hkv;
-  const long long blocks = (tasks + dsa::SA_WARPS - 1) / dsa::SA_WARPS;
-  const int smem = dsa::SA_WARPS * dsa::SA_STAGES * 2 * dsa::SA_CHUNK * d * 2;
+  const long long blocks = (tasks + dsa::BWD_WARPS - 1) / dsa::BWD_WARPS;
+  const int smem = dsa::BWD_WARPS * dsa::BWD_STAGES * 2 * dsa::BWD_CHUNK * d * 2;
   if (blocks > 0) {
     if (d == 128) {
       static bool done = false;
@@ -296,7 +301,7 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
                                  smem); e_ != cudaSuccess) return cuda_fail(e_);
         done = true;
       }
-      dsa::sparse_attn_bwd_kernel<128><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
+      dsa::sparse_attn_bwd_kernel<128><<<(unsigned)blocks, dsa::BWD_WARPS * 32, smem, stream>>>(p);
     } else {
       static bool done = false;
       if (!done) {
@@ -304,7 +309,7 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
                                  smem); e_ != cudaSuccess) return cuda_fail(e_);
         done = true;
       }
-      dsa::sparse_attn_bwd_kernel<64><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
+      dsa::sparse_attn_bwd_kernel<64><<<(unsigned)blocks, dsa::BWD_WARPS * 32, smem, stream>>>(p);
     }
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
   }

@@ -711,6 +711,272 @@ __global__ void __launch_bounds__(FT, 2) topk_fast_kernel(const TopkParams p) {
   if constexpr (C > 1) cg::this_cluster().sync();
 }
 
+
+// ======================================================================================
+// Few long rows (decode: a handful of sequences with 10^5 cached positions each).  A row
+// goes to a cluster of C blocks of 512 threads; every thread loads 64 consecutive scores
+// of the row into registers with 16 float4 loads that are all in flight at once, so the
+// row is read from memory exactly once.
+//   1. While those loads fly, every block takes the same strided sample of 2048 positions
+//      and, by two radix levels, the r_low-th largest sampled key T (a lower bound on the
+//      k-th largest key, with a safety margin).
+//   2. Keys >= T are counted in registers (no atomics); the blocks exchange their counts.
+//      If they add up to at least k and fit rank 0's candidate list, every block writes
+//      its candidates, in position order, into rank 0's shared memory.  Rank 0 then finds
+//      the exact k-th key K* by radix levels over (key - T), whose 2048 bins span exactly
+//      the candidates' range, and writes the selected positions in order.
+//   3. Otherwise (an unlucky sample, or huge ties) all blocks run three radix levels
+//      (11 + 11 + 10 key bits) over the register-resident keys, each level's histogram
+//      summed over the cluster through distributed shared memory, and write in order
+//      from the per-block counts.
+// The sample only decides how the exact K* is found, never which positions are selected.
+// Rows up to C x 32768 positions (C <= 8, the portable cluster size).
+constexpr int RT = 512;           // threads per block
+constexpr int RKEYS = 64;         // keys per thread
+constexpr int RSEG = RT * RKEYS;  // positions per block
+constexpr int RCAP = 16384;       // candidates rank 0 can hold
+
+struct RegsSmem {
+  uint32_t cand_key[RCAP];
+  int cand_pos[RCAP];
+  uint32_t hist[2][2048];  // per level parity (remote blocks read them)
+  uint32_t ghist[2048];    // cluster-wide sum
+  uint32_t warp_sums[32];
+  uint32_t total, bin, above, dmax;
+  uint32_t counts[2];
+};
+
+template <int C>
+__global__ void __launch_bounds__(RT, 1) topk_regs_kernel(const TopkParams p) {
+  constexpr int B = RT;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RegsSmem& S = *reinterpret_cast<RegsSmem*>(smem_raw);
+  auto cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const long long row = p.row_begin + blockIdx.x / C;
+  int lo = 0, hi = p.batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int i = (int)(row - p.cu_q[b]);
+  const int Lq = p.cu_q[b + 1] - p.cu_q[b];
+  const int Lk = p.cu_k[b + 1] - p.cu_k[b];
+  const int vis = min(max(i + Lk - Lq + 1, 0), Lk);
+  const int k = p.k;
+  int* out = p.indices + (row - p.row_begin) * k;
+  const float* src = p.scores + (row - p.row_begin) * p.ld;
+  if (vis <= k) {  // uniform over the cluster
+    if (rank == 0)
+      for (int j = threadIdx.x; j < k; j += B) out[j] = j < vis ? j : -1;
+    return;
+  }
+  // block segment [s_lo, s_hi) (4-aligned starts); this thread: [t_lo, t_lo + RKEYS)
+  const int seg = ((vis + C - 1) / C + 3) & ~3;
+  const int s_lo = min(rank * seg, vis), s_hi = min(s_lo + seg, vis);
+  const int t_lo = s_lo + threadIdx.x * RKEYS;
+  const int nvalid = max(0, min(RKEYS, s_hi - t_lo));  // keys [0, nvalid) of this thread are real
+  float4 x[RKEYS / 4];
+#pragma unroll
+  for (int u = 0; u < RKEYS / 4; ++u)
+    x[u] = (4 * u < nvalid) ? __ldg(reinterpret_cast<const float4*>(src + t_lo) + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+
+  // ---------------------------------------------------------------- 1. sampled bound T
+  uint32_t T;
+  {
+    constexpr int NS = 2048, PER = NS / B;
+    const float m = (float)k * (float)NS / (float)vis;
+    const int r_low = min(NS, (int)ceilf(m + 3.f * sqrtf(m) + 8.f));
+    uint32_t sk[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const long long pos = ((2LL * (threadIdx.x + u * B) + 1) * vis) / (2LL * NS);
+      sk[u] = float_order_key(__ldg(src + pos));
+    }
+    uint32_t sp = 0, sm = 0, rem = (uint32_t)r_low;
+#pragma unroll 1
+    for (int lv = 0; lv < 2; ++lv) {
+      const int shift = lv == 0 ? 21 : 10;
+      for (int j = threadIdx.x; j < 2048; j += B) S.ghist[j] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < PER; ++u)
+        if ((sk[u] & sm) == sp) atomicAdd(&S.ghist[(sk[u] >> shift) & 2047u], 1u);
+      __syncthreads();
+      find_bin<B, 2048>(S.ghist, rem, S.warp_sums, &S.total, &S.bin, &S.above);
+      sp |= S.bin << shift;
+      sm |= 2047u << shift;
+      rem -= S.above;
+    }
+    T = sp;
+  }
+  uint32_t key[RKEYS];
+#pragma unroll
+  for (int u = 0; u < RKEYS / 4; ++u) {
+    key[4 * u + 0] = float_order_key(x[u].x);
+    key[4 * u + 1] = float_order_key(x[u].y);
+    key[4 * u + 2] = float_order_key(x[u].z);
+    key[4 * u + 3] = float_order_key(x[u].w);
+  }
+
+  // ---------------------------------------------------------------- 2. candidates >= T
+  uint32_t n_c = 0;
+#pragma unroll
+  for (int j = 0; j < RKEYS; ++j) n_c += (j < nvalid && key[j] >= T);
+  const uint32_t c_before = block_excl_scan<B>(n_c, S.warp_sums, &S.total);
+  if (threadIdx.x == 0) S.counts[0] = S.total;
+  cl.sync();
+  uint32_t base = 0, N = 0;
+  bool fits = true;
+#pragma unroll
+  for (int r = 0; r < C; ++r) {
+    const uint32_t c = *cl.map_shared_rank(&S.counts[0], r);
+    if (r < rank) base += c;
+    N += c;
+  }
+  fits = N >= (uint32_t)k && N <= (uint32_t)RCAP;
+  if (fits) {
+    uint32_t* rk = cl.map_shared_rank(&S.cand_key[0], 0);
+    int* rp = cl.map_shared_rank(&S.cand_pos[0], 0);
+    uint32_t pos = base + c_before;
+#pragma unroll
+    for (int j = 0; j < RKEYS; ++j) {
+      if (j < nvalid && key[j] >= T) {
+        rk[pos] = key[j];
+        rp[pos] = t_lo + j;
+        ++pos;
+      }
+    }
+    cl.sync();  // the candidates have landed in rank 0; nothing else is read remotely
+    if (rank != 0) return;
+    const int n = (int)N;
+    // exact K* over d = key - T; the first level's bins span [0, max d]
+    uint32_t dm = 0;
+    for (int j = threadIdx.x; j < n; j += B) dm = max(dm, S.cand_key[j] - T);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dm = max(dm, __shfl_xor_sync(0xffffffffu, dm, o));
+    if (threadIdx.x == 0) S.dmax = 0;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) atomicMax(&S.dmax, dm);
+    __syncthreads();
+    const int nbits = 32 - __clz((int)S.dmax);
+    int shift = max(0, nbits - 11);
+    uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
+#pragma unroll 1
+    while (true) {
+      for (int j = threadIdx.x; j < 2048; j += B) S.ghist[j] = 0;
+      __syncthreads();
+      for (int j = threadIdx.x; j < n; j += B) {
+        const uint32_t d = S.cand_key[j] - T;
+        if ((d & pmask) == prefix) atomicAdd(&S.ghist[(d >> shift) & 2047u], 1u);
+      }
+      __syncthreads();
+      find_bin<B, 2048>(S.ghist, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+      prefix |= S.bin << shift;
+      pmask |= 2047u << shift;
+      remaining -= S.above;
+      if (shift == 0) break;
+      shift = max(0, shift - 11);
+    }
+    const uint32_t kstar = T + prefix;
+    constexpr int IT = 4;
+    uint32_t base_gt = 0, base_tie = 0;
+    for (int start = 0; start < n; start += B * IT) {
+      const int j0 = start + threadIdx.x * IT;
+      uint32_t g_ = 0, e_ = 0;
+#pragma unroll
+      for (int j = 0; j < IT; ++j) {
+        if (j0 + j < n) {
+          g_ += S.cand_key[j0 + j] > kstar;
+          e_ += S.cand_key[j0 + j] == kstar;
+        }
+      }
+      const uint32_t excl = block_excl_scan<B>((g_ << 16) | e_, S.warp_sums, &S.total);
+      uint32_t gt_before = base_gt + (excl >> 16), eq_before = base_tie + (excl & 0xFFFFu);
+#pragma unroll
+      for (int j = 0; j < IT; ++j) {
+        if (j0 + j >= n) break;
+        const uint32_t kk = S.cand_key[j0 + j];
+        if (kk > kstar) {
+          out[gt_before + min(eq_before, remaining)] = S.cand_pos[j0 + j];
+          ++gt_before;
+        } else if (kk == kstar) {
+          if (eq_before < remaining) out[gt_before + eq_before] = S.cand_pos[j0 + j];
+          ++eq_before;
+        }
+      }
+      base_gt += S.total >> 16;
+      base_tie += S.total & 0xFFFFu;
+      __syncthreads();
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- 3. exact levels over the registers
+  uint32_t remaining = (uint32_t)k, prefix = 0, pmask = 0;
+#pragma unroll 1
+  for (int level = 0; level < 3; ++level) {
+    const int par = level & 1;
+    const int shift = level == 0 ? 21 : (level == 1 ? 10 : 0);
+    const uint32_t bmask = level == 2 ? 1023u : 2047u;
+    for (int j = threadIdx.x; j < 2048; j += B) S.hist[par][j] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < RKEYS; ++j)
+      if (j < nvalid && (key[j] & pmask) == prefix) atomicAdd(&S.hist[par][(key[j] >> shift) & bmask], 1u);
+    cl.sync();
+    const int nb = level == 2 ? 1024 : 2048;
+    for (int j = threadIdx.x; j < nb; j += B) {
+      uint32_t t = 0;
+#pragma unroll
+      for (int r = 0; r < C; ++r) t += cl.map_shared_rank(&S.hist[par][0], r)[j];
+      S.ghist[j] = t;
+    }
+    __syncthreads();
+    if (level < 2)
+      find_bin<B, 2048>(S.ghist, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    else
+      find_bin<B, 1024>(S.ghist, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
+    prefix |= S.bin << shift;
+    pmask |= bmask << shift;
+    remaining -= S.above;
+  }
+  const uint32_t kstar = prefix;
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int j = 0; j < RKEYS; ++j) {
+    n_gt += (j < nvalid && key[j] > kstar);
+    n_eq += (j < nvalid && key[j] == kstar);
+  }
+  // per-thread counts <= 64 and block totals <= RSEG = 32768 fit the packed 16-bit fields
+  const uint32_t excl = block_excl_scan<B>((n_gt << 16) | n_eq, S.warp_sums, &S.total);
+  if (threadIdx.x == 0) {
+    S.counts[0] = S.total >> 16;
+    S.counts[1] = S.total & 0xFFFFu;
+  }
+  cl.sync();
+  uint32_t gt_before = excl >> 16, eq_before = excl & 0xFFFFu;
+  for (int r = 0; r < rank; ++r) {
+    const uint32_t* rc = cl.map_shared_rank(&S.counts[0], r);
+    gt_before += rc[0];
+    eq_before += rc[1];
+  }
+#pragma unroll
+  for (int j = 0; j < RKEYS; ++j) {
+    if (j < nvalid) {
+      if (key[j] > kstar) {
+        out[gt_before + min(eq_before, remaining)] = t_lo + j;
+        ++gt_before;
+      } else if (key[j] == kstar) {
+        if (eq_before < remaining) out[gt_before + eq_before] = t_lo + j;
+        ++eq_before;
+      }
+    }
+  }
+  cl.sync();  // no block may leave while another still reads its shared memory
+}
+
 }  // namespace dsa
 
 namespace dsa_host {
@@ -751,11 +1017,38 @@ static int topk_launch_c(dsa::TopkParams p, long long rows, cudaStream_t stream)
                         stream);
 }
 
+template <int C>
+static int topk_regs_launch(const dsa::TopkParams& p, long long rows, cudaStream_t stream) {
+  static_assert(C <= 8, "portable cluster sizes only");
+  static bool attr_done = false;
+  if (!attr_done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_regs_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)sizeof(dsa::RegsSmem));
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    attr_done = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
+  cfg.blockDim = dim3(dsa::RT, 1, 1);
+  cfg.dynamicSmemBytes = sizeof(dsa::RegsSmem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (const cudaError_t e_ = cudaLaunchKernelEx(&cfg, dsa::topk_regs_kernel<C>, p); e_ != cudaSuccess)
+    return cuda_fail(e_);
+  return last_launch_status();
+}
+
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
                 long long row_begin, long long row_end, int k, int* indices, int max_vis, cudaStream_t stream) {
   const long long rows = row_end - row_begin;
   if (rows <= 0) return DSA_OK;
-  if (rows > 0x7FFFFFFFLL / 8) return DSA_ERR_UNSUPPORTED;
+  if (rows > 0x7FFFFFFFLL / 16) return DSA_ERR_UNSUPPORTED;
   dsa::TopkParams p;
   p.scores = scores;
   p.ld = ld;
@@ -766,8 +1059,16 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
   p.k = k;
   p.indices = indices;
   p.only_marked = 0;
-  // a cluster per row when the rows are long and few enough blocks would be busy otherwise
   const int sms = sm_count();
+  // few long rows: one cluster per row with the row held in registers, while that takes
+  // at most two waves of one block per SM
+  if (max_vis > 32768) {
+    int C = 4;
+    while (C < 8 && (long long)C * dsa::RSEG < (long long)max_vis) C *= 2;
+    if ((long long)C * dsa::RSEG >= (long long)max_vis && rows * C <= 2LL * sms)
+      return C == 4 ? topk_regs_launch<4>(p, rows, stream) : topk_regs_launch<8>(p, rows, stream);
+  }
+  // a cluster per row when the rows are long and few enough blocks would be busy otherwise
   int C = 1;
   while (C < 8 && (long long)rows * C < 2LL * sms && (long long)max_vis > 16384LL * C) C *= 2;
   switch (C) {

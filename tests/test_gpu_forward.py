@@ -125,6 +125,17 @@ def test_topk_candidate_overflow_paths(n_rows, n):
         assert np.array_equal(idx[r], orc.topk_row(sc[r, :vis[r]].astype(np.float64), 2048)), r
 
 
+def test_topk_many_long_rows_cluster_path():
+    # 120 rows of ~100K positions: too many rows for one cluster per row with the row in
+    # registers, so the sampled-threshold kernel runs with a small cluster per row
+    vis = [100000 - 37 * r for r in range(120)]
+    sc, cu_q, cu_k = _topk_case(vis, 2048, seed=5, ties=True)
+    idx = dsa.topk(torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                   2048).cpu().numpy()
+    for b in range(0, 120, 13):
+        assert np.array_equal(idx[b], orc.topk_row(sc[b, :vis[b]].astype(np.float64), 2048)), b
+
+
 def test_topk_adversarial_rows():
     # rows built so that a strided sample of the row misjudges the threshold: the largest
     # values sit exactly on evenly spaced positions, or everywhere except there; the
@@ -198,6 +209,34 @@ def test_sparse_attention_empty_and_padded_sets():
         Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
         assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL
         assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL
+
+
+def test_sparse_attention_large_rising_logits():
+    """Logits of tens of units that grow along the key order: the running max moves in
+    most chunks, by more than the rescale threshold, and the weights span many octaves."""
+    wl = gen.make_prefill([300], 32, 4, 128, 4, 32, 128, seed=34)
+    Qf = wl.Q.astype(np.uint32) << 16
+    Kf = wl.K.astype(np.uint32) << 16
+    # powers of two keep every value exact in bf16: Q x 8, K x 1/2/4/8 by position band
+    q = (Qf.view(np.float32) * np.float32(8.0)).view(np.uint32)
+    band = np.minimum(np.arange(300) // 75, 3).astype(np.float32)
+    kk = (Kf.view(np.float32) * (np.float32(2.0) ** band)[:, None, None]).view(np.uint32)
+    wl.Q = (q >> 16).astype(np.uint16)
+    wl.K = (kk >> 16).astype(np.uint16)
+    D = orc.Decoded(wl)
+    idx = np.full((300, 128), -1, np.int32)
+    for r in range(300):
+        n = min(r + 1, 128)
+        idx[r, :n] = np.linspace(0, r, n).astype(np.int64)  # step >= 1: distinct, ascending
+    t = to_device(wl)
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"])
+    O = O.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    for r in range(0, 300, 7):
+        sel = idx[r][idx[r] >= 0]
+        Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL, r
+        assert np.max(np.abs(lse[r] - lr)) <= 1e-4 * max(1.0, float(np.max(np.abs(lr)))) + LSE_ATOL, r
 
 
 def test_sparse_attention_decode_given_sets():
