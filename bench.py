@@ -300,6 +300,7 @@ def run_decode(args, device, dist):
     scores = torch.empty((B, ld), dtype=torch.float32, device=device)
     idx = torch.empty((B, k), dtype=torch.int32, device=device)
     ws = torch.empty(dsa.decode_attn_workspace_bytes(B, wl.Hq, wl.d, k), dtype=torch.uint8, device=device)
+    topk_ws = torch.empty(max(1, dsa.topk_workspace_bytes(B, ld, k)), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None):
@@ -308,7 +309,7 @@ def run_decode(args, device, dist):
         dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, 1, N, 0, B, scores=scores)
         if ev is not None:
             ev[1].record(stream)
-        dsa.topk(scores, cu_q, cu_k, k, 0, B, indices=idx)
+        dsa.topk(scores, cu_q, cu_k, k, 0, B, indices=idx, workspace=topk_ws)
         if ev is not None:
             ev[2].record(stream)
         dsa.sparse_attn_decode(t["Q"], t["K"], t["V"], idx, cu_k, workspace=ws)
@@ -329,7 +330,7 @@ def run_decode(args, device, dist):
     us = per.mean(axis=0) * 1e3
     idx_bytes = B * N * wl.d_I * 2 + B * wl.H_I * wl.d_I * 2 + B * wl.H_I * 2
     attn_bytes = B * k * wl.Hkv * wl.d * 2 * 2 + B * wl.Hq * wl.d * 2 * 2 + B * k * 4
-    del t, scores, idx, ws
+    del t, scores, idx, ws, topk_ws
     torch.cuda.empty_cache()
     return {"us_per_step": float(us[3]), "us_per_token": float(us[3]) / B,
             "breakdown_us": {"indexer": float(us[0]), "topk": float(us[1]), "sparse_attn": float(us[2])},

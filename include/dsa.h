@@ -109,11 +109,18 @@ DSA_API int dsa_index(const void* q_idx, const void* k_idx, const void* w,
  * vis(r) <= k every visible position is selected.  Output:
  *   indices device int32 [row_end-row_begin, k]: the selected positions in ascending
  *           order, then -1 in the unused slots.  Bit-for-bit reproducible.
- * Supported: 1 <= k <= 4096.  No workspace.
+ *   workspace  optional caller-owned device scratch (16-byte aligned) of at least
+ *           dsa_topk_workspace_size(row_end-row_begin, ld_scores, k) bytes.  That size is
+ *           non-zero only for a few long rows (the decode shape), where the workspace lets
+ *           the call spread each row over many blocks; NULL (or a smaller buffer) selects
+ *           a method that needs none, with the same result.  Its contents on entry do not
+ *           matter; it must not be shared with work that overlaps this call on the GPU.
+ * Supported: 1 <= k <= 4096.
  * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_topk_workspace_size(int64_t rows, int64_t ld_scores, int k);
 DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_seqlens_q,
                      const int32_t* cu_seqlens_k, int batch, int64_t row_begin, int64_t row_end,
-                     int k, int32_t* indices, void* stream);
+                     int k, int32_t* indices, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * (3) Sparse GQA attention, prefill/varlen.  Source: report summary section 1 (attention

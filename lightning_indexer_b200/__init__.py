@@ -13,7 +13,7 @@ import torch
 from . import _lib
 from ._lib import DSAError, call
 
-__all__ = ["index", "topk", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
+__all__ = ["index", "topk", "topk_workspace_bytes", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
            "sparse_attn_prefill_bwd", "indexer_kl_loss", "device_status", "DSAError"]
 
 
@@ -60,16 +60,28 @@ def index(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_se
     return scores
 
 
+def topk_workspace_bytes(rows: int, ld_scores: int, k: int) -> int:
+    return _lib.load().dsa_topk_workspace_size(rows, ld_scores, k)
+
+
 def topk(scores, cu_seqlens_q, cu_seqlens_k, k: int, row_begin: int = 0, row_end: Optional[int] = None,
-         indices: Optional[torch.Tensor] = None):
-    """Deterministic top-k of each score row: int32 [rows, k], ascending, -1 padded."""
+         indices: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """Deterministic top-k of each score row: int32 [rows, k], ascending, -1 padded.
+
+    A workspace of dsa_topk_workspace_size bytes is allocated when the library asks for
+    one (few long rows) and none is given."""
     _check(scores, "scores", torch.float32, 2)
     row_end = row_begin + scores.shape[0] if row_end is None else row_end
     if indices is None:
         indices = torch.empty((row_end - row_begin, k), dtype=torch.int32, device=scores.device)
     _check(indices, "indices", torch.int32, 2)
+    if workspace is None:
+        nbytes = topk_workspace_bytes(row_end - row_begin, scores.shape[1], k)
+        if nbytes:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=scores.device)
     call("dsa_topk", _ptr(scores), scores.shape[1], _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
-         cu_seqlens_q.numel() - 1, row_begin, row_end, k, _ptr(indices), _stream())
+         cu_seqlens_q.numel() - 1, row_begin, row_end, k, _ptr(indices), _ptr(workspace),
+         0 if workspace is None else workspace.numel(), _stream())
     return indices
 
 

@@ -20,8 +20,10 @@ int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const in
                    int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k,
                    int H_I, int d_I, long long row_begin, long long row_end, float* scores, long long ld,
                    cudaStream_t stream);
+size_t topk_ws_bytes(long long rows, long long max_vis);
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
-                long long row_begin, long long row_end, int k, int* indices, int max_vis, cudaStream_t stream);
+                long long row_begin, long long row_end, int k, int* indices, int max_vis, void* ws,
+                size_t ws_bytes, cudaStream_t stream);
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
                                const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
                                float scale, void* O, float* lse, cudaStream_t stream);
@@ -163,18 +165,24 @@ DSA_API int dsa_index(const void* q_idx, const void* k_idx, const void* w, const
                         static_cast<cudaStream_t>(stream));
 }
 
+DSA_API size_t dsa_topk_workspace_size(int64_t rows, int64_t ld_scores, int k) {
+  if (rows < 1 || ld_scores < 1 || k < 1) return 0;
+  return topk_ws_bytes(rows, ld_scores);
+}
+
 DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_seqlens_q,
                      const int32_t* cu_seqlens_k, int batch, int64_t row_begin, int64_t row_end, int k,
-                     int32_t* indices, void* stream) {
+                     int32_t* indices, void* workspace, size_t workspace_bytes, void* stream) {
   if (!scores || !cu_seqlens_q || !cu_seqlens_k || !indices) return DSA_ERR_INVALID_ARG;
   if (!aligned16(scores) || (ld_scores % 4) != 0 || ld_scores <= 0) return DSA_ERR_INVALID_ARG;
   if (batch < 1 || row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID_ARG;
   if (k < 1) return DSA_ERR_INVALID_ARG;
   if (k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (workspace && !aligned16(workspace)) return DSA_ERR_INVALID_ARG;
   // the row length is bounded by ld_scores (>= the longest visible range)
   const int max_vis = ld_scores > 0x7FFFFFFF ? 0x7FFFFFFF : (int)ld_scores;
   return topk_launch(scores, ld_scores, cu_seqlens_q, cu_seqlens_k, batch, row_begin, row_end, k, indices, max_vis,
-                     static_cast<cudaStream_t>(stream));
+                     workspace, workspace ? workspace_bytes : 0, static_cast<cudaStream_t>(stream));
 }
 
 DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V, const int32_t* indices,
@@ -233,7 +241,7 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
     int st = dsa_index(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                        max_seqlen_k, H_I, d_I, r0, r1, scores, ld, stream);
     if (st != DSA_OK) return st;
-    st = dsa_topk(scores, ld, cu_seqlens_q, cu_seqlens_k, batch, r0, r1, k, indices + r0 * k, stream);
+    st = dsa_topk(scores, ld, cu_seqlens_q, cu_seqlens_k, batch, r0, r1, k, indices + r0 * k, nullptr, 0, stream);
     if (st != DSA_OK) return st;
   }
   return dsa_sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k, scale,
@@ -244,7 +252,7 @@ DSA_API size_t dsa_decode_workspace_size(int batch, int max_seqlen_k, int Hq, in
   if (batch < 1 || max_seqlen_k < 0 || Hq < 1 || d < 1 || k < 1) return 0;
   const size_t ld = round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
   return round_up((size_t)(batch + 1) * sizeof(int), 256) + round_up((size_t)batch * ld * sizeof(float), 256) +
-         round_up(decode_workspace_bytes(batch, Hq, d, k), 256);
+         round_up(topk_ws_bytes(batch, (long long)ld), 256) + round_up(decode_workspace_bytes(batch, Hq, d, k), 256);
 }
 
 DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, const void* Q, const void* K,
@@ -264,12 +272,15 @@ DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, cons
   const int64_t ld = (int64_t)round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
   float* scores = reinterpret_cast<float*>(ws);
   ws += round_up((size_t)batch * ld * sizeof(float), 256);
+  const size_t topk_bytes = topk_ws_bytes(batch, ld);
+  void* topk_ws = topk_bytes ? ws : nullptr;
+  ws += round_up(topk_bytes, 256);
   dsa::iota_kernel<<<(batch + 1 + 255) / 256, 256, 0, s>>>(cu_q, batch, 1);
   if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
   int st = dsa_index(q_idx, k_idx, w, cu_q, cu_seqlens_k, batch, batch, total_k, 1, max_seqlen_k, H_I, d_I, 0, batch,
                      scores, ld, stream);
   if (st != DSA_OK) return st;
-  st = dsa_topk(scores, ld, cu_q, cu_seqlens_k, batch, 0, batch, k, indices, stream);
+  st = dsa_topk(scores, ld, cu_q, cu_seqlens_k, batch, 0, batch, k, indices, topk_ws, topk_bytes, stream);
   if (st != DSA_OK) return st;
   return dsa_sparse_attn_decode(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale, O, lse, ws,
                                 workspace_bytes - (size_t)(ws - static_cast<uint8_t*>(workspace)), stream);

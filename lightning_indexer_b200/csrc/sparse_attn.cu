@@ -314,13 +314,14 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
     }
     if (lane < 4) {
       float* pml = p.part_ml + (((size_t)row * p.nsplit + split) * p.Hq + g * p.G) * 4;
-      if (h0 < p.G) { pml[h0 * 4] = m0; pml[h0 * 4 + 1] = l0; pml[h0 * 4 + 2] = r0; }
-      if (h1 < p.G) { pml[h1 * 4] = m1; pml[h1 * 4 + 1] = l1; pml[h1 * 4 + 2] = r1; }
+      if (h0 < p.G) *reinterpret_cast<float4*>(pml + h0 * 4) = make_float4(m0, l0, r0, 0.f);
+      if (h1 < p.G) *reinterpret_cast<float4*>(pml + h1 * 4) = make_float4(m1, l1, r1, 0.f);
     }
   }
 }
 
-// Merges the per-split partial softmax states of decode: one warp per (row, head).
+// Merges the per-split partial softmax states of decode: one warp per (row, head), lane s
+// holding split s (nsplit <= 32), so every load of the merge is issued at once.
 template <int D>
 __global__ void decode_combine_kernel(const float* part_o, const float* part_ml, int rows, int Hq, int nsplit,
                                       uint16_t* O, float* lse) {
@@ -328,26 +329,39 @@ __global__ void decode_combine_kernel(const float* part_o, const float* part_ml,
   const int lane = threadIdx.x % 32;
   if (gw >= rows * Hq) return;
   const int row = gw / Hq, h = gw % Hq;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, part_ml[(((size_t)row * nsplit + s) * Hq + h) * 4]);
+  const size_t mine = ((size_t)row * nsplit + lane) * Hq + h;  // this lane's split
+  float m = -INFINITY, l = 0.f, rr = 0.f;
+  if (lane < nsplit) {
+    const float4 ml = *reinterpret_cast<const float4*>(part_ml + mine * 4);
+    m = ml.x;
+    l = ml.y;
+    rr = ml.z;
+  }
+  float M = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float Mu = M == -INFINITY ? 0.f : M;
-  float L = 0.f, R = 0.f;
-  float o[D / 32];
+  const float f = (m == -INFINITY) ? 0.f : exp2f(m - Mu);
+  float L = l * f, R = rr * f;
 #pragma unroll
-  for (int j = 0; j < D / 32; ++j) o[j] = 0.f;
+  for (int o = 16; o > 0; o >>= 1) {
+    L += __shfl_xor_sync(0xffffffffu, L, o);
+    R += __shfl_xor_sync(0xffffffffu, R, o);
+  }
+  float o_[D / 32];
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) o_[j] = 0.f;
+#pragma unroll 4
   for (int s = 0; s < nsplit; ++s) {
-    const size_t base = ((size_t)row * nsplit + s) * Hq + h;
-    const float m = part_ml[base * 4], l = part_ml[base * 4 + 1], rr = part_ml[base * 4 + 2];
-    const float f = (m == -INFINITY) ? 0.f : exp2f(m - Mu);
-    L += l * f;
-    R += rr * f;
+    const float fs = __shfl_sync(0xffffffffu, f, s);
+    const float* po = part_o + (((size_t)row * nsplit + s) * Hq + h) * D;
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) o[j] += f * part_o[base * D + j * 32 + lane];
+    for (int j = 0; j < D / 32; ++j) o_[j] += fs * po[j * 32 + lane];
   }
   const float inv = R > 0.f ? 1.f / R : 0.f;
 #pragma unroll
   for (int j = 0; j < D / 32; ++j)
-    O[((size_t)row * Hq + h) * D + j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o[j] * inv));
+    O[((size_t)row * Hq + h) * D + j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o_[j] * inv));
   if (lse && lane == 0) lse[(size_t)row * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
@@ -361,8 +375,10 @@ static int sa_launch_d(const dsa::SAParams& p, long long tasks, cudaStream_t str
   const int smem = dsa::sa_smem_bytes<D>(dsa::SA_WARPS);
   static bool done = false;
   if (!done) {
-    const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                smem);
+    cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // several CTAs per SM need the largest shared-memory carveout
+    if (e_ == cudaSuccess)
+      e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e_ != cudaSuccess) return cuda_fail(e_);
     done = true;
   }
@@ -400,7 +416,7 @@ int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, cons
 }
 
 int decode_nsplit(int k) {
-  int ns = k / 128;  // 128 keys per split
+  int ns = k / 128;  // 128 keys per split; <= 32 for k <= 4096 (the combine kernel's lane-per-split)
   if (ns < 1) ns = 1;
   while (ns > 1 && (k % (ns * dsa::SA_CHUNK)) != 0) --ns;
   return ns;

@@ -117,15 +117,14 @@ struct TopkSmem {
   uint32_t total, bin, above;
   uint32_t flag;     // this block's candidates overflow TOPK_CAP
   uint32_t counts[2];  // (#keys > K*, #ties) of this block's segment
+  uint32_t dmax;
 };
 
+// The exact selection of one row (by a cluster of C blocks).
 template <int C>
-__global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) {
+__device__ void exact_row_select(const TopkParams& p, TopkSmem& S, const long long row) {
   constexpr int B = TOPK_THREADS;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int rank = (C > 1) ? (int)cg::this_cluster().block_rank() : 0;
-  const long long row = p.row_begin + blockIdx.x / C;
   int lo = 0, hi = p.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) / 2;
@@ -447,6 +446,13 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) 
   if constexpr (C > 1) cg::this_cluster().sync();
 }
 
+template <int C>
+__global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  exact_row_select<C>(p, S, p.row_begin + blockIdx.x / C);
+}
+
 // ======================================================================================
 // Fast path.  512 threads, two blocks per SM.  A sampled lower bound T is taken first (the
 // same 2048 strided positions in every block of the row); one streaming pass then
@@ -713,10 +719,144 @@ __global__ void __launch_bounds__(FT, 2) topk_fast_kernel(const TopkParams p) {
 
 
 // ======================================================================================
+// Helpers over a candidate list in shared memory (keys >= T, in position order).
+
+// The exact k-th largest key K* among the n candidates, and how many keys equal to K* are
+// taken, by radix levels over d = key - T.  The first level's 2048 bins span exactly
+// [0, max d], so candidates that share their top key bits (scores in a narrow range) still
+// spread over many bins instead of piling onto a few shared-memory counters.
+template <int B>
+__device__ void select_relative(const uint32_t* ckey, int n, uint32_t T, uint32_t k, uint32_t* hist,
+                                uint32_t* warp_sums, uint32_t* total, uint32_t* bin, uint32_t* above,
+                                uint32_t* dmax, uint32_t& kstar, uint32_t& remaining) {
+  uint32_t dm = 0;
+  for (int j = threadIdx.x; j < n; j += B) dm = max(dm, ckey[j] - T);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dm = max(dm, __shfl_xor_sync(0xffffffffu, dm, o));
+  if (threadIdx.x == 0) *dmax = 0;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) atomicMax(dmax, dm);
+  __syncthreads();
+  const int nbits = 32 - __clz((int)*dmax);
+  int shift = max(0, nbits - 11);
+  uint32_t prefix = 0, pmask = 0, rem = k;
+#pragma unroll 1
+  while (true) {
+    for (int j = threadIdx.x; j < 2048; j += B) hist[j] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += B) {
+      const uint32_t d = ckey[j] - T;
+      if ((d & pmask) == prefix) atomicAdd(&hist[(d >> shift) & 2047u], 1u);
+    }
+    __syncthreads();
+    find_bin<B, 2048>(hist, rem, warp_sums, total, bin, above);
+    prefix |= *bin << shift;
+    pmask |= 2047u << shift;
+    rem -= *above;
+    if (shift == 0) break;
+    shift = max(0, shift - 11);
+  }
+  kstar = T + prefix;
+  remaining = rem;
+}
+
+// Writes the selected candidates (keys > K*, and the first `remaining` keys equal to K*)
+// to out[0..k) in candidate order, which is position order.
+template <int B>
+__device__ void write_selected(const uint32_t* ckey, const int* cpos, int n, uint32_t kstar, uint32_t remaining,
+                               int* out, uint32_t* warp_sums, uint32_t* total) {
+  constexpr int IT = 4;  // tile totals <= B * IT fit the packed 16-bit fields
+  static_assert(B * IT < 65536, "packed counts");
+  uint32_t base_gt = 0, base_tie = 0;
+  for (int start = 0; start < n; start += B * IT) {
+    const int j0 = start + threadIdx.x * IT;
+    uint32_t g_ = 0, e_ = 0;
+#pragma unroll
+    for (int j = 0; j < IT; ++j) {
+      if (j0 + j < n) {
+        g_ += ckey[j0 + j] > kstar;
+        e_ += ckey[j0 + j] == kstar;
+      }
+    }
+    const uint32_t excl = block_excl_scan<B>((g_ << 16) | e_, warp_sums, total);
+    uint32_t gt_before = base_gt + (excl >> 16), eq_before = base_tie + (excl & 0xFFFFu);
+#pragma unroll
+    for (int j = 0; j < IT; ++j) {
+      if (j0 + j >= n) break;
+      const uint32_t kk = ckey[j0 + j];
+      if (kk > kstar) {
+        out[gt_before + min(eq_before, remaining)] = cpos[j0 + j];
+        ++gt_before;
+      } else if (kk == kstar) {
+        if (eq_before < remaining) out[gt_before + eq_before] = cpos[j0 + j];
+        ++eq_before;
+      }
+    }
+    base_gt += *total >> 16;
+    base_tie += *total & 0xFFFFu;
+    __syncthreads();
+  }
+}
+
+// A fixed strided sample of NS positions of a row (PER keys per thread), and from it the
+// r_low-th largest sampled key to 22 bits: a lower bound on the row's k-th largest key
+// with a margin of ~3 sigma + 8 sampled keys.  Every block that samples the same row gets
+// the same value.
+constexpr int SAMPLE_N = 2048;
+
+template <int B>
+__device__ __forceinline__ void load_sample(const float* src, int vis, uint32_t* sk) {
+#pragma unroll
+  for (int u = 0; u < SAMPLE_N / B; ++u) {
+    const long long pos = ((2LL * (threadIdx.x + u * B) + 1) * vis) / (2LL * SAMPLE_N);
+    sk[u] = float_order_key(__ldg(src + pos));
+  }
+}
+
+template <int B>
+__device__ uint32_t bound_from_sample(const uint32_t* sk, int vis, int k, uint32_t* hist, uint32_t* warp_sums,
+                                      uint32_t* total, uint32_t* bin, uint32_t* above) {
+  constexpr int PER = SAMPLE_N / B;
+  static_assert(SAMPLE_N % B == 0, "samples per thread");
+  const float m = (float)k * (float)SAMPLE_N / (float)vis;
+  const int r_low = min(SAMPLE_N, (int)ceilf(m + 3.f * sqrtf(m) + 8.f));
+  uint32_t sp = 0, sm = 0, rem = (uint32_t)r_low;
+#pragma unroll 1
+  for (int lv = 0; lv < 2; ++lv) {
+    const int shift = lv == 0 ? 21 : 10;
+    for (int j = threadIdx.x; j < 2048; j += B) hist[j] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      // samples of a row often share their top bits: one counter update per distinct bin
+      // and warp instead of one per sample
+      const bool act = (sk[u] & sm) == sp;
+      const uint32_t b = act ? (sk[u] >> shift) & 2047u : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, b);
+      if (act && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[b], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    find_bin<B, 2048>(hist, rem, warp_sums, total, bin, above);
+    sp |= *bin << shift;
+    sm |= 2047u << shift;
+    rem -= *above;
+  }
+  return sp;
+}
+
+template <int B>
+__device__ uint32_t sampled_bound(const float* src, int vis, int k, uint32_t* hist, uint32_t* warp_sums,
+                                  uint32_t* total, uint32_t* bin, uint32_t* above) {
+  uint32_t sk[SAMPLE_N / B];
+  load_sample<B>(src, vis, sk);
+  return bound_from_sample<B>(sk, vis, k, hist, warp_sums, total, bin, above);
+}
+
+// ======================================================================================
 // Few long rows (decode: a handful of sequences with 10^5 cached positions each).  A row
-// goes to a cluster of C blocks of 512 threads; every thread loads 64 consecutive scores
-// of the row into registers with 16 float4 loads that are all in flight at once, so the
-// row is read from memory exactly once.
+// goes to a cluster of C blocks of 512 threads; the block reads its segment once with 16
+// coalesced float4 loads per thread (all in flight at once) and hands every thread 64
+// consecutive scores in registers through a swizzled shared-memory transpose.
 //   1. While those loads fly, every block takes the same strided sample of 2048 positions
 //      and, by two radix levels, the r_low-th largest sampled key T (a lower bound on the
 //      k-th largest key, with a safety margin).
@@ -737,8 +877,13 @@ constexpr int RSEG = RT * RKEYS;  // positions per block
 constexpr int RCAP = 16384;       // candidates rank 0 can hold
 
 struct RegsSmem {
-  uint32_t cand_key[RCAP];
-  int cand_pos[RCAP];
+  union {
+    float4 seg[RSEG / 4];  // the block's scores, swizzled 16-byte chunks (load transpose)
+    struct {
+      uint32_t cand_key[RCAP];  // rank 0: the row's candidates in position order
+      int cand_pos[RCAP];
+    };
+  };
   uint32_t hist[2][2048];  // per level parity (remote blocks read them)
   uint32_t ghist[2048];    // cluster-wide sum
   uint32_t warp_sums[32];
@@ -777,47 +922,36 @@ __global__ void __launch_bounds__(RT, 1) topk_regs_kernel(const TopkParams p) {
   const int s_lo = min(rank * seg, vis), s_hi = min(s_lo + seg, vis);
   const int t_lo = s_lo + threadIdx.x * RKEYS;
   const int nvalid = max(0, min(RKEYS, s_hi - t_lo));  // keys [0, nvalid) of this thread are real
-  float4 x[RKEYS / 4];
+  // coalesced loads: 16-byte chunk q = u * B + tid of the segment, stored at chunk
+  // q ^ ((q >> 4) & 7) so that both this store and the per-thread reads below (16
+  // consecutive chunks of one thread) are free of bank conflicts
+  {
+    float4 x[RKEYS / 4];
 #pragma unroll
-  for (int u = 0; u < RKEYS / 4; ++u)
-    x[u] = (4 * u < nvalid) ? __ldg(reinterpret_cast<const float4*>(src + t_lo) + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < RKEYS / 4; ++u) {
+      const int q = u * B + threadIdx.x;
+      x[u] = (s_lo + 4 * q < s_hi) ? __ldg(reinterpret_cast<const float4*>(src + s_lo) + q)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < RKEYS / 4; ++u) {
+      const int q = u * B + threadIdx.x;
+      S.seg[q ^ ((q >> 4) & 7)] = x[u];
+    }
+  }
 
   // ---------------------------------------------------------------- 1. sampled bound T
-  uint32_t T;
-  {
-    constexpr int NS = 2048, PER = NS / B;
-    const float m = (float)k * (float)NS / (float)vis;
-    const int r_low = min(NS, (int)ceilf(m + 3.f * sqrtf(m) + 8.f));
-    uint32_t sk[PER];
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const long long pos = ((2LL * (threadIdx.x + u * B) + 1) * vis) / (2LL * NS);
-      sk[u] = float_order_key(__ldg(src + pos));
-    }
-    uint32_t sp = 0, sm = 0, rem = (uint32_t)r_low;
-#pragma unroll 1
-    for (int lv = 0; lv < 2; ++lv) {
-      const int shift = lv == 0 ? 21 : 10;
-      for (int j = threadIdx.x; j < 2048; j += B) S.ghist[j] = 0;
-      __syncthreads();
-#pragma unroll
-      for (int u = 0; u < PER; ++u)
-        if ((sk[u] & sm) == sp) atomicAdd(&S.ghist[(sk[u] >> shift) & 2047u], 1u);
-      __syncthreads();
-      find_bin<B, 2048>(S.ghist, rem, S.warp_sums, &S.total, &S.bin, &S.above);
-      sp |= S.bin << shift;
-      sm |= 2047u << shift;
-      rem -= S.above;
-    }
-    T = sp;
-  }
+  const uint32_t T = sampled_bound<B>(src, vis, k, S.ghist, S.warp_sums, &S.total, &S.bin, &S.above);
+  __syncthreads();  // the segment is in shared memory
   uint32_t key[RKEYS];
 #pragma unroll
   for (int u = 0; u < RKEYS / 4; ++u) {
-    key[4 * u + 0] = float_order_key(x[u].x);
-    key[4 * u + 1] = float_order_key(x[u].y);
-    key[4 * u + 2] = float_order_key(x[u].z);
-    key[4 * u + 3] = float_order_key(x[u].w);
+    const int q = threadIdx.x * (RKEYS / 4) + u;
+    const float4 x = S.seg[q ^ ((q >> 4) & 7)];
+    key[4 * u + 0] = float_order_key(x.x);
+    key[4 * u + 1] = float_order_key(x.y);
+    key[4 * u + 2] = float_order_key(x.z);
+    key[4 * u + 3] = float_order_key(x.w);
   }
 
   // ---------------------------------------------------------------- 2. candidates >= T
@@ -850,66 +984,10 @@ __global__ void __launch_bounds__(RT, 1) topk_regs_kernel(const TopkParams p) {
     }
     cl.sync();  // the candidates have landed in rank 0; nothing else is read remotely
     if (rank != 0) return;
-    const int n = (int)N;
-    // exact K* over d = key - T; the first level's bins span [0, max d]
-    uint32_t dm = 0;
-    for (int j = threadIdx.x; j < n; j += B) dm = max(dm, S.cand_key[j] - T);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dm = max(dm, __shfl_xor_sync(0xffffffffu, dm, o));
-    if (threadIdx.x == 0) S.dmax = 0;
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) atomicMax(&S.dmax, dm);
-    __syncthreads();
-    const int nbits = 32 - __clz((int)S.dmax);
-    int shift = max(0, nbits - 11);
-    uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
-#pragma unroll 1
-    while (true) {
-      for (int j = threadIdx.x; j < 2048; j += B) S.ghist[j] = 0;
-      __syncthreads();
-      for (int j = threadIdx.x; j < n; j += B) {
-        const uint32_t d = S.cand_key[j] - T;
-        if ((d & pmask) == prefix) atomicAdd(&S.ghist[(d >> shift) & 2047u], 1u);
-      }
-      __syncthreads();
-      find_bin<B, 2048>(S.ghist, remaining, S.warp_sums, &S.total, &S.bin, &S.above);
-      prefix |= S.bin << shift;
-      pmask |= 2047u << shift;
-      remaining -= S.above;
-      if (shift == 0) break;
-      shift = max(0, shift - 11);
-    }
-    const uint32_t kstar = T + prefix;
-    constexpr int IT = 4;
-    uint32_t base_gt = 0, base_tie = 0;
-    for (int start = 0; start < n; start += B * IT) {
-      const int j0 = start + threadIdx.x * IT;
-      uint32_t g_ = 0, e_ = 0;
-#pragma unroll
-      for (int j = 0; j < IT; ++j) {
-        if (j0 + j < n) {
-          g_ += S.cand_key[j0 + j] > kstar;
-          e_ += S.cand_key[j0 + j] == kstar;
-        }
-      }
-      const uint32_t excl = block_excl_scan<B>((g_ << 16) | e_, S.warp_sums, &S.total);
-      uint32_t gt_before = base_gt + (excl >> 16), eq_before = base_tie + (excl & 0xFFFFu);
-#pragma unroll
-      for (int j = 0; j < IT; ++j) {
-        if (j0 + j >= n) break;
-        const uint32_t kk = S.cand_key[j0 + j];
-        if (kk > kstar) {
-          out[gt_before + min(eq_before, remaining)] = S.cand_pos[j0 + j];
-          ++gt_before;
-        } else if (kk == kstar) {
-          if (eq_before < remaining) out[gt_before + eq_before] = S.cand_pos[j0 + j];
-          ++eq_before;
-        }
-      }
-      base_gt += S.total >> 16;
-      base_tie += S.total & 0xFFFFu;
-      __syncthreads();
-    }
+    uint32_t kstar, remaining;
+    select_relative<B>(S.cand_key, (int)N, T, (uint32_t)k, S.ghist, S.warp_sums, &S.total, &S.bin, &S.above, &S.dmax,
+                       kstar, remaining);
+    write_selected<B>(S.cand_key, S.cand_pos, (int)N, kstar, remaining, out, S.warp_sums, &S.total);
     return;
   }
 
@@ -975,6 +1053,177 @@ __global__ void __launch_bounds__(RT, 1) topk_regs_kernel(const TopkParams p) {
     }
   }
   cl.sync();  // no block may leave while another still reads its shared memory
+}
+
+// ======================================================================================
+// Few long rows with a caller workspace (the decode shape: 16 sequences x 262144 cached
+// positions).  Three launches, no clusters, so every SM takes part however the GPCs are
+// filled:
+//   0. row bound: one block per row takes the row's sampled bound T.
+//   1. segment filter: one 256-thread block per (row, 8192-position segment).  The block
+//      reads its segment once (coalesced float4 loads, handed to the threads as 32
+//      consecutive scores each through a swizzled shared-memory transpose) and writes its
+//      keys >= T, in position order, to the workspace with their count.
+//   2. row select: one 1024-thread block per row gathers the segments' candidates in
+//      order, finds the exact K* by radix levels over (key - T) and writes the selected
+//      positions.  A row whose candidates are too few (an unlucky sample), overflow a
+//      segment or the block's list (huge ties) is selected by the exact method from the
+//      scores instead.  Either way the result is the exact top-k.
+constexpr int SF_T = 256;                 // threads of a segment-filter block
+constexpr int SF_SEG = 8192;              // positions per segment
+constexpr int SF_KEYS = SF_SEG / SF_T;    // keys per thread
+constexpr int SF_CAP = 1024;              // candidates kept per segment
+constexpr int SF_MAX_BLOCKS = 1024;       // rows x segments beyond which this path is not used
+
+struct TopkWs {
+  uint32_t* thr;  // [rows] sampled bound T of each row (written for rows with vis > k)
+  uint32_t* cnt;  // [rows, nseg] candidates of each segment (may exceed SF_CAP: overflow)
+  uint2* cand;    // [rows, nseg, SF_CAP] (key, position)
+  int nseg;
+};
+
+struct SegFilterSmem {
+  float4 seg[SF_SEG / 4];
+  uint32_t ghist[2048];
+  uint32_t warp_sums[32];
+  uint32_t total, bin, above;
+};
+
+__device__ __forceinline__ int row_visible(const TopkParams& p, long long row) {
+  int lo = 0, hi = p.batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
+  }
+  const int i = (int)(row - p.cu_q[lo]);
+  const int Lq = p.cu_q[lo + 1] - p.cu_q[lo];
+  const int Lk = p.cu_k[lo + 1] - p.cu_k[lo];
+  return min(max(i + Lk - Lq + 1, 0), Lk);
+}
+
+// The sampled bound T of each row, once per row (a sample read by every filter block of
+// the row would hit the same L2 sectors from all of them at once).
+__global__ void __launch_bounds__(SF_T) topk_rowbound_kernel(const TopkParams p, const TopkWs ws) {
+  constexpr int B = SF_T;
+  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t total, bin, above;
+  const long long rr = blockIdx.x;
+  const int vis = row_visible(p, p.row_begin + rr);
+  if (vis <= p.k) return;
+  const uint32_t T = sampled_bound<B>(p.scores + rr * p.ld, vis, p.k, hist, warp_sums, &total, &bin, &above);
+  if (threadIdx.x == 0) ws.thr[rr] = T;
+}
+
+__global__ void __launch_bounds__(SF_T, 4) topk_segfilter_kernel(const TopkParams p, const TopkWs ws) {
+  constexpr int B = SF_T;
+  __shared__ SegFilterSmem S;
+  const long long rr = blockIdx.x / ws.nseg;
+  const int sg = blockIdx.x % ws.nseg;
+  const long long row = p.row_begin + rr;
+  const int vis = row_visible(p, row);
+  if (vis <= p.k) return;  // the row-select block handles such rows without the workspace
+  uint32_t* cnt = ws.cnt + rr * ws.nseg + sg;
+  const int s_lo = sg * SF_SEG;
+  if (s_lo >= vis) {
+    if (threadIdx.x == 0) *cnt = 0;
+    return;
+  }
+  const int s_hi = min(s_lo + SF_SEG, vis);
+  const float* src = p.scores + rr * p.ld;
+  {
+    // chunk q = u * B + tid, stored at q ^ ((q >> 3) & 7): conflict-free here and for the
+    // per-thread reads of 8 consecutive chunks below
+    float4 x[SF_KEYS / 4];
+#pragma unroll
+    for (int u = 0; u < SF_KEYS / 4; ++u) {
+      const int q = u * B + threadIdx.x;
+      x[u] = (s_lo + 4 * q < s_hi) ? __ldg(reinterpret_cast<const float4*>(src + s_lo) + q)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < SF_KEYS / 4; ++u) {
+      const int q = u * B + threadIdx.x;
+      S.seg[q ^ ((q >> 3) & 7)] = x[u];
+    }
+  }
+  const uint32_t T = ws.thr[rr];
+  __syncthreads();  // the segment is in shared memory
+  const int t_lo = s_lo + threadIdx.x * SF_KEYS;
+  const int nvalid = max(0, min(SF_KEYS, s_hi - t_lo));
+  // this thread's keys are re-read from shared memory (16-byte reads) in each of the two passes
+  auto chunk_at = [&](int u) -> float4 {
+    const int q = threadIdx.x * (SF_KEYS / 4) + u;
+    return S.seg[q ^ ((q >> 3) & 7)];
+  };
+  uint32_t n = 0;
+#pragma unroll
+  for (int u = 0; u < SF_KEYS / 4; ++u) {
+    const float4 x = chunk_at(u);
+    const float v[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) n += (4 * u + e < nvalid && float_order_key(v[e]) >= T);
+  }
+  uint32_t pos = block_excl_scan<B>(n, S.warp_sums, &S.total);
+  uint2* dst = ws.cand + (rr * ws.nseg + sg) * SF_CAP;
+#pragma unroll
+  for (int u = 0; u < SF_KEYS / 4; ++u) {
+    const float4 x = chunk_at(u);
+    const float v[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t kj = float_order_key(v[e]);
+      if (4 * u + e < nvalid && kj >= T) {
+        if (pos < (uint32_t)SF_CAP) dst[pos] = make_uint2(kj, (uint32_t)(t_lo + 4 * u + e));
+        ++pos;
+      }
+    }
+  }
+  if (threadIdx.x == 0) *cnt = S.total;
+}
+
+__global__ void __launch_bounds__(TOPK_THREADS) topk_rowselect_kernel(const TopkParams p, const TopkWs ws) {
+  constexpr int B = TOPK_THREADS;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  const long long rr = blockIdx.x;
+  const long long row = p.row_begin + rr;
+  const int vis = row_visible(p, row);
+  const int k = p.k;
+  int* out = p.indices + rr * k;
+  if (vis <= k) {
+    for (int j = threadIdx.x; j < k; j += B) out[j] = j < vis ? j : -1;
+    return;
+  }
+  const int nseg = (vis + SF_SEG - 1) / SF_SEG;  // <= ws.nseg <= B (host-checked)
+  const uint32_t c = threadIdx.x < nseg ? ws.cnt[rr * ws.nseg + threadIdx.x] : 0u;
+  const bool overflow = __syncthreads_or(c > (uint32_t)SF_CAP) != 0;
+  const uint32_t base = block_excl_scan<B>(c, S.warp_sums, &S.total);
+  const uint32_t N = S.total;
+  if (!overflow && N >= (uint32_t)k && N <= (uint32_t)TOPK_CAP) {
+    if (threadIdx.x < nseg) S.ghist[threadIdx.x] = base;  // segment start in the list
+    __syncthreads();
+    // warp w gathers segments w, w + 32, ...: coalesced, and in position order overall
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int sgi = warp; sgi < nseg; sgi += B / 32) {
+      const uint2* srcc = ws.cand + (rr * ws.nseg + sgi) * SF_CAP;
+      const uint32_t b0 = S.ghist[sgi];
+      const uint32_t cn = ws.cnt[rr * ws.nseg + sgi];
+      for (uint32_t j = lane; j < cn; j += 32) {
+        const uint2 e = srcc[j];
+        S.cand_key[b0 + j] = e.x;
+        S.cand_pos[b0 + j] = (int)e.y;
+      }
+    }
+    __syncthreads();
+    uint32_t kstar, remaining;
+    select_relative<B>(S.cand_key, (int)N, ws.thr[rr], (uint32_t)k, S.hist[0], S.warp_sums, &S.total, &S.bin,
+                       &S.above, &S.dmax, kstar, remaining);
+    write_selected<B>(S.cand_key, S.cand_pos, (int)N, kstar, remaining, out, S.warp_sums, &S.total);
+    return;
+  }
+  __syncthreads();  // S.total and S.warp_sums are reused by the exact method
+  exact_row_select<1>(p, S, row);
 }
 
 }  // namespace dsa
@@ -1044,8 +1293,49 @@ static int topk_regs_launch(const dsa::TopkParams& p, long long rows, cudaStream
   return last_launch_status();
 }
 
+// Workspace of the two-launch path for `rows` rows of up to max_vis positions; 0 where
+// that path is not used (many rows, short rows or rows beyond its segment count).
+size_t topk_ws_bytes(long long rows, long long max_vis) {
+  if (rows <= 0 || max_vis <= 32768) return 0;
+  const long long nseg = (max_vis + dsa::SF_SEG - 1) / dsa::SF_SEG;
+  if (nseg > dsa::TOPK_THREADS || rows * nseg > dsa::SF_MAX_BLOCKS) return 0;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  return up((size_t)rows * 4) + up((size_t)(rows * nseg) * 4) + up((size_t)(rows * nseg) * dsa::SF_CAP * 8);
+}
+
+static int topk_two_launch(const dsa::TopkParams& p, long long rows, long long max_vis, void* ws_ptr,
+                           cudaStream_t stream) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  dsa::TopkWs ws;
+  ws.nseg = (int)((max_vis + dsa::SF_SEG - 1) / dsa::SF_SEG);
+  uint8_t* w = static_cast<uint8_t*>(ws_ptr);
+  ws.thr = reinterpret_cast<uint32_t*>(w);
+  w += up((size_t)rows * 4);
+  ws.cnt = reinterpret_cast<uint32_t*>(w);
+  w += up((size_t)(rows * ws.nseg) * 4);
+  ws.cand = reinterpret_cast<uint2*>(w);
+  static bool attr_done = false;
+  if (!attr_done) {
+    // four filter blocks per SM need the largest shared-memory carveout
+    cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_segfilter_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          100);
+    if (e_ == cudaSuccess)
+      e_ = cudaFuncSetAttribute(dsa::topk_rowselect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(dsa::TopkSmem));
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    attr_done = true;
+  }
+  dsa::topk_rowbound_kernel<<<(unsigned)rows, dsa::SF_T, 0, stream>>>(p, ws);
+  if (const int st = last_launch_status(); st != DSA_OK) return st;
+  dsa::topk_segfilter_kernel<<<(unsigned)(rows * ws.nseg), dsa::SF_T, 0, stream>>>(p, ws);
+  if (const int st = last_launch_status(); st != DSA_OK) return st;
+  dsa::topk_rowselect_kernel<<<(unsigned)rows, dsa::TOPK_THREADS, sizeof(dsa::TopkSmem), stream>>>(p, ws);
+  return last_launch_status();
+}
+
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
-                long long row_begin, long long row_end, int k, int* indices, int max_vis, cudaStream_t stream) {
+                long long row_begin, long long row_end, int k, int* indices, int max_vis, void* ws,
+                size_t ws_bytes, cudaStream_t stream) {
   const long long rows = row_end - row_begin;
   if (rows <= 0) return DSA_OK;
   if (rows > 0x7FFFFFFFLL / 16) return DSA_ERR_UNSUPPORTED;
@@ -1060,6 +1350,9 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
   p.indices = indices;
   p.only_marked = 0;
   const int sms = sm_count();
+  // few long rows with a workspace: segment filter + row select
+  if (const size_t need = topk_ws_bytes(rows, max_vis); need > 0 && ws != nullptr && ws_bytes >= need)
+    return topk_two_launch(p, rows, max_vis, ws, stream);
   // few long rows: one cluster per row with the row held in registers, while that takes
   // at most two waves of one block per SM
   if (max_vis > 32768) {

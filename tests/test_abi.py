@@ -50,8 +50,13 @@ def test_host_side_argument_errors():
     # unsupported indexer shape
     assert lib.dsa_index(fake, fake, fake, fake, fake, 1, 8, 8, 8, 8, 48, 128, 0, 8, fake, 8, None) == -2
     # top-k bounds
-    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 0, fake, None) == -1
-    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 5000, fake, None) == -2
+    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 0, fake, None, 0, None) == -1
+    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 5000, fake, None, 0, None) == -2
+    assert lib.dsa_topk(fake, 8, fake, fake, 1, 0, 8, 16, fake, mis, 1024, None) == -1  # misaligned workspace
+    # top-k workspace: asked for few long rows only
+    assert lib.dsa_topk_workspace_size(16, 262144, 2048) > 0
+    assert lib.dsa_topk_workspace_size(8192, 131072, 2048) == 0
+    assert lib.dsa_topk_workspace_size(16, 4096, 2048) == 0
     # attention shapes
     assert lib.dsa_sparse_attn_prefill(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 96, 64, 0.1, fake,
                                        None, None) == -2

@@ -125,6 +125,31 @@ def test_topk_candidate_overflow_paths(n_rows, n):
         assert np.array_equal(idx[r], orc.topk_row(sc[r, :vis[r]].astype(np.float64), 2048)), r
 
 
+@pytest.mark.parametrize("case", ["decode_length", "adversarial"])
+def test_topk_few_long_rows_without_workspace(case):
+    # an empty workspace selects the single-launch path (one cluster per row, the row held
+    # in registers); the result must equal the two-launch path's and the oracle's
+    if case == "decode_length":
+        vis = [262144, 262143, 131072, 200000]
+        sc, cu_q, cu_k = _topk_case(vis, 2048, seed=13, ties=False)
+    else:
+        n = 131072
+        rng = np.random.default_rng(12)
+        sc = rng.standard_normal((3, n)).astype(np.float32)
+        sc[0, ((2 * np.arange(1024) + 1) * n) // 2048] = 10.0   # the sample sees only huge values
+        sc[1] = 1.0                                            # all ties
+        sc[2, ::3] = 7.0
+        vis = [n] * 3
+        cu_q = np.arange(4, dtype=np.int32)
+        cu_k = (np.arange(4) * n).astype(np.int32)
+    args = (torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(), 2048)
+    a = dsa.topk(*args, workspace=torch.empty(0, dtype=torch.uint8, device="cuda")).cpu().numpy()
+    b = dsa.topk(*args).cpu().numpy()
+    assert np.array_equal(a, b)
+    for r, n in enumerate(vis):
+        assert np.array_equal(a[r], orc.topk_row(sc[r, :n].astype(np.float64), 2048)), r
+
+
 def test_topk_many_long_rows_cluster_path():
     # 120 rows of ~100K positions: too many rows for one cluster per row with the row in
     # registers, so the sampled-threshold kernel runs with a small cluster per row
