@@ -718,6 +718,19 @@ __global__ void __launch_bounds__(FT, 2) topk_fast_kernel(const TopkParams p) {
 }
 
 
+// Visible positions of a row (bottom-right causal alignment).
+__device__ __forceinline__ int row_visible(const TopkParams& p, long long row) {
+  int lo = 0, hi = p.batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
+  }
+  const int i = (int)(row - p.cu_q[lo]);
+  const int Lq = p.cu_q[lo + 1] - p.cu_q[lo];
+  const int Lk = p.cu_k[lo + 1] - p.cu_k[lo];
+  return min(max(i + Lk - Lq + 1, 0), Lk);
+}
+
 // ======================================================================================
 // Helpers over a candidate list in shared memory (keys >= T, in position order).
 
@@ -1056,6 +1069,96 @@ __global__ void __launch_bounds__(RT, 1) topk_regs_kernel(const TopkParams p) {
 }
 
 // ======================================================================================
+// Many rows (prefill chunks: thousands of rows of up to ~10^5 positions).  One 256-thread
+// block per row, four blocks per SM, so the latency-bound steps of some rows overlap the
+// streaming of others:
+//   1. the row's sampled bound T (a strided sample of 2048 scores);
+//   2. one streaming pass over the row in tiles of 4096 positions (16 consecutive per
+//      thread, the next tile's loads issued before this tile is compacted): keys >= T are
+//      appended to a shared-memory list by a block scan per tile, so the list is in
+//      position order;
+//   3. the exact K* by radix levels over (key - T) on the list, and the ordered output.
+// A row whose list would overflow, or holds fewer than k keys (an unlucky sample), gets -2
+// in its first output slot and is finished by the exact kernel.
+constexpr int ST_T = 256;
+constexpr int ST_ITEMS = 16;
+constexpr int ST_TILE = ST_T * ST_ITEMS;
+constexpr int ST_CAP = 4096;
+
+struct StreamSmem {
+  uint32_t cand_key[ST_CAP];
+  int cand_pos[ST_CAP];
+  uint32_t hist[2048];
+  uint32_t warp_sums[32];
+  uint32_t total, bin, above, dmax;
+};
+
+__global__ void __launch_bounds__(ST_T, 4) topk_stream_kernel(const TopkParams p) {
+  constexpr int B = ST_T;
+  __shared__ StreamSmem S;
+  const long long row = p.row_begin + blockIdx.x;
+  const int vis = row_visible(p, row);
+  const int k = p.k;
+  int* out = p.indices + (row - p.row_begin) * k;
+  const float* src = p.scores + (row - p.row_begin) * p.ld;
+  if (vis <= k) {
+    for (int j = threadIdx.x; j < k; j += B) out[j] = j < vis ? j : -1;
+    return;
+  }
+  // loads ST_ITEMS scores of positions [s0, s0 + ST_ITEMS) (s0 4-aligned), 0 past the row
+  auto load = [&](int s0, float4* x) {
+#pragma unroll
+    for (int u = 0; u < ST_ITEMS / 4; ++u)
+      x[u] = (s0 + 4 * u < vis) ? __ldg(reinterpret_cast<const float4*>(src + s0) + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  float4 cur[ST_ITEMS / 4];
+  load(threadIdx.x * ST_ITEMS, cur);  // first tile in flight during the sample
+  const uint32_t T = sampled_bound<B>(src, vis, k, S.hist, S.warp_sums, &S.total, &S.bin, &S.above);
+
+  uint32_t base = 0;
+  for (int tile = 0; tile < vis; tile += ST_TILE) {
+    const int s0 = tile + threadIdx.x * ST_ITEMS;
+    float4 nxt[ST_ITEMS / 4];
+    load(s0 + ST_TILE, nxt);
+    uint32_t key[ST_ITEMS];
+#pragma unroll
+    for (int u = 0; u < ST_ITEMS / 4; ++u) {
+      key[4 * u + 0] = float_order_key(cur[u].x);
+      key[4 * u + 1] = float_order_key(cur[u].y);
+      key[4 * u + 2] = float_order_key(cur[u].z);
+      key[4 * u + 3] = float_order_key(cur[u].w);
+    }
+    uint32_t n = 0;
+#pragma unroll
+    for (int j = 0; j < ST_ITEMS; ++j) n += (s0 + j < vis && key[j] >= T);
+    uint32_t pos = base + block_excl_scan<B>(n, S.warp_sums, &S.total);
+#pragma unroll
+    for (int j = 0; j < ST_ITEMS; ++j) {
+      if (s0 + j < vis && key[j] >= T) {
+        if (pos < (uint32_t)ST_CAP) {
+          S.cand_key[pos] = key[j];
+          S.cand_pos[pos] = s0 + j;
+        }
+        ++pos;
+      }
+    }
+    base += S.total;
+#pragma unroll
+    for (int u = 0; u < ST_ITEMS / 4; ++u) cur[u] = nxt[u];
+    // (S.total is rewritten only after the next scan's first barrier)
+  }
+  __syncthreads();
+  if (base < (uint32_t)k || base > (uint32_t)ST_CAP) {
+    if (threadIdx.x == 0) out[0] = -2;
+    return;
+  }
+  uint32_t kstar, remaining;
+  select_relative<B>(S.cand_key, (int)base, T, (uint32_t)k, S.hist, S.warp_sums, &S.total, &S.bin, &S.above, &S.dmax,
+                     kstar, remaining);
+  write_selected<B>(S.cand_key, S.cand_pos, (int)base, kstar, remaining, out, S.warp_sums, &S.total);
+}
+
+// ======================================================================================
 // Few long rows with a caller workspace (the decode shape: 16 sequences x 262144 cached
 // positions).  Three launches, no clusters, so every SM takes part however the GPCs are
 // filled:
@@ -1089,17 +1192,6 @@ struct SegFilterSmem {
   uint32_t total, bin, above;
 };
 
-__device__ __forceinline__ int row_visible(const TopkParams& p, long long row) {
-  int lo = 0, hi = p.batch;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) / 2;
-    if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
-  }
-  const int i = (int)(row - p.cu_q[lo]);
-  const int Lq = p.cu_q[lo + 1] - p.cu_q[lo];
-  const int Lk = p.cu_k[lo + 1] - p.cu_k[lo];
-  return min(max(i + Lk - Lq + 1, 0), Lk);
-}
 
 // The sampled bound T of each row, once per row (a sample read by every filter block of
 // the row would hit the same L2 sectors from all of them at once).
@@ -1293,6 +1385,22 @@ static int topk_regs_launch(const dsa::TopkParams& p, long long rows, cudaStream
   return last_launch_status();
 }
 
+// One block per row with the streaming kernel, then the exact kernel for rows it marked.
+static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t stream) {
+  static bool attr_done = false, exact_done = false;
+  if (!attr_done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_stream_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    attr_done = true;
+  }
+  p.only_marked = 0;
+  dsa::topk_stream_kernel<<<(unsigned)rows, dsa::ST_T, 0, stream>>>(p);
+  if (const int st = last_launch_status(); st != DSA_OK) return st;
+  p.only_marked = 1;
+  return launch_cluster(dsa::topk_kernel<1>, p, rows, 1, dsa::TOPK_THREADS, (int)sizeof(dsa::TopkSmem), exact_done,
+                        stream);
+}
+
 // Workspace of the two-launch path for `rows` rows of up to max_vis positions; 0 where
 // that path is not used (many rows, short rows or rows beyond its segment count).
 size_t topk_ws_bytes(long long rows, long long max_vis) {
@@ -1365,7 +1473,7 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
   int C = 1;
   while (C < 8 && (long long)rows * C < 2LL * sms && (long long)max_vis > 16384LL * C) C *= 2;
   switch (C) {
-    case 1: return topk_launch_c<1>(p, rows, stream);
+    case 1: return topk_stream_launch(p, rows, stream);
     case 2: return topk_launch_c<2>(p, rows, stream);
     case 4: return topk_launch_c<4>(p, rows, stream);
     default: return topk_launch_c<8>(p, rows, stream);

@@ -150,6 +150,19 @@ def test_topk_few_long_rows_without_workspace(case):
         assert np.array_equal(a[r], orc.topk_row(sc[r, :n].astype(np.float64), 2048)), r
 
 
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_many_rows_stream_path(ties):
+    # 400 rows of 3000..70000 positions, one block per row: ordered candidate lists built
+    # tile by tile (Gaussian scores); with heavy ties most rows overflow the list and are
+    # finished by the exact kernel
+    vis = [3000 + (r * 167) % 67000 for r in range(400)]
+    sc, cu_q, cu_k = _topk_case(vis, 2048, seed=21 + ties, ties=ties)
+    idx = dsa.topk(torch.from_numpy(sc).cuda(), torch.from_numpy(cu_q).cuda(), torch.from_numpy(cu_k).cuda(),
+                   2048).cpu().numpy()
+    for b in range(0, 400, 23):
+        assert np.array_equal(idx[b], orc.topk_row(sc[b, :vis[b]].astype(np.float64), 2048)), b
+
+
 def test_topk_many_long_rows_cluster_path():
     # 120 rows of ~100K positions: too many rows for one cluster per row with the row in
     # registers, so the sampled-threshold kernel runs with a small cluster per row
