@@ -30,6 +30,9 @@ sys.path.insert(0, ROOT)
 from workloads import generators as gen  # noqa: E402
 
 PREFILL_CHUNK = 8192
+# DRAM bytes (read + write) per causal (t, s) pair of the indexer kernel, from one ncu
+# capture of this kernel on the last 4096 rows of a 32K video prefill
+IDX_DRAM_BYTES_PER_PAIR = (144.2e6 + 450.5e6) / 125831168
 METRIC = "DSA prefill tokens/s at 128K ctx (indexer + top-k + sparse attention)"
 
 
@@ -43,7 +46,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-train", action="store_true")
-    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode"],
+    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode", "train"],
                     help="run one kernel on a small case (for profiler captures) instead of the bench")
     ap.add_argument("--case-len", type=int, default=16384, help="sequence length of the --case workload")
     ap.add_argument("--case-chunk", type=int, default=0,
@@ -236,7 +239,8 @@ def run_prefill(args, rank, world, device, dist):
         "breakdown_ms_per_step": {"indexer": t_idx / args.steps, "topk": t_topk / args.steps,
                                   "sparse_attn": t_attn / args.steps},
         "idx_flops_per_launch": idx_flops / len(chunks), "idx_ms_per_launch": t_idx / n_idx_launch,
-        "launches_per_step": 2 * len(chunks) + 1,
+        # per chunk: indexer, streaming top-k, exact top-k for the rows it marked; then attention
+        "launches_per_step": 3 * len(chunks) + 1,
         "flops_per_step": idx_flops + attn_flops, "idx_flops": idx_flops, "attn_flops": attn_flops,
         "scores_bytes_per_step": pairs * 4,
         "gather_bytes_per_step": sel_pairs * wl.Hkv * wl.d * 2 * 2,
@@ -335,14 +339,19 @@ def run_decode(args, device, dist):
     return {"us_per_step": float(us[3]), "us_per_token": float(us[3]) / B,
             "breakdown_us": {"indexer": float(us[0]), "topk": float(us[1]), "sparse_attn": float(us[2])},
             "idx_bytes": idx_bytes, "attn_bytes": attn_bytes, "steps": steps,
-            "launches_per_step": 4}
+            # indexer; top-k row bound, segment filter, row select; attention, split combine
+            "launches_per_step": 6}
 
 
 def run_case(args):
-    """One kernel, steps+warmup launches, on a small video-layout case (profiling aid)."""
+    """One kernel, steps+warmup launches, on a small video-layout case (profiling aid);
+    `train` runs the training step of the varlen 64K workload instead."""
     import torch
     import lightning_indexer_b200 as dsa
     device = torch.device("cuda", 0)
+    if args.case == "train":
+        print(json.dumps(run_train(args, device)))
+        return
     L = args.case_len
     if args.case == "decode":
         wl = gen.make_decode(16, L, 32, 4, 128, 64, 128, 2048, seed=3, layout="video")
@@ -456,9 +465,9 @@ def main():
     train = None if args.no_train else run_train(args, device)
     cpu = None
     if rank == 0 and not args.no_cpu:
-        v, dt, thr, rows = oracle_rate(wl, 24, seed=7)
+        v, dt, thr, rows = oracle_rate(wl, 320, seed=7)
         cpu = {"value": v, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-               "sample": f"24 random query rows of the 131072-row workload ({dt:.1f} s of CPU work); "
+               "sample": f"320 random query rows of the 131072-row workload ({dt:.1f} s of CPU work); "
                          f"whole-workload time extrapolated as mean row time x 131072"}
     if dist is not None:
         dist.barrier()
@@ -477,7 +486,10 @@ def main():
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (q_idx 2 GiB, Q 1 GiB), no flush"},
         "roofline": {"kernel": "indexer (tcgen05)", "bound": "tensor", "achieved": achieved, "peak": peak_tf,
-                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                     "traffic": IDX_DRAM_BYTES_PER_PAIR * res["idx_flops_per_launch"] / (2 * wl.H_I * wl.d_I),
+                     "traffic_source": "ncu dram bytes read+write of the indexer on the last 4096 rows of a 32K "
+                                       "video prefill (4.73 B per causal pair), scaled by the pairs of a launch",
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"},
         "clocks": res["clocks"],
         "gpu_launches": res["launches_per_step"] * args.steps,

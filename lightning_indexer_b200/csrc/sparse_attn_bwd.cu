@@ -12,8 +12,8 @@
 // One warp owns one (token, KV head) and walks its k selected keys in chunks of 16 with
 // the same gather ring and swap-AB warp MMAs as the forward kernel.  The head sums of dK
 // and dV are MMAs with K = 16 (the 8 heads of the group, zero-padded); their 16 x d
-// results go straight to the fp32 workspace with red.global.add.v2.f32, and a final
-// kernel rounds the workspace to bf16.
+// results go straight to the fp32 workspace with 16-byte reductions (red.global.add.v4.f32,
+// after a lane-pair exchange), and a final kernel rounds the workspace to bf16.
 #include "common.cuh"
 
 namespace dsa {
@@ -42,8 +42,9 @@ struct SABwdParams {
   float* dV_acc;
 };
 
-__device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
-  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 template <int D>
@@ -190,23 +191,32 @@ __global__ void __launch_bounds__(BWD_WARPS * 32) sparse_attn_bwd_kernel(const S
         mma_bf16_16816(dq[mt], a0, a1, a2, a3, b0, b1);
       }
     }
-    // dK rows = scale * dS^T[16 x heads] . Q_g[heads x d];  dV rows = P^T . dO_g
-    float* dk0 = p.dK_acc + ((size_t)(kbase + (v0 ? sA : 0)) * p.Hkv + g) * D + 2 * tig;
-    float* dk1 = p.dK_acc + ((size_t)(kbase + (v1 ? sB : 0)) * p.Hkv + g) * D + 2 * tig;
-    float* dv0 = p.dV_acc + ((size_t)(kbase + (v0 ? sA : 0)) * p.Hkv + g) * D + 2 * tig;
-    float* dv1 = p.dV_acc + ((size_t)(kbase + (v1 ? sB : 0)) * p.Hkv + g) * D + 2 * tig;
+    // dK rows = scale * dS^T[16 x heads] . Q_g[heads x d];  dV rows = P^T . dO_g.
+    // A lane holds columns (2*tig, 2*tig+1) of rows gid and gid+8; lanes tig and tig^1
+    // swap halves so that the even lane owns 4 consecutive columns of row gid and the odd
+    // lane the same 4 columns of row gid+8: one 16-byte reduction each.
+    const bool odd = tig & 1;
+    const bool vmine = odd ? v1 : v0;
+    const int smine = odd ? sB : sA;
+    float* dkr = p.dK_acc + ((size_t)(kbase + (vmine ? smine : 0)) * p.Hkv + g) * D + 4 * (tig >> 1);
+    float* dvr = p.dV_acc + ((size_t)(kbase + (vmine ? smine : 0)) * p.Hkv + g) * D + 4 * (tig >> 1);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       float ck[4] = {0.f, 0.f, 0.f, 0.f}, cv[4] = {0.f, 0.f, 0.f, 0.f};
       mma_bf16_16816(ck, dsA0, dsA1, 0u, 0u, qh[nt], 0u);
       mma_bf16_16816(cv, pA0, pA1, 0u, 0u, oh[nt], 0u);
-      if (v0) {
-        red_add_v2(dk0 + nt * 8, ck[0] * p.scale, ck[1] * p.scale);
-        red_add_v2(dv0 + nt * 8, cv[0], cv[1]);
-      }
-      if (v1) {
-        red_add_v2(dk1 + nt * 8, ck[2] * p.scale, ck[3] * p.scale);
-        red_add_v2(dv1 + nt * 8, cv[2], cv[3]);
+      const float k0 = __shfl_xor_sync(0xffffffffu, odd ? ck[0] : ck[2], 1);
+      const float k1 = __shfl_xor_sync(0xffffffffu, odd ? ck[1] : ck[3], 1);
+      const float w0 = __shfl_xor_sync(0xffffffffu, odd ? cv[0] : cv[2], 1);
+      const float w1 = __shfl_xor_sync(0xffffffffu, odd ? cv[1] : cv[3], 1);
+      if (vmine) {
+        if (odd) {
+          red_add_v4(dkr + nt * 8, k0 * p.scale, k1 * p.scale, ck[2] * p.scale, ck[3] * p.scale);
+          red_add_v4(dvr + nt * 8, w0, w1, cv[2], cv[3]);
+        } else {
+          red_add_v4(dkr + nt * 8, ck[0] * p.scale, ck[1] * p.scale, k0 * p.scale, k1 * p.scale);
+          red_add_v4(dvr + nt * 8, cv[0], cv[1], w0, w1);
+        }
       }
     }
     __syncwarp();

@@ -26,6 +26,7 @@
 //      blocks how many keys > K* and ties come before its segment, so its slots are
 //      (#keys > K* before s) + min(#ties before s, remaining): ascending and
 //      bit-reproducible.  No global atomics are used anywhere.
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -451,6 +452,25 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const TopkParams p) 
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
   exact_row_select<C>(p, S, p.row_begin + blockIdx.x / C);
+}
+
+// The exact selection of the rows a one-block-per-row kernel marked with -2 (p.only_marked
+// set): block b first collects the marked rows of its contiguous share (<= TOPK_THREADS
+// rows, one flag read per thread), then selects them one after the other.
+__global__ void __launch_bounds__(TOPK_THREADS) topk_marked_kernel(const TopkParams p, long long rows) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
+  __shared__ int marked[TOPK_THREADS];
+  __shared__ int nmarked;
+  const long long per = (rows + gridDim.x - 1) / gridDim.x;
+  const long long r0 = blockIdx.x * per, r1 = min(rows, r0 + per);
+  if (threadIdx.x == 0) nmarked = 0;
+  __syncthreads();
+  if (r0 + threadIdx.x < r1 && __ldg(p.indices + (r0 + threadIdx.x) * p.k) == -2)
+    marked[atomicAdd(&nmarked, 1)] = (int)threadIdx.x;
+  __syncthreads();
+  const int n = nmarked;
+  for (int j = 0; j < n; ++j) exact_row_select<1>(p, S, p.row_begin + r0 + marked[j]);
 }
 
 // ======================================================================================
@@ -1397,8 +1417,15 @@ static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t st
   dsa::topk_stream_kernel<<<(unsigned)rows, dsa::ST_T, 0, stream>>>(p);
   if (const int st = last_launch_status(); st != DSA_OK) return st;
   p.only_marked = 1;
-  return launch_cluster(dsa::topk_kernel<1>, p, rows, 1, dsa::TOPK_THREADS, (int)sizeof(dsa::TopkSmem), exact_done,
-                        stream);
+  if (!exact_done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_marked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)sizeof(dsa::TopkSmem));
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    exact_done = true;
+  }
+  const long long grid = std::max((rows + dsa::TOPK_THREADS - 1) / dsa::TOPK_THREADS, std::min(rows, (long long)sm_count()));
+  dsa::topk_marked_kernel<<<(unsigned)grid, dsa::TOPK_THREADS, sizeof(dsa::TopkSmem), stream>>>(p, rows);
+  return last_launch_status();
 }
 
 // Workspace of the two-launch path for `rows` rows of up to max_vis positions; 0 where
