@@ -356,14 +356,28 @@ def run_case(args):
     if args.case == "decode":
         wl = gen.make_decode(16, L, 32, 4, 128, 64, 128, 2048, seed=3, layout="video")
     else:
-        wl = gen.make_prefill([L], 32, 4, 128, 64, 128, 2048, seed=2, layout="video")
+        wl = gen.make_prefill([L], 32, 4, 128, 64, 128, 2048, seed=2, layout="video", max_frames=480)
     t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
     cu_q = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
     cu_k = torch.from_numpy(wl.cu_seqlens_k.astype(np.int32)).to(device)
     Tq, Lk = wl.Tq, int(wl.seqlens_k.max())
     r0 = Tq - args.case_chunk if (args.case == "indexer" and args.case_chunk > 0) else 0
-    scores = dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, r0, Tq)
-    idx = dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq)
+    if args.case == "sparse_attn":
+        # the selected sets of every row, from the library's indexer and top-k in chunks of
+        # rows (bounded score scratch); the score buffer is freed before the timed launches
+        mq = int(wl.seqlens_q.max())
+        idx = torch.empty((Tq, wl.topk), dtype=torch.int32, device=device)
+        sc = torch.empty((min(PREFILL_CHUNK, Tq), (Lk + 3) // 4 * 4), dtype=torch.float32, device=device)
+        for c0 in range(0, Tq, PREFILL_CHUNK):
+            c1 = min(Tq, c0 + PREFILL_CHUNK)
+            dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, mq, Lk, c0, c1, scores=sc[: c1 - c0])
+            dsa.topk(sc[: c1 - c0], cu_q, cu_k, wl.topk, c0, c1, indices=idx[c0:c1])
+        torch.cuda.synchronize()
+        del sc, t["q_idx"]
+        torch.cuda.empty_cache()
+    else:
+        scores = dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, r0, Tq)
+        idx = dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for it in range(args.warmup + args.steps):
