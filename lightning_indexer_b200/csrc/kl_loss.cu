@@ -19,8 +19,9 @@
 //   3. row_lse_kernel     log-sum-exp of each I row
 //   4. kl_target_kernel   p from recomputed dense logits, kl[t], g in place [warp MMA]
 //   5. idx_bwd_row_kernel x recomputed per row; dw, dq_idx (row-stationary) [warp MMA]
-//   6. idx_bwd_col_kernel x recomputed per key tile; dk_idx (key-stationary, fp32
-//                         accumulator owned by one CTA per key tile: no atomics)
+//   6. idx_bwd_col_kernel x recomputed per key tile; dk_idx (key-stationary: one CTA per
+//                         key tile and block of 1024 rows owns a partial, then the
+//                         partials are added in a fixed order: no atomics, deterministic)
 //   then dk_idx -> bf16 and loss = mean(kl) (one block, fixed order).
 #include "common.cuh"
 
@@ -423,14 +424,26 @@ __global__ void __launch_bounds__(H_I / 16 * 32)
 }
 
 // ------------------------------------------------------------------ 6. key-stationary
-// One block per (sequence, tile of 128 keys), 8 warps of 16 keys.  Streams the chunk's
-// rows that see the tile; per row t:
+// One block per (sequence, tile of 128 keys, block of KL_COL_ROWS rows of the chunk), 8
+// warps of 16 keys.  Streams its rows that see the tile; per row t:
 //   x^T[16 keys x H_I] = k_w . q_idx[t]^T;  G^T = g w [x > 0];  dk[16 x d_I] += G^T . q_idx[t]
+// and stores its partial dk to dk_part[row block] (plain stores: every (row block, key)
+// entry has one writer); dk_reduce_kernel then adds the row blocks in a fixed order.
+constexpr int KL_COL_ROWS = 1024;
+
+// rows [qlo, qhi) of the chunk [row_begin, row_end) that see key tile `tile` of sequence b
+__device__ __forceinline__ void col_rows(const int* cu_q, const int* cu_k, int b, int tile, long long row_begin,
+                                         long long row_end, long long& qlo, long long& qhi) {
+  const int Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
+  qlo = max((long long)cu_q[b] + max(tile * 128 - (Lk - Lq), 0), row_begin);
+  qhi = min((long long)cu_q[b + 1], row_end);
+}
+
 template <int H_I, int D_I>
 __global__ void __launch_bounds__(256)
     idx_bwd_col_kernel(const uint16_t* q_idx, const uint16_t* k_idx, const uint16_t* w, const int* cu_q,
                        const int* cu_k, int batch, long long row_begin, long long row_end, const float* gbuf,
-                       long long ld, int tiles_per_seq, float* dk_acc) {
+                       long long ld, int tiles_per_seq, int row_blocks, float* dk_part, long long part_stride) {
   constexpr int KT = 128;
   constexpr int SEGS = D_I / 8;
   constexpr int QT = H_I * D_I * 2;  // q_idx[t] tile bytes
@@ -444,17 +457,21 @@ __global__ void __launch_bounds__(256)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int gid = lane / 4, tig = lane % 4;
   const uint32_t sbase = smem_u32(smem);
-  const int b = blockIdx.x / tiles_per_seq;
-  const int tile = blockIdx.x % tiles_per_seq;
+  const int rb = blockIdx.x % row_blocks;
+  const int tile = (blockIdx.x / row_blocks) % tiles_per_seq;
+  const int b = blockIdx.x / (row_blocks * tiles_per_seq);
   if (b >= batch) return;
   const int Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
   const int s0 = tile * KT;
   if (s0 >= Lk) return;
   const int kbase = cu_k[b];
-  // rows of this sequence in [row_begin, row_end) that see key s0: i >= s0 - (Lk - Lq)
-  const long long qlo = max((long long)cu_q[b] + max(s0 - (Lk - Lq), 0), row_begin);
-  const long long qhi = min((long long)cu_q[b + 1], row_end);
+  // this block's rows: block rb of the rows of [row_begin, row_end) that see key s0
+  long long qlo, qhi;
+  col_rows(cu_q, cu_k, b, tile, row_begin, row_end, qlo, qhi);
+  qlo += (long long)rb * KL_COL_ROWS;
+  qhi = min(qhi, qlo + KL_COL_ROWS);
   if (qlo >= qhi) return;
+  float* dk_acc = dk_part + rb * part_stride;
   // A fragments of this warp's 16 keys of k_idx (zero rows past Lk)
   uint32_t ka[KS][4];
   {
@@ -533,17 +550,40 @@ __global__ void __launch_bounds__(256)
   const int kA = s0 + warp * 16 + gid, kB = kA + 8;
 #pragma unroll
   for (int nd = 0; nd < NTD; ++nd) {
-    if (kA < Lk) {
-      float* d0 = dk_acc + (size_t)(kbase + kA) * D_I + nd * 8 + 2 * tig;
-      d0[0] += dk[nd][0];
-      d0[1] += dk[nd][1];
-    }
-    if (kB < Lk) {
-      float* d1 = dk_acc + (size_t)(kbase + kB) * D_I + nd * 8 + 2 * tig;
-      d1[0] += dk[nd][2];
-      d1[1] += dk[nd][3];
-    }
+    if (kA < Lk)
+      *reinterpret_cast<float2*>(dk_acc + (size_t)(kbase + kA) * D_I + nd * 8 + 2 * tig) = make_float2(dk[nd][0], dk[nd][1]);
+    if (kB < Lk)
+      *reinterpret_cast<float2*>(dk_acc + (size_t)(kbase + kB) * D_I + nd * 8 + 2 * tig) = make_float2(dk[nd][2], dk[nd][3]);
   }
+}
+
+// dk_acc[s] += sum over the row blocks that exist for key s's tile (in block order) of
+// dk_part[rb][s]: one thread per 4 consecutive values of one key.
+template <int D_I>
+__global__ void dk_reduce_kernel(const float* dk_part, long long part_stride, const int* cu_q, const int* cu_k,
+                                 int batch, long long row_begin, long long row_end, long long Tk, float* dk_acc) {
+  const long long e = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e >= Tk * D_I) return;
+  const long long key = e / D_I;
+  int lo = 0, hi = batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)cu_k[mid] <= key) lo = mid; else hi = mid;
+  }
+  const int tile = (int)((key - cu_k[lo]) / 128);
+  long long qlo, qhi;
+  col_rows(cu_q, cu_k, lo, tile, row_begin, row_end, qlo, qhi);
+  if (qlo >= qhi) return;
+  const int nrb = (int)((qhi - qlo + KL_COL_ROWS - 1) / KL_COL_ROWS);
+  float4 acc = *reinterpret_cast<const float4*>(dk_acc + e);
+  for (int rb = 0; rb < nrb; ++rb) {
+    const float4 v = *reinterpret_cast<const float4*>(dk_part + rb * part_stride + e);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  *reinterpret_cast<float4*>(dk_acc + e) = acc;
 }
 
 // loss = mean of kl over all rows (one block, fixed summation order)
@@ -575,6 +615,7 @@ int f32_to_bf16_launch(const float* src, void* dst, long long n, cudaStream_t st
 struct KLWorkspace {
   float* lse_att;  // [T, Hq]
   float* dk_acc;   // [Tk, d_I]
+  float* dk_part;  // [ceil(chunk_rows / KL_COL_ROWS), Tk, d_I] per-row-block partials of dk
   float* lseI;     // [chunk_rows]
   float* scores;   // [chunk_rows, ld]
   size_t total;
@@ -592,6 +633,8 @@ KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_s
   off += r256((size_t)T * Hq * 4);
   w.dk_acc = reinterpret_cast<float*>(p + off);
   off += r256((size_t)Tk * d_I * 4);
+  w.dk_part = reinterpret_cast<float*>(p + off);
+  off += r256((size_t)((chunk_rows + dsa::KL_COL_ROWS - 1) / dsa::KL_COL_ROWS) * Tk * d_I * 4);
   w.lseI = reinterpret_cast<float*>(p + off);
   off += r256((size_t)chunk_rows * 4);
   w.scores = reinterpret_cast<float*>(p + off);
@@ -606,8 +649,9 @@ size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, i
 
 template <int H_I, int D_I>
 static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
-                               int batch, long long r0, long long r1, const float* g, long long ld,
-                               int max_seqlen_k, void* dq, void* dw, float* dk_acc, cudaStream_t s) {
+                               int batch, long long r0, long long r1, long long Tk, const float* g, long long ld,
+                               int max_seqlen_k, void* dq, void* dw, float* dk_acc, float* dk_part,
+                               cudaStream_t s) {
   {
     auto kern = dsa::idx_bwd_row_kernel<H_I, D_I>;
     const int smem = 2 * 64 * D_I * 2;
@@ -630,10 +674,18 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
       done = true;
     }
     const int tiles = (max_seqlen_k + 127) / 128;
-    kern<<<(unsigned)((long long)batch * tiles), 256, smem, s>>>(
+    const int row_blocks = (int)((r1 - r0 + dsa::KL_COL_ROWS - 1) / dsa::KL_COL_ROWS);
+    const long long part_stride = Tk * D_I;
+    kern<<<(unsigned)((long long)batch * tiles * row_blocks), 256, smem, s>>>(
         static_cast<const uint16_t*>(q_idx), static_cast<const uint16_t*>(k_idx), static_cast<const uint16_t*>(w),
-        cu_q, cu_k, batch, r0, r1, g, ld, tiles, dk_acc);
+        cu_q, cu_k, batch, r0, r1, g, ld, tiles, row_blocks, dk_part, part_stride);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
+    const long long quads = Tk * D_I / 4;
+    if (quads > 0) {
+      dsa::dk_reduce_kernel<D_I><<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(dk_part, part_stride, cu_q, cu_k, batch,
+                                                                                 r0, r1, Tk, dk_acc);
+      if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
+    }
   }
   return DSA_OK;
 }
@@ -716,8 +768,8 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     }
 #define DSA_KLB(HI, DI)                                                                                   \
   if (H_I == HI && d_I == DI) {                                                                          \
-    st = kl_backward_kernels<HI, DI>(q_idx, k_idx, w, cu_q, cu_k, batch, r0, r1, W.scores, ld, max_seqlen_k, \
-                                     dq, dw, W.dk_acc, s);                                               \
+    st = kl_backward_kernels<HI, DI>(q_idx, k_idx, w, cu_q, cu_k, batch, r0, r1, Tk, W.scores, ld, max_seqlen_k, \
+                                     dq, dw, W.dk_acc, W.dk_part, s);                                    \
     if (st != DSA_OK) return st;                                                                         \
   } else
     DSA_KLB(64, 128) DSA_KLB(32, 128) DSA_KLB(16, 128) { return DSA_ERR_UNSUPPORTED; }
