@@ -19,8 +19,8 @@
 namespace dsa {
 
 // warps per CTA, chunks in flight per warp (the one in use included), keys per chunk
-constexpr int BWD_WARPS = 8;
-constexpr int BWD_STAGES = 3;
+constexpr int BWD_WARPS = 4;
+constexpr int BWD_STAGES = 2;
 constexpr int BWD_CHUNK = 16;
 
 struct SABwdParams {
@@ -48,7 +48,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 }
 
 template <int D>
-__global__ void __launch_bounds__(BWD_WARPS * 32) sparse_attn_bwd_kernel(const SABwdParams p) {
+__global__ void __launch_bounds__(BWD_WARPS * 32, 3) sparse_attn_bwd_kernel(const SABwdParams p) {
   constexpr int SEGS = D / 8;
   constexpr int TILE_BYTES = BWD_CHUNK * D * 2;
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;
@@ -309,6 +309,10 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
       if (!done) {
         if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem); e_ != cudaSuccess) return cuda_fail(e_);
+        // three CTAs per SM need the largest shared-memory carveout
+        if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<128>,
+                                                        cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            e_ != cudaSuccess) return cuda_fail(e_);
         done = true;
       }
       dsa::sparse_attn_bwd_kernel<128><<<(unsigned)blocks, dsa::BWD_WARPS * 32, smem, stream>>>(p);
@@ -317,6 +321,10 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
       if (!done) {
         if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem); e_ != cudaSuccess) return cuda_fail(e_);
+        // three CTAs per SM need the largest shared-memory carveout
+        if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<64>,
+                                                        cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            e_ != cudaSuccess) return cuda_fail(e_);
         done = true;
       }
       dsa::sparse_attn_bwd_kernel<64><<<(unsigned)blocks, dsa::BWD_WARPS * 32, smem, stream>>>(p);
