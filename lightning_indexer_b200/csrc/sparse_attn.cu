@@ -51,13 +51,15 @@ struct SAParams {
   float* part_ml; // [rows, nsplit, Hq, 4]: max (log2 domain), exact sum, sum of bf16-rounded weights
 };
 
-constexpr int SA_WARPS = 4;   // warps per CTA (several CTAs per SM)
+// 4-warp CTAs with 2 stages per warp: 3 CTAs, 12 warps per SM.  (Decode launches only a
+// thousand warps; 1-warp CTAs with 4 stages each, all resident at once, measured slower.)
+constexpr int SA_WARPS = 4;   // warps per CTA
 constexpr int SA_STAGES = 2;  // chunks in flight per warp, the one in use included
 constexpr int SA_CHUNK = 16;
 
-template <int D>
+template <int D, int STAGES>
 constexpr int sa_smem_bytes(int warps) {
-  return warps * SA_STAGES * 2 * SA_CHUNK * D * 2;
+  return warps * STAGES * 2 * SA_CHUNK * D * 2;
 }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -95,7 +97,7 @@ __device__ __forceinline__ uint32_t tile_off(int row, int seg) {
   return (uint32_t)(row * (D * 2) + ((seg ^ (row & 7)) << 4));
 }
 
-template <int D>
+template <int D, int SA_STAGES, int SA_WARPS>
 __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAParams p) {
   constexpr int SEGS = D / 8;                   // 16-byte segments per row
   constexpr int TILE_BYTES = SA_CHUNK * D * 2;  // one K or V chunk
@@ -369,27 +371,30 @@ __global__ void decode_combine_kernel(const float* part_o, const float* part_ml,
 
 namespace dsa_host {
 
-template <int D>
+template <int D, int STAGES, int WARPS>
 static int sa_launch_d(const dsa::SAParams& p, long long tasks, cudaStream_t stream) {
-  const long long blocks = (tasks + dsa::SA_WARPS - 1) / dsa::SA_WARPS;
-  const int smem = dsa::sa_smem_bytes<D>(dsa::SA_WARPS);
+  const long long blocks = (tasks + WARPS - 1) / WARPS;
+  const int smem = dsa::sa_smem_bytes<D, STAGES>(WARPS);
   static bool done = false;
   if (!done) {
-    cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D, STAGES, WARPS>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     // several CTAs per SM need the largest shared-memory carveout
     if (e_ == cudaSuccess)
-      e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D, STAGES, WARPS>,
+                                cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e_ != cudaSuccess) return cuda_fail(e_);
     done = true;
   }
-  dsa::sparse_attn_kernel<D><<<(unsigned)blocks, dsa::SA_WARPS * 32, smem, stream>>>(p);
+  dsa::sparse_attn_kernel<D, STAGES, WARPS><<<(unsigned)blocks, WARPS * 32, smem, stream>>>(p);
   return last_launch_status();
 }
 
 static int sa_launch_common(dsa::SAParams& p, int d, cudaStream_t stream) {
   const long long tasks = p.rows * p.Hkv * p.nsplit;
   if (tasks <= 0) return DSA_OK;
-  return d == 128 ? sa_launch_d<128>(p, tasks, stream) : sa_launch_d<64>(p, tasks, stream);
+  return d == 128 ? sa_launch_d<128, dsa::SA_STAGES, dsa::SA_WARPS>(p, tasks, stream)
+                  : sa_launch_d<64, dsa::SA_STAGES, dsa::SA_WARPS>(p, tasks, stream);
 }
 
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
