@@ -1,0 +1,415 @@
+// Key-stationary indexer backward of the KL loss on tcgen05 tensor cores (sm_100a).
+//
+// Source: Keye-VL-2.0 report summary (mqxn.cn/news/1966), section 1: in the dense warm-up
+// only the indexer is trained, by the KL divergence to the full attention distribution.
+// With g[t,s] = dloss/dI[t,s] (from the KL target pass) and x[t,j,s] = q_idx[t,j].k_idx[s],
+//   dk_idx[s] = sum_t sum_j g[t,s] w[t,j] [x[t,j,s] > 0] q_idx[t,j,:].
+//
+// One work item is (sequence, tile of 128 keys, block of up to 1024 query rows of the row
+// chunk that see the tile); its partial dk (128 keys x d_I, fp32) goes to the row block's
+// slice of the partial workspace, and a second kernel adds the row blocks in a fixed order.
+// Per block of 2 query rows (N = 2 x 64 heads = 128 columns), two chained MMAs:
+//   MMA1  X[128 keys x 128 (t,j)] = K_tile . Q_blk^T          (TMEM, two buffers)
+//   epilogue  G = g w [X > 0] -> bf16, written to shared memory in the 128-byte swizzled
+//             K-major layout the tensor core reads (row = key, 16-byte chunk c of a row
+//             at chunk c ^ (row % 8))
+//   MMA2  dk[128 keys x 128 d] += G . (Q_blk^T)^T             (TMEM accumulator)
+// Every operand is K-major: MMA2's B is the same query block transposed, which TMA reads
+// from a transposed copy of q_idx ([d_I, T*H_I], written once per loss call).
+// MMA1 of the next block is issued before MMA2 of this one, so the tensor pipe computes X
+// while the epilogue turns the previous X into G.  Warp roles: warp 0 TMA producer, warp 1
+// MMA issuer and TMEM owner, warps 2-9 epilogue (one TMEM lane, i.e. one key, per thread;
+// two warps per lane quarter, one per query row of the block).
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace dsa {
+
+struct KlDkParams {
+  const uint16_t* w;  // [T, 64] bf16
+  long long total_q;
+  const int* cu_q;
+  const int* cu_k;
+  int batch;
+  long long row_begin, row_end;  // the row chunk
+  const float* g;                // [row_end - row_begin, ld] fp32 dloss/dI
+  long long ld;
+  int tiles_per_seq, row_blocks, rows_per_block;
+  long long n_items;
+  float* dk_part;  // [row_blocks][Tk][128] fp32
+  long long part_stride;
+};
+
+struct KlDkItem {
+  int b, tile, rb, kbase, Lq, Lk;
+  long long qlo, qhi;  // the item's query rows
+  int nb;              // blocks of 2 rows
+};
+
+__device__ __forceinline__ bool kl_dk_item(long long item, const KlDkParams& p, KlDkItem& it) {
+  const int rb = (int)(item % p.row_blocks);
+  const int tile = (int)((item / p.row_blocks) % p.tiles_per_seq);
+  const int b = (int)(item / ((long long)p.row_blocks * p.tiles_per_seq));
+  if (b >= p.batch) return false;
+  const int Lq = p.cu_q[b + 1] - p.cu_q[b], Lk = p.cu_k[b + 1] - p.cu_k[b];
+  if (tile * 128 >= Lk) return false;
+  long long qlo = max((long long)p.cu_q[b] + max(tile * 128 - (Lk - Lq), 0), p.row_begin);
+  long long qhi = min((long long)p.cu_q[b + 1], p.row_end);
+  qlo += (long long)rb * p.rows_per_block;
+  qhi = min(qhi, qlo + p.rows_per_block);
+  if (qlo >= qhi) return false;
+  it.b = b;
+  it.tile = tile;
+  it.rb = rb;
+  it.kbase = p.cu_k[b];
+  it.Lq = Lq;
+  it.Lk = Lk;
+  it.qlo = qlo;
+  it.qhi = qhi;
+  it.nb = (int)((qhi - qlo + 1) / 2);
+  return true;
+}
+
+struct KlDkCfg {
+  static constexpr int H_I = 64, D_I = 128, NTOK = 2, N = NTOK * H_I;  // 128 columns
+  static constexpr int TILE_BYTES = 128 * 128 * 2;                      // any 128 x 128 bf16 operand
+  static constexpr int PANEL_BYTES = 128 * 128;                         // 128 rows x 128 B
+  static constexpr int OFF_A = 0;                                       // key tile
+  static constexpr int OFF_Q = OFF_A + TILE_BYTES;                      // 2 stages x (Q_blk, Q_blk^T)
+  static constexpr int STAGE_STRIDE = 2 * TILE_BYTES;
+  static constexpr int OFF_G = OFF_Q + 2 * STAGE_STRIDE;                // 2 G buffers
+  static constexpr int OFF_W = OFF_G + 2 * TILE_BYTES;                  // 2 stages x w of the block's rows
+  static constexpr int W_BYTES = 2 * 64 * 2;
+  static constexpr int OFF_BAR = OFF_W + 2 * W_BYTES;
+  static constexpr int NUM_BARS = 2 + 4 + 4 + 4 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter: one per block row (64 columns)
+  static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  static constexpr int TMEM_COLS = 512;  // X buffers [0,128) [128,256), dk [256,384)
+  static constexpr uint32_t IDESC = idesc_bf16_f32(128, 128);
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+__global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
+    kl_dk_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_qt, const KlDkParams p) {
+  using C = KlDkCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sG = smem + C::OFF_G;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = bars + 1;
+  uint64_t* q_full = bars + 2;   // [2]
+  uint64_t* q_empty = bars + 4;  // [2]
+  uint64_t* x_full = bars + 6;   // [2]
+  uint64_t* x_empty = bars + 8;  // [2]
+  uint64_t* g_full = bars + 10;   // [2]
+  uint64_t* g_empty = bars + 12;  // [2]
+  uint64_t* dk_full = bars + 14;
+  uint64_t* dk_empty = bars + 15;
+  uint64_t* mma_done = bars + 16;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], C::EPI_WARPS);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&g_full[i], C::EPI_WARPS);
+      mbar_init(&g_empty[i], 1);
+    }
+    mbar_init(dk_full, 1);
+    mbar_init(dk_empty, C::EPI_WARPS);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_qt);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      long long n = 0;  // blocks loaded so far (stage n % 2)
+      long long m = 0;  // non-empty items so far
+      bool ok = true;
+      for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        KlDkItem it;
+        if (!kl_dk_item(item, p, it)) continue;
+        if (!(ok = mbar_wait(a_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 40))) break;
+        mbar_arrive_expect_tx(a_full, C::TILE_BYTES);
+        for (int pn = 0; pn < 2; ++pn)
+          tma_load_2d(sA + pn * C::PANEL_BYTES, &tmap_k, a_full, pn * 64, it.kbase + it.tile * 128);
+        ++m;
+        for (int i = 0; i < it.nb; ++i, ++n) {
+          const int st = (int)(n & 1);
+          if (!(ok = mbar_wait(&q_empty[st], (uint32_t)((n >> 1) & 1) ^ 1u, abort_flag, 41))) break;
+          const long long t0 = it.qlo + 2 * i;
+          // head weights of the block's rows that exist in the tensor (the second may not)
+          const uint32_t wbytes = (uint32_t)(min(2LL, p.total_q - t0) * C::H_I * 2);
+          mbar_arrive_expect_tx(&q_full[st], 2 * C::TILE_BYTES + wbytes);
+          uint8_t* sq = sQ + st * C::STAGE_STRIDE;
+          const int col = (int)(t0 * C::H_I);  // first (t, j) row of the block
+          for (int pn = 0; pn < 2; ++pn) {
+            tma_load_2d(sq + pn * C::PANEL_BYTES, &tmap_q, &q_full[st], pn * 64, col);
+            tma_load_2d(sq + C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_qt, &q_full[st], col + pn * 64, 0);
+          }
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_u32(smem + C::OFF_W + st * C::W_BYTES)),
+              "l"(p.w + t0 * C::H_I), "r"(wbytes), "r"(smem_u32(&q_full[st]))
+              : "memory");
+        }
+      }
+      if (!ok) {
+        // drain: the loads this thread issued land before the CTA can exit
+        const uint64_t t0 = globaltimer_ns();
+        for (int i = 0; i < 2; ++i)
+          while (!mbar_try_wait(smem_u32(&q_full[i]), (uint32_t)(((n - (n & 1) + i) >> 1) & 1)) &&
+                 globaltimer_ns() - t0 < 200000000ull) {
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      long long n = 0;  // blocks whose MMA1 was issued
+      long long m = 0;  // non-empty items
+      long long gcount = 0;
+      bool ok = true;
+      const uint32_t a_base = smem_u32(sA);
+      const uint32_t g_base = smem_u32(sG);
+      const uint32_t dk_tmem = tmem_base + 256;
+      auto mma1 = [&](long long blk) -> bool {
+        const int st = (int)(blk & 1);
+        if (!mbar_wait(&q_full[st], (uint32_t)((blk >> 1) & 1), abort_flag, 42)) return false;
+        if (!mbar_wait(&x_empty[st], (uint32_t)((blk >> 1) & 1) ^ 1u, abort_flag, 43)) return false;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(sQ + st * C::STAGE_STRIDE);
+        const uint32_t d_tmem = tmem_base + st * 128;
+#pragma unroll
+        for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(d_tmem, smem_desc_kmajor(a_base + pn * C::PANEL_BYTES + kk * 32, 128),
+                      smem_desc_kmajor(q_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC, (pn | kk) != 0);
+        umma_commit(&x_full[st]);
+        return true;
+      };
+      for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        KlDkItem it;
+        if (!kl_dk_item(item, p, it)) continue;
+        if (!(ok = mbar_wait(a_full, (uint32_t)(m & 1), abort_flag, 44))) break;
+        tc_fence_after();
+        const long long n0 = n;
+        if (!(ok = mma1(n))) break;
+        ++n;
+        for (int i = 0; i < it.nb && ok; ++i) {
+          if (i + 1 < it.nb) {
+            if (!(ok = mma1(n))) break;
+            ++n;
+          }
+          if (i + 1 == it.nb) umma_commit(a_empty);  // the key tile is free once these MMAs finish
+          const int gb = (int)(gcount & 1);
+          if (!(ok = mbar_wait(&g_full[gb], (uint32_t)((gcount >> 1) & 1), abort_flag, 45))) break;
+          if (i == 0 && !(ok = mbar_wait(dk_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 46))) break;
+          tc_fence_after();
+          const long long blk = n0 + i;
+          const uint32_t qt_base = smem_u32(sQ + (int)(blk & 1) * C::STAGE_STRIDE + C::TILE_BYTES);
+#pragma unroll
+          for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(dk_tmem, smem_desc_kmajor(g_base + gb * C::TILE_BYTES + pn * C::PANEL_BYTES + kk * 32, 128),
+                        smem_desc_kmajor(qt_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC,
+                        (i | pn | kk) != 0);
+          umma_commit(&g_empty[gb]);
+          umma_commit(&q_empty[(int)(blk & 1)]);
+          ++gcount;
+        }
+        if (!ok) break;
+        umma_commit(dk_full);
+        ++m;
+      }
+      umma_commit(mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (8 warps)
+    const int lane_grp = warp % 4;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) / 4;           // block row (and column half) of this warp
+    const int r = lane_grp * 32 + lane;        // key row of this thread within the tile
+    const uint32_t lane_off = (uint32_t)(lane_grp * 32) << 16;
+    const uint32_t g_row0 = smem_u32(sG) + half * C::PANEL_BYTES + r * 128;
+    long long n = 0, m = 0, gcount = 0;
+    bool ok = true;
+    for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      KlDkItem it;
+      if (!kl_dk_item(item, p, it)) continue;
+      const int s = it.tile * 128 + r;  // this thread's key (sequence-local)
+      const int dvis = it.Lk - it.Lq + 1;
+      for (int i = 0; i < it.nb; ++i, ++n) {
+        const long long t = it.qlo + 2 * i + half;  // this warp's query row
+        const int vis = min(max((int)(t - p.cu_q[it.b]) + dvis, 0), it.Lk);
+        const bool tv = t < it.qhi;  // else its G columns are 0
+        const float gv = (tv && s < vis) ? p.g[(t - p.row_begin) * p.ld + s] : 0.f;
+        const int st = (int)(n & 1);
+        // the block's head weights arrive with its query tiles: observe that phase here too
+        // (the stage cannot be refilled before this block's G is written, so the phase seen
+        // is this block's)
+        if (!(ok = mbar_wait(&q_full[st], (uint32_t)((n >> 1) & 1), abort_flag, 50))) break;
+        const uint16_t* sW = reinterpret_cast<const uint16_t*>(smem + C::OFF_W + st * C::W_BYTES) + half * C::H_I;
+        if (!(ok = mbar_wait(&x_full[st], (uint32_t)((n >> 1) & 1), abort_flag, 47))) break;
+        tc_fence_after();
+        float x[64];
+        tmem_ld_x32_sync(tmem_base + lane_off + st * 128 + half * 64, x);
+        tmem_ld_x32_sync(tmem_base + lane_off + st * 128 + half * 64 + 32, x + 32);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&x_empty[st]);
+        // G buffer gb may be overwritten once the MMA2 that read it two blocks ago is done
+        const int gb = (int)(gcount & 1);
+        if (!(ok = mbar_wait(&g_empty[gb], (uint32_t)((gcount >> 1) & 1) ^ 1u, abort_flag, 48))) break;
+        const uint32_t g_row = g_row0 + gb * C::TILE_BYTES;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of this row's panel: columns 8q .. 8q+7
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = q * 8 + 2 * e;
+            const float v0 = (tv && x[c] > 0.f) ? gv * bf16_bits_to_f32(sW[c]) : 0.f;
+            const float v1 = (tv && x[c + 1] > 0.f) ? gv * bf16_bits_to_f32(sW[c + 1]) : 0.f;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(g_row + ((q ^ (r & 7)) * 16)),
+                       "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+        }
+        fence_proxy_async_shared();  // the tensor core reads G through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&g_full[gb]);
+        ++gcount;
+      }
+      if (!ok) break;
+      // the item's dk: one key row per thread, this warp's 64 of its 128 fp32 values
+      if (!(ok = mbar_wait(dk_full, (uint32_t)(m & 1), abort_flag, 49))) break;
+      tc_fence_after();
+      float* dst = p.dk_part + it.rb * p.part_stride + (size_t)(it.kbase + s) * C::D_I + half * 64;
+#pragma unroll 1
+      for (int c = 0; c < 64; c += 32) {
+        float v[32];
+        tmem_ld_x32_sync(tmem_base + lane_off + 256 + half * 64 + c, v);
+        if (s < it.Lk) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dk_empty);
+      ++m;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// q_idx [rows, 128] -> q_idx^T [128, rows] (bf16), 32 x 32 tiles through shared memory
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, long long rows) {
+  __shared__ uint16_t t[32][33];
+  const long long r0 = (long long)blockIdx.x * 32;
+  const int c0 = blockIdx.y * 32;
+  for (int y = threadIdx.y; y < 32; y += blockDim.y)
+    if (r0 + y < rows) t[y][threadIdx.x] = src[(r0 + y) * 128 + c0 + threadIdx.x];
+  __syncthreads();
+  for (int y = threadIdx.y; y < 32; y += blockDim.y)
+    if (r0 + threadIdx.x < rows) dst[(long long)(c0 + y) * rows + r0 + threadIdx.x] = t[threadIdx.x][y];
+}
+
+}  // namespace dsa
+
+namespace dsa_host {
+
+int kl_transpose_q_launch(const void* q_idx, void* q_t, long long rows, cudaStream_t s) {
+  if (rows <= 0) return DSA_OK;
+  dsa::transpose_bf16_kernel<<<dim3((unsigned)((rows + 31) / 32), 4), dim3(32, 8), 0, s>>>(
+      static_cast<const uint16_t*>(q_idx), static_cast<uint16_t*>(q_t), rows);
+  return last_launch_status();
+}
+
+// dk partials of the row chunk [r0, r1) for H_I = 64, d_I = 128 (see the file comment);
+// q_t is q_idx transposed ([128, total_q * 64]).
+int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const void* w, const int* cu_q,
+                    const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
+                    long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
+                    long long part_stride, cudaStream_t s) {
+  using C = dsa::KlDkCfg;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_dk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    C::SMEM_BYTES);
+        e_ != cudaSuccess)
+      return cuda_fail(e_);
+    attr_done = true;
+  }
+  CUtensorMap tk, tq, tqt;
+  int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)total_k, 128, 256, 128, 64, 128);
+  if (st != DSA_OK) return st;
+  st = make_tmap_bf16_2d(&tq, q_idx, (uint64_t)total_q * 64, 128, 256, 128, 64, 128);
+  if (st != DSA_OK) return st;
+  st = make_tmap_bf16_2d(&tqt, q_t, 128, (uint64_t)total_q * 64, (uint64_t)total_q * 64 * 2, 128, 64, 128);
+  if (st != DSA_OK) return st;
+  dsa::KlDkParams p;
+  p.w = static_cast<const uint16_t*>(w);
+  p.total_q = total_q;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.row_begin = r0;
+  p.row_end = r1;
+  p.g = g;
+  p.ld = ld;
+  p.tiles_per_seq = (max_seqlen_k + 127) / 128;
+  p.rows_per_block = rows_per_block;
+  p.row_blocks = (int)((r1 - r0 + rows_per_block - 1) / rows_per_block);
+  p.n_items = (long long)batch * p.tiles_per_seq * p.row_blocks;
+  p.dk_part = dk_part;
+  p.part_stride = part_stride;
+  const long long grid = std::min<long long>(p.n_items, (long long)sm_count());
+  if (grid <= 0) return DSA_OK;
+  dsa::kl_dk_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, tqt, p);
+  return last_launch_status();
+}
+
+}  // namespace dsa_host

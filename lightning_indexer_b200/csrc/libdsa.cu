@@ -6,5 +6,6 @@
 #include "topk.cu"
 #include "sparse_attn.cu"
 #include "sparse_attn_bwd.cu"
+#include "kl_bwd_tc.cu"
 #include "kl_loss.cu"
 #include "decode_noalloc.cu"
