@@ -307,14 +307,14 @@ def run_decode(args, device, dist):
     topk_ws = torch.empty(max(1, dsa.topk_workspace_bytes(B, ld, k)), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step(ev=None):
+    def step(ev=None, inner=True):
         if ev is not None:
             ev[0].record(stream)
         dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, 1, N, 0, B, scores=scores)
-        if ev is not None:
+        if ev is not None and inner:
             ev[1].record(stream)
         dsa.topk(scores, cu_q, cu_k, k, 0, B, indices=idx, workspace=topk_ws)
-        if ev is not None:
+        if ev is not None and inner:
             ev[2].record(stream)
         dsa.sparse_attn_decode(t["Q"], t["K"], t["V"], idx, cu_k, workspace=ws)
         if ev is not None:
@@ -325,18 +325,47 @@ def run_decode(args, device, dist):
         step()
     torch.cuda.synchronize(device)
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    # per-call breakdown: events between the calls (they also stop the launches from
+    # overlapping across calls)
     evs = [[E(), E(), E(), E()] for _ in range(steps)]
     for s in range(steps):
         step(evs[s])
     torch.cuda.synchronize(device)
-    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
-                     e[0].elapsed_time(e[3])] for e in evs])
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
     us = per.mean(axis=0) * 1e3
+    # the step: events only around it, so its 6 launches chain as they do in a server
+    evs = [[E(), None, None, E()] for _ in range(steps)]
+    for s in range(steps):
+        step(evs[s], inner=False)
+    torch.cuda.synchronize(device)
+    step_us = float(np.mean([e[0].elapsed_time(e[3]) for e in evs])) * 1e3
+    # the same step captured once in a CUDA graph and replayed back to back (host work per
+    # step: one graph launch); reported beside the step time
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        step()  # warm the caching allocator on the capture stream
+        torch.cuda.synchronize(device)
+        with torch.cuda.graph(graph, stream=side):
+            step()
+    torch.cuda.synchronize(device)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(device)
+    g0, g1 = E(), E()
+    g0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize(device)
+    graph_us = g0.elapsed_time(g1) / steps * 1e3
+    del graph
     idx_bytes = B * N * wl.d_I * 2 + B * wl.H_I * wl.d_I * 2 + B * wl.H_I * 2
     attn_bytes = B * k * wl.Hkv * wl.d * 2 * 2 + B * wl.Hq * wl.d * 2 * 2 + B * k * 4
     del t, scores, idx, ws, topk_ws
     torch.cuda.empty_cache()
-    return {"us_per_step": float(us[3]), "us_per_token": float(us[3]) / B,
+    return {"us_per_step": step_us, "us_per_token": step_us / B, "graph_replay_us_per_step": graph_us,
             "breakdown_us": {"indexer": float(us[0]), "topk": float(us[1]), "sparse_attn": float(us[2])},
             "idx_bytes": idx_bytes, "attn_bytes": attn_bytes, "steps": steps,
             # indexer; top-k row bound, segment filter, row select; attention, split combine
@@ -520,7 +549,11 @@ def main():
         line["decode"] = {
             "metric": "DSA decode us/step at 256K ctx (16 sequences, one token each)",
             "workload": "decode_256k", "value": dec["us_per_step"], "unit": "us/step",
-            "us_per_token": dec["us_per_token"], "breakdown_us": dec["breakdown_us"],
+            "timing": "device time from an event before the step's first launch to one after its last, "
+                      "mean over steps; breakdown from a run with events between the calls; graph_replay: "
+                      "the step as a CUDA graph replayed back to back, per replay",
+            "us_per_token": dec["us_per_token"], "graph_replay_us_per_step": dec["graph_replay_us_per_step"],
+            "breakdown_us": dec["breakdown_us"],
             "roofline": {"kernel": "whole decode step", "bound": "hbm",
                          "achieved": dec_bytes / (dec["us_per_step"] / 1e6) / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": dec_bytes / (dec["us_per_step"] / 1e6) / 1e9 / hbm},

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/dsa.h"
 
 namespace dsa {
@@ -272,6 +274,18 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with the programmatic-serialization attribute may be scheduled before
+// the previous kernel of the stream finishes; pdl_wait() blocks (in hardware) until that
+// kernel has completed and its memory is visible, and is a no-op otherwise.  Every kernel
+// that is launched that way calls pdl_wait() before touching global memory.
+// pdl_trigger() lets the next kernel of the stream be scheduled early; kernels call it only
+// after their own pdl_wait() returned, so at most one kernel waits ahead of the running
+// one (a chain of early triggers would park later kernels' blocks on SMs the running
+// kernel needs).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
@@ -301,5 +315,28 @@ int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 int sm_count();
 int last_launch_status();    // DSA_ERR_CUDA if the last launch failed, else DSA_OK
 int cuda_fail(cudaError_t e);  // records e for dsa_last_cuda_error(); returns DSA_ERR_CUDA
+
+// Launches `kern`, with programmatic stream serialization when `pdl` is set (the kernel
+// must then call pdl_wait() before its first global memory access).  The library sets it
+// only between the launches of one entry point (the top-k passes, attention and its split
+// combine): measured on the decode step, letting a call's first kernel overlap the
+// previous call's last one made the step slower.  Returns DSA_OK or DSA_ERR_CUDA.
+template <typename... KArgs, typename... Args>
+int launch_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...); e != cudaSuccess)
+    return cuda_fail(e);
+  return last_launch_status();
+}
 
 }  // namespace dsa_host

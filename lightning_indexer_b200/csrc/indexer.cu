@@ -122,6 +122,8 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_ST
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                    const IndexerParams p) {
   using C = IndexerCfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + C::OFF_A;
@@ -372,8 +374,7 @@ static int launch_indexer(const void* q_idx, const void* k_idx, const void* w, c
   (void)max_seqlen_q;
   const long long grid = std::min<long long>(p.n_items, (long long)sm_count());
   if (grid <= 0) return DSA_OK;
-  kern<<<(unsigned)grid, C::THREADS, smem, stream>>>(tk, tq, p);
-  return last_launch_status();
+  return launch_pdl(false, kern, dim3((unsigned)grid), dim3(C::THREADS), (size_t)smem, stream, tk, tq, p);
 }
 
 int indexer2_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,

@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   constexpr int MT = D / 16;                    // m-tiles of O^T, k-steps of S^T
   static_assert(MT % 2 == 0, "two interleaved S chains");
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t my_s = smem_u32(smem + warp * SA_STAGES * STAGE_BYTES);
@@ -327,6 +329,8 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
 template <int D>
 __global__ void decode_combine_kernel(const float* part_o, const float* part_ml, int rows, int Hq, int nsplit,
                                       uint16_t* O, float* lse) {
+  pdl_wait();
+  pdl_trigger();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (gw >= rows * Hq) return;
@@ -386,8 +390,8 @@ static int sa_launch_d(const dsa::SAParams& p, long long tasks, cudaStream_t str
     if (e_ != cudaSuccess) return cuda_fail(e_);
     done = true;
   }
-  dsa::sparse_attn_kernel<D, STAGES, WARPS><<<(unsigned)blocks, WARPS * 32, smem, stream>>>(p);
-  return last_launch_status();
+  return launch_pdl(false, dsa::sparse_attn_kernel<D, STAGES, WARPS>, dim3((unsigned)blocks), dim3(WARPS * 32),
+                    (size_t)smem, stream, p);
 }
 
 static int sa_launch_common(dsa::SAParams& p, int d, cudaStream_t stream) {
@@ -460,13 +464,15 @@ int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const
   const int warps = batch * Hq;
   const int threads = 256;
   const int blocks = (warps * 32 + threads - 1) / threads;
+  const float* part_o = p.part_o;
+  const float* part_ml = p.part_ml;
+  uint16_t* O_ = p.O;
+  const int nsplit = p.nsplit;
   if (d == 128)
-    dsa::decode_combine_kernel<128><<<blocks, threads, 0, stream>>>(p.part_o, p.part_ml, batch, Hq, p.nsplit,
-                                                                   p.O, lse);
-  else
-    dsa::decode_combine_kernel<64><<<blocks, threads, 0, stream>>>(p.part_o, p.part_ml, batch, Hq, p.nsplit,
-                                                                  p.O, lse);
-  return last_launch_status();
+    return launch_pdl(true, dsa::decode_combine_kernel<128>, dim3(blocks), dim3(threads), 0, stream, part_o, part_ml, batch,
+                      Hq, nsplit, O_, lse);
+  return launch_pdl(true, dsa::decode_combine_kernel<64>, dim3(blocks), dim3(threads), 0, stream, part_o, part_ml, batch,
+                    Hq, nsplit, O_, lse);
 }
 
 }  // namespace dsa_host

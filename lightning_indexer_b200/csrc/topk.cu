@@ -1217,6 +1217,8 @@ struct SegFilterSmem {
 // the row would hit the same L2 sectors from all of them at once).
 __global__ void __launch_bounds__(SF_T) topk_rowbound_kernel(const TopkParams p, const TopkWs ws) {
   constexpr int B = SF_T;
+  pdl_wait();
+  pdl_trigger();
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t total, bin, above;
@@ -1229,6 +1231,7 @@ __global__ void __launch_bounds__(SF_T) topk_rowbound_kernel(const TopkParams p,
 
 __global__ void __launch_bounds__(SF_T, 4) topk_segfilter_kernel(const TopkParams p, const TopkWs ws) {
   constexpr int B = SF_T;
+  pdl_wait();
   __shared__ SegFilterSmem S;
   const long long rr = blockIdx.x / ws.nseg;
   const int sg = blockIdx.x % ws.nseg;
@@ -1292,10 +1295,13 @@ __global__ void __launch_bounds__(SF_T, 4) topk_segfilter_kernel(const TopkParam
     }
   }
   if (threadIdx.x == 0) *cnt = S.total;
+  pdl_trigger();  // late: the next kernel's blocks would take this one's SM slots
 }
 
 __global__ void __launch_bounds__(TOPK_THREADS) topk_rowselect_kernel(const TopkParams p, const TopkWs ws) {
   constexpr int B = TOPK_THREADS;
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem& S = *reinterpret_cast<TopkSmem*>(smem_raw);
   const long long rr = blockIdx.x;
@@ -1460,12 +1466,17 @@ static int topk_two_launch(const dsa::TopkParams& p, long long rows, long long m
     if (e_ != cudaSuccess) return cuda_fail(e_);
     attr_done = true;
   }
-  dsa::topk_rowbound_kernel<<<(unsigned)rows, dsa::SF_T, 0, stream>>>(p, ws);
-  if (const int st = last_launch_status(); st != DSA_OK) return st;
-  dsa::topk_segfilter_kernel<<<(unsigned)(rows * ws.nseg), dsa::SF_T, 0, stream>>>(p, ws);
-  if (const int st = last_launch_status(); st != DSA_OK) return st;
-  dsa::topk_rowselect_kernel<<<(unsigned)rows, dsa::TOPK_THREADS, sizeof(dsa::TopkSmem), stream>>>(p, ws);
-  return last_launch_status();
+  // the second and third launches overlap their launch latency with the previous kernel's
+  // tail (programmatic dependent launch)
+  if (const int st = launch_pdl(false, dsa::topk_rowbound_kernel, dim3((unsigned)rows), dim3(dsa::SF_T), 0, stream, p, ws);
+      st != DSA_OK)
+    return st;
+  if (const int st = launch_pdl(true, dsa::topk_segfilter_kernel, dim3((unsigned)(rows * ws.nseg)), dim3(dsa::SF_T), 0,
+                                stream, p, ws);
+      st != DSA_OK)
+    return st;
+  return launch_pdl(true, dsa::topk_rowselect_kernel, dim3((unsigned)rows), dim3(dsa::TOPK_THREADS), sizeof(dsa::TopkSmem),
+                    stream, p, ws);
 }
 
 int topk_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
