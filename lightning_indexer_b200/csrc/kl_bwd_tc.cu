@@ -274,11 +274,19 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
       if (!kl_dk_item(item, p, it)) continue;
       const int s = it.tile * 128 + r;  // this thread's key (sequence-local)
       const int dvis = it.Lk - it.Lq + 1;
+      const long long q0 = p.cu_q[it.b];
+      // g of this warp's row and this thread's key; 0 past the item or the row's visible keys
+      auto load_g = [&](int blk) -> float {
+        const long long t = it.qlo + 2 * blk + half;
+        const int vis = min(max((int)(t - q0) + dvis, 0), it.Lk);
+        return (t < it.qhi && s < vis) ? p.g[(t - p.row_begin) * p.ld + s] : 0.f;
+      };
+      float g_next = load_g(0);  // one block ahead, so the load's latency hides behind a block
       for (int i = 0; i < it.nb; ++i, ++n) {
         const long long t = it.qlo + 2 * i + half;  // this warp's query row
-        const int vis = min(max((int)(t - p.cu_q[it.b]) + dvis, 0), it.Lk);
         const bool tv = t < it.qhi;  // else its G columns are 0
-        const float gv = (tv && s < vis) ? p.g[(t - p.row_begin) * p.ld + s] : 0.f;
+        const float gv = g_next;
+        if (i + 1 < it.nb) g_next = load_g(i + 1);
         const int st = (int)(n & 1);
         // the block's head weights arrive with its query tiles: observe that phase here too
         // (the stage cannot be refilled before this block's G is written, so the phase seen
