@@ -13,7 +13,7 @@ import torch
 from . import _lib
 from ._lib import DSAError, call
 
-__all__ = ["index", "topk", "topk_workspace_bytes", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
+__all__ = ["index", "topk", "topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
            "sparse_attn_prefill_bwd", "indexer_kl_loss", "device_status", "DSAError"]
 
 
@@ -86,16 +86,21 @@ def topk(scores, cu_seqlens_q, cu_seqlens_k, k: int, row_begin: int = 0, row_end
 
 
 def sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, scale: Optional[float] = None,
-                        with_lse: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Sparse GQA attention of every packed query row over its selected keys."""
+                        with_lse: bool = True, out=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Sparse GQA attention of every packed query row over its selected keys.  `out` may
+    give (O, lse) tensors to write (lse may be None)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _check(t, n, torch.bfloat16, 3)
     _check(indices, "indices", torch.int32, 2)
     T, Hq, d = Q.shape
     Hkv = K.shape[1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    O = torch.empty_like(Q)
-    lse = torch.empty((T, Hq), dtype=torch.float32, device=Q.device) if with_lse else None
+    if out is not None:
+        O, lse = out
+        _check(O, "O", torch.bfloat16, 3)
+    else:
+        O = torch.empty_like(Q)
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=Q.device) if with_lse else None
     call("dsa_sparse_attn_prefill", _ptr(Q), _ptr(K), _ptr(V), _ptr(indices), _ptr(cu_seqlens_q),
          _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Hq, Hkv, d, indices.shape[1], scale, _ptr(O),
          _ptr(lse), _stream())
@@ -151,6 +156,85 @@ def prefill(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: 
          H_I, d_I, k, scale, chunk_rows, _ptr(indices), _ptr(O), _ptr(lse), _ptr(workspace), workspace.numel(),
          _stream())
     return indices, O, lse
+
+
+_aux_streams = {}
+
+
+def _streams(device: torch.device):
+    key = device.index
+    if key not in _aux_streams:
+        _aux_streams[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
+    return _aux_streams[key]
+
+
+def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                      k: int, chunk_rows: int = 8192, scale: Optional[float] = None, O=None,
+                      device: Optional[torch.device] = None, buffers: Optional[dict] = None):
+    """Whole DSA prefill whose inputs and output live in host memory (pin them for overlap).
+
+    The key-side tensors (k_idx, K, V) are copied first; then the query rows of each row
+    chunk are copied on a copy stream while the previous chunk runs its indexer, top-k and
+    attention on the current stream, and each chunk's O rows go back on a third stream
+    while the next chunk runs.  The kernels and their results are those of `prefill`.
+    `buffers` (a dict, filled on first use) keeps the device copies between calls.
+    Returns O (host, bf16 [T, Hq, d]); the current stream is ordered after every copy.
+    """
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    T, Hq, d = Q.shape
+    L = max_seqlen_k
+    chunk_rows = max(1, min(chunk_rows, T))
+    chunks = [(r0, min(T, r0 + chunk_rows)) for r0 in range(0, T, chunk_rows)]
+    buf = {} if buffers is None else buffers
+    for name, h in (("q_idx", q_idx), ("k_idx", k_idx), ("w", w), ("Q", Q), ("K", K), ("V", V),
+                    ("cu_q", cu_seqlens_q), ("cu_k", cu_seqlens_k)):
+        if name not in buf or buf[name].shape != h.shape:
+            buf[name] = torch.empty(h.shape, dtype=h.dtype, device=dev)
+    B = cu_seqlens_q.numel() - 1
+    # per chunk: the query offsets shifted to the chunk's first row (attention runs per chunk)
+    cq = cu_seqlens_q.to(torch.int64)
+    cu_chunks = torch.stack([(cq - r0).clamp(0, r1 - r0) for r0, r1 in chunks]).to(torch.int32)
+    if "cu_chunks" not in buf or buf["cu_chunks"].shape != cu_chunks.shape:
+        buf["cu_chunks"] = torch.empty(cu_chunks.shape, dtype=torch.int32, device=dev)
+    if "scores" not in buf or buf["scores"].shape[0] < chunk_rows or buf["scores"].shape[1] < _ld(L):
+        buf["scores"] = torch.empty((chunk_rows, _ld(L)), dtype=torch.float32, device=dev)
+    if "idx" not in buf or buf["idx"].shape != (T, k):
+        buf["idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if "O" not in buf or buf["O"].shape != Q.shape:
+        buf["O"] = torch.empty(Q.shape, dtype=torch.bfloat16, device=dev)
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16, pin_memory=True)
+    main = torch.cuda.current_stream(dev)
+    h2d, d2h = _streams(dev)
+    h2d.wait_stream(main)  # the buffers are free once earlier work on this stream is done
+    d2h.wait_stream(main)
+    ev_keys = torch.cuda.Event()
+    ev_in = [torch.cuda.Event() for _ in chunks]
+    with torch.cuda.stream(h2d):
+        for name, h in (("cu_q", cu_seqlens_q), ("cu_k", cu_seqlens_k), ("k_idx", k_idx), ("K", K), ("V", V)):
+            buf[name].copy_(h, non_blocking=True)
+        buf["cu_chunks"].copy_(cu_chunks, non_blocking=True)
+        ev_keys.record(h2d)
+        for (r0, r1), ev in zip(chunks, ev_in):
+            for name, h in (("q_idx", q_idx), ("w", w), ("Q", Q)):
+                buf[name][r0:r1].copy_(h[r0:r1], non_blocking=True)
+            ev.record(h2d)
+    main.wait_event(ev_keys)
+    for c, (r0, r1) in enumerate(chunks):
+        main.wait_event(ev_in[c])
+        sc = buf["scores"][: r1 - r0]
+        index(buf["q_idx"], buf["k_idx"], buf["w"], buf["cu_q"], buf["cu_k"], max_seqlen_q, L, r0, r1, scores=sc)
+        topk(sc, buf["cu_q"], buf["cu_k"], k, r0, r1, indices=buf["idx"][r0:r1])
+        sparse_attn_prefill(buf["Q"][r0:r1], buf["K"], buf["V"], buf["idx"][r0:r1], buf["cu_chunks"][c],
+                            buf["cu_k"], scale, out=(buf["O"][r0:r1], None))
+        ev_out = torch.cuda.Event()
+        ev_out.record(main)
+        d2h.wait_event(ev_out)
+        with torch.cuda.stream(d2h):
+            O[r0:r1].copy_(buf["O"][r0:r1], non_blocking=True)
+    main.wait_stream(d2h)
+    main.wait_stream(h2d)
+    return O
 
 
 def decode_workspace_bytes(batch: int, max_seqlen_k: int, Hq: int, d: int, k: int) -> int:
