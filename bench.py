@@ -54,6 +54,24 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's `value` (the job is as slow as its slowest rank);
+    `value` itself with no process group.  `device` holds the reduction tensor (a CUDA
+    device under NCCL, the CPU under gloo)."""
+    if dist is None:
+        return value
+    import torch
+    x = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return float(x.item())
+
+
+def whole_job_rate(tokens_per_rank: int, ms_per_step: float, world: int) -> float:
+    """Tokens per second of the whole job: every rank processes its own replica's tokens
+    in each step, and a step lasts as long as the slowest rank's."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def measured_peaks():
     try:
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
@@ -222,12 +240,9 @@ def run_prefill(args, rank, world, device, dist):
             t_idx += e0.elapsed_time(e1)
             t_topk += e1.elapsed_time(e2)
         t_attn += evs[s][len(chunks) - 1][2].elapsed_time(evs[s][-1][0])
-    if dist is not None:
-        x = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms = float(x.item())
+    ms = max_over_ranks(ms, dist, device)
     ms_step = ms / args.steps
-    value = world * L / (ms_step / 1e3)
+    value = whole_job_rate(L, ms_step, world)
 
     pairs = wl.causal_pairs()
     sel_pairs = wl.selected_pairs()
@@ -276,11 +291,8 @@ def run_prefill(args, rank, world, device, dist):
         b.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms = a.elapsed_time(b) / args.steps
-        if dist is not None:
-            x = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(x, op=dist.ReduceOp.MAX)
-            e2e_ms = float(x.item())
-        res["e2e"] = {"value": world * L / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks(e2e_ms, dist, device)
+        res["e2e"] = {"value": whole_job_rate(L, e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "api": "lightning_indexer_b200.prefill_from_host"}
         del host, bufs
     else:
