@@ -13,7 +13,8 @@
 //   dw[t,j] = sum_s g max(0,x),  dq_idx[t,j] = sum_s G k_idx[s],  dk_idx[s] = sum_t,j G q_idx[t,j]
 //
 // Passes (rows processed in chunks that bound the fp32 score scratch):
-//   1. dense_lse_kernel   LSE of the dense causal logits for every (t, h)   [warp MMA]
+//   1. dense LSE          LSE of the dense causal logits for every (t, h)   [tcgen05 for d = 128,
+//                         Hq/Hkv = 8 (kl_dense_tc.cu); warp MMA otherwise]
 //   per chunk:
 //   2. dsa_index          I for the chunk rows                              [tcgen05]
 //   3. row_lse_kernel     log-sum-exp of each I row
@@ -612,6 +613,9 @@ int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const in
                    cudaStream_t stream);
 int f32_to_bf16_launch(const float* src, void* dst, long long n, cudaStream_t stream);
 int kl_transpose_q_launch(const void* q_idx, void* q_t, long long rows, cudaStream_t s);
+int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
+                     long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
+                     cudaStream_t s);
 int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const void* w, const int* cu_q,
                     const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
                     long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
@@ -714,8 +718,11 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
   const long long ld = ((long long)(max_seqlen_k > 0 ? max_seqlen_k : 1) + 3) / 4 * 4;
   const float scale_log2 = scale * 1.4426950408889634f;
   if (const cudaError_t e_ = cudaMemsetAsync(W.dk_acc, 0, (size_t)Tk * d_I * 4, s); e_ != cudaSuccess) return cuda_fail(e_);
-  // 1. dense LSE
-  {
+  // 1. dense LSE (tensor cores for d = 128 and 8 query heads per KV head)
+  if (d == 128 && Hq == 8 * Hkv) {
+    const int st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, T, Tk, Hq, Hkv, max_seqlen_q, scale_log2, W.lse_att, s);
+    if (st != DSA_OK) return st;
+  } else {
     const long long tasks = T * Hkv;
     const long long blocks = (tasks + dsa::KL_WARPS - 1) / dsa::KL_WARPS;
     const int smem = dsa::KL_WARPS * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;

@@ -7,5 +7,6 @@
 #include "sparse_attn.cu"
 #include "sparse_attn_bwd.cu"
 #include "kl_bwd_tc.cu"
+#include "kl_dense_tc.cu"
 #include "kl_loss.cu"
 #include "decode_noalloc.cu"
