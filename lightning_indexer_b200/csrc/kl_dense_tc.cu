@@ -1,4 +1,5 @@
-// Dense attention LSE of the KL target on tcgen05 tensor cores (sm_100a).
+// Dense attention of the KL target on tcgen05 tensor cores (sm_100a): the LSE pass and the
+// target / KL / gradient pass.
 //
 // Source: Keye-VL-2.0 report summary (mqxn.cn/news/1966), section 1: the dense warm-up
 // trains the indexer against the full attention distribution; its target needs, for every
@@ -241,6 +242,343 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
+
+// ---------------------------------------------------------------------------- target
+// Dense target p, the row's KL term and g = dloss/dI for the rows [row_begin, row_end) of
+// one score chunk (same source and definitions as the LSE above):
+//   p[t,s]  = (1/Hq) sum_h exp(scale Q[t,h].K[s,g(h)] - lse[t,h])
+//   kl[t]   = sum_{s visible} p (log p - log q),  log q = I[t,s] - lseI[t]
+//   I[t,s] <- (q - p) / T   (in place)
+// A work item is 8 query rows of one sequence.  Orientation is key-stationary per tile:
+// the A operand is 128 keys of one KV head (M = 128), the B operand the 8 rows x 8 query
+// heads of that KV head (N = 64, one 3-D TMA box of Q), so a TMEM lane is a key and the
+// sum over heads stays inside a thread.  All Hkv (<= 4) heads of a key tile go to one
+// 256-column TMEM buffer; two buffers alternate.  Eight epilogue warps: warp w reads lanes
+// 32 (w % 4) .. (keys) for rows 4 ((w - 2) / 4) .. + 3.  Each (row, warp-quarter) keeps its
+// own partial of kl[t], written once to kl_part[t][quarter] (a fixed-order sum follows).
+struct KlTgtParams {
+  const int* cu_q;
+  const int* cu_k;
+  int batch;
+  int Hq, Hkv;
+  float scale_log2;
+  long long row_begin, row_end;
+  const float* lse_att;  // [T, Hq] natural log
+  const float* lseI;     // [row_end - row_begin]
+  float* scores;         // [row_end - row_begin, ld]: I in, g out
+  long long ld;
+  float inv_T;
+  float* kl_part;        // [T, 4]
+  long long n_blocks;    // bound on the 8-row blocks of the chunk
+  long long n_slots;     // n_blocks rounded up to whole rounds of gridDim.x
+};
+
+struct KlTgtItem {
+  long long t0;
+  int ntok, i0, Lq, Lk, kbase, ntiles;
+};
+
+// Items in snake order over rounds of gridDim.x (CTA c takes position c of even rounds and
+// gridDim.x - 1 - c of odd ones); within the order blocks run from the chunk's last one,
+// so long rows come first.
+__device__ __forceinline__ bool kl_tgt_item(long long item, const KlTgtParams& p, KlTgtItem& it) {
+  const long long G = gridDim.x, k = item / G, pos = item % G;
+  const long long idx = k * G + ((k & 1) ? G - 1 - pos : pos);
+  if (idx >= p.n_blocks) return false;
+  long long r = p.n_blocks - 1 - idx;
+  for (int b = 0; b < p.batch; ++b) {
+    const long long lo = max((long long)p.cu_q[b], p.row_begin), hi = min((long long)p.cu_q[b + 1], p.row_end);
+    if (hi <= lo) continue;
+    const long long nb = (hi - lo + 7) / 8;
+    if (r < nb) {
+      it.t0 = lo + r * 8;
+      it.ntok = (int)min(8LL, hi - it.t0);
+      it.i0 = (int)(it.t0 - p.cu_q[b]);
+      it.Lq = p.cu_q[b + 1] - p.cu_q[b];
+      it.Lk = p.cu_k[b + 1] - p.cu_k[b];
+      it.kbase = p.cu_k[b];
+      const int vis_last = min(max(it.i0 + it.ntok - 1 + it.Lk - it.Lq + 1, 0), it.Lk);
+      it.ntiles = (vis_last + 127) / 128;
+      return true;
+    }
+    r -= nb;
+  }
+  return false;
+}
+
+struct KlTgtCfg {
+  static constexpr int K_TILE_BYTES = 128 * 128 * 2;  // 128 keys x 128 dims
+  static constexpr int K_PANEL_BYTES = 128 * 128;
+  static constexpr int Q_GROUP_BYTES = 64 * 128 * 2;  // 8 rows x 8 heads x 128 dims
+  static constexpr int Q_PANEL_BYTES = 64 * 128;
+  static constexpr int MAX_HKV = 4;
+  static constexpr int B_STAGES = 4;
+  static constexpr int L_BYTES = 8 * 8 * MAX_HKV * 4;  // lse of 8 rows x Hq heads
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_B = OFF_Q + MAX_HKV * Q_GROUP_BYTES;
+  static constexpr int OFF_L = OFF_B + B_STAGES * K_TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_L + 2 * L_BYTES;
+  // q_full, q_empty, l_full[2], l_empty[2], b_full[S], b_empty[S], acc_full[2], acc_empty[2], done
+  static constexpr int NUM_BARS = 2 + 4 + 2 * B_STAGES + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int ACC_COLS = 256;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(128, 64);
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+__global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
+    kl_target_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                        const KlTgtParams p) {
+  using C = KlTgtCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sB = smem + C::OFF_B;
+  float* sL = reinterpret_cast<float*>(smem + C::OFF_L);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* l_full = bars + 2;   // [2]
+  uint64_t* l_empty = bars + 4;  // [2]
+  uint64_t* b_full = bars + 6;   // [B_STAGES]
+  uint64_t* b_empty = b_full + C::B_STAGES;
+  uint64_t* acc_full = b_empty + C::B_STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint64_t* mma_done = acc_full + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int Hkv = p.Hkv;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&l_full[i], 1);
+      mbar_init(&l_empty[i], C::EPI_WARPS);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::EPI_WARPS);
+    }
+    for (int i = 0; i < C::B_STAGES; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      long long m = 0, n = 0;  // items, (key tile, KV head) stages
+      bool ok = true;
+      for (long long item = blockIdx.x; item < p.n_slots && ok; item += gridDim.x) {
+        KlTgtItem it;
+        if (!kl_tgt_item(item, p, it)) continue;
+        const int lb = (int)(m & 1);
+        if (!(ok = mbar_wait(&l_empty[lb], (uint32_t)((m >> 1) & 1) ^ 1u, abort_flag, 70))) break;
+        {
+          const uint32_t lbytes = (uint32_t)(it.ntok * p.Hq * 4);
+          mbar_arrive_expect_tx(&l_full[lb], lbytes);
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                  smem_u32(sL + lb * (C::L_BYTES / 4))),
+              "l"(p.lse_att + it.t0 * p.Hq), "r"(lbytes), "r"(smem_u32(&l_full[lb]))
+              : "memory");
+        }
+        if (!(ok = mbar_wait(q_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 71))) break;
+        mbar_arrive_expect_tx(q_full, Hkv * C::Q_GROUP_BYTES);
+        for (int g = 0; g < Hkv; ++g)
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(sQ + g * C::Q_GROUP_BYTES + pn * C::Q_PANEL_BYTES, &tmap_q, q_full, pn * 64, g * 8,
+                        (int)it.t0);
+        ++m;
+        for (int j = 0; j < it.ntiles && ok; ++j) {
+          for (int g = 0; g < Hkv; ++g, ++n) {
+            const int st = (int)(n % C::B_STAGES);
+            if (!(ok = mbar_wait(&b_empty[st], (uint32_t)((n / C::B_STAGES) & 1) ^ 1u, abort_flag, 72))) break;
+            mbar_arrive_expect_tx(&b_full[st], C::K_TILE_BYTES);
+            for (int pn = 0; pn < 2; ++pn)
+              tma_load_3d(sB + st * C::K_TILE_BYTES + pn * C::K_PANEL_BYTES, &tmap_k, &b_full[st], pn * 64, g,
+                          it.kbase + j * 128);
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies this thread issued land before the CTA exits (bounded)
+        const uint64_t t0 = globaltimer_ns();
+        for (long long k = max(0LL, n - C::B_STAGES); k < n; ++k)
+          while (!mbar_try_wait(smem_u32(&b_full[k % C::B_STAGES]), (uint32_t)((k / C::B_STAGES) & 1)) &&
+                 globaltimer_ns() - t0 < 100000000ull) {
+          }
+        if (m > 0) {
+          while (!mbar_try_wait(smem_u32(q_full), (uint32_t)((m - 1) & 1)) && globaltimer_ns() - t0 < 100000000ull) {
+          }
+          const long long k = m - 1;
+          while (!mbar_try_wait(smem_u32(&l_full[k & 1]), (uint32_t)((k >> 1) & 1)) &&
+                 globaltimer_ns() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      long long m = 0, n = 0, nt = 0;
+      bool ok = true;
+      const uint32_t q_base = smem_u32(sQ);
+      for (long long item = blockIdx.x; item < p.n_slots && ok; item += gridDim.x) {
+        KlTgtItem it;
+        if (!kl_tgt_item(item, p, it)) continue;
+        if (!(ok = mbar_wait(q_full, (uint32_t)(m & 1), abort_flag, 73))) break;
+        tc_fence_after();
+        for (int j = 0; j < it.ntiles && ok; ++j, ++nt) {
+          const int ab = (int)(nt & 1);
+          if (!(ok = mbar_wait(&acc_empty[ab], (uint32_t)((nt >> 1) & 1) ^ 1u, abort_flag, 74))) break;
+          tc_fence_after();
+          for (int g = 0; g < Hkv; ++g, ++n) {
+            const int st = (int)(n % C::B_STAGES);
+            if (!(ok = mbar_wait(&b_full[st], (uint32_t)((n / C::B_STAGES) & 1), abort_flag, 75))) break;
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(sB + st * C::K_TILE_BYTES);
+            const uint32_t d = tmem_base + ab * C::ACC_COLS + g * 64;
+#pragma unroll
+            for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(d, smem_desc_kmajor(k_base + pn * C::K_PANEL_BYTES + kk * 32, 128),
+                          smem_desc_kmajor(q_base + g * C::Q_GROUP_BYTES + pn * C::Q_PANEL_BYTES + kk * 32, 128),
+                          C::IDESC, (pn | kk) != 0);
+            umma_commit(&b_empty[st]);
+          }
+          if (!ok) break;
+          umma_commit(&acc_full[ab]);
+        }
+        if (!ok) break;
+        umma_commit(q_empty);
+        ++m;
+      }
+      umma_commit(mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (8 warps)
+    const int quarter = warp % 4;
+    const int half = (warp - 2) / 4;  // rows 4 half .. 4 half + 3
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float inv_Hq = 1.f / (float)p.Hq;
+    constexpr float kLog2e = 1.4426950408889634f;
+    long long m = 0, nt = 0;
+    bool ok = true;
+    for (long long item = blockIdx.x; item < p.n_slots && ok; item += gridDim.x) {
+      KlTgtItem it;
+      if (!kl_tgt_item(item, p, it)) continue;
+      const int lb = (int)(m & 1);
+      int vis[4];
+      float lI[4], kl[4];
+      float* Irow[4];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int u = 4 * half + rr;
+        const bool valid = u < it.ntok;
+        vis[rr] = valid ? min(max(it.i0 + u + it.Lk - it.Lq + 1, 0), it.Lk) : 0;
+        const long long lr = it.t0 + (valid ? u : 0) - p.row_begin;
+        lI[rr] = p.lseI[lr];
+        Irow[rr] = p.scores + lr * p.ld;
+        kl[rr] = 0.f;
+      }
+      if (!(ok = mbar_wait(&l_full[lb], (uint32_t)((m >> 1) & 1), abort_flag, 76))) break;
+      const float* Lrow = sL + lb * (C::L_BYTES / 4) + 4 * half * p.Hq;
+      for (int j = 0; j < it.ntiles; ++j, ++nt) {
+        const int ab = (int)(nt & 1);
+        const int key = j * 128 + quarter * 32 + lane;
+        float Iv[4];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) Iv[rr] = key < vis[rr] ? Irow[rr][key] : 0.f;
+        if (!(ok = mbar_wait(&acc_full[ab], (uint32_t)((nt >> 1) & 1), abort_flag, 77))) break;
+        tc_fence_after();
+        float pr[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int g = 0; g < Hkv; ++g) {
+          float v[32];
+          tmem_ld_x32_sync(tmem_base + lane_off + ab * C::ACC_COLS + g * 64 + half * 32, v);
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            const float4 La = *reinterpret_cast<const float4*>(Lrow + rr * p.Hq + g * 8);
+            const float4 Lb = *reinterpret_cast<const float4*>(Lrow + rr * p.Hq + g * 8 + 4);
+            const float* x = v + rr * 8;
+            float a0 = exp2f(fmaf(x[0], p.scale_log2, -La.x * kLog2e));
+            float a1 = exp2f(fmaf(x[1], p.scale_log2, -La.y * kLog2e));
+            a0 += exp2f(fmaf(x[2], p.scale_log2, -La.z * kLog2e));
+            a1 += exp2f(fmaf(x[3], p.scale_log2, -La.w * kLog2e));
+            a0 += exp2f(fmaf(x[4], p.scale_log2, -Lb.x * kLog2e));
+            a1 += exp2f(fmaf(x[5], p.scale_log2, -Lb.y * kLog2e));
+            a0 += exp2f(fmaf(x[6], p.scale_log2, -Lb.z * kLog2e));
+            a1 += exp2f(fmaf(x[7], p.scale_log2, -Lb.w * kLog2e));
+            pr[rr] += a0 + a1;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          if (key < vis[rr]) {
+            const float pp = pr[rr] * inv_Hq;
+            const float lq = Iv[rr] - lI[rr];  // log q
+            if (pp > 0.f) kl[rr] += pp * (logf(pp) - lq);
+            Irow[rr][key] = (expf(lq) - pp) * p.inv_T;
+          }
+        }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&l_empty[lb]);
+      ++m;
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        float s = kl[rr];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0 && 4 * half + rr < it.ntok) p.kl_part[(it.t0 + 4 * half + rr) * 4 + quarter] = s;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// kl[t] = sum of its four key-quarter partials, in a fixed order
+__global__ void kl_parts_sum_kernel(const float4* part, long long T, float* kl) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < T) {
+    const float4 v = part[t];
+    kl[t] = ((v.x + v.y) + v.z) + v.w;
+  }
+}
+
 }  // namespace dsa
 
 namespace dsa_host {
@@ -286,6 +624,65 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
   const long long grid = std::min<long long>(p.n_items, (long long)sm_count());
   if (grid <= 0) return DSA_OK;
   dsa::kl_lse_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, p);
+  return last_launch_status();
+}
+
+// Dense target, kl partials and g for the chunk rows [r0, r1) (d = 128, Hq = 8 Hkv, Hkv <= 4).
+int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
+                        long long Tk, int Hq, int Hkv, long long r0, long long r1, float scale_log2,
+                        const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
+                        float* kl_part, cudaStream_t s) {
+  using C = dsa::KlTgtCfg;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_tc_kernel,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        e_ != cudaSuccess)
+      return cuda_fail(e_);
+    attr_done = true;
+  }
+  if (Hkv < 1 || Hkv > C::MAX_HKV || Hq != 8 * Hkv) return DSA_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk;
+  {
+    const uint64_t dims[3] = {128, (uint64_t)Hq, (uint64_t)T};
+    const uint64_t strides[2] = {256, (uint64_t)Hq * 256};
+    const uint32_t box[3] = {64, 8, 8};
+    if (const int st = make_tmap_bf16_3d(&tq, Q, dims, strides, box); st != DSA_OK) return st;
+  }
+  {
+    const uint64_t dims[3] = {128, (uint64_t)Hkv, (uint64_t)Tk};
+    const uint64_t strides[2] = {256, (uint64_t)Hkv * 256};
+    const uint32_t box[3] = {64, 1, 128};
+    if (const int st = make_tmap_bf16_3d(&tk, K, dims, strides, box); st != DSA_OK) return st;
+  }
+  dsa::KlTgtParams p;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.scale_log2 = scale_log2;
+  p.row_begin = r0;
+  p.row_end = r1;
+  p.lse_att = lse_att;
+  p.lseI = lseI;
+  p.scores = scores;
+  p.ld = ld;
+  p.inv_T = inv_T;
+  p.kl_part = kl_part;
+  // an upper bound on the 8-row blocks (each sequence piece rounds up once)
+  p.n_blocks = (r1 - r0 + 7) / 8 + batch;
+  const long long grid = std::min<long long>(p.n_blocks, (long long)sm_count());
+  if (grid <= 0) return DSA_OK;
+  p.n_slots = (p.n_blocks + grid - 1) / grid * grid;
+  dsa::kl_target_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, p);
+  return last_launch_status();
+}
+
+int kl_parts_sum_launch(const float* kl_part, long long T, float* kl, cudaStream_t s) {
+  if (T <= 0) return DSA_OK;
+  dsa::kl_parts_sum_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4*>(kl_part), T,
+                                                                       kl);
   return last_launch_status();
 }
 

@@ -18,7 +18,8 @@
 //   per chunk:
 //   2. dsa_index          I for the chunk rows                              [tcgen05]
 //   3. row_lse_kernel     log-sum-exp of each I row
-//   4. kl_target_kernel   p from recomputed dense logits, kl[t], g in place [warp MMA]
+//   4. kl_target_kernel   p from recomputed dense logits, kl[t], g in place [tcgen05 for d = 128,
+//                         Hq/Hkv = 8, Hkv <= 4 (kl_dense_tc.cu); warp MMA otherwise]
 //   5. idx_bwd_row_kernel x recomputed per row; dw, dq_idx (row-stationary) [warp MMA]
 //   6. idx_bwd_col_kernel x recomputed per key tile; dk_idx (key-stationary: one CTA per
 //                         key tile and block of 1024 rows owns a partial, then the
@@ -616,6 +617,11 @@ int kl_transpose_q_launch(const void* q_idx, void* q_t, long long rows, cudaStre
 int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
                      cudaStream_t s);
+int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
+                        long long Tk, int Hq, int Hkv, long long r0, long long r1, float scale_log2,
+                        const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
+                        float* kl_part, cudaStream_t s);
+int kl_parts_sum_launch(const float* kl_part, long long T, float* kl, cudaStream_t s);
 int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const void* w, const int* cu_q,
                     const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
                     long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
@@ -628,6 +634,7 @@ struct KLWorkspace {
   uint16_t* q_t;   // [d_I, T * H_I] q_idx transposed (tensor-core dk path, H_I = 64, d_I = 128)
   float* lseI;     // [chunk_rows]
   float* scores;   // [chunk_rows, ld]
+  float* kl_part;  // [T, 4] per-key-quarter partials of kl (tensor-core target path)
   size_t total;
 };
 
@@ -651,6 +658,8 @@ KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_s
   off += r256((size_t)chunk_rows * 4);
   w.scores = reinterpret_cast<float*>(p + off);
   off += r256((size_t)chunk_rows * ld * 4);
+  w.kl_part = reinterpret_cast<float*>(p + off);
+  off += r256((size_t)T * 4 * 4);
   w.total = off;
   return w;
 }
@@ -758,6 +767,8 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     if (st != DSA_OK) return st;
   }
   const float inv_T = T > 0 ? 1.f / (float)T : 0.f;
+  // 4. on tensor cores for d = 128 and 8 query heads per KV head (at most 4 KV heads)
+  const bool target_tc = d == 128 && Hq == 8 * Hkv && Hkv <= 4;
   for (long long r0 = 0; r0 < T; r0 += chunk_rows) {
     const long long r1 = std::min(T, r0 + chunk_rows);
     int st = indexer_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, max_seqlen_q, max_seqlen_k, H_I, d_I, r0, r1,
@@ -765,7 +776,11 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     if (st != DSA_OK) return st;
     dsa::row_lse_kernel<<<(unsigned)(r1 - r0), 256, 0, s>>>(W.scores, ld, cu_q, cu_k, batch, r0, W.lseI);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
-    {
+    if (target_tc) {
+      st = kl_target_tc_launch(Q, K, cu_q, cu_k, batch, T, Tk, Hq, Hkv, r0, r1, scale_log2, W.lse_att, W.lseI,
+                               W.scores, ld, inv_T, W.kl_part, s);
+      if (st != DSA_OK) return st;
+    } else {
       const int smem = Hkv * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;
       if (d == 128) {
         static bool done = false;
@@ -803,6 +818,10 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
   }
   int st = f32_to_bf16_launch(W.dk_acc, dk, Tk * d_I, s);
   if (st != DSA_OK) return st;
+  if (target_tc) {
+    st = kl_parts_sum_launch(W.kl_part, T, kl, s);
+    if (st != DSA_OK) return st;
+  }
   dsa::mean_kernel<<<1, 1024, 0, s>>>(kl, T, loss);
   return last_launch_status();
 }

@@ -61,7 +61,7 @@ def test_sparse_attention_backward_padded_sets():
     assert _rel_err(dV.float().cpu().numpy(), ref["dV"]) <= 1.5e-2
 
 
-@pytest.mark.parametrize("H_I,Hq,Hkv,d", [(16, 8, 2, 64), (64, 32, 4, 128), (32, 16, 4, 128)])
+@pytest.mark.parametrize("H_I,Hq,Hkv,d", [(16, 8, 2, 64), (64, 32, 4, 128), (32, 16, 4, 128), (64, 16, 2, 128)])
 def test_indexer_kl_loss(H_I, Hq, Hkv, d):
     wl = gen.make_prefill([260, 1, 129, 75], Hq, Hkv, d, H_I, 128, 64, seed=53, layout="video")
     D = orc.Decoded(wl)
