@@ -203,6 +203,17 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, int swizzle
   return start | (lbo << 16) | (sbo << 32) | (1ull << 46) | (layout << 61);
 }
 
+// Shared-memory matrix descriptor for an MN-major operand in the 128-byte swizzled layout:
+// each 128-byte row holds 64 consecutive M (or N) elements of one k, 8 rows (k .. k+7) form
+// a 1024-byte swizzle atom.  `mn_block_bytes` is the distance between blocks of 64 M/N
+// elements (the leading byte offset), 8-row k groups are 1024 bytes apart (stride offset).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t mn_block_bytes) {
+  const uint64_t start = (saddr >> 4) & 0x3FFFu;
+  const uint64_t lbo = (mn_block_bytes >> 4) & 0x3FFFu;
+  const uint64_t sbo = 1024 >> 4;
+  return start | (lbo << 16) | (sbo << 32) | (1ull << 46) | (2ull << 61);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A/B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                       // D format: f32
@@ -211,6 +222,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
+// Instruction-descriptor bit that marks the B operand as MN-major (N contiguous).
+constexpr uint32_t kIdescBMnMajor = 1u << 16;
 
 // ------------------------------------------------------------------ CTA pairs (cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -304,6 +317,50 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+// Query rows [row_begin, row_end) of a varlen batch split, per sequence, into blocks of R
+// rows; block 0 is the range's last block (the longest causal rows of the last sequence).
+struct RowBlock {
+  long long t0;  // first row (global)
+  int ntok;      // rows in the block (1..R)
+  int i0;        // t0's position in its sequence
+  int Lq, Lk, kbase;
+};
+
+// `from_last`-th block of the range, or false past its end (n_blocks may be an upper bound).
+template <int R>
+__device__ __forceinline__ bool chunk_row_block(long long from_last, const int* cu_q, const int* cu_k, int batch,
+                                                long long row_begin, long long row_end, long long n_blocks,
+                                                RowBlock& rb) {
+  if (from_last >= n_blocks) return false;
+  long long r = n_blocks - 1 - from_last;
+  for (int b = 0; b < batch; ++b) {
+    const long long lo = max((long long)cu_q[b], row_begin), hi = min((long long)cu_q[b + 1], row_end);
+    if (hi <= lo) continue;
+    const long long nb = (hi - lo + R - 1) / R;
+    if (r < nb) {
+      rb.t0 = lo + r * R;
+      rb.ntok = (int)min((long long)R, hi - rb.t0);
+      rb.i0 = (int)(rb.t0 - cu_q[b]);
+      rb.Lq = cu_q[b + 1] - cu_q[b];
+      rb.Lk = cu_k[b + 1] - cu_k[b];
+      rb.kbase = cu_k[b];
+      return true;
+    }
+    r -= nb;
+  }
+  return false;
+}
+
+// Persistent-grid slot -> work index in snake order: CTA c takes position c of even rounds
+// of gridDim.x slots and gridDim.x - 1 - c of odd ones, which evens out a descending cost.
+__device__ __forceinline__ long long snake_slot(long long slot) {
+  const long long G = gridDim.x, k = slot / G, pos = slot % G;
+  return k * G + ((k & 1) ? G - 1 - pos : pos);
+}
+
+// Visible keys of query position i (causal, queries aligned to the end of the keys).
+__device__ __forceinline__ int causal_vis(int i, int Lq, int Lk) { return min(max(i + Lk - Lq + 1, 0), Lk); }
 
 // Order-preserving map of fp32 to uint32 (larger float -> larger key); -0.0 maps like +0.0.
 __device__ __forceinline__ uint32_t float_order_key(float f) {

@@ -353,6 +353,365 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
+// ---------------------------------------------------------------------------- rows
+// Row-stationary half of the same backward (H_I = 64, d_I = 128):
+//   dw[t,j]     = sum_s g[t,s] max(0, x[t,j,s])
+//   dq_idx[t,j] = sum_s g[t,s] w[t,j] [x[t,j,s] > 0] k_idx[s]
+// One work item is 2 query rows of one sequence of the row chunk (M = 2 x 64 (t,j) pairs
+// = 128 TMEM lanes); the item's key tiles of 128 stream through three stages, each with
+// the g values of its two rows.  Per key tile:
+//   MMA1  X[128 (t,j) x 128 keys] = Q_blk . K_tile^T       (TMEM, two buffers)
+//   epilogue  dw += g max(0, X) (thread-local: one (t,j) per lane), G = g w [X > 0] -> bf16
+//             in the 128-byte swizzled K-major layout (K = keys)
+//   MMA2  dq[128 (t,j) x 128 d] += G . K_tile             (TMEM accumulator)
+// MMA2's B operand is the key tile itself read MN-major (d contiguous), so no transposed
+// copy of k_idx is needed.  MMA1 of the next tile is issued before MMA2 of this one.
+// Warps: 0 TMA, 1 MMA issuer and TMEM owner, 2-9 epilogue (two per lane quarter, one per
+// 64-key half of the tile; the two dw halves meet in shared memory, added in a fixed order).
+struct KlDqParams {
+  const uint16_t* w;  // [T, 64] bf16
+  const int* cu_q;
+  const int* cu_k;
+  int batch;
+  long long row_begin, row_end;  // the row chunk
+  const float* g;                // [row_end - row_begin, ld] fp32 dloss/dI
+  long long ld;
+  uint16_t* dq;  // [T, 64, 128] bf16
+  uint16_t* dw;  // [T, 64] bf16
+  long long n_blocks, n_slots;
+};
+
+struct KlDqItem {
+  long long t0;
+  int ntok, i0, Lq, Lk, kbase, ntiles;
+};
+
+__device__ __forceinline__ bool kl_dq_item(long long slot, const KlDqParams& p, KlDqItem& it) {
+  RowBlock rb;
+  if (!chunk_row_block<2>(snake_slot(slot), p.cu_q, p.cu_k, p.batch, p.row_begin, p.row_end, p.n_blocks, rb))
+    return false;
+  it.t0 = rb.t0;
+  it.ntok = rb.ntok;
+  it.i0 = rb.i0;
+  it.Lq = rb.Lq;
+  it.Lk = rb.Lk;
+  it.kbase = rb.kbase;
+  it.ntiles = (causal_vis(it.i0 + it.ntok - 1, it.Lq, it.Lk) + 127) / 128;
+  return true;
+}
+
+struct KlDqCfg {
+  static constexpr int H_I = 64, D_I = 128;
+  static constexpr int TILE_BYTES = 128 * 128 * 2;
+  static constexpr int PANEL_BYTES = 128 * 128;
+  static constexpr int K_STAGES = 3;
+  static constexpr int GS_BYTES = 2 * 128 * 4;  // g of the 2 rows for one key tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_G = OFF_K + K_STAGES * TILE_BYTES;  // 2 G buffers
+  static constexpr int OFF_GS = OFF_G + 2 * TILE_BYTES;
+  static constexpr int OFF_DW = OFF_GS + K_STAGES * GS_BYTES;  // 128 fp32 dw halves
+  static constexpr int OFF_BAR = OFF_DW + 128 * 4;
+  // q_full, q_empty, k_full[S], k_empty[S], x_full[2], x_empty[2], g_full[2], g_empty[2],
+  // dq_full, dq_empty, dw_full, dw_empty, done
+  static constexpr int NUM_BARS = 2 + 2 * K_STAGES + 8 + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  static constexpr int TMEM_COLS = 512;  // X buffers [0,128) [128,256), dq [256,384)
+  static constexpr uint32_t IDESC1 = idesc_bf16_f32(128, 128);
+  static constexpr uint32_t IDESC2 = idesc_bf16_f32(128, 128) | kIdescBMnMajor;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+__global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
+    kl_dq_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                    const KlDqParams p) {
+  using C = KlDqCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sG = smem + C::OFF_G;
+  float* sGs = reinterpret_cast<float*>(smem + C::OFF_GS);
+  float* sDw = reinterpret_cast<float*>(smem + C::OFF_DW);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;                 // [K_STAGES]
+  uint64_t* k_empty = k_full + C::K_STAGES;    // [K_STAGES]
+  uint64_t* x_full = k_empty + C::K_STAGES;    // [2]
+  uint64_t* x_empty = x_full + 2;              // [2]
+  uint64_t* g_full = x_full + 4;               // [2]
+  uint64_t* g_empty = x_full + 6;              // [2]
+  uint64_t* dq_full = x_full + 8;
+  uint64_t* dq_empty = x_full + 9;
+  uint64_t* dw_full = x_full + 10;
+  uint64_t* dw_empty = x_full + 11;
+  uint64_t* mma_done = x_full + 12;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < C::K_STAGES; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], C::EPI_WARPS);
+      mbar_init(&g_full[i], C::EPI_WARPS);
+      mbar_init(&g_empty[i], 1);
+    }
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, C::EPI_WARPS);
+    mbar_init(dw_full, C::EPI_WARPS / 2);
+    mbar_init(dw_empty, C::EPI_WARPS / 2);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      long long m = 0, n = 0;  // items with key tiles, key tiles
+      bool ok = true;
+      for (long long slot = blockIdx.x; slot < p.n_slots && ok; slot += gridDim.x) {
+        KlDqItem it;
+        if (!kl_dq_item(slot, p, it) || it.ntiles == 0) continue;
+        if (!(ok = mbar_wait(q_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 80))) break;
+        mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+        for (int pn = 0; pn < 2; ++pn)
+          tma_load_2d(sQ + pn * C::PANEL_BYTES, &tmap_q, q_full, pn * 64, (int)(it.t0 * C::H_I));
+        ++m;
+        for (int j = 0; j < it.ntiles; ++j, ++n) {
+          const int st = (int)(n % C::K_STAGES);
+          if (!(ok = mbar_wait(&k_empty[st], (uint32_t)((n / C::K_STAGES) & 1) ^ 1u, abort_flag, 81))) break;
+          // g of the block's rows for this tile's keys (the row ends at ld; ld % 4 == 0)
+          const uint32_t gbytes = (uint32_t)(min(128LL, p.ld - (long long)j * 128) * 4);
+          mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES + it.ntok * gbytes);
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_2d(sK + st * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &k_full[st], pn * 64,
+                        it.kbase + j * 128);
+          for (int r = 0; r < it.ntok; ++r)
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                    smem_u32(sGs + st * (C::GS_BYTES / 4) + r * 128)),
+                "l"(p.g + (it.t0 + r - p.row_begin) * p.ld + (long long)j * 128), "r"(gbytes),
+                "r"(smem_u32(&k_full[st]))
+                : "memory");
+        }
+      }
+      if (!ok) {
+        // let the copies this thread issued land before the CTA exits (bounded)
+        const uint64_t t0 = globaltimer_ns();
+        for (long long k = max(0LL, n - C::K_STAGES); k < n; ++k)
+          while (!mbar_try_wait(smem_u32(&k_full[k % C::K_STAGES]), (uint32_t)((k / C::K_STAGES) & 1)) &&
+                 globaltimer_ns() - t0 < 100000000ull) {
+          }
+        if (m > 0)
+          while (!mbar_try_wait(smem_u32(q_full), (uint32_t)((m - 1) & 1)) && globaltimer_ns() - t0 < 100000000ull) {
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      long long m = 0, n = 0;
+      bool ok = true;
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t g_base = smem_u32(sG);
+      const uint32_t dq_tmem = tmem_base + 256;
+      auto mma1 = [&](long long u) -> bool {
+        const int st = (int)(u % C::K_STAGES), xb = (int)(u & 1);
+        if (!mbar_wait(&k_full[st], (uint32_t)((u / C::K_STAGES) & 1), abort_flag, 82)) return false;
+        if (!mbar_wait(&x_empty[xb], (uint32_t)((u >> 1) & 1) ^ 1u, abort_flag, 83)) return false;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(sK + st * C::TILE_BYTES);
+#pragma unroll
+        for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_base + xb * 128, smem_desc_kmajor(q_base + pn * C::PANEL_BYTES + kk * 32, 128),
+                      smem_desc_kmajor(k_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC1, (pn | kk) != 0);
+        umma_commit(&x_full[xb]);
+        return true;
+      };
+      auto mma2 = [&](long long u, bool first) -> bool {
+        const int st = (int)(u % C::K_STAGES), gb = (int)(u & 1);
+        if (!mbar_wait(&g_full[gb], (uint32_t)((u >> 1) & 1), abort_flag, 84)) return false;
+        if (first && !mbar_wait(dq_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 85)) return false;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(sK + st * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // 16 keys per step
+          umma_bf16(dq_tmem,
+                    smem_desc_kmajor(g_base + gb * C::TILE_BYTES + (kk / 4) * C::PANEL_BYTES + (kk % 4) * 32, 128),
+                    smem_desc_mn_sw128(k_base + kk * 16 * 128, C::PANEL_BYTES), C::IDESC2, !(first && kk == 0));
+        umma_commit(&k_empty[st]);
+        umma_commit(&g_empty[gb]);
+        return true;
+      };
+      for (long long slot = blockIdx.x; slot < p.n_slots && ok; slot += gridDim.x) {
+        KlDqItem it;
+        if (!kl_dq_item(slot, p, it) || it.ntiles == 0) continue;
+        if (!(ok = mbar_wait(q_full, (uint32_t)(m & 1), abort_flag, 86))) break;
+        tc_fence_after();
+        for (int j = 0; j < it.ntiles && ok; ++j) {
+          if (!(ok = mma1(n + j))) break;
+          if (j + 1 == it.ntiles) umma_commit(q_empty);  // the query block is free after these
+          if (j > 0 && !(ok = mma2(n + j - 1, j == 1))) break;
+        }
+        if (!ok) break;
+        if (!(ok = mma2(n + it.ntiles - 1, it.ntiles == 1))) break;
+        umma_commit(dq_full);
+        n += it.ntiles;
+        ++m;
+      }
+      umma_commit(mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (8 warps)
+    const int quarter = warp % 4;          // TMEM lane quarter: rows 32 quarter .. of the block
+    const int half = (warp - 2) / 4;       // keys 64 half .. 64 half + 63 of each tile
+    const int mrow = quarter * 32 + lane;  // (t,j) row of the block: t = t0 + mrow / 64
+    const int rsel = quarter >> 1;
+    const int head = mrow % 64;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t g_row0 = smem_u32(sG) + half * C::PANEL_BYTES + mrow * 128;
+    long long m = 0, n = 0;
+    bool ok = true;
+    for (long long slot = blockIdx.x; slot < p.n_slots && ok; slot += gridDim.x) {
+      KlDqItem it;
+      if (!kl_dq_item(slot, p, it)) continue;
+      const long long t = it.t0 + rsel;
+      const bool tv = rsel < it.ntok;
+      uint16_t* dq_dst = p.dq + ((size_t)t * C::H_I + head) * C::D_I + half * 64;
+      if (it.ntiles == 0) {  // no visible key: dq = 0, dw = 0
+        if (tv) {
+#pragma unroll
+          for (int e = 0; e < 64; e += 8) *reinterpret_cast<uint4*>(dq_dst + e) = make_uint4(0u, 0u, 0u, 0u);
+          if (half == 0) p.dw[t * C::H_I + head] = 0;
+        }
+        continue;
+      }
+      const int vis = tv ? causal_vis(it.i0 + rsel, it.Lq, it.Lk) : 0;
+      const float wv = tv ? bf16_bits_to_f32(p.w[t * C::H_I + head]) : 0.f;
+      float dw = 0.f;
+      for (int j = 0; j < it.ntiles; ++j, ++n) {
+        const int st = (int)(n % C::K_STAGES), xb = (int)(n & 1);
+        // the tile's g values arrive with its keys
+        if (!(ok = mbar_wait(&k_full[st], (uint32_t)((n / C::K_STAGES) & 1), abort_flag, 87))) break;
+        if (!(ok = mbar_wait(&x_full[xb], (uint32_t)((n >> 1) & 1), abort_flag, 88))) break;
+        tc_fence_after();
+        float x[64];
+        tmem_ld_x32_sync(tmem_base + lane_off + xb * 128 + half * 64, x);
+        tmem_ld_x32_sync(tmem_base + lane_off + xb * 128 + half * 64 + 32, x + 32);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&x_empty[xb]);
+        const float* gs = sGs + st * (C::GS_BYTES / 4) + rsel * 128 + half * 64;
+        const int s0 = j * 128 + half * 64;
+        if (!(ok = mbar_wait(&g_empty[xb], (uint32_t)((n >> 1) & 1) ^ 1u, abort_flag, 89))) break;
+        const uint32_t g_row = g_row0 + xb * C::TILE_BYTES;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of this row's panel: keys 8q .. 8q+7
+          const float4 ga = *reinterpret_cast<const float4*>(gs + q * 8);
+          const float4 gb = *reinterpret_cast<const float4*>(gs + q * 8 + 4);
+          const float gq[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = q * 8 + 2 * e;
+            const float g0 = (s0 + c < vis) ? gq[2 * e] : 0.f;
+            const float g1 = (s0 + c + 1 < vis) ? gq[2 * e + 1] : 0.f;
+            dw = fmaf(g0, fmaxf(x[c], 0.f), dw);
+            dw = fmaf(g1, fmaxf(x[c + 1], 0.f), dw);
+            const float v0 = x[c] > 0.f ? g0 * wv : 0.f;
+            const float v1 = x[c + 1] > 0.f ? g1 * wv : 0.f;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(g_row + ((q ^ (mrow & 7)) * 16)),
+                       "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+        }
+        fence_proxy_async_shared();  // the tensor core reads G through the async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&g_full[xb]);
+      }
+      if (!ok) break;
+      // dq of this thread's (t,j): 64 of its 128 columns, as bf16
+      if (!(ok = mbar_wait(dq_full, (uint32_t)(m & 1), abort_flag, 90))) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 64; c += 32) {
+        float v[32];
+        tmem_ld_x32_sync(tmem_base + lane_off + 256 + half * 64 + c, v);
+        if (tv) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 o;
+            uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[e + 2 * f], v[e + 2 * f + 1]);
+              po[f] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(dq_dst + c + e) = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_empty);
+      // dw = (keys 0..63 half) + (keys 64..127 half), added in this order
+      if (half == 1) {
+        if (!(ok = mbar_wait(dw_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 91))) break;
+        sDw[mrow] = dw;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dw_full);
+      } else {
+        if (!(ok = mbar_wait(dw_full, (uint32_t)(m & 1), abort_flag, 92))) break;
+        const float total = dw + sDw[mrow];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dw_empty);
+        if (tv) {
+          __nv_bfloat16 b = __float2bfloat16_rn(total);
+          p.dw[t * C::H_I + head] = *reinterpret_cast<uint16_t*>(&b);
+        }
+      }
+      ++m;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
 // q_idx [rows, 128] -> q_idx^T [128, rows] (bf16), 32 x 32 tiles through shared memory
 __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, long long rows) {
   __shared__ uint16_t t[32][33];
@@ -417,6 +776,44 @@ int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const
   const long long grid = std::min<long long>(p.n_items, (long long)sm_count());
   if (grid <= 0) return DSA_OK;
   dsa::kl_dk_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, tqt, p);
+  return last_launch_status();
+}
+
+// dw and dq_idx of the row chunk [r0, r1) for H_I = 64, d_I = 128 (row-stationary, above).
+int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
+                    long long total_q, long long total_k, long long r0, long long r1, const float* g, long long ld,
+                    void* dq, void* dw, cudaStream_t s) {
+  using C = dsa::KlDqCfg;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    C::SMEM_BYTES);
+        e_ != cudaSuccess)
+      return cuda_fail(e_);
+    attr_done = true;
+  }
+  CUtensorMap tk, tq;
+  int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)total_k, 128, 256, 128, 64, 128);
+  if (st != DSA_OK) return st;
+  st = make_tmap_bf16_2d(&tq, q_idx, (uint64_t)total_q * 64, 128, 256, 128, 64, 128);
+  if (st != DSA_OK) return st;
+  dsa::KlDqParams p;
+  p.w = static_cast<const uint16_t*>(w);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.row_begin = r0;
+  p.row_end = r1;
+  p.g = g;
+  p.ld = ld;
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dw = static_cast<uint16_t*>(dw);
+  // an upper bound on the 2-row blocks (each sequence piece rounds up once)
+  p.n_blocks = (r1 - r0 + 1) / 2 + batch;
+  const long long grid = std::min<long long>(p.n_blocks, (long long)sm_count());
+  if (grid <= 0) return DSA_OK;
+  p.n_slots = (p.n_blocks + grid - 1) / grid * grid;
+  dsa::kl_dq_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, p);
   return last_launch_status();
 }
 

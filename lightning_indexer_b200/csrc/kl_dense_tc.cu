@@ -278,32 +278,20 @@ struct KlTgtItem {
   int ntok, i0, Lq, Lk, kbase, ntiles;
 };
 
-// Items in snake order over rounds of gridDim.x (CTA c takes position c of even rounds and
-// gridDim.x - 1 - c of odd ones); within the order blocks run from the chunk's last one,
-// so long rows come first.
+// Items in snake order over rounds of gridDim.x; within the order blocks run from the
+// chunk's last one, so long rows come first.
 __device__ __forceinline__ bool kl_tgt_item(long long item, const KlTgtParams& p, KlTgtItem& it) {
-  const long long G = gridDim.x, k = item / G, pos = item % G;
-  const long long idx = k * G + ((k & 1) ? G - 1 - pos : pos);
-  if (idx >= p.n_blocks) return false;
-  long long r = p.n_blocks - 1 - idx;
-  for (int b = 0; b < p.batch; ++b) {
-    const long long lo = max((long long)p.cu_q[b], p.row_begin), hi = min((long long)p.cu_q[b + 1], p.row_end);
-    if (hi <= lo) continue;
-    const long long nb = (hi - lo + 7) / 8;
-    if (r < nb) {
-      it.t0 = lo + r * 8;
-      it.ntok = (int)min(8LL, hi - it.t0);
-      it.i0 = (int)(it.t0 - p.cu_q[b]);
-      it.Lq = p.cu_q[b + 1] - p.cu_q[b];
-      it.Lk = p.cu_k[b + 1] - p.cu_k[b];
-      it.kbase = p.cu_k[b];
-      const int vis_last = min(max(it.i0 + it.ntok - 1 + it.Lk - it.Lq + 1, 0), it.Lk);
-      it.ntiles = (vis_last + 127) / 128;
-      return true;
-    }
-    r -= nb;
-  }
-  return false;
+  RowBlock rb;
+  if (!chunk_row_block<8>(snake_slot(item), p.cu_q, p.cu_k, p.batch, p.row_begin, p.row_end, p.n_blocks, rb))
+    return false;
+  it.t0 = rb.t0;
+  it.ntok = rb.ntok;
+  it.i0 = rb.i0;
+  it.Lq = rb.Lq;
+  it.Lk = rb.Lk;
+  it.kbase = rb.kbase;
+  it.ntiles = (causal_vis(it.i0 + it.ntok - 1, it.Lq, it.Lk) + 127) / 128;
+  return true;
 }
 
 struct KlTgtCfg {
@@ -501,7 +489,7 @@ __global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
       for (int rr = 0; rr < 4; ++rr) {
         const int u = 4 * half + rr;
         const bool valid = u < it.ntok;
-        vis[rr] = valid ? min(max(it.i0 + u + it.Lk - it.Lq + 1, 0), it.Lk) : 0;
+        vis[rr] = valid ? causal_vis(it.i0 + u, it.Lq, it.Lk) : 0;
         const long long lr = it.t0 + (valid ? u : 0) - p.row_begin;
         lI[rr] = p.lseI[lr];
         Irow[rr] = p.scores + lr * p.ld;

@@ -20,7 +20,8 @@
 //   3. row_lse_kernel     log-sum-exp of each I row
 //   4. kl_target_kernel   p from recomputed dense logits, kl[t], g in place [tcgen05 for d = 128,
 //                         Hq/Hkv = 8, Hkv <= 4 (kl_dense_tc.cu); warp MMA otherwise]
-//   5. idx_bwd_row_kernel x recomputed per row; dw, dq_idx (row-stationary) [warp MMA]
+//   5. idx_bwd_row_kernel x recomputed per row; dw, dq_idx (row-stationary) [tcgen05 for
+//                         H_I = 64, d_I = 128 (kl_dq_tc_kernel); warp MMA otherwise]
 //   6. idx_bwd_col_kernel x recomputed per key tile; dk_idx (key-stationary: one CTA per
 //                         key tile and block of 1024 rows owns a partial, then the
 //                         partials are added in a fixed order: no atomics, deterministic)
@@ -622,6 +623,9 @@ int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int
                         const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
                         float* kl_part, cudaStream_t s);
 int kl_parts_sum_launch(const float* kl_part, long long T, float* kl, cudaStream_t s);
+int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
+                    long long total_q, long long total_k, long long r0, long long r1, const float* g, long long ld,
+                    void* dq, void* dw, cudaStream_t s);
 int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const void* w, const int* cu_q,
                     const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
                     long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
@@ -673,7 +677,11 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
                                int batch, long long r0, long long r1, long long T, long long Tk, const float* g,
                                long long ld, int max_seqlen_k, void* dq, void* dw, float* dk_acc, float* dk_part,
                                const void* q_t, cudaStream_t s) {
-  {
+  if constexpr (H_I == 64 && D_I == 128) {
+    // tensor-core row-stationary kernel
+    const int st = kl_dq_tc_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, r0, r1, g, ld, dq, dw, s);
+    if (st != DSA_OK) return st;
+  } else {
     auto kern = dsa::idx_bwd_row_kernel<H_I, D_I>;
     const int smem = 2 * 64 * D_I * 2;
     static bool done = false;
