@@ -13,9 +13,9 @@
 //   epilogue  G = g w [X > 0] -> bf16, written to shared memory in the 128-byte swizzled
 //             K-major layout the tensor core reads (row = key, 16-byte chunk c of a row
 //             at chunk c ^ (row % 8))
-//   MMA2  dk[128 keys x 128 d] += G . (Q_blk^T)^T             (TMEM accumulator)
-// Every operand is K-major: MMA2's B is the same query block transposed, which TMA reads
-// from a transposed copy of q_idx ([d_I, T*H_I], written once per loss call).
+//   MMA2  dk[128 keys x 128 d] += G . Q_blk                   (TMEM accumulator)
+// MMA2's B operand is the same query block read MN-major (d contiguous), so the block is
+// loaded once for both MMAs.
 // MMA1 of the next block is issued before MMA2 of this one, so the tensor pipe computes X
 // while the epilogue turns the previous X into G.  Warp roles: warp 0 TMA producer, warp 1
 // MMA issuer and TMEM owner, warps 2-9 epilogue (one TMEM lane, i.e. one key, per thread;
@@ -75,26 +75,31 @@ struct KlDkCfg {
   static constexpr int H_I = 64, D_I = 128, NTOK = 2, N = NTOK * H_I;  // 128 columns
   static constexpr int TILE_BYTES = 128 * 128 * 2;                      // any 128 x 128 bf16 operand
   static constexpr int PANEL_BYTES = 128 * 128;                         // 128 rows x 128 B
+  static constexpr int Q_STAGES = 3;
   static constexpr int OFF_A = 0;                                       // key tile
-  static constexpr int OFF_Q = OFF_A + TILE_BYTES;                      // 2 stages x (Q_blk, Q_blk^T)
-  static constexpr int STAGE_STRIDE = 2 * TILE_BYTES;
-  static constexpr int OFF_G = OFF_Q + 2 * STAGE_STRIDE;                // 2 G buffers
-  static constexpr int OFF_W = OFF_G + 2 * TILE_BYTES;                  // 2 stages x w of the block's rows
+  static constexpr int OFF_Q = OFF_A + TILE_BYTES;                      // Q_STAGES x Q_blk
+  static constexpr int OFF_G = OFF_Q + Q_STAGES * TILE_BYTES;           // 2 G buffers
+  static constexpr int OFF_W = OFF_G + 2 * TILE_BYTES;                  // Q_STAGES x w of the block's rows
   static constexpr int W_BYTES = 2 * 64 * 2;
-  static constexpr int OFF_BAR = OFF_W + 2 * W_BYTES;
-  static constexpr int NUM_BARS = 2 + 4 + 4 + 4 + 2 + 1;
+  static constexpr int OFF_GS = OFF_W + Q_STAGES * W_BYTES;            // Q_STAGES x g of the block's rows
+  static constexpr int GS_BYTES = 2 * 128 * 4;
+  static constexpr int OFF_BAR = OFF_GS + Q_STAGES * GS_BYTES;
+  // a_full, a_empty, q_full[S], q_empty[S], x_full[2], x_empty[2], g_full[2], g_empty[2],
+  // dk_full, dk_empty, done
+  static constexpr int NUM_BARS = 2 + 2 * Q_STAGES + 8 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter: one per block row (64 columns)
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
   static constexpr int TMEM_COLS = 512;  // X buffers [0,128) [128,256), dk [256,384)
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, 128);
+  static constexpr uint32_t IDESC2 = idesc_bf16_f32(128, 128) | kIdescBMnMajor;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
     kl_dk_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
-                    const __grid_constant__ CUtensorMap tmap_qt, const KlDkParams p) {
+                    const KlDkParams p) {
   using C = KlDkCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -104,15 +109,15 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
-  uint64_t* q_full = bars + 2;   // [2]
-  uint64_t* q_empty = bars + 4;  // [2]
-  uint64_t* x_full = bars + 6;   // [2]
-  uint64_t* x_empty = bars + 8;  // [2]
-  uint64_t* g_full = bars + 10;   // [2]
-  uint64_t* g_empty = bars + 12;  // [2]
-  uint64_t* dk_full = bars + 14;
-  uint64_t* dk_empty = bars + 15;
-  uint64_t* mma_done = bars + 16;
+  uint64_t* q_full = bars + 2;                  // [Q_STAGES]
+  uint64_t* q_empty = q_full + C::Q_STAGES;     // [Q_STAGES]
+  uint64_t* x_full = q_empty + C::Q_STAGES;     // [2]
+  uint64_t* x_empty = x_full + 2;               // [2]
+  uint64_t* g_full = x_full + 4;                // [2]
+  uint64_t* g_empty = x_full + 6;               // [2]
+  uint64_t* dk_full = x_full + 8;
+  uint64_t* dk_empty = x_full + 9;
+  uint64_t* mma_done = x_full + 10;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const int warp = threadIdx.x / 32;
@@ -121,9 +126,11 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(a_full, 1);
     mbar_init(a_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::Q_STAGES; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&x_full[i], 1);
       mbar_init(&x_empty[i], C::EPI_WARPS);
     }
@@ -144,7 +151,6 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_q);
-    tma_prefetch_desc(&tmap_qt);
   }
   tc_fence_before();
   __syncthreads();
@@ -154,7 +160,7 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      long long n = 0;  // blocks loaded so far (stage n % 2)
+      long long n = 0;  // blocks loaded so far (stage n % Q_STAGES)
       long long m = 0;  // non-empty items so far
       bool ok = true;
       for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -166,30 +172,37 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
           tma_load_2d(sA + pn * C::PANEL_BYTES, &tmap_k, a_full, pn * 64, it.kbase + it.tile * 128);
         ++m;
         for (int i = 0; i < it.nb; ++i, ++n) {
-          const int st = (int)(n & 1);
-          if (!(ok = mbar_wait(&q_empty[st], (uint32_t)((n >> 1) & 1) ^ 1u, abort_flag, 41))) break;
+          const int st = (int)(n % C::Q_STAGES);
+          if (!(ok = mbar_wait(&q_empty[st], (uint32_t)((n / C::Q_STAGES) & 1) ^ 1u, abort_flag, 41))) break;
           const long long t0 = it.qlo + 2 * i;
           // head weights of the block's rows that exist in the tensor (the second may not)
           const uint32_t wbytes = (uint32_t)(min(2LL, p.total_q - t0) * C::H_I * 2);
-          mbar_arrive_expect_tx(&q_full[st], 2 * C::TILE_BYTES + wbytes);
-          uint8_t* sq = sQ + st * C::STAGE_STRIDE;
+          // g of the block's rows in the item for the tile's keys (rows end at ld; ld % 4 == 0)
+          const int grows = (int)min(2LL, it.qhi - t0);
+          const uint32_t gbytes = (uint32_t)(min(128LL, p.ld - (long long)it.tile * 128) * 4);
+          mbar_arrive_expect_tx(&q_full[st], C::TILE_BYTES + wbytes + grows * gbytes);
+          uint8_t* sq = sQ + st * C::TILE_BYTES;
           const int col = (int)(t0 * C::H_I);  // first (t, j) row of the block
-          for (int pn = 0; pn < 2; ++pn) {
-            tma_load_2d(sq + pn * C::PANEL_BYTES, &tmap_q, &q_full[st], pn * 64, col);
-            tma_load_2d(sq + C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_qt, &q_full[st], col + pn * 64, 0);
-          }
+          for (int pn = 0; pn < 2; ++pn) tma_load_2d(sq + pn * C::PANEL_BYTES, &tmap_q, &q_full[st], pn * 64, col);
           asm volatile(
               "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                   smem_u32(smem + C::OFF_W + st * C::W_BYTES)),
               "l"(p.w + t0 * C::H_I), "r"(wbytes), "r"(smem_u32(&q_full[st]))
               : "memory");
+          for (int r = 0; r < grows; ++r)
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                    smem_u32(smem + C::OFF_GS + st * C::GS_BYTES + r * 512)),
+                "l"(p.g + (t0 + r - p.row_begin) * p.ld + (long long)it.tile * 128), "r"(gbytes),
+                "r"(smem_u32(&q_full[st]))
+                : "memory");
         }
       }
       if (!ok) {
         // drain: the loads this thread issued land before the CTA can exit
         const uint64_t t0 = globaltimer_ns();
-        for (int i = 0; i < 2; ++i)
-          while (!mbar_try_wait(smem_u32(&q_full[i]), (uint32_t)(((n - (n & 1) + i) >> 1) & 1)) &&
+        for (long long k = max(0LL, n - C::Q_STAGES); k < n; ++k)
+          while (!mbar_try_wait(smem_u32(&q_full[k % C::Q_STAGES]), (uint32_t)((k / C::Q_STAGES) & 1)) &&
                  globaltimer_ns() - t0 < 200000000ull) {
           }
       }
@@ -205,19 +218,19 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
       const uint32_t g_base = smem_u32(sG);
       const uint32_t dk_tmem = tmem_base + 256;
       auto mma1 = [&](long long blk) -> bool {
-        const int st = (int)(blk & 1);
-        if (!mbar_wait(&q_full[st], (uint32_t)((blk >> 1) & 1), abort_flag, 42)) return false;
-        if (!mbar_wait(&x_empty[st], (uint32_t)((blk >> 1) & 1) ^ 1u, abort_flag, 43)) return false;
+        const int st = (int)(blk % C::Q_STAGES), xb = (int)(blk & 1);
+        if (!mbar_wait(&q_full[st], (uint32_t)((blk / C::Q_STAGES) & 1), abort_flag, 42)) return false;
+        if (!mbar_wait(&x_empty[xb], (uint32_t)((blk >> 1) & 1) ^ 1u, abort_flag, 43)) return false;
         tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + st * C::STAGE_STRIDE);
-        const uint32_t d_tmem = tmem_base + st * 128;
+        const uint32_t q_base = smem_u32(sQ + st * C::TILE_BYTES);
+        const uint32_t d_tmem = tmem_base + xb * 128;
 #pragma unroll
         for (int pn = 0; pn < 2; ++pn)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(d_tmem, smem_desc_kmajor(a_base + pn * C::PANEL_BYTES + kk * 32, 128),
                       smem_desc_kmajor(q_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC, (pn | kk) != 0);
-        umma_commit(&x_full[st]);
+        umma_commit(&x_full[xb]);
         return true;
       };
       for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -239,16 +252,15 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
           if (i == 0 && !(ok = mbar_wait(dk_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 46))) break;
           tc_fence_after();
           const long long blk = n0 + i;
-          const uint32_t qt_base = smem_u32(sQ + (int)(blk & 1) * C::STAGE_STRIDE + C::TILE_BYTES);
+          const int qs = (int)(blk % C::Q_STAGES);
+          const uint32_t q_base = smem_u32(sQ + qs * C::TILE_BYTES);
 #pragma unroll
-          for (int pn = 0; pn < 2; ++pn)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(dk_tmem, smem_desc_kmajor(g_base + gb * C::TILE_BYTES + pn * C::PANEL_BYTES + kk * 32, 128),
-                        smem_desc_kmajor(qt_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC,
-                        (i | pn | kk) != 0);
+          for (int kk = 0; kk < 8; ++kk)  // 16 (t,j) rows of the block per step
+            umma_bf16(dk_tmem,
+                      smem_desc_kmajor(g_base + gb * C::TILE_BYTES + (kk / 4) * C::PANEL_BYTES + (kk % 4) * 32, 128),
+                      smem_desc_mn_sw128(q_base + kk * 16 * 128, C::PANEL_BYTES), C::IDESC2, (i | kk) != 0);
           umma_commit(&g_empty[gb]);
-          umma_commit(&q_empty[(int)(blk & 1)]);
+          umma_commit(&q_empty[qs]);
           ++gcount;
         }
         if (!ok) break;
@@ -275,32 +287,25 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
       const int s = it.tile * 128 + r;  // this thread's key (sequence-local)
       const int dvis = it.Lk - it.Lq + 1;
       const long long q0 = p.cu_q[it.b];
-      // g of this warp's row and this thread's key; 0 past the item or the row's visible keys
-      auto load_g = [&](int blk) -> float {
-        const long long t = it.qlo + 2 * blk + half;
-        const int vis = min(max((int)(t - q0) + dvis, 0), it.Lk);
-        return (t < it.qhi && s < vis) ? p.g[(t - p.row_begin) * p.ld + s] : 0.f;
-      };
-      float g_next = load_g(0);  // one block ahead, so the load's latency hides behind a block
       for (int i = 0; i < it.nb; ++i, ++n) {
         const long long t = it.qlo + 2 * i + half;  // this warp's query row
-        const bool tv = t < it.qhi;  // else its G columns are 0
-        const float gv = g_next;
-        if (i + 1 < it.nb) g_next = load_g(i + 1);
-        const int st = (int)(n & 1);
-        // the block's head weights arrive with its query tiles: observe that phase here too
+        // its G columns are 0 past the item or the row's visible keys
+        const bool tv = t < it.qhi && s < min(max((int)(t - q0) + dvis, 0), it.Lk);
+        const int st = (int)(n % C::Q_STAGES), xb = (int)(n & 1);
+        // the block's head weights arrive with its query tile: observe that phase here too
         // (the stage cannot be refilled before this block's G is written, so the phase seen
         // is this block's)
-        if (!(ok = mbar_wait(&q_full[st], (uint32_t)((n >> 1) & 1), abort_flag, 50))) break;
-        const uint16_t* sW = reinterpret_cast<const uint16_t*>(smem + C::OFF_W + st * C::W_BYTES) + half * C::H_I;
-        if (!(ok = mbar_wait(&x_full[st], (uint32_t)((n >> 1) & 1), abort_flag, 47))) break;
+        if (!(ok = mbar_wait(&q_full[st], (uint32_t)((n / C::Q_STAGES) & 1), abort_flag, 50))) break;
+        const uint4* sW = reinterpret_cast<const uint4*>(smem + C::OFF_W + st * C::W_BYTES + half * C::H_I * 2);
+        const float gv = tv ? reinterpret_cast<const float*>(smem + C::OFF_GS + st * C::GS_BYTES)[half * 128 + r] : 0.f;
+        if (!(ok = mbar_wait(&x_full[xb], (uint32_t)((n >> 1) & 1), abort_flag, 47))) break;
         tc_fence_after();
         float x[64];
-        tmem_ld_x32_sync(tmem_base + lane_off + st * 128 + half * 64, x);
-        tmem_ld_x32_sync(tmem_base + lane_off + st * 128 + half * 64 + 32, x + 32);
+        tmem_ld_x32_sync(tmem_base + lane_off + xb * 128 + half * 64, x);
+        tmem_ld_x32_sync(tmem_base + lane_off + xb * 128 + half * 64 + 32, x + 32);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&x_empty[st]);
+        if (lane == 0) mbar_arrive(&x_empty[xb]);
         // G buffer gb may be overwritten once the MMA2 that read it two blocks ago is done
         const int gb = (int)(gcount & 1);
         if (!(ok = mbar_wait(&g_empty[gb], (uint32_t)((gcount >> 1) & 1) ^ 1u, abort_flag, 48))) break;
@@ -308,11 +313,13 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of this row's panel: columns 8q .. 8q+7
           uint32_t pk[4];
+          const uint4 w8 = sW[q];  // head weights of columns 8q .. 8q+7
+          const uint32_t wp[4] = {w8.x, w8.y, w8.z, w8.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = q * 8 + 2 * e;
-            const float v0 = (tv && x[c] > 0.f) ? gv * bf16_bits_to_f32(sW[c]) : 0.f;
-            const float v1 = (tv && x[c + 1] > 0.f) ? gv * bf16_bits_to_f32(sW[c + 1]) : 0.f;
+            const float v0 = x[c] > 0.f ? gv * __uint_as_float(wp[e] << 16) : 0.f;
+            const float v1 = x[c + 1] > 0.f ? gv * __uint_as_float(wp[e] & 0xFFFF0000u) : 0.f;
             __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
             pk[e] = *reinterpret_cast<uint32_t*>(&b2);
           }
@@ -712,32 +719,12 @@ __global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
-// q_idx [rows, 128] -> q_idx^T [128, rows] (bf16), 32 x 32 tiles through shared memory
-__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, long long rows) {
-  __shared__ uint16_t t[32][33];
-  const long long r0 = (long long)blockIdx.x * 32;
-  const int c0 = blockIdx.y * 32;
-  for (int y = threadIdx.y; y < 32; y += blockDim.y)
-    if (r0 + y < rows) t[y][threadIdx.x] = src[(r0 + y) * 128 + c0 + threadIdx.x];
-  __syncthreads();
-  for (int y = threadIdx.y; y < 32; y += blockDim.y)
-    if (r0 + threadIdx.x < rows) dst[(long long)(c0 + y) * rows + r0 + threadIdx.x] = t[threadIdx.x][y];
-}
-
 }  // namespace dsa
 
 namespace dsa_host {
 
-int kl_transpose_q_launch(const void* q_idx, void* q_t, long long rows, cudaStream_t s) {
-  if (rows <= 0) return DSA_OK;
-  dsa::transpose_bf16_kernel<<<dim3((unsigned)((rows + 31) / 32), 4), dim3(32, 8), 0, s>>>(
-      static_cast<const uint16_t*>(q_idx), static_cast<uint16_t*>(q_t), rows);
-  return last_launch_status();
-}
-
-// dk partials of the row chunk [r0, r1) for H_I = 64, d_I = 128 (see the file comment);
-// q_t is q_idx transposed ([128, total_q * 64]).
-int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const void* w, const int* cu_q,
+// dk partials of the row chunk [r0, r1) for H_I = 64, d_I = 128 (see the file comment).
+int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q,
                     const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
                     long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
                     long long part_stride, cudaStream_t s) {
@@ -750,12 +737,10 @@ int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const
       return cuda_fail(e_);
     attr_done = true;
   }
-  CUtensorMap tk, tq, tqt;
+  CUtensorMap tk, tq;
   int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)total_k, 128, 256, 128, 64, 128);
   if (st != DSA_OK) return st;
   st = make_tmap_bf16_2d(&tq, q_idx, (uint64_t)total_q * 64, 128, 256, 128, 64, 128);
-  if (st != DSA_OK) return st;
-  st = make_tmap_bf16_2d(&tqt, q_t, 128, (uint64_t)total_q * 64, (uint64_t)total_q * 64 * 2, 128, 64, 128);
   if (st != DSA_OK) return st;
   dsa::KlDkParams p;
   p.w = static_cast<const uint16_t*>(w);
@@ -775,7 +760,7 @@ int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const
   p.part_stride = part_stride;
   const long long grid = std::min<long long>(p.n_items, (long long)sm_count());
   if (grid <= 0) return DSA_OK;
-  dsa::kl_dk_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, tqt, p);
+  dsa::kl_dk_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, p);
   return last_launch_status();
 }
 

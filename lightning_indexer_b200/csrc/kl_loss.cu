@@ -614,7 +614,6 @@ int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const in
                    int H_I, int d_I, long long row_begin, long long row_end, float* scores, long long ld,
                    cudaStream_t stream);
 int f32_to_bf16_launch(const float* src, void* dst, long long n, cudaStream_t stream);
-int kl_transpose_q_launch(const void* q_idx, void* q_t, long long rows, cudaStream_t s);
 int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
                      cudaStream_t s);
@@ -626,7 +625,7 @@ int kl_parts_sum_launch(const float* kl_part, long long T, float* kl, cudaStream
 int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
                     long long total_q, long long total_k, long long r0, long long r1, const float* g, long long ld,
                     void* dq, void* dw, cudaStream_t s);
-int kl_dk_tc_launch(const void* q_idx, const void* q_t, const void* k_idx, const void* w, const int* cu_q,
+int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q,
                     const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
                     long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
                     long long part_stride, cudaStream_t s);
@@ -635,7 +634,6 @@ struct KLWorkspace {
   float* lse_att;  // [T, Hq]
   float* dk_acc;   // [Tk, d_I]
   float* dk_part;  // [ceil(chunk_rows / KL_COL_ROWS), Tk, d_I] per-row-block partials of dk
-  uint16_t* q_t;   // [d_I, T * H_I] q_idx transposed (tensor-core dk path, H_I = 64, d_I = 128)
   float* lseI;     // [chunk_rows]
   float* scores;   // [chunk_rows, ld]
   float* kl_part;  // [T, 4] per-key-quarter partials of kl (tensor-core target path)
@@ -656,8 +654,6 @@ KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_s
   off += r256((size_t)Tk * d_I * 4);
   w.dk_part = reinterpret_cast<float*>(p + off);
   off += r256((size_t)((chunk_rows + dsa::KL_COL_ROWS - 1) / dsa::KL_COL_ROWS) * Tk * d_I * 4);
-  w.q_t = reinterpret_cast<uint16_t*>(p + off);
-  off += r256((size_t)T * 64 * d_I * 2);
   w.lseI = reinterpret_cast<float*>(p + off);
   off += r256((size_t)chunk_rows * 4);
   w.scores = reinterpret_cast<float*>(p + off);
@@ -676,7 +672,7 @@ template <int H_I, int D_I>
 static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                                int batch, long long r0, long long r1, long long T, long long Tk, const float* g,
                                long long ld, int max_seqlen_k, void* dq, void* dw, float* dk_acc, float* dk_part,
-                               const void* q_t, cudaStream_t s) {
+                               cudaStream_t s) {
   if constexpr (H_I == 64 && D_I == 128) {
     // tensor-core row-stationary kernel
     const int st = kl_dq_tc_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, r0, r1, g, ld, dq, dw, s);
@@ -697,7 +693,7 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
   const long long part_stride = Tk * D_I;
   if constexpr (H_I == 64 && D_I == 128) {
     // tensor-core key-stationary kernel
-    const int st = kl_dk_tc_launch(q_idx, q_t, k_idx, w, cu_q, cu_k, batch, T, Tk, max_seqlen_k, r0, r1, g, ld,
+    const int st = kl_dk_tc_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, max_seqlen_k, r0, r1, g, ld,
                                    dsa::KL_COL_ROWS, dk_part, part_stride, s);
     if (st != DSA_OK) return st;
   } else {
@@ -770,10 +766,6 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
       if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
     }
   }
-  if (H_I == 64 && d_I == 128) {
-    const int st = kl_transpose_q_launch(q_idx, W.q_t, T * 64, s);
-    if (st != DSA_OK) return st;
-  }
   const float inv_T = T > 0 ? 1.f / (float)T : 0.f;
   // 4. on tensor cores for d = 128 and 8 query heads per KV head (at most 4 KV heads)
   const bool target_tc = d == 128 && Hq == 8 * Hkv && Hkv <= 4;
@@ -818,7 +810,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
 #define DSA_KLB(HI, DI)                                                                                   \
   if (H_I == HI && d_I == DI) {                                                                          \
     st = kl_backward_kernels<HI, DI>(q_idx, k_idx, w, cu_q, cu_k, batch, r0, r1, T, Tk, W.scores, ld,         \
-                                     max_seqlen_k, dq, dw, W.dk_acc, W.dk_part, W.q_t, s);               \
+                                     max_seqlen_k, dq, dw, W.dk_acc, W.dk_part, s);               \
     if (st != DSA_OK) return st;                                                                         \
   } else
     DSA_KLB(64, 128) DSA_KLB(32, 128) DSA_KLB(16, 128) { return DSA_ERR_UNSUPPORTED; }
