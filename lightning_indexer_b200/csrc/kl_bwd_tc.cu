@@ -21,6 +21,7 @@
 // MMA issuer and TMEM owner, warps 2-9 epilogue (one TMEM lane, i.e. one key, per thread;
 // two warps per lane quarter, one per query row of the block).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -364,19 +365,23 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
 // Row-stationary half of the same backward (H_I = 64, d_I = 128):
 //   dw[t,j]     = sum_s g[t,s] max(0, x[t,j,s])
 //   dq_idx[t,j] = sum_s g[t,s] w[t,j] [x[t,j,s] > 0] k_idx[s]
+// Both come from one product: with u[t,j] = sum_s g[t,s] [x[t,j,s] > 0] k_idx[s],
+// dq_idx = w u, and since x is linear in q_idx, dw = sum_s g [x > 0] (q_idx . k_idx[s])
+// = q_idx[t,j] . u[t,j], a 128-term dot per (t,j) instead of a term per key.
 // One work item is 2 query rows of one sequence of the row chunk (M = 2 x 64 (t,j) pairs
 // = 128 TMEM lanes); the item's key tiles of 128 stream through three stages, each with
 // the g values of its two rows.  Per key tile:
 //   MMA1  X[128 (t,j) x 128 keys] = Q_blk . K_tile^T       (TMEM, two buffers)
-//   epilogue  dw += g max(0, X) (thread-local: one (t,j) per lane), G = g w [X > 0] -> bf16
-//             in the 128-byte swizzled K-major layout (K = keys)
-//   MMA2  dq[128 (t,j) x 128 d] += G . K_tile             (TMEM accumulator)
+//   epilogue  G = g [X > 0] -> bf16 in the 128-byte swizzled K-major layout (K = keys)
+//   MMA2  u[128 (t,j) x 128 d] += G . K_tile              (TMEM accumulator)
+// and per item dq_idx = w u, dw = q_idx . u (one (t,j) per TMEM lane).
 // MMA2's B operand is the key tile itself read MN-major (d contiguous), so no transposed
 // copy of k_idx is needed.  MMA1 of the next tile is issued before MMA2 of this one.
 // Warps: 0 TMA, 1 MMA issuer and TMEM owner, 2-9 epilogue (two per lane quarter, one per
 // 64-key half of the tile; the two dw halves meet in shared memory, added in a fixed order).
 struct KlDqParams {
-  const uint16_t* w;  // [T, 64] bf16
+  const uint16_t* q_idx;  // [T, 64, 128] bf16
+  const uint16_t* w;      // [T, 64] bf16
   const int* cu_q;
   const int* cu_k;
   int batch;
@@ -625,7 +630,6 @@ __global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
       }
       const int vis = tv ? causal_vis(it.i0 + rsel, it.Lq, it.Lk) : 0;
       const float wv = tv ? bf16_bits_to_f32(p.w[t * C::H_I + head]) : 0.f;
-      float dw = 0.f;
       for (int j = 0; j < it.ntiles; ++j, ++n) {
         const int st = (int)(n % C::K_STAGES), xb = (int)(n & 1);
         // the tile's g values arrive with its keys
@@ -640,38 +644,47 @@ __global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
         if (lane == 0) mbar_arrive(&x_empty[xb]);
         const float* gs = sGs + st * (C::GS_BYTES / 4) + rsel * 128 + half * 64;
         const int s0 = j * 128 + half * 64;
+        const int nvis = vis - s0;  // keys of this half the row sees (all 64 unless at its end)
         if (!(ok = mbar_wait(&g_empty[xb], (uint32_t)((n >> 1) & 1) ^ 1u, abort_flag, 89))) break;
         const uint32_t g_row = g_row0 + xb * C::TILE_BYTES;
+        // G = g [x > 0]; keys past the row's visible ones (only in its last tile) give 0
+        auto write_g = [&](auto masked) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of this row's panel: keys 8q .. 8q+7
-          const float4 ga = *reinterpret_cast<const float4*>(gs + q * 8);
-          const float4 gb = *reinterpret_cast<const float4*>(gs + q * 8 + 4);
-          const float gq[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-          uint32_t pk[4];
+          for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of this row's panel: keys 8q .. 8q+7
+            const float4 ga = *reinterpret_cast<const float4*>(gs + q * 8);
+            const float4 gb = *reinterpret_cast<const float4*>(gs + q * 8 + 4);
+            const float gq[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = q * 8 + 2 * e;
-            const float g0 = (s0 + c < vis) ? gq[2 * e] : 0.f;
-            const float g1 = (s0 + c + 1 < vis) ? gq[2 * e + 1] : 0.f;
-            dw = fmaf(g0, fmaxf(x[c], 0.f), dw);
-            dw = fmaf(g1, fmaxf(x[c + 1], 0.f), dw);
-            const float v0 = x[c] > 0.f ? g0 * wv : 0.f;
-            const float v1 = x[c + 1] > 0.f ? g1 * wv : 0.f;
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-            pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+            for (int e = 0; e < 4; ++e) {
+              const int c = q * 8 + 2 * e;
+              bool k0 = x[c] > 0.f, k1 = x[c + 1] > 0.f;
+              if constexpr (decltype(masked)::value) {
+                k0 = k0 && c < nvis;
+                k1 = k1 && c + 1 < nvis;
+              }
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(k0 ? gq[2 * e] : 0.f, k1 ? gq[2 * e + 1] : 0.f);
+              pk[e] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(g_row + ((q ^ (mrow & 7)) * 16)),
+                         "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                         : "memory");
           }
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(g_row + ((q ^ (mrow & 7)) * 16)),
-                       "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                       : "memory");
-        }
+        };
+        if (nvis >= 64)
+          write_g(std::false_type{});
+        else
+          write_g(std::true_type{});
         fence_proxy_async_shared();  // the tensor core reads G through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&g_full[xb]);
       }
       if (!ok) break;
-      // dq of this thread's (t,j): 64 of its 128 columns, as bf16
+      // u of this thread's (t,j), 64 of its 128 columns: dq_idx = w u (bf16), dw part = q_idx . u
       if (!(ok = mbar_wait(dq_full, (uint32_t)(m & 1), abort_flag, 90))) break;
       tc_fence_after();
+      float dw = 0.f;
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q_idx + ((size_t)t * C::H_I + head) * C::D_I + half * 64);
 #pragma unroll 1
       for (int c = 0; c < 64; c += 32) {
         float v[32];
@@ -679,11 +692,16 @@ __global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
         if (tv) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
+            const uint4 q8 = qrow[(c + e) / 8];
+            const uint32_t qp[4] = {q8.x, q8.y, q8.z, q8.w};
             uint4 o;
             uint32_t* po = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
             for (int f = 0; f < 4; ++f) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[e + 2 * f], v[e + 2 * f + 1]);
+              const float u0 = v[e + 2 * f], u1 = v[e + 2 * f + 1];
+              dw = fmaf(__uint_as_float(qp[f] << 16), u0, dw);
+              dw = fmaf(__uint_as_float(qp[f] & 0xFFFF0000u), u1, dw);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(wv * u0, wv * u1);
               po[f] = *reinterpret_cast<uint32_t*>(&b2);
             }
             *reinterpret_cast<uint4*>(dq_dst + c + e) = o;
@@ -693,7 +711,7 @@ __global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_empty);
-      // dw = (keys 0..63 half) + (keys 64..127 half), added in this order
+      // dw = (d 0..63 half) + (d 64..127 half), added in this order
       if (half == 1) {
         if (!(ok = mbar_wait(dw_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 91))) break;
         sDw[mrow] = dw;
@@ -783,6 +801,7 @@ int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const i
   st = make_tmap_bf16_2d(&tq, q_idx, (uint64_t)total_q * 64, 128, 256, 128, 64, 128);
   if (st != DSA_OK) return st;
   dsa::KlDqParams p;
+  p.q_idx = static_cast<const uint16_t*>(q_idx);
   p.w = static_cast<const uint16_t*>(w);
   p.cu_q = cu_q;
   p.cu_k = cu_k;

@@ -4,14 +4,17 @@
 // Source: Keye-VL-2.0 report summary (mqxn.cn/news/1966), section 1: the dense warm-up
 // trains the indexer against the full attention distribution; its target needs, for every
 // query row t and head h, the log-sum-exp of the dense causal logits
-//   lse[t,h] = log sum_{s visible to t} exp(scale * Q[t,h] . K[s, h / (Hq/Hkv)]).
+//   lse[t,h] = log sum_{s visible to t} exp(scale * Q[t,h] . K[s, h / (Hq/Hkv)]),
+// kept in base 2 (lse / ln 2) for the exp2-based passes that read it.
 //
 // One work item is (16 query rows of one sequence, one KV head g): the A operand is the
 // 16 rows x 8 query heads of group g (M = 128, read by a 3-D TMA box straight from
 // Q [T, Hq, d]), the B operand a tile of 128 keys of K [Tk, Hkv, d] (3-D box, head g),
 // K = d = 128.  Each TMEM lane is one (row, head), so the online log-sum-exp over the keys
 // is thread-local in the epilogue.  Persistent CTAs, warp-specialised: warp 0 TMA, warp 1
-// MMA issuer and TMEM owner, warps 2-5 epilogue; two accumulator buffers, four key stages.
+// MMA issuer and TMEM owner, warps 2-9 epilogue (two per TMEM lane quarter, one per
+// 64-key half of each tile; their two running (max, sum) pairs merge at the item's end);
+// two accumulator buffers, four key stages.
 #include <algorithm>
 
 #include "common.cuh"
@@ -24,7 +27,7 @@ struct KlLseParams {
   int batch;
   int Hq, Hkv;
   float scale_log2;
-  float* lse_out;  // [T, Hq] natural log
+  float* lse_out;  // [T, Hq] base-2 log
   long long n_blocks;  // 16-row blocks over all sequences
   long long n_items;   // n_blocks * Hkv
 };
@@ -64,10 +67,13 @@ struct KlLseCfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + TILE_BYTES;
   static constexpr int OFF_BAR = OFF_B + B_STAGES * TILE_BYTES;
-  static constexpr int NUM_BARS = 2 + 2 * B_STAGES + 4 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  // a_full, a_empty, b_full[S], b_empty[S], acc_full[2], acc_empty[2], done, ml_full, ml_empty
+  static constexpr int NUM_BARS = 2 + 2 * B_STAGES + 4 + 1 + 2;
+  static constexpr int OFF_ML = OFF_BAR + NUM_BARS * 8;  // 128 (max, sum) pairs of the second half
+  static constexpr int OFF_MISC = OFF_ML + 128 * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int THREADS = 64 + 128;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 64 + EPI_WARPS * 32;
   static constexpr int TMEM_COLS = 256;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, 128);
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -89,6 +95,9 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
   uint64_t* acc_full = bars + 2 + 2 * C::B_STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;               // [2]
   uint64_t* mma_done = acc_full + 4;
+  uint64_t* ml_full = acc_full + 5;
+  uint64_t* ml_empty = acc_full + 6;
+  float2* sML = reinterpret_cast<float2*>(smem + C::OFF_ML);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const int warp = threadIdx.x / 32;
@@ -103,9 +112,11 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], C::EPI_WARPS);
     }
     mbar_init(mma_done, 1);
+    mbar_init(ml_full, C::EPI_WARPS / 2);
+    mbar_init(ml_empty, C::EPI_WARPS / 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -183,56 +194,75 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (4 warps)
+    // ------------------------------------------------------------ epilogue (8 warps)
     const int lane_grp = warp % 4;
+    const int half = (warp - 2) / 4;     // keys 64 half .. 64 half + 63 of each tile
     const int r = lane_grp * 32 + lane;  // (row, head) of this thread: row r / 8, head r % 8
     const uint32_t lane_off = (uint32_t)(lane_grp * 32) << 16;
-    long long n = 0;
+    long long n = 0, m = 0;
     bool ok = true;
     for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       KlLseItem it;
       if (!kl_lse_item(item, p, it)) continue;
       const int u = r / 8;
       const bool valid = u < it.ntok;
-      const int vis = min(max(it.i0 + u + it.Lk - it.Lq + 1, 0), it.Lk);
+      const int vis = valid ? causal_vis(it.i0 + u, it.Lq, it.Lk) : 0;
+      // running max of the raw logits and sum of 2^(scale (x - max)) (scale > 0)
       float mx = -INFINITY, l = 0.f;
       for (int j = 0; j < it.ntiles; ++j, ++n) {
         const int ab = (int)(n & 1);
         if (!(ok = mbar_wait(&acc_full[ab], (uint32_t)((n >> 1) & 1), abort_flag, 65))) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          float v[32];
-          tmem_ld_x32_sync(tmem_base + lane_off + ab * 128 + c0, v);
-          const int sb = j * 128 + c0;  // first key of the chunk
-          float cm = -INFINITY;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            v[q] = (sb + q < vis) ? v[q] * p.scale_log2 : -INFINITY;
-            cm = fmaxf(cm, v[q]);
-          }
-          if (cm > mx) {
-            l *= exp2f(mx - cm);  // mx = -inf: l is 0
-            mx = cm;
-          }
-          if (mx > -INFINITY) {
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int q = 0; q < 32; q += 2) {
-              a0 += exp2f(v[q] - mx);
-              a1 += exp2f(v[q + 1] - mx);
-            }
-            l += a0 + a1;
-          }
-        }
+        float v[64];
+        tmem_ld_x32_sync(tmem_base + lane_off + ab * 128 + half * 64, v);
+        tmem_ld_x32_sync(tmem_base + lane_off + ab * 128 + half * 64 + 32, v + 32);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        const int nvis = vis - (j * 128 + half * 64);  // keys of this half the row sees
+        if (nvis < 64) {
+#pragma unroll
+          for (int q = 0; q < 64; ++q)
+            if (q >= nvis) v[q] = -INFINITY;
+        }
+        float cm = v[0];
+#pragma unroll
+        for (int q = 1; q < 64; ++q) cm = fmaxf(cm, v[q]);
+        if (cm > mx) {
+          l *= ex2_ftz((mx - cm) * p.scale_log2);  // mx = -inf: l is 0
+          mx = cm;
+        }
+        if (mx > -INFINITY) {
+          const float nb = -mx * p.scale_log2;
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+          for (int q = 0; q < 64; q += 4) {
+            a0 += ex2_ftz(fmaf(v[q], p.scale_log2, nb));
+            a1 += ex2_ftz(fmaf(v[q + 1], p.scale_log2, nb));
+            a2 += ex2_ftz(fmaf(v[q + 2], p.scale_log2, nb));
+            a3 += ex2_ftz(fmaf(v[q + 3], p.scale_log2, nb));
+          }
+          l += (a0 + a1) + (a2 + a3);
+        }
       }
       if (!ok) break;
-      if (valid)
-        p.lse_out[(it.t0 + u) * p.Hq + it.g * G + (r % 8)] =
-            l > 0.f ? (mx + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      // merge the two halves: (mx, l) of keys 64..127 of each tile into those of 0..63
+      if (half == 1) {
+        if (!(ok = mbar_wait(ml_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 66))) break;
+        sML[r] = make_float2(mx, l);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ml_full);
+      } else {
+        if (!(ok = mbar_wait(ml_full, (uint32_t)(m & 1), abort_flag, 67))) break;
+        const float2 o = sML[r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ml_empty);
+        const float M = fmaxf(mx, o.x);
+        float L = 0.f;
+        if (M > -INFINITY) L = l * ex2_ftz((mx - M) * p.scale_log2) + o.y * ex2_ftz((o.x - M) * p.scale_log2);
+        if (valid) p.lse_out[(it.t0 + u) * p.Hq + it.g * G + (r % 8)] = L > 0.f ? M * p.scale_log2 + log2f(L) : -INFINITY;
+      }
+      ++m;
     }
   }
 
@@ -253,8 +283,8 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
 // the A operand is 128 keys of one KV head (M = 128), the B operand the 8 rows x 8 query
 // heads of that KV head (N = 64, one 3-D TMA box of Q), so a TMEM lane is a key and the
 // sum over heads stays inside a thread.  All Hkv (<= 4) heads of a key tile go to one
-// 256-column TMEM buffer; two buffers alternate.  Eight epilogue warps: warp w reads lanes
-// 32 (w % 4) .. (keys) for rows 4 ((w - 2) / 4) .. + 3.  Each (row, warp-quarter) keeps its
+// 256-column TMEM buffer; two buffers alternate.  Sixteen epilogue warps: warp w reads lanes
+// 32 (w % 4) .. (keys) for rows 2 ((w - 2) / 4) .. + 1.  Each (row, warp-quarter) keeps its
 // own partial of kl[t], written once to kl_part[t][quarter] (a fixed-order sum follows).
 struct KlTgtParams {
   const int* cu_q;
@@ -263,7 +293,7 @@ struct KlTgtParams {
   int Hq, Hkv;
   float scale_log2;
   long long row_begin, row_end;
-  const float* lse_att;  // [T, Hq] natural log
+  const float* lse_att;  // [T, Hq] base-2 log
   const float* lseI;     // [row_end - row_begin]
   float* scores;         // [row_end - row_begin, ld]: I in, g out
   long long ld;
@@ -310,7 +340,9 @@ struct KlTgtCfg {
   static constexpr int NUM_BARS = 2 + 4 + 2 * B_STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARPS = 16;
+  static constexpr int ROWS_PER_WARP = 8 / (EPI_WARPS / 4);
+  static_assert(ROWS_PER_WARP == 2, "one 16-column TMEM load per KV head and warp");
   static constexpr int THREADS = 64 + EPI_WARPS * 32;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_COLS = 256;
@@ -470,24 +502,24 @@ __global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (8 warps)
+    // ------------------------------------------------------------ epilogue (16 warps)
+    constexpr int R = C::ROWS_PER_WARP;
     const int quarter = warp % 4;
-    const int half = (warp - 2) / 4;  // rows 4 half .. 4 half + 3
+    const int rgrp = (warp - 2) / 4;  // rows R rgrp .. R rgrp + R - 1
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float inv_Hq = 1.f / (float)p.Hq;
-    constexpr float kLog2e = 1.4426950408889634f;
     long long m = 0, nt = 0;
     bool ok = true;
     for (long long item = blockIdx.x; item < p.n_slots && ok; item += gridDim.x) {
       KlTgtItem it;
       if (!kl_tgt_item(item, p, it)) continue;
       const int lb = (int)(m & 1);
-      int vis[4];
-      float lI[4], kl[4];
-      float* Irow[4];
+      int vis[R];
+      float lI[R], kl[R];
+      float* Irow[R];
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const int u = 4 * half + rr;
+      for (int rr = 0; rr < R; ++rr) {
+        const int u = R * rgrp + rr;
         const bool valid = u < it.ntok;
         vis[rr] = valid ? causal_vis(it.i0 + u, it.Lq, it.Lk) : 0;
         const long long lr = it.t0 + (valid ? u : 0) - p.row_begin;
@@ -496,32 +528,35 @@ __global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
         kl[rr] = 0.f;
       }
       if (!(ok = mbar_wait(&l_full[lb], (uint32_t)((m >> 1) & 1), abort_flag, 76))) break;
-      const float* Lrow = sL + lb * (C::L_BYTES / 4) + 4 * half * p.Hq;
+      const float* Lrow = sL + lb * (C::L_BYTES / 4) + R * rgrp * p.Hq;
       for (int j = 0; j < it.ntiles; ++j, ++nt) {
         const int ab = (int)(nt & 1);
         const int key = j * 128 + quarter * 32 + lane;
-        float Iv[4];
+        float Iv[R];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) Iv[rr] = key < vis[rr] ? Irow[rr][key] : 0.f;
+        for (int rr = 0; rr < R; ++rr) Iv[rr] = key < vis[rr] ? Irow[rr][key] : 0.f;
         if (!(ok = mbar_wait(&acc_full[ab], (uint32_t)((nt >> 1) & 1), abort_flag, 77))) break;
         tc_fence_after();
-        float pr[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int g = 0; g < Hkv; ++g) {
-          float v[32];
-          tmem_ld_x32_sync(tmem_base + lane_off + ab * C::ACC_COLS + g * 64 + half * 32, v);
+        float pr[R];
 #pragma unroll
-          for (int rr = 0; rr < 4; ++rr) {
+        for (int rr = 0; rr < R; ++rr) pr[rr] = 0.f;
+        for (int g = 0; g < Hkv; ++g) {
+          float v[8 * R];
+          tmem_ld_x16_sync(tmem_base + lane_off + ab * C::ACC_COLS + g * 64 + rgrp * 8 * R, v);
+#pragma unroll
+          for (int rr = 0; rr < R; ++rr) {
+            // 2^(scale log2(e) x - lse2) of the 8 heads of group g, summed
             const float4 La = *reinterpret_cast<const float4*>(Lrow + rr * p.Hq + g * 8);
             const float4 Lb = *reinterpret_cast<const float4*>(Lrow + rr * p.Hq + g * 8 + 4);
             const float* x = v + rr * 8;
-            float a0 = exp2f(fmaf(x[0], p.scale_log2, -La.x * kLog2e));
-            float a1 = exp2f(fmaf(x[1], p.scale_log2, -La.y * kLog2e));
-            a0 += exp2f(fmaf(x[2], p.scale_log2, -La.z * kLog2e));
-            a1 += exp2f(fmaf(x[3], p.scale_log2, -La.w * kLog2e));
-            a0 += exp2f(fmaf(x[4], p.scale_log2, -Lb.x * kLog2e));
-            a1 += exp2f(fmaf(x[5], p.scale_log2, -Lb.y * kLog2e));
-            a0 += exp2f(fmaf(x[6], p.scale_log2, -Lb.z * kLog2e));
-            a1 += exp2f(fmaf(x[7], p.scale_log2, -Lb.w * kLog2e));
+            float a0 = ex2_ftz(fmaf(x[0], p.scale_log2, -La.x));
+            float a1 = ex2_ftz(fmaf(x[1], p.scale_log2, -La.y));
+            a0 += ex2_ftz(fmaf(x[2], p.scale_log2, -La.z));
+            a1 += ex2_ftz(fmaf(x[3], p.scale_log2, -La.w));
+            a0 += ex2_ftz(fmaf(x[4], p.scale_log2, -Lb.x));
+            a1 += ex2_ftz(fmaf(x[5], p.scale_log2, -Lb.y));
+            a0 += ex2_ftz(fmaf(x[6], p.scale_log2, -Lb.z));
+            a1 += ex2_ftz(fmaf(x[7], p.scale_log2, -Lb.w));
             pr[rr] += a0 + a1;
           }
         }
@@ -529,7 +564,7 @@ __global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
+        for (int rr = 0; rr < R; ++rr) {
           if (key < vis[rr]) {
             const float pp = pr[rr] * inv_Hq;
             const float lq = Iv[rr] - lI[rr];  // log q
@@ -543,11 +578,11 @@ __global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
       if (lane == 0) mbar_arrive(&l_empty[lb]);
       ++m;
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
+      for (int rr = 0; rr < R; ++rr) {
         float s = kl[rr];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0 && 4 * half + rr < it.ntok) p.kl_part[(it.t0 + 4 * half + rr) * 4 + quarter] = s;
+        if (lane == 0 && R * rgrp + rr < it.ntok) p.kl_part[(it.t0 + R * rgrp + rr) * 4 + quarter] = s;
       }
     }
   }

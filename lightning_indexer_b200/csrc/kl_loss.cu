@@ -54,6 +54,7 @@ __device__ __forceinline__ int seq_of_row(const int* cu, int batch, long long ro
 
 // ------------------------------------------------------------------ 1. dense LSE
 // One warp per (row, KV head): streams the row's visible keys (contiguous) in chunks of 16.
+// Writes the base-2 LSE log2 sum_s 2^(scale log2(e) Q.K).
 template <int D>
 __global__ void __launch_bounds__(KL_WARPS * 32)
     dense_lse_kernel(const uint16_t* Q, const uint16_t* K, const int* cu_q, const int* cu_k, int batch,
@@ -147,9 +148,8 @@ __global__ void __launch_bounds__(KL_WARPS * 32)
   }
   if (lane < 4) {
     const int h0 = 2 * tig, h1 = h0 + 1;
-    const float ln2 = 0.69314718055994531f;
-    if (h0 < G) lse_out[row * Hq + g * G + h0] = l0 > 0.f ? (m0 + log2f(l0)) * ln2 : -INFINITY;
-    if (h1 < G) lse_out[row * Hq + g * G + h1] = l1 > 0.f ? (m1 + log2f(l1)) * ln2 : -INFINITY;
+    if (h0 < G) lse_out[row * Hq + g * G + h0] = l0 > 0.f ? m0 + log2f(l0) : -INFINITY;
+    if (h1 < G) lse_out[row * Hq + g * G + h1] = l1 > 0.f ? m1 + log2f(l1) : -INFINITY;
   }
 }
 
@@ -225,8 +225,8 @@ __global__ void __launch_bounds__(256)
     }
   }
   const int h0 = 2 * tig, h1 = h0 + 1;
-  const float L0 = h0 < G ? lse_att[row * Hq + g * G + h0] * 1.4426950408889634f : -INFINITY;
-  const float L1 = h1 < G ? lse_att[row * Hq + g * G + h1] * 1.4426950408889634f : -INFINITY;
+  const float L0 = h0 < G ? lse_att[row * Hq + g * G + h0] : -INFINITY;
+  const float L1 = h1 < G ? lse_att[row * Hq + g * G + h1] : -INFINITY;
   const int nchunks = (vis + KL_CHUNK - 1) / KL_CHUNK;
   auto issue = [&](int c, int st) {
 #pragma unroll
@@ -631,7 +631,7 @@ int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const i
                     long long part_stride, cudaStream_t s);
 
 struct KLWorkspace {
-  float* lse_att;  // [T, Hq]
+  float* lse_att;  // [T, Hq] base-2 LSE: log2 sum_s 2^(scale log2(e) Q.K)
   float* dk_acc;   // [Tk, d_I]
   float* dk_part;  // [ceil(chunk_rows / KL_COL_ROWS), Tk, d_I] per-row-block partials of dk
   float* lseI;     // [chunk_rows]
