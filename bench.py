@@ -460,7 +460,7 @@ def run_train(args, device):
                                   chunk_rows=chunk, workspace=ws)
         if ev:
             ev[1].record(stream)
-        dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse, idx, cu, cu)
+        dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse, idx, cu, cu, max_seqlen_k=mq)
         if ev:
             ev[2].record(stream)
         dsa.indexer_kl_loss(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], cu, cu, mq, mq, chunk_rows=chunk)

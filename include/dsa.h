@@ -216,18 +216,25 @@ DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, cons
  *     dQ[r,h] = scale * sum_s dS[s] K[s,g]
  *     dK[s,g] += scale * dS[s] Q[r,h],   dV[s,g] += P[s] dO[r,h]   (over all r, h)
  *   dQ device bf16 [total_q, Hq, d]; dK, dV device bf16 [total_k, Hkv, d].
- *   dK/dV are accumulated in fp32 in the workspace (float atomics: the summation order,
- *   and so the last bits, can vary between runs) and rounded to bf16 once at the end.
- *   workspace: dsa_sparse_attn_bwd_workspace_size(total_q, total_k, Hq, Hkv, d) bytes.
+ *   max_seqlen_k: the longest sequence of keys (bounds the selected positions).
+ *   Two paths, chosen from the shapes: when d = 128, Hq = 8 Hkv and 8 k >= max_seqlen_k
+ *   (dense selected sets), a masked dense pass on tensor cores: each key's dK and dV are
+ *   written once, dQ is accumulated in fp32 (float atomics); otherwise one warp per (token,
+ *   KV head) over its selected keys, with dK and dV accumulated in fp32 (float atomics).
+ *   Float atomics make the summation order, and so the last bits, vary between runs; every
+ *   fp32 accumulator is rounded to bf16 once at the end.  Selected positions outside
+ *   [0, max_seqlen_k) and -1 slots are ignored.
+ *   workspace: dsa_sparse_attn_bwd_workspace_size(total_q, total_k, Hq, Hkv, d,
+ *   max_seqlen_k) bytes (enough for either path).
  * ------------------------------------------------------------------------------- */
 DSA_API size_t dsa_sparse_attn_bwd_workspace_size(int64_t total_q, int64_t total_k, int Hq,
-                                                  int Hkv, int d);
+                                                  int Hkv, int d, int max_seqlen_k);
 DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void* V,
                                         const void* O, const void* dO, const float* lse,
                                         const int32_t* indices, const int32_t* cu_seqlens_q,
                                         const int32_t* cu_seqlens_k, int batch, int64_t total_q,
-                                        int64_t total_k, int Hq, int Hkv, int d, int k,
-                                        float scale, void* dQ, void* dK, void* dV,
+                                        int64_t total_k, int max_seqlen_k, int Hq, int Hkv, int d,
+                                        int k, float scale, void* dQ, void* dK, void* dV,
                                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------

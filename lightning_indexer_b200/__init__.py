@@ -265,18 +265,24 @@ def decode(q_idx, k_idx, w, Q, K, V, cu_seqlens_k, max_seqlen_k: int, k: int, sc
 
 
 def sparse_attn_prefill_bwd(Q, K, V, O, dO, lse, indices, cu_seqlens_q, cu_seqlens_k,
-                            scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None):
-    """Gradients dQ, dK, dV of sparse attention for fixed selected sets."""
+                            scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                            max_seqlen_k: Optional[int] = None):
+    """Gradients dQ, dK, dV of sparse attention for fixed selected sets.
+
+    max_seqlen_k: the longest key sequence; read from cu_seqlens_k (a device sync) if None.
+    """
     T, Hq, d = Q.shape
     Tk, Hkv, _ = K.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    nbytes = _lib.load().dsa_sparse_attn_bwd_workspace_size(T, Tk, Hq, Hkv, d)
+    if max_seqlen_k is None:
+        max_seqlen_k = int((cu_seqlens_k[1:] - cu_seqlens_k[:-1]).max().item()) if cu_seqlens_k.numel() > 1 else 0
+    nbytes = _lib.load().dsa_sparse_attn_bwd_workspace_size(T, Tk, Hq, Hkv, d, max_seqlen_k)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=Q.device)
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
     call("dsa_sparse_attn_prefill_bwd", _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse), _ptr(indices),
-         _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Tk, Hq, Hkv, d, indices.shape[1],
-         scale, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace), workspace.numel(), _stream())
+         _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Tk, max_seqlen_k, Hq, Hkv, d,
+         indices.shape[1], scale, _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace), workspace.numel(), _stream())
     return dQ, dK, dV
 
 

@@ -1,6 +1,7 @@
 // C ABI of libdsa_b200 (declared in include/dsa.h): argument checks, launch selection,
 // and the chunked prefill / decode pipelines.  Every check happens on the host before
 // anything is enqueued; the library never allocates and never synchronises.
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -33,6 +34,12 @@ int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const
                               void* ws, cudaStream_t stream);
 
 size_t sparse_attn_bwd_workspace_bytes(long long total_k, int Hkv, int d);
+bool sa_bwd_tc_eligible(int Hq, int Hkv, int d, int k, int max_seqlen_k);
+size_t sa_bwd_tc_workspace_bytes(long long total_q, int Hq, int max_seqlen_k);
+int sa_bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* lse,
+                     const int* indices, const int* cu_q, const int* cu_k, int batch, long long total_q,
+                     long long total_k, int Hq, int Hkv, int k, int max_seqlen_k, float scale, void* dQ, void* dK,
+                     void* dV, void* ws, cudaStream_t s);
 int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                            const float* lse, const int* indices, const int* cu_q, const int* cu_k, int batch,
                            long long total_q, long long total_k, int Hq, int Hkv, int d, int k, float scale,
@@ -308,27 +315,35 @@ DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, cons
                                 workspace_bytes - (size_t)(ws - static_cast<uint8_t*>(workspace)), stream);
 }
 
-DSA_API size_t dsa_sparse_attn_bwd_workspace_size(int64_t total_q, int64_t total_k, int Hq, int Hkv, int d) {
-  (void)total_q;
-  (void)Hq;
-  if (total_k < 0 || Hkv < 1 || d < 1) return 0;
-  return sparse_attn_bwd_workspace_bytes(total_k, Hkv, d);
+DSA_API size_t dsa_sparse_attn_bwd_workspace_size(int64_t total_q, int64_t total_k, int Hq, int Hkv, int d,
+                                                  int max_seqlen_k) {
+  if (total_q < 0 || total_k < 0 || Hq < 1 || Hkv < 1 || d < 1 || max_seqlen_k < 0) return 0;
+  size_t bytes = sparse_attn_bwd_workspace_bytes(total_k, Hkv, d);
+  if (d == 128 && Hq == 8 * Hkv) bytes = std::max(bytes, sa_bwd_tc_workspace_bytes(total_q, Hq, max_seqlen_k));
+  return bytes;
 }
 
 DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                                         const float* lse, const int32_t* indices, const int32_t* cu_seqlens_q,
                                         const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
-                                        int Hq, int Hkv, int d, int k, float scale, void* dQ, void* dK, void* dV,
-                                        void* workspace, size_t workspace_bytes, void* stream) {
+                                        int max_seqlen_k, int Hq, int Hkv, int d, int k, float scale, void* dQ,
+                                        void* dK, void* dV, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
   if (!Q || !K || !V || !O || !dO || !lse || !indices || !cu_seqlens_q || !cu_seqlens_k || !dQ || !dK || !dV)
     return DSA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
       !aligned16(dK) || !aligned16(dV))
     return DSA_ERR_INVALID_ARG;
-  if (batch < 1 || total_q < 0 || total_k < 0 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || k < 1 || !(scale > 0.f) || max_seqlen_k < 0)
+    return DSA_ERR_INVALID_ARG;
   if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
-  if (!workspace || !aligned16(workspace) || workspace_bytes < sparse_attn_bwd_workspace_bytes(total_k, Hkv, d))
-    return DSA_ERR_WORKSPACE;
+  if (!workspace || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  if (sa_bwd_tc_eligible(Hq, Hkv, d, k, max_seqlen_k)) {
+    if (workspace_bytes < sa_bwd_tc_workspace_bytes(total_q, Hq, max_seqlen_k)) return DSA_ERR_WORKSPACE;
+    return sa_bwd_tc_launch(Q, K, V, O, dO, lse, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, Hq,
+                            Hkv, k, max_seqlen_k, scale, dQ, dK, dV, workspace, static_cast<cudaStream_t>(stream));
+  }
+  if (workspace_bytes < sparse_attn_bwd_workspace_bytes(total_k, Hkv, d)) return DSA_ERR_WORKSPACE;
   return sparse_attn_bwd_launch(Q, K, V, O, dO, lse, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                                 Hq, Hkv, d, k, scale, dQ, dK, dV, workspace, static_cast<cudaStream_t>(stream));
 }

@@ -222,7 +222,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
-// Instruction-descriptor bit that marks the B operand as MN-major (N contiguous).
+// Instruction-descriptor bits that mark the A operand as MN-major (M contiguous) and the
+// B operand as MN-major (N contiguous).
+constexpr uint32_t kIdescAMnMajor = 1u << 15;
 constexpr uint32_t kIdescBMnMajor = 1u << 16;
 
 // ------------------------------------------------------------------ CTA pairs (cta_group::2)

@@ -6,6 +6,7 @@
 #include "topk.cu"
 #include "sparse_attn.cu"
 #include "sparse_attn_bwd.cu"
+#include "sparse_attn_bwd_tc.cu"
 #include "kl_bwd_tc.cu"
 #include "kl_dense_tc.cu"
 #include "kl_loss.cu"

@@ -17,8 +17,9 @@ def _rel_err(got, ref):
     return float(np.max(np.abs(got - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
-@pytest.mark.parametrize("Hq,Hkv,d,k", [(8, 2, 64, 32), (32, 4, 128, 64), (16, 4, 64, 48)])
+@pytest.mark.parametrize("Hq,Hkv,d,k", [(8, 2, 64, 32), (32, 4, 128, 64), (16, 4, 64, 48), (32, 4, 128, 16)])
 def test_sparse_attention_backward(Hq, Hkv, d, k):
+    # d = 128, 8 heads per KV head: k = 64 takes the masked dense path (8 k >= 211), k = 16 the gather path
     wl = gen.make_prefill([150, 33, 211], Hq, Hkv, d, 4, 32, k, seed=51, with_dO=True, layout="video")
     D = orc.Decoded(wl)
     ref_f = orc.forward(D, k=k)
@@ -38,8 +39,10 @@ def test_sparse_attention_backward(Hq, Hkv, d, k):
     np.testing.assert_allclose(dV.sum(0), grp, rtol=2e-2, atol=2e-2 * np.abs(grp).max())
 
 
-def test_sparse_attention_backward_padded_sets():
-    wl = gen.make_prefill([40], 8, 2, 64, 4, 32, 32, seed=52, with_dO=True)
+@pytest.mark.parametrize("Hq,Hkv,d", [(8, 2, 64), (16, 2, 128)])
+def test_sparse_attention_backward_padded_sets(Hq, Hkv, d):
+    # d = 128 with 8 query heads per KV head takes the masked dense tensor-core path
+    wl = gen.make_prefill([40], Hq, Hkv, d, 4, 32, 32, seed=52, with_dO=True)
     D = orc.Decoded(wl)
     idx = np.full((40, 32), -1, np.int64)
     for r in range(40):
