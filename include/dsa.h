@@ -254,11 +254,12 @@ DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void
  *   workspace: dsa_indexer_kl_loss_workspace_size(...) bytes.
  * Supported: H_I in {16, 32, 64} with d_I = 128; d in {64, 128}; Hq/Hkv in {4, 8}; Hkv <= 8;
  * self-attention packing (Lq == Lk per sequence).  dk_idx is accumulated in fp32 in the
- * workspace by one thread block per key tile (no atomics: bit-reproducible).
+ * workspace from per-(key tile, row block) partials added in a fixed order (no atomics:
+ * bit-reproducible).
  * ------------------------------------------------------------------------------- */
 DSA_API size_t dsa_indexer_kl_loss_workspace_size(int64_t total_q, int64_t total_k,
                                                   int max_seqlen_k, int Hq, int H_I, int d_I,
-                                                  int64_t chunk_rows);
+                                                  int64_t chunk_rows, int batch);
 DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx, const void* k_idx,
                                 const void* w, const int32_t* cu_seqlens_q,
                                 const int32_t* cu_seqlens_k, int batch, int64_t total_q,

@@ -298,7 +298,8 @@ def indexer_kl_loss(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, max_seqle
     H_I, d_I = q_idx.shape[1], q_idx.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     chunk_rows = max(1, min(chunk_rows, T))
-    nbytes = _lib.load().dsa_indexer_kl_loss_workspace_size(T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows)
+    nbytes = _lib.load().dsa_indexer_kl_loss_workspace_size(T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows,
+                                                            cu_seqlens_q.numel() - 1)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=Q.device)
     loss = torch.empty(1, dtype=torch.float32, device=Q.device)

@@ -46,7 +46,8 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
                            void* dQ, void* dK, void* dV, void* ws, cudaStream_t stream);
 
 struct KLWorkspace;
-size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int d_I, long long chunk_rows);
+size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I, long long chunk_rows,
+                          int batch);
 int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
                            const int* cu_q, const int* cu_k, int batch, long long T, long long Tk,
                            int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I,
@@ -349,10 +350,10 @@ DSA_API int dsa_sparse_attn_prefill_bwd(const void* Q, const void* K, const void
 }
 
 DSA_API size_t dsa_indexer_kl_loss_workspace_size(int64_t total_q, int64_t total_k, int max_seqlen_k, int Hq,
-                                                  int H_I, int d_I, int64_t chunk_rows) {
-  (void)H_I;
-  if (total_q < 0 || total_k < 0 || max_seqlen_k < 0 || Hq < 1 || d_I < 1 || chunk_rows < 1) return 0;
-  return kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, d_I, chunk_rows);
+                                                  int H_I, int d_I, int64_t chunk_rows, int batch) {
+  if (total_q < 0 || total_k < 0 || max_seqlen_k < 0 || Hq < 1 || H_I < 1 || d_I < 1 || chunk_rows < 1 || batch < 1)
+    return 0;
+  return kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch);
 }
 
 DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
@@ -372,7 +373,7 @@ DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx,
   if (!((H_I == 64 || H_I == 32 || H_I == 16) && d_I == 128)) return DSA_ERR_UNSUPPORTED;
   if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace) ||
-      workspace_bytes < kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, d_I, chunk_rows))
+      workspace_bytes < kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch))
     return DSA_ERR_WORKSPACE;
   return indexer_kl_loss_launch(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                                 max_seqlen_q, max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, loss, kl, dq_idx,

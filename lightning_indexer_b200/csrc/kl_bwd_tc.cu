@@ -5,9 +5,11 @@
 // With g[t,s] = dloss/dI[t,s] (from the KL target pass) and x[t,j,s] = q_idx[t,j].k_idx[s],
 //   dk_idx[s] = sum_t sum_j g[t,s] w[t,j] [x[t,j,s] > 0] q_idx[t,j,:].
 //
-// One work item is (sequence, tile of 128 keys, block of up to 1024 query rows of the row
-// chunk that see the tile); its partial dk (128 keys x d_I, fp32) goes to the row block's
-// slice of the partial workspace, and a second kernel adds the row blocks in a fixed order.
+// One work item is (sequence, tile of 128 keys, block of up to KL_DK_ROWS query rows of the
+// row chunk that see the tile).  The items of a chunk are counted on the device (a prefix
+// sum over (sequence, tile) pairs), so their partial dk (128 keys x d_I, fp32) sit in one
+// compact slot each, and a second kernel adds a tile's slots in item order (deterministic).
+// Small items keep the persistent CTAs evenly loaded on chunks of short sequences.
 // Per block of 2 query rows (N = 2 x 64 heads = 128 columns), two chained MMAs:
 //   MMA1  X[128 keys x 128 (t,j)] = K_tile . Q_blk^T          (TMEM, two buffers)
 //   epilogue  G = g w [X > 0] -> bf16, written to shared memory in the 128-byte swizzled
@@ -27,6 +29,94 @@
 
 namespace dsa {
 
+// query rows per dk work item (a multiple of 2)
+constexpr int KL_DK_ROWS = 256;
+// (sequence, tile) pairs whose item offsets are cached in shared memory
+constexpr int KL_DK_SMEM_PAIRS = 4095;
+
+// rows [qlo, qhi) of the chunk [row_begin, row_end) that see key tile `tile` of sequence b
+__device__ __forceinline__ void dk_tile_rows(const int* cu_q, const int* cu_k, int b, int tile, long long row_begin,
+                                             long long row_end, long long& qlo, long long& qhi) {
+  const int Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
+  qlo = max((long long)cu_q[b] + max(tile * 128 - (Lk - Lq), 0), row_begin);
+  qhi = min((long long)cu_q[b + 1], row_end);
+  if (tile * 128 >= Lk) qhi = qlo;
+}
+
+// offs[pair] = first item of (sequence, tile) pair = b * tiles_per_seq + tile, offs[n_pairs]
+// = the chunk's item count (one block; exclusive scan in rounds of blockDim.x pairs)
+__global__ void dk_items_kernel(const int* cu_q, const int* cu_k, int batch, int tiles_per_seq, long long row_begin,
+                                long long row_end, int* offs) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry;
+  const long long n_pairs = (long long)batch * tiles_per_seq;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (long long base = 0; base < n_pairs; base += blockDim.x) {
+    const long long pr = base + threadIdx.x;
+    int cnt = 0;
+    if (pr < n_pairs) {
+      long long qlo, qhi;
+      dk_tile_rows(cu_q, cu_k, (int)(pr / tiles_per_seq), (int)(pr % tiles_per_seq), row_begin, row_end, qlo, qhi);
+      cnt = qhi > qlo ? (int)((qhi - qlo + KL_DK_ROWS - 1) / KL_DK_ROWS) : 0;
+    }
+    // inclusive warp scan, then across warps
+    int v = cnt;
+    const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_sums[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+      int ws = lane < (int)(blockDim.x / 32) ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += y;
+      }
+      warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    const int before = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + v - cnt;
+    if (pr < n_pairs) offs[pr] = before;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = before + cnt;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offs[n_pairs] = carry;
+}
+
+// dk_acc[key] += the slots of key's (sequence, tile) pair, in item order (one thread per 4
+// consecutive values of one key)
+__global__ void dk_reduce_items_kernel(const float* __restrict__ dk_part, const int* __restrict__ offs,
+                                       int tiles_per_seq, const int* cu_k, int batch, long long Tk, float* dk_acc) {
+  const long long e = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e >= Tk * 128) return;
+  const long long key = e / 128;
+  const int c = (int)(e % 128);
+  int lo = 0, hi = batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)cu_k[mid] <= key) lo = mid; else hi = mid;
+  }
+  const int sl = (int)(key - cu_k[lo]);
+  const int pair = lo * tiles_per_seq + sl / 128, r = sl % 128;
+  const int i0 = offs[pair], i1 = offs[pair + 1];
+  if (i0 == i1) return;
+  float4 acc = *reinterpret_cast<const float4*>(dk_acc + e);
+  for (int i = i0; i < i1; ++i) {
+    const float4 v = *reinterpret_cast<const float4*>(dk_part + ((size_t)i * 128 + r) * 128 + c);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  *reinterpret_cast<float4*>(dk_acc + e) = acc;
+}
+
 struct KlDkParams {
   const uint16_t* w;  // [T, 64] bf16
   long long total_q;
@@ -36,40 +126,40 @@ struct KlDkParams {
   long long row_begin, row_end;  // the row chunk
   const float* g;                // [row_end - row_begin, ld] fp32 dloss/dI
   long long ld;
-  int tiles_per_seq, row_blocks, rows_per_block;
-  long long n_items;
-  float* dk_part;  // [row_blocks][Tk][128] fp32
-  long long part_stride;
+  int tiles_per_seq;
+  int n_pairs;                   // batch * tiles_per_seq
+  const int* offs;               // [n_pairs + 1] first item of each pair (dk_items_kernel)
+  float* dk_part;                // [items][128 keys][128] fp32
 };
 
 struct KlDkItem {
-  int b, tile, rb, kbase, Lq, Lk;
+  long long slot;      // partial slot (the item index)
+  int b, tile, kbase, Lq, Lk;
   long long qlo, qhi;  // the item's query rows
   int nb;              // blocks of 2 rows
 };
 
-__device__ __forceinline__ bool kl_dk_item(long long item, const KlDkParams& p, KlDkItem& it) {
-  const int rb = (int)(item % p.row_blocks);
-  const int tile = (int)((item / p.row_blocks) % p.tiles_per_seq);
-  const int b = (int)(item / ((long long)p.row_blocks * p.tiles_per_seq));
-  if (b >= p.batch) return false;
-  const int Lq = p.cu_q[b + 1] - p.cu_q[b], Lk = p.cu_k[b + 1] - p.cu_k[b];
-  if (tile * 128 >= Lk) return false;
-  long long qlo = max((long long)p.cu_q[b] + max(tile * 128 - (Lk - Lq), 0), p.row_begin);
-  long long qhi = min((long long)p.cu_q[b + 1], p.row_end);
-  qlo += (long long)rb * p.rows_per_block;
-  qhi = min(qhi, qlo + p.rows_per_block);
-  if (qlo >= qhi) return false;
+// item index -> (pair, row block) by a search over the pair offsets `offs` (shared or global)
+__device__ __forceinline__ void kl_dk_item(long long item, const KlDkParams& p, const int* offs, KlDkItem& it) {
+  int lo = 0, hi = p.n_pairs;  // offs[lo] <= item < offs[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if (offs[mid] <= item) lo = mid; else hi = mid;
+  }
+  const int b = lo / p.tiles_per_seq, tile = lo % p.tiles_per_seq;
+  long long qlo, qhi;
+  dk_tile_rows(p.cu_q, p.cu_k, b, tile, p.row_begin, p.row_end, qlo, qhi);
+  qlo += (item - offs[lo]) * KL_DK_ROWS;
+  qhi = min(qhi, qlo + KL_DK_ROWS);
+  it.slot = item;
   it.b = b;
   it.tile = tile;
-  it.rb = rb;
   it.kbase = p.cu_k[b];
-  it.Lq = Lq;
-  it.Lk = Lk;
+  it.Lq = p.cu_q[b + 1] - p.cu_q[b];
+  it.Lk = p.cu_k[b + 1] - it.kbase;
   it.qlo = qlo;
   it.qhi = qhi;
   it.nb = (int)((qhi - qlo + 1) / 2);
-  return true;
 }
 
 struct KlDkCfg {
@@ -84,7 +174,8 @@ struct KlDkCfg {
   static constexpr int W_BYTES = 2 * 64 * 2;
   static constexpr int OFF_GS = OFF_W + Q_STAGES * W_BYTES;            // Q_STAGES x g of the block's rows
   static constexpr int GS_BYTES = 2 * 128 * 4;
-  static constexpr int OFF_BAR = OFF_GS + Q_STAGES * GS_BYTES;
+  static constexpr int OFF_OFFS = OFF_GS + Q_STAGES * GS_BYTES;       // cached item offsets
+  static constexpr int OFF_BAR = OFF_OFFS + (KL_DK_SMEM_PAIRS + 1) * 4;
   // a_full, a_empty, q_full[S], q_empty[S], x_full[2], x_empty[2], g_full[2], g_empty[2],
   // dk_full, dk_empty, done
   static constexpr int NUM_BARS = 2 + 2 * Q_STAGES + 8 + 2 + 1;
@@ -153,10 +244,18 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_q);
   }
+  // the chunk's item offsets: shared-memory copy when they fit
+  int* s_offs = reinterpret_cast<int*>(smem + C::OFF_OFFS);
+  const bool offs_in_smem = p.n_pairs <= KL_DK_SMEM_PAIRS;
+  if (offs_in_smem)
+    for (int i = threadIdx.x; i <= p.n_pairs; i += blockDim.x) s_offs[i] = p.offs[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  const int* offs = offs_in_smem ? s_offs : p.offs;
+  const long long n_items = offs[p.n_pairs];
+  const long long n_slots = (n_items + gridDim.x - 1) / gridDim.x * gridDim.x;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -164,9 +263,11 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
       long long n = 0;  // blocks loaded so far (stage n % Q_STAGES)
       long long m = 0;  // non-empty items so far
       bool ok = true;
-      for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (long long slot = blockIdx.x; slot < n_slots && ok; slot += gridDim.x) {
+        const long long item = snake_slot(slot);
+        if (item >= n_items) continue;
         KlDkItem it;
-        if (!kl_dk_item(item, p, it)) continue;
+        kl_dk_item(item, p, offs, it);
         if (!(ok = mbar_wait(a_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 40))) break;
         mbar_arrive_expect_tx(a_full, C::TILE_BYTES);
         for (int pn = 0; pn < 2; ++pn)
@@ -234,9 +335,11 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
         umma_commit(&x_full[xb]);
         return true;
       };
-      for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (long long slot = blockIdx.x; slot < n_slots && ok; slot += gridDim.x) {
+        const long long item = snake_slot(slot);
+        if (item >= n_items) continue;
         KlDkItem it;
-        if (!kl_dk_item(item, p, it)) continue;
+        kl_dk_item(item, p, offs, it);
         if (!(ok = mbar_wait(a_full, (uint32_t)(m & 1), abort_flag, 44))) break;
         tc_fence_after();
         const long long n0 = n;
@@ -282,9 +385,11 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
     const uint32_t g_row0 = smem_u32(sG) + half * C::PANEL_BYTES + r * 128;
     long long n = 0, m = 0, gcount = 0;
     bool ok = true;
-    for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (long long slot = blockIdx.x; slot < n_slots && ok; slot += gridDim.x) {
+      const long long item = snake_slot(slot);
+      if (item >= n_items) continue;
       KlDkItem it;
-      if (!kl_dk_item(item, p, it)) continue;
+      kl_dk_item(item, p, offs, it);
       const int s = it.tile * 128 + r;  // this thread's key (sequence-local)
       const int dvis = it.Lk - it.Lq + 1;
       const long long q0 = p.cu_q[it.b];
@@ -337,7 +442,7 @@ __global__ void __launch_bounds__(KlDkCfg::THREADS, 1)
       // the item's dk: one key row per thread, this warp's 64 of its 128 fp32 values
       if (!(ok = mbar_wait(dk_full, (uint32_t)(m & 1), abort_flag, 49))) break;
       tc_fence_after();
-      float* dst = p.dk_part + it.rb * p.part_stride + (size_t)(it.kbase + s) * C::D_I + half * 64;
+      float* dst = p.dk_part + ((size_t)it.slot * 128 + r) * C::D_I + half * 64;
 #pragma unroll 1
       for (int c = 0; c < 64; c += 32) {
         float v[32];
@@ -741,11 +846,19 @@ __global__ void __launch_bounds__(KlDqCfg::THREADS, 1)
 
 namespace dsa_host {
 
-// dk partials of the row chunk [r0, r1) for H_I = 64, d_I = 128 (see the file comment).
-int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q,
-                    const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
-                    long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
-                    long long part_stride, cudaStream_t s) {
+// Upper bound on the dk work items of one row chunk: every item but the last of each
+// (sequence, tile) pair covers KL_DK_ROWS rows of the chunk.
+size_t kl_dk_tc_max_items(long long chunk_rows, long long total_k, int batch, int max_seqlen_k) {
+  const long long tiles = (max_seqlen_k + 127) / 128;
+  return (size_t)((total_k + 127) / 128 + batch + (chunk_rows * tiles + dsa::KL_DK_ROWS - 1) / dsa::KL_DK_ROWS);
+}
+
+// dk_acc += dk of the row chunk [r0, r1) for H_I = 64, d_I = 128 (see the file comment), by
+// partials in dk_part (kl_dk_tc_max_items slots of 128 x 128 fp32) with the item offsets in
+// offs (batch * ceil(max_seqlen_k / 128) + 1 ints).
+int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
+                    int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0, long long r1,
+                    const float* g, long long ld, float* dk_part, int* offs, float* dk_acc, cudaStream_t s) {
   using C = dsa::KlDkCfg;
   static bool attr_done = false;
   if (!attr_done) {
@@ -755,6 +868,10 @@ int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const i
       return cuda_fail(e_);
     attr_done = true;
   }
+  const int tiles = (max_seqlen_k + 127) / 128;
+  if (tiles <= 0 || r1 <= r0) return DSA_OK;
+  dsa::dk_items_kernel<<<1, 1024, 0, s>>>(cu_q, cu_k, batch, tiles, r0, r1, offs);
+  if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
   CUtensorMap tk, tq;
   int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)total_k, 128, 256, 128, 64, 128);
   if (st != DSA_OK) return st;
@@ -770,16 +887,20 @@ int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const i
   p.row_end = r1;
   p.g = g;
   p.ld = ld;
-  p.tiles_per_seq = (max_seqlen_k + 127) / 128;
-  p.rows_per_block = rows_per_block;
-  p.row_blocks = (int)((r1 - r0 + rows_per_block - 1) / rows_per_block);
-  p.n_items = (long long)batch * p.tiles_per_seq * p.row_blocks;
+  p.tiles_per_seq = tiles;
+  p.n_pairs = batch * tiles;
+  p.offs = offs;
   p.dk_part = dk_part;
-  p.part_stride = part_stride;
-  const long long grid = std::min<long long>(p.n_items, (long long)sm_count());
-  if (grid <= 0) return DSA_OK;
-  dsa::kl_dk_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, p);
-  return last_launch_status();
+  dsa::kl_dk_tc_kernel<<<(unsigned)sm_count(), C::THREADS, C::SMEM_BYTES, s>>>(tk, tq, p);
+  if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
+  // dk_acc += the pairs' slots in item order
+  const long long quads = total_k * 32;
+  if (quads > 0) {
+    dsa::dk_reduce_items_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(dk_part, offs, tiles, cu_k, batch,
+                                                                               total_k, dk_acc);
+    if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
 }
 
 // dw and dq_idx of the row chunk [r0, r1) for H_I = 64, d_I = 128 (row-stationary, above).

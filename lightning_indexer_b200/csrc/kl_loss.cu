@@ -625,15 +625,17 @@ int kl_parts_sum_launch(const float* kl_part, long long T, float* kl, cudaStream
 int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
                     long long total_q, long long total_k, long long r0, long long r1, const float* g, long long ld,
                     void* dq, void* dw, cudaStream_t s);
-int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q,
-                    const int* cu_k, int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0,
-                    long long r1, const float* g, long long ld, int rows_per_block, float* dk_part,
-                    long long part_stride, cudaStream_t s);
+int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
+                    int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0, long long r1,
+                    const float* g, long long ld, float* dk_part, int* offs, float* dk_acc, cudaStream_t s);
+size_t kl_dk_tc_max_items(long long chunk_rows, long long total_k, int batch, int max_seqlen_k);
 
 struct KLWorkspace {
   float* lse_att;  // [T, Hq] base-2 LSE: log2 sum_s 2^(scale log2(e) Q.K)
   float* dk_acc;   // [Tk, d_I]
-  float* dk_part;  // [ceil(chunk_rows / KL_COL_ROWS), Tk, d_I] per-row-block partials of dk
+  float* dk_part;  // partials of dk: tensor-core path [items][128][d_I], else
+                   // [ceil(chunk_rows / KL_COL_ROWS), Tk, d_I] per row block
+  int* dk_offs;    // tensor-core path: first item of each (sequence, key tile) pair
   float* lseI;     // [chunk_rows]
   float* scores;   // [chunk_rows, ld]
   float* kl_part;  // [T, 4] per-key-quarter partials of kl (tensor-core target path)
@@ -642,8 +644,11 @@ struct KLWorkspace {
 
 static size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
-KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_seqlen_k, int Hq, int d_I,
-                                long long chunk_rows) {
+// the tensor-core backward kernels serve H_I = 64, d_I = 128
+static bool kl_tc_backward(int H_I, int d_I) { return H_I == 64 && d_I == 128; }
+
+KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I,
+                                long long chunk_rows, int batch) {
   KLWorkspace w{};
   uint8_t* p = static_cast<uint8_t*>(base);
   const size_t ld = ((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1) + 3) / 4 * 4;
@@ -653,7 +658,12 @@ KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_s
   w.dk_acc = reinterpret_cast<float*>(p + off);
   off += r256((size_t)Tk * d_I * 4);
   w.dk_part = reinterpret_cast<float*>(p + off);
-  off += r256((size_t)((chunk_rows + dsa::KL_COL_ROWS - 1) / dsa::KL_COL_ROWS) * Tk * d_I * 4);
+  if (kl_tc_backward(H_I, d_I))
+    off += r256(kl_dk_tc_max_items(chunk_rows, Tk, batch, max_seqlen_k) * 128 * d_I * 4);
+  else
+    off += r256((size_t)((chunk_rows + dsa::KL_COL_ROWS - 1) / dsa::KL_COL_ROWS) * Tk * d_I * 4);
+  w.dk_offs = reinterpret_cast<int*>(p + off);
+  off += r256(((size_t)batch * ((max_seqlen_k + 127) / 128) + 1) * 4);
   w.lseI = reinterpret_cast<float*>(p + off);
   off += r256((size_t)chunk_rows * 4);
   w.scores = reinterpret_cast<float*>(p + off);
@@ -664,15 +674,16 @@ KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_s
   return w;
 }
 
-size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int d_I, long long chunk_rows) {
-  return kl_workspace_layout(nullptr, T, Tk, max_seqlen_k, Hq, d_I, chunk_rows).total;
+size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I, long long chunk_rows,
+                          int batch) {
+  return kl_workspace_layout(nullptr, T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch).total;
 }
 
 template <int H_I, int D_I>
 static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                                int batch, long long r0, long long r1, long long T, long long Tk, const float* g,
                                long long ld, int max_seqlen_k, void* dq, void* dw, float* dk_acc, float* dk_part,
-                               cudaStream_t s) {
+                               int* dk_offs, cudaStream_t s) {
   if constexpr (H_I == 64 && D_I == 128) {
     // tensor-core row-stationary kernel
     const int st = kl_dq_tc_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, r0, r1, g, ld, dq, dw, s);
@@ -690,13 +701,13 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
         cu_q, cu_k, batch, r0, g, ld, static_cast<uint16_t*>(dq), static_cast<uint16_t*>(dw));
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
   }
-  const long long part_stride = Tk * D_I;
   if constexpr (H_I == 64 && D_I == 128) {
-    // tensor-core key-stationary kernel
-    const int st = kl_dk_tc_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, max_seqlen_k, r0, r1, g, ld,
-                                   dsa::KL_COL_ROWS, dk_part, part_stride, s);
-    if (st != DSA_OK) return st;
+    // tensor-core key-stationary kernel (adds its partials into dk_acc itself)
+    return kl_dk_tc_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, max_seqlen_k, r0, r1, g, ld, dk_part, dk_offs,
+                           dk_acc, s);
   } else {
+    (void)dk_offs;
+    const long long part_stride = Tk * D_I;
     auto kern = dsa::idx_bwd_col_kernel<H_I, D_I>;
     const int smem = 2 * H_I * D_I * 2 + 2 * H_I * 4 + 2 * 128 * 4;
     static bool done = false;
@@ -710,8 +721,6 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
         static_cast<const uint16_t*>(q_idx), static_cast<const uint16_t*>(k_idx), static_cast<const uint16_t*>(w),
         cu_q, cu_k, batch, r0, r1, g, ld, tiles, row_blocks, dk_part, part_stride);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
-  }
-  {
     const long long quads = Tk * D_I / 4;
     if (quads > 0) {
       dsa::dk_reduce_kernel<D_I><<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(dk_part, part_stride, cu_q, cu_k, batch,
@@ -727,7 +736,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
                            int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I,
                            float scale, long long chunk_rows, float* loss, float* kl, void* dq, void* dk, void* dw,
                            void* ws, cudaStream_t s) {
-  KLWorkspace W = kl_workspace_layout(ws, T, Tk, max_seqlen_k, Hq, d_I, chunk_rows);
+  KLWorkspace W = kl_workspace_layout(ws, T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch);
   const long long ld = ((long long)(max_seqlen_k > 0 ? max_seqlen_k : 1) + 3) / 4 * 4;
   const float scale_log2 = scale * 1.4426950408889634f;
   if (const cudaError_t e_ = cudaMemsetAsync(W.dk_acc, 0, (size_t)Tk * d_I * 4, s); e_ != cudaSuccess) return cuda_fail(e_);
@@ -810,7 +819,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
 #define DSA_KLB(HI, DI)                                                                                   \
   if (H_I == HI && d_I == DI) {                                                                          \
     st = kl_backward_kernels<HI, DI>(q_idx, k_idx, w, cu_q, cu_k, batch, r0, r1, T, Tk, W.scores, ld,         \
-                                     max_seqlen_k, dq, dw, W.dk_acc, W.dk_part, s);               \
+                                     max_seqlen_k, dq, dw, W.dk_acc, W.dk_part, W.dk_offs, s);               \
     if (st != DSA_OK) return st;                                                                         \
   } else
     DSA_KLB(64, 128) DSA_KLB(32, 128) DSA_KLB(16, 128) { return DSA_ERR_UNSUPPORTED; }
