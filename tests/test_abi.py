@@ -70,6 +70,26 @@ def test_host_side_argument_errors():
     assert lib.dsa_sparse_attn_decode(fake, fake, fake, fake, fake, 16, 32, 4, 128, 2048, 0.1, fake, None,
                                       fake, need - 1, None) == -3
     assert lib.dsa_prefill_workspace_size(8192, 131072) >= 8192 * 131072 * 4
+    # sparse backward: the masked dense path (d = 128, 8 heads per KV head) needs the fp32 dQ
+    # accumulator; the gather path the fp32 dK and dV accumulators
+    T, Tk = 4096, 4096
+    dense = lib.dsa_sparse_attn_bwd_workspace_size(T, Tk, 32, 4, 128, 4096)
+    assert dense >= T * 32 * 128 * 4 + T * 32 * 8
+    gather = lib.dsa_sparse_attn_bwd_workspace_size(T, Tk, 8, 2, 64, 4096)
+    assert gather >= 2 * Tk * 2 * 64 * 4
+    assert lib.dsa_sparse_attn_bwd_workspace_size(T, Tk, 32, 4, 128, -1) == 0
+    # dense path chosen (8 k >= max_seqlen_k) with a workspace only the gather path fits
+    small = 2 * Tk * 4 * 128 * 4
+    assert small < dense
+    assert lib.dsa_sparse_attn_prefill_bwd(fake, fake, fake, fake, fake, fake, fake, fake, fake, 1, T, Tk, 4096,
+                                           32, 4, 128, 512, 0.1, fake, fake, fake, fake, small, None) == -3
+    assert lib.dsa_sparse_attn_prefill_bwd(fake, fake, fake, fake, fake, fake, fake, fake, fake, 1, T, Tk, -1,
+                                           32, 4, 128, 512, 0.1, fake, fake, fake, fake, dense, None) == -1
+    # KL loss workspace: needs the batch (dk work items per row chunk), grows with it
+    assert lib.dsa_indexer_kl_loss_workspace_size(T, Tk, 4096, 32, 64, 128, 1024, 0) == 0
+    w1 = lib.dsa_indexer_kl_loss_workspace_size(T, Tk, 4096, 32, 64, 128, 1024, 1)
+    w8 = lib.dsa_indexer_kl_loss_workspace_size(T, Tk, 4096, 32, 64, 128, 1024, 8)
+    assert 0 < w1 < w8
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
