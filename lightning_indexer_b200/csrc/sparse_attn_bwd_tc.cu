@@ -19,8 +19,8 @@
 //   epilogue  P^T, dS^T -> bf16, 128-byte swizzled rows of 64 (token, head) values
 //   dV += P^T . dO_blk,  dK += dS^T . Q_blk                         (B read MN-major)
 //   dQ^T[d x rows] = K_tile^T . dS^T                                (A and B read MN-major)
-// dQ^T goes to an fp32 accumulator with coalesced float reductions (their order can vary
-// between runs; dK and dV are deterministic).  Items are taken from a global counter, tile-
+// dQ^T goes to an fp32 accumulator with 16-byte float reductions after a 4 x 4 lane
+// transpose (their order can vary between runs; dK and dV are deterministic).  Items are taken from a global counter, tile-
 // major, so the long early tiles start first.  Warps: 0 TMA, 1 MMA issuer and TMEM owner,
 // 2-9 epilogue (warp w: keys 32 (w % 4) .., rows 32 ((w - 2) / 4) .. of each block).
 #include <algorithm>
@@ -36,9 +36,10 @@ struct SABwdTcParams {
   int tiles_max;           // ceil(max_seqlen_k / 128)
   long long n_items;       // tiles_max * batch * Hkv
   float scale, scale_log2;
-  const float2* LD;        // [T, Hq] (lse in base 2, dO . O)
-  const uint32_t* mask;    // [T, mask_words] selection bits, bit s % 32 of word s / 32
-  int mask_words;          // multiple of 4
+  long long total_q;       // T
+  const float2* LD;        // [Hkv, T, 8] (lse in base 2, dO . O) of head 8 g + i
+  const uint32_t* mask;    // [tiles_max, T, 4] selection bits: key s is bit s % 32 of word
+                           // (s % 128) / 32 of tile s / 128
   float* dQ_acc;           // [T, Hq, 128] fp32, zeroed
   uint16_t* dK;            // [Tk, Hkv, 128] bf16
   uint16_t* dV;
@@ -79,12 +80,13 @@ struct SABwdTcCfg {
   static constexpr int PT_BYTES = 128 * 64 * 2;  // P^T or dS^T: 128 keys x 64 rows
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
-  static constexpr int OFF_ST = OFF_V + KV_TILE;          // 2 stages
-  static constexpr int OFF_P = OFF_ST + 2 * STAGE;        // 2 x (P^T, dS^T)
-  static constexpr int OFF_BAR = OFF_P + 4 * PT_BYTES;
-  // kv_full, kv_empty, qd_full[2], qd_empty[2], s_full, s_empty, p_full[2], p_empty[2],
+  static constexpr int QD_STAGES = 3;
+  static constexpr int OFF_ST = OFF_V + KV_TILE;                  // QD_STAGES stages
+  static constexpr int OFF_P = OFF_ST + QD_STAGES * STAGE;        // P^T, dS^T
+  static constexpr int OFF_BAR = OFF_P + 2 * PT_BYTES;
+  // kv_full, kv_empty, qd_full[S], qd_empty[S], s_full, s_empty, p_full, p_empty,
   // dq_full[2], dq_empty[2], acc_full, acc_empty, item_full[2], item_empty[2], done
-  static constexpr int NUM_BARS = 2 + 4 + 2 + 4 + 4 + 2 + 4 + 1;
+  static constexpr int NUM_BARS = 2 + 2 * QD_STAGES + 2 + 2 + 4 + 2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
   static constexpr int EPI_WARPS = 8;
@@ -103,10 +105,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                : "memory");
 }
 
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
-}
-
 __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
     sa_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_do,
                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -117,19 +115,19 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* qd_full = bars + 2;     // [2]
-  uint64_t* qd_empty = bars + 4;    // [2]
-  uint64_t* s_full = bars + 6;
-  uint64_t* s_empty = bars + 7;
-  uint64_t* p_full = bars + 8;      // [2]
-  uint64_t* p_empty = bars + 10;    // [2]
-  uint64_t* dq_full = bars + 12;    // [2]
-  uint64_t* dq_empty = bars + 14;   // [2]
-  uint64_t* acc_full = bars + 16;
-  uint64_t* acc_empty = bars + 17;
-  uint64_t* item_full = bars + 18;  // [2]
-  uint64_t* item_empty = bars + 20; // [2]
-  uint64_t* mma_done = bars + 22;
+  uint64_t* qd_full = bars + 2;                    // [QD_STAGES]
+  uint64_t* qd_empty = qd_full + C::QD_STAGES;     // [QD_STAGES]
+  uint64_t* s_full = qd_empty + C::QD_STAGES;
+  uint64_t* s_empty = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* p_empty = s_full + 3;
+  uint64_t* dq_full = s_full + 4;                  // [2]
+  uint64_t* dq_empty = s_full + 6;                 // [2]
+  uint64_t* acc_full = s_full + 8;
+  uint64_t* acc_empty = s_full + 9;
+  uint64_t* item_full = s_full + 10;               // [2]
+  uint64_t* item_empty = s_full + 12;              // [2]
+  uint64_t* mma_done = s_full + 14;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   volatile int* item_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 16);  // [2]
@@ -139,11 +137,13 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::QD_STAGES; ++i) {
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], 1);
-      mbar_init(&p_full[i], C::EPI_WARPS);
-      mbar_init(&p_empty[i], 1);
+    }
+    mbar_init(p_full, C::EPI_WARPS);
+    mbar_init(p_empty, 1);
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&dq_full[i], 1);
       mbar_init(&dq_empty[i], C::EPI_WARPS);
       mbar_init(&item_full[i], 1);
@@ -213,8 +213,8 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
         }
         ++m;
         for (int q = 0; q < it.nq; ++q, ++u) {
-          const int st = (int)(u & 1);
-          if (!(ok = mbar_wait(&qd_empty[st], (uint32_t)((u >> 1) & 1) ^ 1u, abort_flag, 102))) break;
+          const int st = (int)(u % C::QD_STAGES);
+          if (!(ok = mbar_wait(&qd_empty[st], (uint32_t)((u / C::QD_STAGES) & 1) ^ 1u, abort_flag, 102))) break;
           const int i0 = (it.blk0 + q) * 8;
           const int ntok = min(8, it.Lq - i0);
           const int t0 = it.qbase + i0;
@@ -224,18 +224,17 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
             tma_load_3d(sst + pn * C::QD_PANEL, &tmap_q, &qd_full[st], pn * 64, it.g * 8, t0);
             tma_load_3d(sst + C::QD_TILE + pn * C::QD_PANEL, &tmap_do, &qd_full[st], pn * 64, it.g * 8, t0);
           }
-          for (int tk = 0; tk < ntok; ++tk) {
-            bulk_g2s(sst + 2 * C::QD_TILE + tk * 64, p.LD + (size_t)(t0 + tk) * p.Hq + it.g * 8, 64, &qd_full[st]);
-            bulk_g2s(sst + 2 * C::QD_TILE + C::LD_BYTES + tk * 16,
-                     p.mask + (size_t)(t0 + tk) * p.mask_words + it.j * 4, 16, &qd_full[st]);
-          }
+          // the block's (lse, D) rows and selection words are contiguous: one copy each
+          bulk_g2s(sst + 2 * C::QD_TILE, p.LD + ((size_t)it.g * p.total_q + t0) * 8, ntok * 64, &qd_full[st]);
+          bulk_g2s(sst + 2 * C::QD_TILE + C::LD_BYTES, p.mask + ((size_t)it.j * p.total_q + t0) * 4, ntok * 16,
+                   &qd_full[st]);
         }
       }
       if (!ok) {
         // let the copies this thread issued land before the CTA exits (bounded)
         const uint64_t t0 = globaltimer_ns();
-        for (long long k = max(0LL, u - 2); k < u; ++k)
-          while (!mbar_try_wait(smem_u32(&qd_full[k & 1]), (uint32_t)((k >> 1) & 1)) &&
+        for (long long k = max(0LL, u - C::QD_STAGES); k < u; ++k)
+          while (!mbar_try_wait(smem_u32(&qd_full[k % C::QD_STAGES]), (uint32_t)((k / C::QD_STAGES) & 1)) &&
                  globaltimer_ns() - t0 < 100000000ull) {
           }
         if (m > 0)
@@ -251,8 +250,8 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
     const uint32_t v_base = smem_u32(smem + C::OFF_V);
     // S^T and dP^T of block uu (its stage must have landed and S/dP must be free)
     auto mma_s = [&](long long uu) -> bool {
-      const int st = (int)(uu & 1);
-      if (!mbar_wait(&qd_full[st], (uint32_t)((uu >> 1) & 1), abort_flag, 103)) return false;
+      const int st = (int)(uu % C::QD_STAGES);
+      if (!mbar_wait(&qd_full[st], (uint32_t)((uu / C::QD_STAGES) & 1), abort_flag, 103)) return false;
       if (!mbar_wait(s_empty, (uint32_t)(uu & 1) ^ 1u, abort_flag, 104)) return false;
       tc_fence_after();
       const uint32_t q_base = smem_u32(smem + C::OFF_ST + st * C::STAGE);
@@ -282,14 +281,14 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
         if (!(ok = mma_s(u))) break;
         for (int q = 0; q < it.nq && ok; ++q, ++u) {
           if (q + 1 < it.nq && !(ok = mma_s(u + 1))) break;
-          const int st = (int)(u & 1);
-          if (!(ok = mbar_wait(&p_full[st], (uint32_t)((u >> 1) & 1), abort_flag, 107))) break;
+          const int st = (int)(u % C::QD_STAGES), db = (int)(u & 1);
+          if (!(ok = mbar_wait(p_full, (uint32_t)(u & 1), abort_flag, 107))) break;
           if (q == 0 && !(ok = mbar_wait(acc_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 108))) break;
-          if (!(ok = mbar_wait(&dq_empty[st], (uint32_t)((u >> 1) & 1) ^ 1u, abort_flag, 109))) break;
+          if (!(ok = mbar_wait(&dq_empty[db], (uint32_t)((u >> 1) & 1) ^ 1u, abort_flag, 109))) break;
           tc_fence_after();
           const uint32_t q_base = smem_u32(smem + C::OFF_ST + st * C::STAGE);
           const uint32_t do_base = q_base + C::QD_TILE;
-          const uint32_t pt_base = smem_u32(smem + C::OFF_P + st * 2 * C::PT_BYTES);
+          const uint32_t pt_base = smem_u32(smem + C::OFF_P);
           const uint32_t ds_base = pt_base + C::PT_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // K = 64 rows, 16 per step
@@ -301,11 +300,11 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
           }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step
-            umma_bf16(tmem_base + 384 + st * 64, smem_desc_mn_sw128(k_base + kk * 16 * 128, C::KV_PANEL),
+            umma_bf16(tmem_base + 384 + db * 64, smem_desc_mn_sw128(k_base + kk * 16 * 128, C::KV_PANEL),
                       smem_desc_mn_sw128(ds_base + kk * 16 * 128, C::PT_BYTES), C::IDESC_Q, kk != 0);
-          umma_commit(&dq_full[st]);
+          umma_commit(&dq_full[db]);
           umma_commit(&qd_empty[st]);
-          umma_commit(&p_empty[st]);
+          umma_commit(p_empty);
         }
         if (!ok) break;
         umma_commit(acc_full);
@@ -335,13 +334,40 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&dq_empty[st]);
+      // 4 x 4 transposes among lanes 4a .. 4a + 3 (two xor-shuffle steps) give lane 4a + b the
+      // dims 32 quarter + 4a .. + 3 of row 4 grp + b, so each reduction carries 16 bytes
+      const int a = lane >> 2, b = lane & 3;
       const int i0 = (it.blk0 + q) * 8 + 4 * half;
 #pragma unroll
-      for (int tk = 0; tk < 4; ++tk) {
-        if (i0 + tk >= it.Lq) break;
-        float* dst = p.dQ_acc + ((size_t)(it.qbase + i0 + tk) * p.Hq + it.g * 8) * 128 + key;
-#pragma unroll
-        for (int hd = 0; hd < 8; ++hd) red_add_f32(dst + hd * 128, v[tk * 8 + hd] * p.scale);
+      for (int grp = 0; grp < 8; ++grp) {
+        float x0 = v[4 * grp], x1 = v[4 * grp + 1], x2 = v[4 * grp + 2], x3 = v[4 * grp + 3];
+        {
+          const float r0 = __shfl_xor_sync(0xffffffffu, (b & 1) ? x0 : x1, 1);
+          const float r1 = __shfl_xor_sync(0xffffffffu, (b & 1) ? x2 : x3, 1);
+          if (b & 1) {
+            x0 = r0;
+            x2 = r1;
+          } else {
+            x1 = r0;
+            x3 = r1;
+          }
+        }
+        {
+          const float r0 = __shfl_xor_sync(0xffffffffu, (b & 2) ? x0 : x2, 2);
+          const float r1 = __shfl_xor_sync(0xffffffffu, (b & 2) ? x1 : x3, 2);
+          if (b & 2) {
+            x0 = r0;
+            x1 = r1;
+          } else {
+            x2 = r0;
+            x3 = r1;
+          }
+        }
+        const int c = 4 * grp + b;  // column: token 4 half + c / 8, head c % 8
+        if (i0 + (c >> 3) < it.Lq)
+          red_add_v4(p.dQ_acc + ((size_t)(it.qbase + i0 + (c >> 3)) * p.Hq + it.g * 8 + (c & 7)) * 128 + quarter * 32 +
+                         4 * a,
+                     x0 * p.scale, x1 * p.scale, x2 * p.scale, x3 * p.scale);
       }
       return true;
     };
@@ -352,9 +378,9 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
       SABwdItem it;
       sa_bwd_item(id, p, it);
       for (int q = 0; q < it.nq; ++q, ++u) {
-        const int st = (int)(u & 1);
+        const int st = (int)(u % C::QD_STAGES);
         // this block's lse / D / selection bits arrive with its query tiles
-        if (!(ok = mbar_wait(&qd_full[st], (uint32_t)((u >> 1) & 1), abort_flag, 112))) break;
+        if (!(ok = mbar_wait(&qd_full[st], (uint32_t)((u / C::QD_STAGES) & 1), abort_flag, 112))) break;
         if (!(ok = mbar_wait(s_full, (uint32_t)(u & 1), abort_flag, 113))) break;
         tc_fence_after();
         float sv[32], dp[32];
@@ -388,9 +414,9 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
             pk_d[tk * 4 + hp] = *reinterpret_cast<uint32_t*>(&bd);
           }
         }
-        if (!(ok = mbar_wait(&p_empty[st], (uint32_t)((u >> 1) & 1) ^ 1u, abort_flag, 114))) break;
+        if (!(ok = mbar_wait(p_empty, (uint32_t)(u & 1) ^ 1u, abort_flag, 114))) break;
         // row `key` of P^T and dS^T: 16-byte chunks 4 half .. 4 half + 3 of its 128 bytes
-        const uint32_t pt_row = smem_u32(smem + C::OFF_P + st * 2 * C::PT_BYTES) + key * 128;
+        const uint32_t pt_row = smem_u32(smem + C::OFF_P) + key * 128;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           const uint32_t off = (uint32_t)(((4 * half + c4) ^ (key & 7)) * 16);
@@ -403,7 +429,7 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
         }
         fence_proxy_async_shared();  // the tensor core reads P^T and dS^T through the async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[st]);
+        if (lane == 0) mbar_arrive(p_full);
         if (q > 0 && !(ok = dq_out(u - 1, it, q - 1))) break;
       }
       if (!ok) break;
@@ -449,9 +475,11 @@ __global__ void __launch_bounds__(SABwdTcCfg::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
-// LD[t,h] = (lse[t,h] log2(e), dO[t,h] . O[t,h]); one warp per (t, h), d = 128
+// LD[g, t, i] = (lse[t,h] log2(e), dO[t,h] . O[t,h]) for h = 8 g + i; one warp per (t, h),
+// d = 128
 __global__ void sa_bwd_prep_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
-                                   const float* __restrict__ lse, long long rows, float2* __restrict__ LD) {
+                                   const float* __restrict__ lse, long long T, int Hq, float2* __restrict__ LD) {
+  const long long rows = T * Hq;
   const long long r = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (r >= rows) return;
@@ -463,17 +491,19 @@ __global__ void sa_bwd_prep_kernel(const uint16_t* __restrict__ O, const uint16_
   acc = fmaf(__uint_as_float(a.y & 0xFFFF0000u), __uint_as_float(b.y & 0xFFFF0000u), acc);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) LD[r] = make_float2(lse[r] * 1.4426950408889634f, acc);
+  const long long t = r / Hq;
+  const int h = (int)(r % Hq);
+  if (lane == 0) LD[((long long)(h / 8) * T + t) * 8 + (h % 8)] = make_float2(lse[r] * 1.4426950408889634f, acc);
 }
 
 // selection bits: one thread per (row, slot); -1 slots (and out-of-range values) are skipped
 __global__ void sa_bwd_mask_kernel(const int* __restrict__ indices, long long rows, int k, uint32_t* mask,
-                                   int mask_words) {
+                                   int tiles) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * k) return;
   const int s = indices[i];
-  if (s < 0 || s >= mask_words * 32) return;
-  atomicOr(mask + (i / k) * mask_words + (s >> 5), 1u << (s & 31));
+  if (s < 0 || s >= tiles * 128) return;
+  atomicOr(mask + ((long long)(s >> 7) * rows + i / k) * 4 + ((s >> 5) & 3), 1u << (s & 31));
 }
 
 }  // namespace dsa
@@ -528,10 +558,10 @@ int sa_bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O,
   if (total_q > 0) {
     const long long rows = total_q * Hq;
     dsa::sa_bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
-        static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), lse, rows, LD);
+        static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), lse, total_q, Hq, LD);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
     const long long n = total_q * k;
-    dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, total_q, k, mask, mw);
+    dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, total_q, k, mask, mw / 4);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
   }
   CUtensorMap tq, tdo, tk, tv;
@@ -559,9 +589,9 @@ int sa_bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O,
   p.n_items = (long long)p.tiles_max * batch * Hkv;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.total_q = total_q;
   p.LD = LD;
   p.mask = mask;
-  p.mask_words = mw;
   p.dQ_acc = dq_acc;
   p.dK = static_cast<uint16_t*>(dK);
   p.dV = static_cast<uint16_t*>(dV);
