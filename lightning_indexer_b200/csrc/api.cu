@@ -35,6 +35,11 @@ int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const
 
 size_t sparse_attn_bwd_workspace_bytes(long long total_k, int Hkv, int d);
 bool sa_bwd_tc_eligible(int Hq, int Hkv, int d, int k, int max_seqlen_k);
+bool sa_fwd_tc_eligible(int Hq, int Hkv, int d, int k, int max_seqlen_k);
+size_t sa_fwd_tc_scratch_bytes(long long total_q, int Hq, int max_seqlen_k);
+int sa_fwd_tc_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                     const int* cu_k, int batch, long long total_q, long long total_k, int Hq, int Hkv, int k,
+                     int max_seqlen_k, float scale, void* O, float* lse, void* mask_ws, cudaStream_t s);
 size_t sa_bwd_tc_workspace_bytes(long long total_q, int Hq, int max_seqlen_k);
 int sa_bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* lse,
                      const int* indices, const int* cu_q, const int* cu_k, int batch, long long total_q,
@@ -273,6 +278,15 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
     if (st != DSA_OK) return st;
     st = dsa_topk(scores, ld, cu_seqlens_q, cu_seqlens_k, batch, r0, r1, k, indices + r0 * k, nullptr, 0, stream);
     if (st != DSA_OK) return st;
+  }
+  // dense selected sets: masked dense tensor-core passes, their selection words and row
+  // maxima in the score scratch (free once the last chunk is selected)
+  if (lse && sa_fwd_tc_eligible(Hq, Hkv, d, k, max_seqlen_k) &&
+      sa_fwd_tc_scratch_bytes(total_q, Hq, max_seqlen_k) <= workspace_bytes) {
+    if (batch < 1 || total_q < 0 || total_k < 0 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DSA_ERR_INVALID_ARG;
+    return sa_fwd_tc_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, Hq, Hkv, k,
+                            max_seqlen_k, scale, O, lse, workspace, static_cast<cudaStream_t>(stream));
   }
   return dsa_sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k, scale,
                                  O, lse, stream);

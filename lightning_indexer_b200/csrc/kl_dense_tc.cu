@@ -27,9 +27,16 @@ struct KlLseParams {
   int batch;
   int Hq, Hkv;
   float scale_log2;
-  float* lse_out;  // [T, Hq] base-2 log
+  float* lse_out;  // [T, Hq]: base-2 log times out_scale
+  float out_scale;     // 1 (base 2) or ln 2 (natural log)
   long long n_blocks;  // 16-row blocks over all sequences
   long long n_items;   // n_blocks * Hkv
+  // optional selection: only keys whose bit is set count (bit s % 32 of word
+  // ((s / 128) * T + t) * 4 + (s % 128) / 32); blocks with no visible key are kept then,
+  // so that their rows get -inf
+  const uint32_t* mask;
+  long long total_q;
+  float* max_out;  // optional [T, Hq]: the row maxima of the scaled logits in base 2
 };
 
 struct KlLseItem {
@@ -53,7 +60,7 @@ __device__ __forceinline__ bool kl_lse_item(long long item, const KlLseParams& p
       it.kbase = p.cu_k[b];
       const int vis_last = min(max(it.i0 + it.ntok - 1 + it.Lk - it.Lq + 1, 0), it.Lk);
       it.ntiles = (vis_last + 127) / 128;
-      return it.ntiles > 0;
+      return it.ntiles > 0 || p.mask != nullptr;
     }
     r -= nb;
   }
@@ -209,8 +216,15 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
       const int vis = valid ? causal_vis(it.i0 + u, it.Lq, it.Lk) : 0;
       // running max of the raw logits and sum of 2^(scale (x - max)) (scale > 0)
       float mx = -INFINITY, l = 0.f;
+      const uint32_t* mrow = p.mask ? p.mask + (it.t0 + (valid ? u : 0)) * 4 + 2 * half : nullptr;
       for (int j = 0; j < it.ntiles; ++j, ++n) {
         const int ab = (int)(n & 1);
+        // selection words of this row for the half's 64 keys (all set without a selection)
+        uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
+        if (mrow) {
+          w0 = mrow[(long long)j * p.total_q * 4];
+          w1 = mrow[(long long)j * p.total_q * 4 + 1];
+        }
         if (!(ok = mbar_wait(&acc_full[ab], (uint32_t)((n >> 1) & 1), abort_flag, 65))) break;
         tc_fence_after();
         float v[64];
@@ -224,6 +238,11 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
 #pragma unroll
           for (int q = 0; q < 64; ++q)
             if (q >= nvis) v[q] = -INFINITY;
+        }
+        if ((w0 & w1) != 0xffffffffu) {
+#pragma unroll
+          for (int q = 0; q < 64; ++q)
+            if (!(((q < 32 ? w0 : w1) >> (q & 31)) & 1u)) v[q] = -INFINITY;
         }
         float cm = v[0];
 #pragma unroll
@@ -260,7 +279,11 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
         const float M = fmaxf(mx, o.x);
         float L = 0.f;
         if (M > -INFINITY) L = l * ex2_ftz((mx - M) * p.scale_log2) + o.y * ex2_ftz((o.x - M) * p.scale_log2);
-        if (valid) p.lse_out[(it.t0 + u) * p.Hq + it.g * G + (r % 8)] = L > 0.f ? M * p.scale_log2 + log2f(L) : -INFINITY;
+        if (valid) {
+          const long long o = (it.t0 + u) * p.Hq + it.g * G + (r % 8);
+          p.lse_out[o] = L > 0.f ? (M * p.scale_log2 + log2f(L)) * p.out_scale : -INFINITY;
+          if (p.max_out) p.max_out[o] = L > 0.f ? M * p.scale_log2 : -INFINITY;
+        }
       }
       ++m;
     }
@@ -607,9 +630,10 @@ __global__ void kl_parts_sum_kernel(const float4* part, long long T, float* kl) 
 namespace dsa_host {
 
 // Dense LSE of every (row, head) for d = 128 and 8 query heads per KV head.
+// lse_out = base-2 LSE times out_scale; with `mask`, over the selected keys only.
 int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
-                     cudaStream_t s) {
+                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out) {
   using C = dsa::KlLseCfg;
   static bool attr_done = false;
   if (!attr_done) {
@@ -640,6 +664,10 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
   p.Hkv = Hkv;
   p.scale_log2 = scale_log2;
   p.lse_out = lse_out;
+  p.out_scale = out_scale;
+  p.mask = mask;
+  p.total_q = T;
+  p.max_out = max_out;
   // an upper bound on the 16-row blocks (each sequence rounds up once)
   p.n_blocks = (T + 15) / 16 + batch;
   p.n_items = p.n_blocks * Hkv;

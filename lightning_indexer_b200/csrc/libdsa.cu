@@ -9,5 +9,6 @@
 #include "sparse_attn_bwd_tc.cu"
 #include "kl_bwd_tc.cu"
 #include "kl_dense_tc.cu"
+#include "sparse_attn_tc.cu"
 #include "kl_loss.cu"
 #include "decode_noalloc.cu"

@@ -514,6 +514,19 @@ int f32_to_bf16_launch(const float* src, void* dst, long long n, cudaStream_t st
 
 static size_t r256b(size_t x) { return (x + 255) / 256 * 256; }
 
+// selection words of `indices` (layout of SABwdTcParams::mask) into `mask`, which it clears
+// first (total_q * ceil(max_seqlen_k / 128) * 16 bytes)
+int sa_bwd_mask_build(const int* indices, long long total_q, int k, int max_seqlen_k, uint32_t* mask,
+                      cudaStream_t s) {
+  const int tiles = (max_seqlen_k + 127) / 128;
+  if (const cudaError_t e_ = cudaMemsetAsync(mask, 0, (size_t)total_q * tiles * 16, s); e_ != cudaSuccess)
+    return cuda_fail(e_);
+  const long long n = total_q * k;
+  if (n <= 0) return DSA_OK;
+  dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, total_q, k, mask, tiles);
+  return last_launch_status();
+}
+
 bool sa_bwd_tc_eligible(int Hq, int Hkv, int d, int k, int max_seqlen_k) {
   return d == 128 && Hq == 8 * Hkv && max_seqlen_k > 0 && 8LL * k >= (long long)max_seqlen_k;
 }

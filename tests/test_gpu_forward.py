@@ -310,11 +310,17 @@ def test_prefill_pipeline_integer_bit_exact_sets():
 
 
 def test_prefill_pipeline_gaussian_varlen():
+    # d = 128, 8 heads per KV head and 8 k >= the longest sequence: the pipeline takes the
+    # masked dense attention passes; the gather kernel on the same sets must agree on every row
     wl = gen.make_prefill([1500, 700, 2300], 32, 4, 128, 64, 128, 512, seed=41, layout="video")
     t = to_device(wl)
-    idx, O, lse = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_q"], t["cu_k"],
-                              t["max_q"], t["max_k"], wl.topk, chunk_rows=1024)
-    idx, O = idx.cpu().numpy(), O.float().cpu().numpy()
+    idx_t, O_t, lse_t = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_q"], t["cu_k"],
+                                    t["max_q"], t["max_k"], wl.topk, chunk_rows=1024)
+    O_g, lse_g = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx_t, t["cu_q"], t["cu_k"])
+    # two bf16-rounded results, each within ATTN_ATOL of the exact value
+    assert torch.max(torch.abs(O_t.float() - O_g.float())).item() <= 2 * ATTN_ATOL
+    assert torch.max(torch.abs(lse_t - lse_g)).item() <= LSE_ATOL
+    idx, O, lse = idx_t.cpu().numpy(), O_t.float().cpu().numpy(), lse_t.cpu().numpy()
     D = orc.Decoded(wl)
     rows = orc.sample_rows(wl.Tq, seed=5, n_first=32, n_last=32, n_mid=96) + [1499, 1500, 2199, 2200]
     swaps = 0
@@ -326,6 +332,7 @@ def test_prefill_pipeline_gaussian_varlen():
         if nsw == 0:
             assert np.array_equal(idx[r], ref["idx"])
             assert np.max(np.abs(O[r] - ref["O"])) <= ATTN_ATOL, r
+            assert np.max(np.abs(lse[r] - ref["lse"])) <= LSE_ATOL, r
 
 
 def test_prefill_from_host_matches_device_prefill():
