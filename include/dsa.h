@@ -183,6 +183,11 @@ DSA_API int dsa_sparse_attn_decode_noalloc(const void* Q, const void* K, const v
  *   max_seqlen_q / max_seqlen_k: host ints >= every Lq / Lk.
  *   indices device int32 [total_q, k] receives the selected sets.
  *   workspace: dsa_prefill_workspace_size(chunk_rows, max_seqlen_k) bytes.
+ *   Step (3) is the gather kernel of (3), except when the selected sets are dense (d = 128,
+ *   Hq = 8 Hkv, 8 k >= max_seqlen_k), lse is not NULL and the score scratch also holds
+ *   total_q * ceil(max_seqlen_k / 128) * 16 bytes of selection bits plus total_q * Hq * 4
+ *   bytes: then masked dense tensor-core passes compute the same O and lse (within the
+ *   same rounding bound).
  * ------------------------------------------------------------------------------- */
 DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k);
 DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, const void* Q,
