@@ -35,14 +35,17 @@ struct SAFwdTcParams {
 struct SAFwdTcCfg {
   static constexpr int TILE_BYTES = 128 * 128 * 2;
   static constexpr int PANEL_BYTES = 128 * 128;
-  static constexpr int KV_STAGES = 2;
+  // K tiles are free after their S MMA, V tiles only after P.V: separate rings, the K ring
+  // one deeper so the next tiles' keys load while the epilogue works
+  static constexpr int K_STAGES = 3, V_STAGES = 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + TILE_BYTES;                       // stages of (K, V)
-  static constexpr int OFF_P = OFF_KV + KV_STAGES * 2 * TILE_BYTES;      // P
+  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + K_STAGES * TILE_BYTES;
+  static constexpr int OFF_P = OFF_V + V_STAGES * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_P + TILE_BYTES;
-  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], s_empty[2], p_full, p_empty,
-  // o_full, o_empty, done
-  static constexpr int NUM_BARS = 2 + 2 * KV_STAGES + 4 + 2 + 2 + 1;
+  // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2], s_empty[2],
+  // p_full, p_empty, o_full, o_empty, done
+  static constexpr int NUM_BARS = 2 + 2 * K_STAGES + 2 * V_STAGES + 4 + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int EPI_WARPS = 8;
@@ -63,9 +66,11 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;                   // [KV_STAGES]
-  uint64_t* kv_empty = kv_full + C::KV_STAGES;    // [KV_STAGES]
-  uint64_t* s_full = kv_empty + C::KV_STAGES;     // [2]
+  uint64_t* k_full = bars + 2;                    // [K_STAGES]
+  uint64_t* k_empty = k_full + C::K_STAGES;       // [K_STAGES]
+  uint64_t* v_full = k_empty + C::K_STAGES;       // [V_STAGES]
+  uint64_t* v_empty = v_full + C::V_STAGES;       // [V_STAGES]
+  uint64_t* s_full = v_empty + C::V_STAGES;       // [2]
   uint64_t* s_empty = s_full + 2;                 // [2]
   uint64_t* p_full = s_full + 4;
   uint64_t* p_empty = s_full + 5;
@@ -80,9 +85,13 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < C::KV_STAGES; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+    for (int i = 0; i < C::K_STAGES; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < C::V_STAGES; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -125,22 +134,31 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
           tma_load_3d(smem + C::OFF_Q + pn * C::PANEL_BYTES, &tmap_q, q_full, pn * 64, it.g * G, (int)it.t0);
         ++m;
         for (int j = 0; j < it.ntiles; ++j, ++n) {
-          const int st = (int)(n % C::KV_STAGES);
-          if (!(ok = mbar_wait(&kv_empty[st], (uint32_t)((n / C::KV_STAGES) & 1) ^ 1u, abort_flag, 121))) break;
-          mbar_arrive_expect_tx(&kv_full[st], 2 * C::TILE_BYTES);
-          uint8_t* sk = smem + C::OFF_KV + st * 2 * C::TILE_BYTES;
-          for (int pn = 0; pn < 2; ++pn) {
-            tma_load_3d(sk + pn * C::PANEL_BYTES, &tmap_k, &kv_full[st], pn * 64, it.g, it.kbase + j * 128);
-            tma_load_3d(sk + C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_v, &kv_full[st], pn * 64, it.g,
-                        it.kbase + j * 128);
+          const int ks = (int)(n % C::K_STAGES), vs = (int)(n % C::V_STAGES);
+          if (!(ok = mbar_wait(&k_empty[ks], (uint32_t)((n / C::K_STAGES) & 1) ^ 1u, abort_flag, 121))) break;
+          mbar_arrive_expect_tx(&k_full[ks], C::TILE_BYTES);
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(smem + C::OFF_K + ks * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &k_full[ks], pn * 64,
+                        it.g, it.kbase + j * 128);
+          if (!(ok = mbar_wait(&v_empty[vs], (uint32_t)((n / C::V_STAGES) & 1) ^ 1u, abort_flag, 130))) {
+            ++n;  // this tile's K copy is in flight: the drain below waits for it
+            break;
           }
+          mbar_arrive_expect_tx(&v_full[vs], C::TILE_BYTES);
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(smem + C::OFF_V + vs * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_v, &v_full[vs], pn * 64,
+                        it.g, it.kbase + j * 128);
         }
       }
       if (!ok) {
         // let the copies this thread issued land before the CTA exits (bounded)
         const uint64_t t0 = globaltimer_ns();
-        for (long long k = max(0LL, n - C::KV_STAGES); k < n; ++k)
-          while (!mbar_try_wait(smem_u32(&kv_full[k % C::KV_STAGES]), (uint32_t)((k / C::KV_STAGES) & 1)) &&
+        for (long long k = max(0LL, n - C::K_STAGES); k < n; ++k)
+          while (!mbar_try_wait(smem_u32(&k_full[k % C::K_STAGES]), (uint32_t)((k / C::K_STAGES) & 1)) &&
+                 globaltimer_ns() - t0 < 100000000ull) {
+          }
+        for (long long k = max(0LL, n - C::V_STAGES); k < n; ++k)
+          while (!mbar_try_wait(smem_u32(&v_full[k % C::V_STAGES]), (uint32_t)((k / C::V_STAGES) & 1)) &&
                  globaltimer_ns() - t0 < 100000000ull) {
           }
         if (m > 0)
@@ -157,11 +175,11 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
       const uint32_t p_base = smem_u32(smem + C::OFF_P);
       // S of key tile number nn (its stage landed, its TMEM buffer free)
       auto mma_s = [&](long long nn) -> bool {
-        const int st = (int)(nn % C::KV_STAGES), sb = (int)(nn & 1);
-        if (!mbar_wait(&kv_full[st], (uint32_t)((nn / C::KV_STAGES) & 1), abort_flag, 122)) return false;
+        const int ks = (int)(nn % C::K_STAGES), sb = (int)(nn & 1);
+        if (!mbar_wait(&k_full[ks], (uint32_t)((nn / C::K_STAGES) & 1), abort_flag, 122)) return false;
         if (!mbar_wait(&s_empty[sb], (uint32_t)((nn >> 1) & 1) ^ 1u, abort_flag, 123)) return false;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(smem + C::OFF_KV + st * 2 * C::TILE_BYTES);
+        const uint32_t k_base = smem_u32(smem + C::OFF_K + ks * C::TILE_BYTES);
 #pragma unroll
         for (int pn = 0; pn < 2; ++pn)
 #pragma unroll
@@ -169,6 +187,7 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
             umma_bf16(tmem_base + sb * 128, smem_desc_kmajor(q_base + pn * C::PANEL_BYTES + kk * 32, 128),
                       smem_desc_kmajor(k_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC_S, (pn | kk) != 0);
         umma_commit(&s_full[sb]);
+        umma_commit(&k_empty[ks]);
         return true;
       };
       for (long long item = blockIdx.x; item < ip.n_items && ok; item += gridDim.x) {
@@ -184,14 +203,16 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
           if (!(ok = mbar_wait(p_full, (uint32_t)(nn & 1), abort_flag, 125))) break;
           if (j == 0 && !(ok = mbar_wait(o_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 126))) break;
           tc_fence_after();
-          const int st = (int)(nn % C::KV_STAGES);
-          const uint32_t v_base = smem_u32(smem + C::OFF_KV + st * 2 * C::TILE_BYTES + C::TILE_BYTES);
+          const int vs = (int)(nn % C::V_STAGES);
+          if (!(ok = mbar_wait(&v_full[vs], (uint32_t)((nn / C::V_STAGES) & 1), abort_flag, 131))) break;
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step
             umma_bf16(tmem_base + 256,
                       smem_desc_kmajor(p_base + (kk / 4) * C::PANEL_BYTES + (kk % 4) * 32, 128),
                       smem_desc_mn_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES), C::IDESC_O, (j | kk) != 0);
-          umma_commit(&kv_empty[st]);
+          umma_commit(&v_empty[vs]);
           umma_commit(p_empty);
         }
         if (!ok) break;
