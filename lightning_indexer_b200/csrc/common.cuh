@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "../../include/dsa.h"
@@ -390,6 +391,35 @@ int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 
 int make_tmap_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
                       const uint32_t box[3]);
+
+// A one-time-setup flag kept per GPU: cudaFuncSetAttribute applies to the current device
+// only, and one process may drive several GPUs.  Reads and writes go to the current
+// device's bit (devices past 63 always read false, so their setup simply repeats).
+class DeviceFlag {
+ public:
+  constexpr DeviceFlag() = default;
+  operator bool() const {
+    const int d = device();
+    return d < 64 && ((bits_.load(std::memory_order_acquire) >> d) & 1ull);
+  }
+  DeviceFlag& operator=(bool v) {
+    const int d = device();
+    if (d < 64) {
+      if (v)
+        bits_.fetch_or(1ull << d, std::memory_order_acq_rel);
+      else
+        bits_.fetch_and(~(1ull << d), std::memory_order_acq_rel);
+    }
+    return *this;
+  }
+
+ private:
+  static int device() {
+    int d = 0;
+    return cudaGetDevice(&d) == cudaSuccess && d >= 0 ? d : 64;
+  }
+  std::atomic<unsigned long long> bits_{0};
+};
 
 int sm_count();
 int last_launch_status();    // DSA_ERR_CUDA if the last launch failed, else DSA_OK

@@ -343,7 +343,7 @@ static int launch_indexer(const void* q_idx, const void* k_idx, const void* w, c
                           float* scores, long long ld, int tiles_per_split, cudaStream_t stream) {
   using C = dsa::IndexerCfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
   auto kern = dsa::indexer_kernel<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   const int smem = std::max(C::SMEM_BYTES, 120 * 1024);  // one CTA per SM (TMEM ownership)
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);

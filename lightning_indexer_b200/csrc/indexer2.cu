@@ -283,7 +283,7 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
                            cudaStream_t stream) {
   using C = dsa::Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
   auto kern = dsa::indexer2_kernel<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   const int smem = std::max(C::SMEM_BYTES, 120 * 1024);
   if (!attr_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

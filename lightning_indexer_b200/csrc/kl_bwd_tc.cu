@@ -860,7 +860,7 @@ int kl_dk_tc_launch(const void* q_idx, const void* k_idx, const void* w, const i
                     int batch, long long total_q, long long total_k, int max_seqlen_k, long long r0, long long r1,
                     const float* g, long long ld, float* dk_part, int* offs, float* dk_acc, cudaStream_t s) {
   using C = dsa::KlDkCfg;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_dk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);
@@ -908,7 +908,7 @@ int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const i
                     long long total_q, long long total_k, long long r0, long long r1, const float* g, long long ld,
                     void* dq, void* dw, cudaStream_t s) {
   using C = dsa::KlDqCfg;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);

@@ -635,7 +635,7 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
                      cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out) {
   using C = dsa::KlLseCfg;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_lse_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);
@@ -684,7 +684,7 @@ int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int
                         const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
                         float* kl_part, cudaStream_t s) {
   using C = dsa::KlTgtCfg;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_tc_kernel,
                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);

@@ -691,7 +691,7 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
   } else {
     auto kern = dsa::idx_bwd_row_kernel<H_I, D_I>;
     const int smem = 2 * 64 * D_I * 2;
-    static bool done = false;
+    static DeviceFlag done;
     if (!done) {
       if (const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
       done = true;
@@ -710,7 +710,7 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
     const long long part_stride = Tk * D_I;
     auto kern = dsa::idx_bwd_col_kernel<H_I, D_I>;
     const int smem = 2 * H_I * D_I * 2 + 2 * H_I * 4 + 2 * 128 * 4;
-    static bool done = false;
+    static DeviceFlag done;
     if (!done) {
       if (const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); e_ != cudaSuccess) return cuda_fail(e_);
       done = true;
@@ -751,7 +751,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     const int smem = dsa::KL_WARPS * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;
     if (blocks > 0) {
       if (d == 128) {
-        static bool done = false;
+        static DeviceFlag done;
         if (!done) {
           const cudaError_t e_ = cudaFuncSetAttribute(dsa::dense_lse_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           smem);
@@ -762,7 +762,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, T, Hq, Hkv,
             scale_log2, W.lse_att);
       } else {
-        static bool done = false;
+        static DeviceFlag done;
         if (!done) {
           const cudaError_t e_ = cudaFuncSetAttribute(dsa::dense_lse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           smem);
@@ -793,7 +793,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     } else {
       const int smem = Hkv * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;
       if (d == 128) {
-        static bool done = false;
+        static DeviceFlag done;
         if (!done) {
           const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           8 * dsa::KL_STAGES * dsa::KL_CHUNK * 128 * 2);
@@ -804,7 +804,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
             static_cast<const uint16_t*>(Q), static_cast<const uint16_t*>(K), cu_q, cu_k, batch, r0, Hq, Hkv,
             scale_log2, W.lse_att, W.lseI, W.scores, ld, inv_T, kl);
       } else {
-        static bool done = false;
+        static DeviceFlag done;
         if (!done) {
           const cudaError_t e_ = cudaFuncSetAttribute(dsa::kl_target_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           8 * dsa::KL_STAGES * dsa::KL_CHUNK * 64 * 2);

@@ -379,7 +379,7 @@ template <int D, int STAGES, int WARPS>
 static int sa_launch_d(const dsa::SAParams& p, long long tasks, cudaStream_t stream) {
   const long long blocks = (tasks + WARPS - 1) / WARPS;
   const int smem = dsa::sa_smem_bytes<D, STAGES>(WARPS);
-  static bool done = false;
+  static DeviceFlag done;
   if (!done) {
     cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_kernel<D, STAGES, WARPS>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

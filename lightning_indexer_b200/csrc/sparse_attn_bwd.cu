@@ -305,7 +305,7 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
   const int smem = dsa::BWD_WARPS * dsa::BWD_STAGES * 2 * dsa::BWD_CHUNK * d * 2;
   if (blocks > 0) {
     if (d == 128) {
-      static bool done = false;
+      static DeviceFlag done;
       if (!done) {
         if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem); e_ != cudaSuccess) return cuda_fail(e_);
@@ -317,7 +317,7 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
       }
       dsa::sparse_attn_bwd_kernel<128><<<(unsigned)blocks, dsa::BWD_WARPS * 32, smem, stream>>>(p);
     } else {
-      static bool done = false;
+      static DeviceFlag done;
       if (!done) {
         if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sparse_attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem); e_ != cudaSuccess) return cuda_fail(e_);

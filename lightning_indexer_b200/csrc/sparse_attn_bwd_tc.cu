@@ -542,7 +542,7 @@ int sa_bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O,
                      long long total_k, int Hq, int Hkv, int k, int max_seqlen_k, float scale, void* dQ, void* dK,
                      void* dV, void* ws, cudaStream_t s) {
   using C = dsa::SABwdTcCfg;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sa_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);

@@ -349,7 +349,7 @@ int sa_fwd_tc_launch(const void* Q, const void* K, const void* V, const int* ind
                      const int* cu_k, int batch, long long total_q, long long total_k, int Hq, int Hkv, int k,
                      int max_seqlen_k, float scale, void* O, float* lse, void* mask_ws, cudaStream_t s) {
   using C = dsa::SAFwdTcCfg;
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sa_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     C::SMEM_BYTES);

@@ -1350,7 +1350,7 @@ namespace dsa_host {
 
 template <typename Kern>
 static int launch_cluster(Kern kern, const dsa::TopkParams& p, long long rows, int C, int threads, int smem,
-                          bool& attr_done, cudaStream_t stream) {
+                          DeviceFlag& attr_done, cudaStream_t stream) {
   if (!attr_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e_ != cudaSuccess) return cuda_fail(e_);
@@ -1374,7 +1374,7 @@ static int launch_cluster(Kern kern, const dsa::TopkParams& p, long long rows, i
 
 template <int C>
 static int topk_launch_c(dsa::TopkParams p, long long rows, cudaStream_t stream) {
-  static bool fast_done = false, exact_done = false;
+  static DeviceFlag fast_done, exact_done;
   p.only_marked = 0;
   int st = launch_cluster(dsa::topk_fast_kernel<C>, p, rows, C, dsa::FT, (int)sizeof(dsa::FastSmem), fast_done,
                           stream);
@@ -1387,7 +1387,7 @@ static int topk_launch_c(dsa::TopkParams p, long long rows, cudaStream_t stream)
 template <int C>
 static int topk_regs_launch(const dsa::TopkParams& p, long long rows, cudaStream_t stream) {
   static_assert(C <= 8, "portable cluster sizes only");
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_regs_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 (int)sizeof(dsa::RegsSmem));
@@ -1413,7 +1413,7 @@ static int topk_regs_launch(const dsa::TopkParams& p, long long rows, cudaStream
 
 // One block per row with the streaming kernel, then the exact kernel for rows it marked.
 static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t stream) {
-  static bool attr_done = false, exact_done = false;
+  static DeviceFlag attr_done, exact_done;
   if (!attr_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_stream_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e_ != cudaSuccess) return cuda_fail(e_);
@@ -1455,7 +1455,7 @@ static int topk_two_launch(const dsa::TopkParams& p, long long rows, long long m
   ws.cnt = reinterpret_cast<uint32_t*>(w);
   w += up((size_t)(rows * ws.nseg) * 4);
   ws.cand = reinterpret_cast<uint2*>(w);
-  static bool attr_done = false;
+  static DeviceFlag attr_done;
   if (!attr_done) {
     // four filter blocks per SM need the largest shared-memory carveout
     cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_segfilter_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
