@@ -1,4 +1,5 @@
-// Key-stationary indexer backward of the KL loss on tcgen05 tensor cores (sm_100a).
+// Indexer backward of the KL loss on tcgen05 tensor cores (sm_100a): the key-stationary
+// dk_idx kernel (first below) and the row-stationary dw / dq_idx kernel (second).
 //
 // Source: Keye-VL-2.0 report summary (mqxn.cn/news/1966), section 1: in the dense warm-up
 // only the indexer is trained, by the KL divergence to the full attention distribution.
