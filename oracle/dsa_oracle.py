@@ -315,15 +315,16 @@ def sparse_attention_backward(D: Decoded, idx: np.ndarray, O: np.ndarray, lse: n
         sel = idx[r][idx[r] >= 0] + k0
         if sel.size == 0:
             continue
-        for h in range(Hq):
-            g = h // G
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)  # the query heads that read KV head g
             Ks = K[sel, g, :]
             Vs = V[sel, g, :]
-            P = np.exp(D.scale * (Ks @ Q[r, h]) - lse[r, h])
-            dS = P * (Vs @ dO[r, h] - float(dO[r, h] @ O[r, h]))
-            dQ[r, h] = D.scale * (dS @ Ks)
-            np.add.at(dK[:, g, :], sel, D.scale * dS[:, None] * Q[r, h][None, :])
-            np.add.at(dV[:, g, :], sel, P[:, None] * dO[r, h][None, :])
+            P = np.exp(D.scale * (Ks @ Q[r, hs].T) - lse[r, hs])                   # [n, G]
+            dS = P * (Vs @ dO[r, hs].T - np.sum(dO[r, hs] * O[r, hs], axis=1))    # [n, G]
+            dQ[r, hs] = D.scale * (dS.T @ Ks)
+            # the sums over the group's heads (dS.Q and P.dO) are matrix products
+            np.add.at(dK[:, g, :], sel, D.scale * (dS @ Q[r, hs]))
+            np.add.at(dV[:, g, :], sel, P @ dO[r, hs])
     return {"dQ": dQ, "dK": dK, "dV": dV}
 
 

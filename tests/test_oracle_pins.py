@@ -240,6 +240,32 @@ def test_dense_target_closed_forms():
     assert abs(p.sum() - 1.0) < 1e-14 and np.all(p > 0)
 
 
+def test_dense_target_hand_worked_gqa():
+    # two KV heads, two query heads each: catches a wrong query-head -> KV-head mapping
+    # and a dropped softmax scale (the derivation lists what each mistake would give)
+    g = GOLD["dense_target_gqa"]
+    p = orc.dense_target_row(f64(g["Q"]), f64(g["K_vis"]), g["scale"])
+    np.testing.assert_allclose(p, f64(g["expected_p"]), rtol=0, atol=1e-15)
+
+
+def test_dense_target_is_head_mean_of_sdpa_with_identity_values():
+    # With V = the identity over the visible keys, attention of head h returns its softmax
+    # row itself, so the head mean of torch's SDPA outputs (fp64, GQA by repeat_interleave,
+    # the same scale) is the target p.  A dropped scale or KV head h % Hkv fails here.
+    rng = np.random.default_rng(12)
+    for Hq, Hkv, d, n in ((8, 2, 16, 11), (32, 4, 8, 5), (4, 1, 32, 9)):
+        G = Hq // Hkv
+        Q = rng.standard_normal((Hq, d))
+        K = rng.standard_normal((n, Hkv, d))
+        scale = 1.0 / math.sqrt(d)
+        p = orc.dense_target_row(Q, K, scale)
+        q = torch.from_numpy(Q)[:, None, :]                                         # [Hq, 1, d]
+        k = torch.from_numpy(K).repeat_interleave(G, dim=1).permute(1, 0, 2)       # [Hq, n, d]
+        v = torch.eye(n, dtype=torch.float64).expand(Hq, n, n)                     # [Hq, n, n]
+        out = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=scale)
+        np.testing.assert_allclose(p, out[:, 0, :].mean(0).numpy(), rtol=1e-12, atol=1e-15)
+
+
 def test_kl_gradients_by_finite_differences():
     wl = gen.make_prefill([9, 14], 4, 2, 8, 3, 4, 4, seed=9)
     D = orc.Decoded(wl)
