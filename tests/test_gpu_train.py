@@ -8,7 +8,7 @@ import lightning_indexer_b200 as dsa
 from oracle import dsa_oracle as orc
 from workloads import generators as gen
 
-from dsa_testutil import to_device
+from dsa_testutil import set_mismatch_ok, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -93,3 +93,50 @@ def test_indexer_kl_gradient_homogeneity_identity():
     c = float((t["q_idx"].float() * dq.float()).sum())
     scale = max(abs(a), abs(b), abs(c), 1e-30)
     assert abs(a - b) <= 3e-2 * scale and abs(a - c) <= 3e-2 * scale
+
+
+def test_training_medium_varlen_elementwise():
+    # Four packed sequences [2048, 1024, 512, 512], k = 512, Hq = 8, Hkv = 1, d = 128,
+    # H_I = 64, d_I = 128: every training kernel takes its tensor-core path (8 k >= 2048),
+    # the 2048-long sequence spans 16 key tiles of 128 and 8 KL dk items of 256 rows per
+    # tile, rows past 512 select a sparse set, and the later sequences sit at non-zero
+    # offsets of the pack.  Every element of dQ, dK, dV, dq_idx, dk_idx and dw is compared
+    # with the oracle.
+    wl = gen.make_prefill([2048, 1024, 512, 512], 8, 1, 128, 64, 128, 512, seed=55, with_dO=True,
+                          layout="video")
+    D = orc.Decoded(wl)
+    ref_f = orc.forward(D)
+    t = to_device(wl)
+    # the pipeline (indexer, top-k, masked dense attention) on the selected sets
+    idx_p, O_p, lse_p = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_q"], t["cu_k"],
+                                    t["max_q"], t["max_k"], wl.topk, chunk_rows=1024)
+    idx_p, O_p, lse_p = idx_p.cpu().numpy(), O_p.float().cpu().numpy(), lse_p.cpu().numpy()
+    exact = 0
+    for r in range(wl.Tq):
+        ok, nsw = set_mismatch_ok(idx_p[r], ref_f["idx"][r], ref_f["scores"][r])
+        assert ok, r
+        if nsw == 0:
+            exact += 1
+            assert np.max(np.abs(O_p[r] - ref_f["O"][r])) <= 1e-2, r
+            assert np.max(np.abs(lse_p[r] - ref_f["lse"][r])) <= 2e-3, r
+    assert exact >= 0.9 * wl.Tq
+    # backward on the oracle's sets, from the GPU forward's O and lse
+    ref_b = orc.sparse_attention_backward(D, ref_f["idx"], ref_f["O"], ref_f["lse"], D.full("dO"))
+    idx = torch.from_numpy(ref_f["idx"].astype(np.int32)).cuda()
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, t["cu_q"], t["cu_k"])
+    dQ, dK, dV = dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse, idx, t["cu_q"], t["cu_k"],
+                                             max_seqlen_k=t["max_k"])
+    assert _rel_err(dQ.float().cpu().numpy(), ref_b["dQ"]) <= 1.5e-2
+    assert _rel_err(dK.float().cpu().numpy(), ref_b["dK"]) <= 1.5e-2
+    assert _rel_err(dV.float().cpu().numpy(), ref_b["dV"]) <= 1.5e-2
+    # indexer KL loss and its gradients, in row chunks of 1024 and in one chunk
+    ref = orc.indexer_kl_loss(D)
+    for chunk in (1024, wl.Tq):
+        loss, kl, dq, dk, dw = dsa.indexer_kl_loss(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], t["cu_q"],
+                                                   t["cu_k"], t["max_q"], t["max_k"], chunk_rows=chunk)
+        kl = kl.cpu().numpy()
+        assert abs(loss.item() - ref["loss"]) <= 1e-4 * abs(ref["loss"]) + 1e-6
+        assert np.max(np.abs(kl - ref["kl"])) <= 1e-4 * np.max(np.abs(ref["kl"])) + 1e-6
+        assert _rel_err(dq.float().cpu().numpy(), ref["dq_idx"]) <= 1.5e-2
+        assert _rel_err(dk.float().cpu().numpy(), ref["dk_idx"]) <= 1.5e-2
+        assert _rel_err(dw.float().cpu().numpy(), ref["dw"]) <= 1.5e-2
