@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-train", action="store_true")
-    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode", "train"],
+    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode", "train", "index_topk"],
                     help="run one kernel on a small case (for profiler captures) instead of the bench")
     ap.add_argument("--case-len", type=int, default=16384, help="sequence length of the --case workload")
     ap.add_argument("--case-chunk", type=int, default=0,
@@ -391,6 +391,9 @@ def run_case(args):
     if args.case == "train":
         print(json.dumps(run_train(args, device)))
         return
+    if args.case == "index_topk":
+        print(json.dumps(run_index_topk_case(args, device)))
+        return
     L = args.case_len
     if args.case == "decode":
         wl = gen.make_decode(16, L, 32, 4, 128, 64, 128, 2048, seed=3, layout="video")
@@ -436,6 +439,38 @@ def run_case(args):
     ms = a.elapsed_time(b) / max(1, args.steps)
     print(json.dumps({"case": args.case, "len": L, "rows": [r0, Tq], "ms_per_iter": ms, "causal_pairs_in_rows": pairs,
                       "indexer_tflops": pairs * wl.H_I * wl.d_I * 2 / (ms / 1e3) / 1e12}))
+
+
+def run_index_topk_case(args, device):
+    """Selected sets of a video-layout prefill of --case-len tokens through dsa_index_topk:
+    the fused path against the separate indexer + top-k passes, same chunking, with the
+    two results compared for identity."""
+    import torch
+    import lightning_indexer_b200 as dsa
+    L = args.case_len
+    wl = gen.make_prefill([L], 32, 4, 128, 64, 128, 2048, seed=2, layout="video", max_frames=480)
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w")}
+    cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+    chunk = min(PREFILL_CHUNK, L)
+    ws = torch.empty(dsa.index_topk_workspace_bytes(chunk, L), dtype=torch.uint8, device=device)
+    out = {}
+    res = {"case": "index_topk", "len": L, "chunk_rows": chunk}
+    for name, path in (("fused", dsa.PATH_AUTO), ("separate", dsa.PATH_SEPARATE)):
+        idx = torch.empty((L, wl.topk), dtype=torch.int32, device=device)
+        run = lambda: dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, wl.topk,  # noqa: E731
+                                     chunk_rows=chunk, path=path, indices=idx, workspace=ws)
+        for _ in range(args.warmup):
+            run()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        res[name + "_ms"] = a.elapsed_time(b) / max(1, args.steps)
+        out[name] = idx
+    res["identical"] = bool(torch.equal(out["fused"], out["separate"]))
+    return res
 
 
 def run_train(args, device):

@@ -62,6 +62,12 @@ typedef enum {
   DSA_ERR_TIMEOUT = -5      /* a bounded device-side wait ran out (device status word) */
 } dsa_status;
 
+/* How dsa_index_topk finds the selected sets. */
+typedef enum {
+  DSA_PATH_AUTO = 0,     /* the fused indexer -> top-k where it applies, else the separate passes */
+  DSA_PATH_SEPARATE = 1  /* always the separate passes: dsa_index then dsa_topk per row chunk */
+} dsa_path;
+
 /* Human-readable name of a dsa_status value.  Never returns NULL. */
 DSA_API const char* dsa_status_string(int status);
 
@@ -77,6 +83,15 @@ DSA_API int dsa_last_cuda_error(const char** message);
  * DSA_ERR_TIMEOUT; *detail_out (may be NULL) receives a kernel-specific code of where
  * the wait ran out.  Returns DSA_ERR_CUDA if the synchronisation itself failed. */
 DSA_API int dsa_get_device_status(int* status_out, int* detail_out);
+
+/* Self-test of the bounded device waits (a diagnostic; the method has no counterpart).
+ * Launches one small kernel that waits, with the same bounded-wait routine the pipelined
+ * kernels use, on a barrier that nothing arrives at, for limit_ns nanoseconds (1 ns .. 1 s);
+ * the wait then gives up, records DSA_ERR_TIMEOUT with detail code 900 in the device status
+ * word, and the kernel returns.  Read the result with dsa_get_device_status().  The kernel
+ * holds no copies, tensor-core work or tensor memory when it gives up, so the context stays
+ * usable.  Returns DSA_ERR_INVALID_ARG for a limit outside that range. */
+DSA_API int dsa_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * (1) Lightning indexer scores.  Source: report summary section 1 (an MQA-shared
@@ -123,10 +138,37 @@ DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_s
                      int k, int32_t* indices, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * (2b) Indexer and top-k together: the selected sets of every query row, i.e. (2) applied
+ * to the scores of (1), without handing the scores to the caller.  Source: report summary
+ * section 1 (the indexer scans every position; each token keeps its k best) and section 8
+ * (deterministic top-k).  Rows are processed in chunks of at most `chunk_rows`.
+ *   indices device int32 [total_q, k]: as (2), ascending, -1 padded, bit-for-bit the sets
+ *           (2) returns on the scores of (1) (the same scores, the same tie rule).
+ *   path    DSA_PATH_AUTO: for (H_I, d_I) in {(64,128), (32,128)} with score rows of at
+ *           most 524288 positions and room for 2k candidates per row in the scratch, the
+ *           fused form: the indexer first scores every S-th key (S a power of two, about
+ *           1024 samples per full row) to bound each row's k-th largest score from below,
+ *           then scores every key again but keeps only the (score, position) pairs that
+ *           reach the bound, and an exact select over those pairs writes the sets; rows the
+ *           bound failed for (fewer than k pairs kept, or more than fit) are recomputed
+ *           in full and selected by the exact method.  Otherwise, and with
+ *           DSA_PATH_SEPARATE, (1) then (2) per chunk.
+ *   workspace  device scratch of dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k)
+ *           bytes (16-byte aligned): one chunk of fp32 score rows plus 256 bytes.
+ * Supported: the shapes of (1); 1 <= k <= 4096.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_index_topk_workspace_size(int64_t chunk_rows, int max_seqlen_k);
+DSA_API int dsa_index_topk(const void* q_idx, const void* k_idx, const void* w, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
+                           int max_seqlen_q, int max_seqlen_k, int H_I, int d_I, int k, int64_t chunk_rows,
+                           int path, int32_t* indices, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * (3) Sparse GQA attention, prefill/varlen.  Source: report summary section 1 (attention
  * only over the selected positions, O(L*k); GQA adapted to DSA: the one selected set of a
  * token is shared by all its query heads).  For row r, head h, KV head g = h/(Hq/Hkv),
- * set S = {indices[r,:] >= 0}:
+ * set S = the entries of indices[r,:] inside [0, vis(r)) (a -1 slot, or a position the
+ * row cannot see, including one past the end of its sequence, is ignored):
  *     O[r,h,:]  = sum_{s in S} softmax_s(scale * Q[r,h,:].K[k0+s,g,:]) V[k0+s,g,:]
  *     lse[r,h]  = natural log of sum_{s in S} exp(scale * Q[r,h,:].K[k0+s,g,:])
  * An empty set gives O = 0 and lse = -inf.
@@ -145,7 +187,8 @@ DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
  * (4) Sparse GQA attention, decode.  Source: report summary section 8 (a decode path
  * specific to DSA).  Same arithmetic as (3) for one query row per sequence (Lq == 1), with
  * the k selected keys split over several thread blocks and their partial softmax states
- * merged by log-sum-exp.
+ * merged by log-sum-exp.  The query of sequence b sees its whole cache (vis = Lk_b):
+ * entries of indices outside [0, Lk_b) are ignored like -1.
  *   Q device bf16 [batch, Hq, d]; K, V device bf16 [total_k, Hkv, d] (sequence b's cache
  *   is rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1); indices device int32 [batch, k];
  *   O device bf16 [batch, Hq, d]; lse device fp32 [batch, Hq] (may be NULL).
@@ -164,9 +207,12 @@ DSA_API int dsa_sparse_attn_decode(const void* Q, const void* K, const void* V,
  * latency-critical loop that must not call cudaMalloc) and have no scratch buffer to pass.
  * Same inputs, outputs and arithmetic as (4); the split-K scratch lives in a fixed 8 MiB
  * device array inside the library, held on every GPU that loads the library until exit.
- *   - Returns DSA_ERR_WORKSPACE when (4) would need more than 8 MiB of scratch, i.e. when
- *     dsa_sparse_attn_decode_workspace_size(batch, Hq, d, k) > 8388608 (at d = 128 and
- *     k = 2048 that allows batch * Hq <= 992).
+ *   - Arguments are checked as in (4), in the same order (DSA_ERR_INVALID_ARG, then
+ *     DSA_ERR_UNSUPPORTED); then it returns DSA_ERR_WORKSPACE when (4) would need more than
+ *     8 MiB of scratch, i.e. when dsa_sparse_attn_decode_workspace_size(batch, Hq, d, k) >
+ *     8388608 (at d = 128 and k = 2048 that allows batch * Hq <= 992).
+ *   - Device ordinals 0..63 are served; on a device numbered 64 or more it returns
+ *     DSA_ERR_UNSUPPORTED.
  *   - The first call on a device looks up the array's device address with that device
  *     current (a one-time set-up); make that first call before any stream capture.
  *   - All calls on a device share the one array; calls that can overlap on the GPU race
@@ -178,7 +224,7 @@ DSA_API int dsa_sparse_attn_decode_noalloc(const void* Q, const void* K, const v
                                            void* O, float* lse, void* stream);
 
 /* ---------------------------------------------------------------------------------
- * (5) Whole DSA forward for prefill: (1) then (2) over row chunks of at most
+ * (5) Whole DSA forward for prefill: (2b) with DSA_PATH_SEPARATE over row chunks of at most
  * `chunk_rows` query rows (bounding the fp32 score scratch), then (3).
  *   max_seqlen_q / max_seqlen_k: host ints >= every Lq / Lk.
  *   indices device int32 [total_q, k] receives the selected sets.
@@ -227,8 +273,8 @@ DSA_API int dsa_decode(const void* q_idx, const void* k_idx, const void* w, cons
  *   written once, dQ is accumulated in fp32 (float atomics); otherwise one warp per (token,
  *   KV head) over its selected keys, with dK and dV accumulated in fp32 (float atomics).
  *   Float atomics make the summation order, and so the last bits, vary between runs; every
- *   fp32 accumulator is rounded to bf16 once at the end.  Selected positions outside
- *   [0, max_seqlen_k) and -1 slots are ignored.
+ *   fp32 accumulator is rounded to bf16 once at the end.  As in (3), -1 slots and
+ *   positions outside [0, vis(r)) are ignored.
  *   workspace: dsa_sparse_attn_bwd_workspace_size(total_q, total_k, Hq, Hkv, d,
  *   max_seqlen_k) bytes (enough for either path).
  * ------------------------------------------------------------------------------- */

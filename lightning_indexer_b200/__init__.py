@@ -13,7 +13,7 @@ import torch
 from . import _lib
 from ._lib import DSAError, call
 
-__all__ = ["index", "topk", "topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
+__all__ = ["index", "topk", "topk_workspace_bytes", "index_topk", "index_topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
            "sparse_attn_prefill_bwd", "indexer_kl_loss", "device_status", "DSAError"]
 
 
@@ -82,6 +82,35 @@ def topk(scores, cu_seqlens_q, cu_seqlens_k, k: int, row_begin: int = 0, row_end
     call("dsa_topk", _ptr(scores), scores.shape[1], _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
          cu_seqlens_q.numel() - 1, row_begin, row_end, k, _ptr(indices), _ptr(workspace),
          0 if workspace is None else workspace.numel(), _stream())
+    return indices
+
+
+PATH_AUTO, PATH_SEPARATE = 0, 1
+
+
+def index_topk_workspace_bytes(chunk_rows: int, max_seqlen_k: int) -> int:
+    return _lib.load().dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k)
+
+
+def index_topk(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, k: int,
+               chunk_rows: int = 8192, path: int = PATH_AUTO, indices: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None):
+    """Selected sets of every query row (indexer + top-k, fused where it applies):
+    int32 [T, k], ascending, -1 padded (see dsa_index_topk)."""
+    _check(q_idx, "q_idx", torch.bfloat16, 3)
+    _check(k_idx, "k_idx", torch.bfloat16, 2)
+    _check(w, "w", torch.bfloat16, 2)
+    total_q, H_I, d_I = q_idx.shape
+    chunk_rows = max(1, min(chunk_rows, max(total_q, 1)))
+    if indices is None:
+        indices = torch.empty((total_q, k), dtype=torch.int32, device=q_idx.device)
+    _check(indices, "indices", torch.int32, 2)
+    if workspace is None:
+        workspace = torch.empty(index_topk_workspace_bytes(chunk_rows, max_seqlen_k), dtype=torch.uint8,
+                                device=q_idx.device)
+    call("dsa_index_topk", _ptr(q_idx), _ptr(k_idx), _ptr(w), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+         cu_seqlens_q.numel() - 1, total_q, k_idx.shape[0], max_seqlen_q, max_seqlen_k, H_I, d_I, k, chunk_rows,
+         path, _ptr(indices), _ptr(workspace), workspace.numel(), _stream())
     return indices
 
 

@@ -17,10 +17,14 @@ SIGNATURES = {
     "dsa_version": (c_int, []),
     "dsa_last_cuda_error": (c_int, [ctypes.POINTER(ctypes.c_char_p)]),
     "dsa_get_device_status": (c_int, [ctypes.POINTER(c_int), ctypes.POINTER(c_int)]),
+    "dsa_selftest_bounded_wait": (c_int, [ctypes.c_uint64, c_vp]),
     "dsa_index": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int,
                           c_i64, c_i64, c_vp, c_i64, c_vp]),
     "dsa_topk_workspace_size": (c_size, [c_i64, c_i64, c_int]),
     "dsa_topk": (c_int, [c_vp, c_i64, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
+    "dsa_index_topk_workspace_size": (c_size, [c_i64, c_int]),
+    "dsa_index_topk": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_int,
+                               c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "dsa_sparse_attn_prefill": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_int, c_int, c_int,
                                         c_int, c_f32, c_vp, c_vp, c_vp]),
     "dsa_sparse_attn_decode_workspace_size": (c_size, [c_int, c_int, c_int, c_int]),

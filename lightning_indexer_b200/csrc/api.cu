@@ -12,6 +12,24 @@ __global__ void iota_kernel(int* dst, int n, int step) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i <= n) dst[i] = i * step;
 }
+
+// Self-test of the bounded wait every pipelined kernel uses: one thread waits, through the
+// same mbar_wait, on a shared-memory barrier that nothing ever arrives at.  The wait runs
+// out after limit_ns and records DSA_ERR_TIMEOUT with the site code kSelftestWaitSite; the
+// kernel then returns.  No copy, tensor-core or tensor-memory work is in flight.
+constexpr int kSelftestWaitSite = 900;
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, kSelftestWaitSite, limit_ns);
+  __syncthreads();
+}
 }  // namespace dsa
 
 namespace dsa_host {
@@ -49,6 +67,11 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
                            const float* lse, const int* indices, const int* cu_q, const int* cu_k, int batch,
                            long long total_q, long long total_k, int Hq, int Hkv, int d, int k, float scale,
                            void* dQ, void* dK, void* dV, void* ws, cudaStream_t stream);
+
+size_t index_topk_workspace_bytes(long long chunk_rows, int max_seqlen_k);
+int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
+                      int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k, int H_I,
+                      int d_I, int k, long long chunk_rows, int* indices, void* ws, int fused, cudaStream_t stream);
 
 struct KLWorkspace;
 size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I, long long chunk_rows,
@@ -144,6 +167,19 @@ static bool attn_shape_supported(int Hq, int Hkv, int d) {
   return (d == 64 || d == 128) && (G == 4 || G == 8);
 }
 
+// Argument checks of the decode attention calls, in their documented order: pointers and
+// alignment, then sizes (DSA_ERR_INVALID_ARG), then shapes without a kernel
+// (DSA_ERR_UNSUPPORTED).
+int decode_attn_args_status(const void* Q, const void* K, const void* V, const int32_t* indices,
+                            const int32_t* cu_seqlens_k, int batch, int Hq, int Hkv, int d, int k, float scale,
+                            const void* O) {
+  if (!Q || !K || !V || !indices || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
 }  // namespace dsa_host
 
 using namespace dsa_host;
@@ -181,6 +217,13 @@ DSA_API int dsa_get_device_status(int* status_out, int* detail_out) {
   *status_out = st;
   if (detail_out) *detail_out = det;
   return DSA_OK;
+}
+
+DSA_API int dsa_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return DSA_ERR_INVALID_ARG;
+  dsa::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_ns);
+  return last_launch_status();
 }
 
 DSA_API int dsa_index(const void* q_idx, const void* k_idx, const void* w, const int32_t* cu_seqlens_q,
@@ -243,20 +286,41 @@ DSA_API int dsa_sparse_attn_decode(const void* Q, const void* K, const void* V, 
                                    const int32_t* cu_seqlens_k, int batch, int Hq, int Hkv, int d, int k,
                                    float scale, void* O, float* lse, void* workspace, size_t workspace_bytes,
                                    void* stream) {
-  if (!Q || !K || !V || !indices || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return DSA_ERR_INVALID_ARG;
-  if (batch < 1 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
-  if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (const int st = decode_attn_args_status(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale, O);
+      st != DSA_OK)
+    return st;
   if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(batch, Hq, d, k))
     return DSA_ERR_WORKSPACE;
   return sparse_attn_decode_launch(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale, O, lse, workspace,
                                    static_cast<cudaStream_t>(stream));
 }
 
-DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k) {
+DSA_API size_t dsa_index_topk_workspace_size(int64_t chunk_rows, int max_seqlen_k) {
   if (chunk_rows < 1 || max_seqlen_k < 0) return 0;
-  const size_t ld = round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
-  return round_up((size_t)chunk_rows * ld * sizeof(float), 256);
+  return index_topk_workspace_bytes(chunk_rows, max_seqlen_k);
+}
+
+DSA_API int dsa_index_topk(const void* q_idx, const void* k_idx, const void* w, const int32_t* cu_seqlens_q,
+                           const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                           int max_seqlen_k, int H_I, int d_I, int k, int64_t chunk_rows, int path, int32_t* indices,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_idx || !k_idx || !w || !cu_seqlens_q || !cu_seqlens_k || !indices) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || chunk_rows < 1 || k < 1)
+    return DSA_ERR_INVALID_ARG;
+  if (path != DSA_PATH_AUTO && path != DSA_PATH_SEPARATE) return DSA_ERR_INVALID_ARG;
+  if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  if (!index_shape_supported(H_I, d_I) || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k))
+    return DSA_ERR_WORKSPACE;
+  if (total_q == 0) return DSA_OK;
+  return index_topk_launch(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                           max_seqlen_k, H_I, d_I, k, chunk_rows, indices, workspace, path == DSA_PATH_AUTO ? 1 : 0,
+                           static_cast<cudaStream_t>(stream));
+}
+
+DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k) {
+  return dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k);
 }
 
 DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, const void* Q, const void* K,
@@ -269,16 +333,11 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
     return DSA_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace) || workspace_bytes < dsa_prefill_workspace_size(chunk_rows, max_seqlen_k))
     return DSA_ERR_WORKSPACE;
-  const int64_t ld = (int64_t)round_up((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), 4);
-  float* scores = static_cast<float*>(workspace);
-  for (int64_t r0 = 0; r0 < total_q; r0 += chunk_rows) {
-    const int64_t r1 = r0 + chunk_rows < total_q ? r0 + chunk_rows : total_q;
-    int st = dsa_index(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
-                       max_seqlen_k, H_I, d_I, r0, r1, scores, ld, stream);
-    if (st != DSA_OK) return st;
-    st = dsa_topk(scores, ld, cu_seqlens_q, cu_seqlens_k, batch, r0, r1, k, indices + r0 * k, nullptr, 0, stream);
-    if (st != DSA_OK) return st;
-  }
+  if (const int st = dsa_index_topk(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                    max_seqlen_q, max_seqlen_k, H_I, d_I, k, chunk_rows, DSA_PATH_SEPARATE, indices,
+                                    workspace, workspace_bytes, stream);
+      st != DSA_OK)
+    return st;
   // dense selected sets: masked dense tensor-core passes, their selection words and row
   // maxima in the score scratch (free once the last chunk is selected)
   if (lse && sa_fwd_tc_eligible(Hq, Hkv, d, k, max_seqlen_k) &&

@@ -26,23 +26,34 @@ static __device__ __align__(256) uint8_t g_decode_scratch[kDecodeScratchBytes];
 
 namespace dsa_host {
 
+int decode_attn_args_status(const void* Q, const void* K, const void* V, const int32_t* indices,
+                            const int32_t* cu_seqlens_k, int batch, int Hq, int Hkv, int d, int k, float scale,
+                            const void* O);
+
+constexpr int kMaxScratchDevices = 64;  // device ordinals this entry point serves
+
 // Device address of the scratch array, looked up once per device (with that device
 // current).  In host code the array's name is only a host-side stand-in, so the kernel
-// must be given this address, never the symbol itself.
+// must be given this address, never the symbol itself.  A failed CUDA call is recorded
+// for dsa_last_cuda_error(); a device ordinal of kMaxScratchDevices or more is
+// DSA_ERR_UNSUPPORTED.
 static void* decode_scratch_address(int* status) {
-  constexpr int kMaxDevices = 64;
-  static void* addr[kMaxDevices] = {};
+  static void* addr[kMaxScratchDevices] = {};
   static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    *status = DSA_ERR_CUDA;
+  if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) {
+    *status = cuda_fail(e);
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxScratchDevices) {
+    *status = DSA_ERR_UNSUPPORTED;
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, dsa::g_decode_scratch) != cudaSuccess || !p) {
-      *status = DSA_ERR_CUDA;
+    if (const cudaError_t e = cudaGetSymbolAddress(&p, dsa::g_decode_scratch); e != cudaSuccess || !p) {
+      *status = e != cudaSuccess ? cuda_fail(e) : DSA_ERR_CUDA;
       return nullptr;
     }
     addr[dev] = p;
@@ -57,8 +68,11 @@ extern "C" DSA_API int dsa_sparse_attn_decode_noalloc(const void* Q, const void*
                                                       const int32_t* indices, const int32_t* cu_seqlens_k,
                                                       int batch, int Hq, int Hkv, int d, int k, float scale,
                                                       void* O, float* lse, void* stream) {
-  if (!Q || !K || !V || !indices || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
-  if (batch < 1 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  // the same checks, in the same order, as dsa_sparse_attn_decode; then the scratch limit
+  if (const int st = dsa_host::decode_attn_args_status(Q, K, V, indices, cu_seqlens_k, batch, Hq, Hkv, d, k, scale,
+                                                       O);
+      st != DSA_OK)
+    return st;
   const size_t need = dsa_sparse_attn_decode_workspace_size(batch, Hq, d, k);
   if (need == 0) return DSA_ERR_INVALID_ARG;
   if (need > dsa::kDecodeScratchBytes) return DSA_ERR_WORKSPACE;  // beyond the fixed scratch

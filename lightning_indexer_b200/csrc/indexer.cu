@@ -35,6 +35,22 @@ struct IndexerParams {
   int tiles_per_split;
   int max_splits;
   long long n_items;
+  // Sampled scores: with key_stride S > 1 the keys are the k_idx rows 0, S, 2S, ... (the
+  // key tensor map steps S rows at a time) and score column j of a row is the key at
+  // packed row (ceil(k0 / S) + j) * S, for the visible ones.
+  int key_stride = 1;
+  // Repair pass: only blocks holding a row r with mark[(r - row_begin) * mark_ld] == -2
+  // are processed, and nothing at all while *run_flag == 0.
+  const int* mark = nullptr;
+  int mark_ld = 0;
+  const int* run_flag = nullptr;
+  // Fused top-k candidates (CTA-pair kernel, fused form): scores whose order key is at
+  // least thr[r - row_begin] are appended as (key, position) to cand[(r - row_begin) * cap ..]
+  // with the running count in cnt[r - row_begin]; no score matrix is written.
+  const uint32_t* thr = nullptr;
+  uint32_t* cnt = nullptr;
+  uint2* cand = nullptr;
+  int cap = 0;
 };
 
 struct Item {
@@ -42,9 +58,18 @@ struct Item {
   int ntok;      // valid rows in the block
   int i0;        // sequence-local index of row t0
   int Lq, Lk;
-  int k0;        // first packed key row of the sequence
+  int kg;        // first packed key row of the sequence
+  int k0;        // first key-tensor-map row of the sequence (kg, or ceil(kg / S) when sampled)
   int tile_begin, tile_end;
 };
+
+// Visible keys of a row in the key-tensor-map rows of the item: the causal count, or for
+// sampled scores the number of sampled rows j * S inside [kg, kg + vis).
+__device__ __forceinline__ int item_visible(const IndexerParams& p, const Item& it, int vis) {
+  if (p.key_stride == 1) return vis;
+  const long long S = p.key_stride;
+  return (int)((it.kg + (long long)vis + S - 1) / S - it.k0);
+}
 
 // Work item -> (token block, key-tile range).  Items are numbered split-major
 // (item = split * blocks + block) with blocks heaviest-first, so consecutive item numbers,
@@ -76,13 +101,20 @@ __device__ __forceinline__ bool decode_item(long long item, const IndexerParams&
       it.i0 = (int)(it.t0 - p.cu_q[b]);
       it.Lq = p.cu_q[b + 1] - p.cu_q[b];
       it.Lk = p.cu_k[b + 1] - p.cu_k[b];
-      it.k0 = p.cu_k[b];
+      it.kg = p.cu_k[b];
+      it.k0 = p.key_stride == 1 ? it.kg : (int)(((long long)it.kg + p.key_stride - 1) / p.key_stride);
       const int last = it.i0 + it.ntok - 1;
-      const int vis = min(max(last + it.Lk - it.Lq + 1, 0), it.Lk);
+      const int vis = item_visible(p, it, min(max(last + it.Lk - it.Lq + 1, 0), it.Lk));
       const int ntiles = (vis + TILE_KEYS - 1) / TILE_KEYS;
       it.tile_begin = split * p.tiles_per_split;
       it.tile_end = min(ntiles, it.tile_begin + p.tiles_per_split);
-      return it.tile_begin < it.tile_end;
+      if (it.tile_begin >= it.tile_end) return false;
+      if (p.mark) {
+        bool any = false;
+        for (int j = 0; j < it.ntok; ++j) any |= p.mark[(it.t0 + j - p.row_begin) * p.mark_ld] == -2;
+        return any;
+      }
+      return true;
     }
     r -= nb;
   }

@@ -15,11 +15,23 @@
 //   warps 2+ epilogue (both): tcgen05.ld -> fp32 ReLU/FMA over heads -> stores
 // Releases go back through multicast commits (stage free, accumulator full) to both CTAs
 // and through remote arrivals (accumulator drained) to the even CTA.
+//
+// Three forms share the kernel (IndexerParams selects them):
+//   - scores: every visible score is written to the fp32 score rows (dsa_index);
+//   - sampled scores (key_stride S > 1): the keys are every S-th indexer key, so a row gets
+//     about vis / S scores, from which the fused top-k takes a lower bound on the row's
+//     k-th largest score;
+//   - fused top-k (FUSED): no score is written; scores whose order key reaches the row's
+//     bound are appended to the row's candidate list as (key, position).  Each epilogue
+//     warp stages its candidates per token in a 64-entry shared-memory ring and moves 32
+//     at a time to global memory behind one atomicAdd on the row's count, so the count's
+//     round trip is paid once per 32 candidates, not once per key tile.  The order of a
+//     row's list depends on timing; the selection made from it does not.
 #include "common.cuh"
 
 namespace dsa {
 
-template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES>
+template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES, bool FUSED = false>
 struct Indexer2Cfg {
   static constexpr int N = NTOK * H_I;  // MMA N over the pair
   static constexpr int NH = N / 2;      // q_idx rows held by each CTA
@@ -42,17 +54,25 @@ struct Indexer2Cfg {
   static constexpr int OFF_BAR = OFF_W + 2 * N * 2;  // two bf16 weight buffers
   static constexpr int NUM_BARS = 2 * A_STAGES + 2 * B_STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // fused form: a 64-entry (key, position) ring per epilogue warp and token it handles
+  static constexpr int TPW = CPT / H_I;  // tokens per epilogue thread
+  static constexpr int RING = 64;
+  static constexpr int OFF_RING = OFF_MISC + 16;
+  static constexpr int RING_BYTES = FUSED ? NUM_EPI_WARPS * TPW * RING * 8 : 0;
+  static constexpr int SMEM_BYTES = OFF_RING + RING_BYTES + 1024;
   static constexpr uint32_t IDESC = idesc_bf16_f32(256, N);
   static_assert(SMEM_BYTES <= 232448, "exceeds the 227 KB per-block shared memory limit");
 };
 
-template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES>
-__global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>::THREADS, 1)
+template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES, bool FUSED>
+__global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES, FUSED>::THREADS, 1)
     indexer2_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                     const IndexerParams p) {
-  using C = Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
+  using C = Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES, FUSED>;
   constexpr int TILE_KEYS = 256;
+  // a repair pass with nothing to repair: both CTAs of every pair read the same flag and
+  // leave before touching any barrier or tensor memory
+  if (p.run_flag && *(volatile const int*)p.run_flag == 0) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + C::OFF_A;
@@ -232,6 +252,31 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
         wr[c] = tk0 < it.ntok ? __uint_as_float(pr << 16) : 0.f;
         wr[c + 1] = tk1 < it.ntok ? __uint_as_float(pr & 0xFFFF0000u) : 0.f;
       }
+      // visible keys (key-tensor-map rows) of this thread's tokens, 0 past the block's rows;
+      // in the fused form also each token's bound and its ring state (warp-uniform)
+      int vtok[C::TPW];
+      uint32_t thr_t[C::TPW], rhead[C::TPW], rcount[C::TPW];
+#pragma unroll
+      for (int j = 0; j < C::TPW; ++j) {
+        const int tok = col0 / H_I + j;
+        vtok[j] = tok < it.ntok ? item_visible(p, it, min(max(it.i0 + tok + dvis, 0), it.Lk)) : 0;
+        thr_t[j] = FUSED && tok < it.ntok ? __ldg(p.thr + (it.t0 + tok - p.row_begin)) : 0xFFFFFFFFu;
+        rhead[j] = 0;
+        rcount[j] = 0;
+      }
+      // moves the oldest n (<= 32) staged candidates of token slot j to the row's list
+      auto flush = [&](int j, uint32_t n) {
+        uint2* ring = reinterpret_cast<uint2*>(smem + C::OFF_RING) + (ep * C::TPW + j) * C::RING;
+        const long long rr = it.t0 + col0 / H_I + j - p.row_begin;
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(p.cnt + rr, n);
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if ((uint32_t)lane < n && base + lane < (uint32_t)p.cap)
+          p.cand[rr * p.cap + base + lane] = ring[(rhead[j] + lane) & (C::RING - 1)];
+        rhead[j] = (rhead[j] + n) & (C::RING - 1);
+        rcount[j] -= n;
+        __syncwarp();  // the ring slots just read may be refilled
+      };
       for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
         if (!(ok = mbar_wait(&acc_full[ab], abph, abort_flag, 16))) break;
         tc_fence_after();
@@ -241,6 +286,7 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
 #pragma unroll
         for (int c = 0; c < C::CPT; c += H_I) {
           const int tok = (col0 + c) / H_I;
+          const int j = c / H_I;
           float acc = 0.f;
 #pragma unroll
           for (int h0 = 0; h0 < H_I; h0 += 16) {
@@ -249,13 +295,34 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
 #pragma unroll
             for (int q = 0; q < 16; ++q) acc = fmaf(wr[c + h0 + q], fmaxf(v[q], 0.f), acc);
           }
-          const int vis = min(max(it.i0 + tok + dvis, 0), it.Lk);
-          if (tok < it.ntok && s < vis) out_row0[(long long)tok * p.ld] = acc;
+          if constexpr (!FUSED) {
+            if (s < vtok[j]) out_row0[(long long)tok * p.ld] = acc;
+          } else {
+            const uint32_t key = float_order_key(acc);
+            const bool pass = s < vtok[j] && key >= thr_t[j];
+            const uint32_t m = __ballot_sync(0xffffffffu, pass);
+            if (m) {
+              uint2* ring = reinterpret_cast<uint2*>(smem + C::OFF_RING) + (ep * C::TPW + j) * C::RING;
+              if (pass)
+                ring[(rhead[j] + rcount[j] + __popc(m & ((1u << lane) - 1u))) & (C::RING - 1)] =
+                    make_uint2(key, (uint32_t)s);
+              rcount[j] += __popc(m);
+              __syncwarp();
+              if (rcount[j] >= 32) flush(j, 32);
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(ab == 0 ? acc_empty0 : acc_empty1);
         if (++ab == 2) { ab = 0; abph ^= 1; }
+      }
+      if constexpr (FUSED) {
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < C::TPW; ++j)
+            if (rcount[j] > 0) flush(j, rcount[j]);
+        }
       }
       item = nitem;
       it = nx;
@@ -276,13 +343,25 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
 
 namespace dsa_host {
 
-template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES>
+// Which form of the CTA-pair kernel a launch runs (see the kernel's header comment).
+struct Indexer2Pass {
+  int key_stride = 1;             // > 1: sampled scores over every key_stride-th key
+  const int* mark = nullptr;      // repair: rows marked -2 in mark[(r - row_begin) * mark_ld]
+  int mark_ld = 0;
+  const int* run_flag = nullptr;  // repair: nothing to do while *run_flag == 0
+  const uint32_t* thr = nullptr;  // fused: per-row bound, candidate counts and lists
+  uint32_t* cnt = nullptr;
+  uint2* cand = nullptr;
+  int cap = 0;
+};
+
+template <int H_I, int D_I, int NTOK, int NUM_EPI_WARPS, int A_STAGES, int B_STAGES, bool FUSED>
 static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                            int batch, long long total_q, long long total_k, int max_seqlen_k, long long row_begin,
                            long long row_end, float* scores, long long ld, int tiles_per_split,
-                           cudaStream_t stream) {
-  using C = dsa::Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
-  auto kern = dsa::indexer2_kernel<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES>;
+                           const Indexer2Pass& pass, cudaStream_t stream) {
+  using C = dsa::Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES, FUSED>;
+  auto kern = dsa::indexer2_kernel<H_I, D_I, NTOK, NUM_EPI_WARPS, A_STAGES, B_STAGES, FUSED>;
   static DeviceFlag attr_done;
   const int smem = std::max(C::SMEM_BYTES, 120 * 1024);
   if (!attr_done) {
@@ -290,8 +369,11 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
     if (e_ != cudaSuccess) return cuda_fail(e_);
     attr_done = true;
   }
+  const long long S = std::max(1, pass.key_stride);
   CUtensorMap tk, tq;
-  int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)total_k, D_I, (uint64_t)D_I * 2, 128, C::PANEL, C::SWZ);
+  // sampled scores: the key map steps S rows of k_idx per row (rows past the end read 0)
+  int st = make_tmap_bf16_2d(&tk, k_idx, (uint64_t)((total_k + S - 1) / S), D_I, (uint64_t)(S * D_I * 2), 128,
+                             C::PANEL, C::SWZ);
   if (st != DSA_OK) return st;
   st = make_tmap_bf16_2d(&tq, q_idx, (uint64_t)total_q * H_I, D_I, (uint64_t)D_I * 2, C::NH, C::PANEL, C::SWZ);
   if (st != DSA_OK) return st;
@@ -306,8 +388,17 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
   p.scores = scores;
   p.ld = ld;
   p.tiles_per_split = tiles_per_split;
-  const int max_tiles = (max_seqlen_k + 255) / 256;
-  p.max_splits = std::max(1, (max_tiles + tiles_per_split - 1) / tiles_per_split);
+  p.key_stride = (int)S;
+  p.mark = pass.mark;
+  p.mark_ld = pass.mark_ld;
+  p.run_flag = pass.run_flag;
+  p.thr = pass.thr;
+  p.cnt = pass.cnt;
+  p.cand = pass.cand;
+  p.cap = pass.cap;
+  const long long max_keys = S == 1 ? max_seqlen_k : max_seqlen_k / S + 2;
+  const long long max_tiles = (max_keys + 255) / 256;
+  p.max_splits = (int)std::max(1LL, (max_tiles + tiles_per_split - 1) / tiles_per_split);
   const long long rows = row_end - row_begin;
   const long long nblk = (rows + NTOK - 1) / NTOK + batch;
   p.n_items = nblk * p.max_splits;
@@ -329,17 +420,36 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
   return last_launch_status();
 }
 
-// 128K-class prefill shapes on CTA pairs; returns DSA_ERR_UNSUPPORTED for other shapes
+// True for the indexer shapes that have the CTA-pair kernel (and so the fused top-k).
+bool indexer2_shape(int H_I, int d_I) { return d_I == 128 && (H_I == 64 || H_I == 32); }
+
+// Any form of the CTA-pair kernel for the 128K-class prefill shapes; fused = candidates
+// instead of scores.  DSA_ERR_UNSUPPORTED for other shapes.
+int indexer2_pass_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
+                         int batch, long long total_q, long long total_k, int max_seqlen_k, int H_I, int d_I,
+                         long long row_begin, long long row_end, float* scores, long long ld, bool fused,
+                         const Indexer2Pass& pass, cudaStream_t stream) {
+#define DSA_IDX2(HI, NT, FU)                                                                                  \
+  return launch_indexer2<HI, 128, NT, 8, 4, 2, FU>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k,      \
+                                                   max_seqlen_k, row_begin, row_end, scores, ld, 64, pass, stream)
+  if (H_I == 64 && d_I == 128) {
+    if (fused) DSA_IDX2(64, 4, true);
+    DSA_IDX2(64, 4, false);
+  }
+  if (H_I == 32 && d_I == 128) {
+    if (fused) DSA_IDX2(32, 8, true);
+    DSA_IDX2(32, 8, false);
+  }
+#undef DSA_IDX2
+  return DSA_ERR_UNSUPPORTED;
+}
+
+// 128K-class prefill shapes on CTA pairs, scores form; DSA_ERR_UNSUPPORTED for other shapes
 int indexer2_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
                     long long total_q, long long total_k, int max_seqlen_k, int H_I, int d_I, long long row_begin,
                     long long row_end, float* scores, long long ld, cudaStream_t stream) {
-  if (H_I == 64 && d_I == 128)
-    return launch_indexer2<64, 128, 4, 8, 4, 2>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k,
-                                                row_begin, row_end, scores, ld, 64, stream);
-  if (H_I == 32 && d_I == 128)
-    return launch_indexer2<32, 128, 8, 8, 4, 2>(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k,
-                                                row_begin, row_end, scores, ld, 64, stream);
-  return DSA_ERR_UNSUPPORTED;
+  return indexer2_pass_launch(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_k, H_I, d_I,
+                              row_begin, row_end, scores, ld, false, Indexer2Pass{}, stream);
 }
 
 }  // namespace dsa_host

@@ -110,14 +110,17 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t my_s = smem_u32(smem + warp * SA_STAGES * STAGE_BYTES);
 
+  // Tasks run KV head by KV head (the head is the slowest index): the warps resident at
+  // one time then gather from one head's K/V rows only, a quarter of the K/V bytes, which
+  // stays in L2 at 128K context (64 MiB per head) where all four heads' rows would not.
   const long long task = (long long)blockIdx.x * SA_WARPS + warp;
-  const long long per_row = (long long)p.Hkv * p.nsplit;
-  const long long row = task / per_row;
-  if (row >= p.rows) return;  // warp-uniform; the kernel has no CTA-wide barrier
-  const int rem = (int)(task % per_row);
-  const int split = rem / p.Hkv;
-  const int g = rem % p.Hkv;
-  int kbase = 0;
+  const long long per_head = p.rows * p.nsplit;
+  const int g = (int)(task / per_head);
+  if (g >= p.Hkv) return;  // warp-uniform; the kernel has no CTA-wide barrier
+  const long long rem = task - (long long)g * per_head;
+  const long long row = rem / p.nsplit;
+  const int split = (int)(rem % p.nsplit);
+  int kbase = 0, vis = 0;
   if (p.cu_q) {
     int lo = 0, hi = p.batch;
     while (hi - lo > 1) {
@@ -125,8 +128,10 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
       if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
     }
     kbase = p.cu_k[lo];
+    vis = causal_vis((int)(row - p.cu_q[lo]), p.cu_q[lo + 1] - p.cu_q[lo], p.cu_k[lo + 1] - kbase);
   } else {
     kbase = p.cu_k[row];
+    vis = p.cu_k[row + 1] - kbase;
   }
   const int keys_per_split = p.k / p.nsplit;
   const int* idx = p.indices + row * p.k + split * keys_per_split;
@@ -158,13 +163,13 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
       const int e = j * 32 + lane;
       const int r = e / SEGS, seg = e % SEGS;
       const int s = __shfl_sync(0xffffffffu, my_idx, r);
-      const bool valid = s >= 0;
+      const bool valid = (unsigned)s < (unsigned)vis;  // -1 and positions the row cannot see
       const size_t off = valid ? (size_t)(kbase + s) * kv_row_stride + seg * 8 : 0;
       cp_async_16(kdst + tile_off<D>(r, seg), Kg + off, valid);
       cp_async_16(vdst + tile_off<D>(r, seg), Vg + off, valid);
     }
     cp_async_commit();
-    return __ballot_sync(0xffffffffu, my_idx >= 0) & 0xFFFFu;
+    return __ballot_sync(0xffffffffu, (unsigned)my_idx < (unsigned)vis) & 0xFFFFu;
   };
 
   float acc[MT][4];

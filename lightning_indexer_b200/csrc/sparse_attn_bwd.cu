@@ -59,16 +59,18 @@ __global__ void __launch_bounds__(BWD_WARPS * 32, 3) sparse_attn_bwd_kernel(cons
   const int gid = lane / 4, tig = lane % 4;
   const uint32_t my_s = smem_u32(smem + warp * BWD_STAGES * STAGE_BYTES);
 
+  // KV head slowest: the resident warps gather from, and reduce into, one head's rows
   const long long task = (long long)blockIdx.x * BWD_WARPS + warp;
-  const long long row = task / p.Hkv;
-  if (row >= p.rows) return;
-  const int g = (int)(task % p.Hkv);
+  const int g = (int)(task / p.rows);
+  if (g >= p.Hkv) return;
+  const long long row = task - (long long)g * p.rows;
   int lo = 0, hi = p.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) / 2;
     if ((long long)p.cu_q[mid] <= row) lo = mid; else hi = mid;
   }
   const int kbase = p.cu_k[lo];
+  const int vis = causal_vis((int)(row - p.cu_q[lo]), p.cu_q[lo + 1] - p.cu_q[lo], p.cu_k[lo + 1] - kbase);
   const int* idx = p.indices + row * p.k;
   const int nchunks = p.k / BWD_CHUNK;
   const size_t kv_row_stride = (size_t)p.Hkv * D;
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(BWD_WARPS * 32, 3) sparse_attn_bwd_kernel(cons
       const int e = j * 32 + lane;
       const int r = e / SEGS, seg = e % SEGS;
       const int s = __shfl_sync(0xffffffffu, my_idx, r);
-      const bool valid = s >= 0;
+      const bool valid = (unsigned)s < (unsigned)vis;  // -1 and positions the row cannot see
       const size_t off = valid ? (size_t)(kbase + s) * kv_row_stride + seg * 8 : 0;
       cp_async_16(kdst + tile_off<D>(r, seg), Kg + off, valid);
       cp_async_16(vdst + tile_off<D>(r, seg), Vg + off, valid);
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(BWD_WARPS * 32, 3) sparse_attn_bwd_kernel(cons
     const int myi = __ldg(idx + c * BWD_CHUNK + (lane & 15));
     const int sA = __shfl_sync(0xffffffffu, myi, gid);      // key of accumulator row gid
     const int sB = __shfl_sync(0xffffffffu, myi, gid + 8);  // key of row gid + 8
-    const bool v0 = sA >= 0, v1 = sB >= 0;
+    const bool v0 = (unsigned)sA < (unsigned)vis, v1 = (unsigned)sB < (unsigned)vis;
     const float p00 = (v0 && live0) ? exp2f(s[0] * p.scale_log2 - L0) : 0.f;
     const float p01 = (v0 && live1) ? exp2f(s[1] * p.scale_log2 - L1) : 0.f;
     const float p10 = (v1 && live0) ? exp2f(s[2] * p.scale_log2 - L0) : 0.f;

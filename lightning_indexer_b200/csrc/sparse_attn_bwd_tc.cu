@@ -496,14 +496,24 @@ __global__ void sa_bwd_prep_kernel(const uint16_t* __restrict__ O, const uint16_
   if (lane == 0) LD[((long long)(h / 8) * T + t) * 8 + (h % 8)] = make_float2(lse[r] * 1.4426950408889634f, acc);
 }
 
-// selection bits: one thread per (row, slot); -1 slots (and out-of-range values) are skipped
-__global__ void sa_bwd_mask_kernel(const int* __restrict__ indices, long long rows, int k, uint32_t* mask,
+// selection bits: one thread per (row, slot); -1 slots and positions the row cannot see
+// (outside [0, vis)) are skipped, as in the gather kernels
+__global__ void sa_bwd_mask_kernel(const int* __restrict__ indices, const int* __restrict__ cu_q,
+                                   const int* __restrict__ cu_k, int batch, long long rows, int k, uint32_t* mask,
                                    int tiles) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * k) return;
   const int s = indices[i];
   if (s < 0 || s >= tiles * 128) return;
-  atomicOr(mask + ((long long)(s >> 7) * rows + i / k) * 4 + ((s >> 5) & 3), 1u << (s & 31));
+  const long long row = i / k;
+  int lo = 0, hi = batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if ((long long)cu_q[mid] <= row) lo = mid; else hi = mid;
+  }
+  const int vis = causal_vis((int)(row - cu_q[lo]), cu_q[lo + 1] - cu_q[lo], cu_k[lo + 1] - cu_k[lo]);
+  if (s >= vis) return;
+  atomicOr(mask + ((long long)(s >> 7) * rows + row) * 4 + ((s >> 5) & 3), 1u << (s & 31));
 }
 
 }  // namespace dsa
@@ -516,14 +526,15 @@ static size_t r256b(size_t x) { return (x + 255) / 256 * 256; }
 
 // selection words of `indices` (layout of SABwdTcParams::mask) into `mask`, which it clears
 // first (total_q * ceil(max_seqlen_k / 128) * 16 bytes)
-int sa_bwd_mask_build(const int* indices, long long total_q, int k, int max_seqlen_k, uint32_t* mask,
-                      cudaStream_t s) {
+int sa_bwd_mask_build(const int* indices, const int* cu_q, const int* cu_k, int batch, long long total_q, int k,
+                      int max_seqlen_k, uint32_t* mask, cudaStream_t s) {
   const int tiles = (max_seqlen_k + 127) / 128;
   if (const cudaError_t e_ = cudaMemsetAsync(mask, 0, (size_t)total_q * tiles * 16, s); e_ != cudaSuccess)
     return cuda_fail(e_);
   const long long n = total_q * k;
   if (n <= 0) return DSA_OK;
-  dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, total_q, k, mask, tiles);
+  dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, cu_q, cu_k, batch, total_q, k, mask,
+                                                                        tiles);
   return last_launch_status();
 }
 
@@ -574,7 +585,8 @@ int sa_bwd_tc_launch(const void* Q, const void* K, const void* V, const void* O,
         static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), lse, total_q, Hq, LD);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
     const long long n = total_q * k;
-    dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, total_q, k, mask, mw / 4);
+    dsa::sa_bwd_mask_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(indices, cu_q, cu_k, batch, total_q, k, mask,
+                                                                        mw / 4);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
   }
   CUtensorMap tq, tdo, tk, tv;

@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      long long m = 0, n = 0;  // items with key tiles, key tiles
+      long long m = 0, n = 0;    // items with key tiles, key tiles
+      long long nk = 0, nv = 0;  // K and V tile copies issued (they differ after an abort)
       bool ok = true;
       for (long long item = blockIdx.x; item < ip.n_items && ok; item += gridDim.x) {
         KlLseItem it;
@@ -140,27 +141,29 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
           for (int pn = 0; pn < 2; ++pn)
             tma_load_3d(smem + C::OFF_K + ks * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &k_full[ks], pn * 64,
                         it.g, it.kbase + j * 128);
-          if (!(ok = mbar_wait(&v_empty[vs], (uint32_t)((n / C::V_STAGES) & 1) ^ 1u, abort_flag, 130))) {
-            ++n;  // this tile's K copy is in flight: the drain below waits for it
-            break;
-          }
+          ++nk;
+          if (!(ok = mbar_wait(&v_empty[vs], (uint32_t)((n / C::V_STAGES) & 1) ^ 1u, abort_flag, 130))) break;
           mbar_arrive_expect_tx(&v_full[vs], C::TILE_BYTES);
           for (int pn = 0; pn < 2; ++pn)
             tma_load_3d(smem + C::OFF_V + vs * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_v, &v_full[vs], pn * 64,
                         it.g, it.kbase + j * 128);
+          ++nv;
         }
       }
       if (!ok) {
-        // let the copies this thread issued land before the CTA exits (bounded)
-        const uint64_t t0 = globaltimer_ns();
-        for (long long k = max(0LL, n - C::K_STAGES); k < n; ++k)
+        // let the copies this thread issued land before the CTA exits (bounded; each ring
+        // waits only for copies it really issued, each with its own time budget)
+        uint64_t t0 = globaltimer_ns();
+        for (long long k = max(0LL, nk - C::K_STAGES); k < nk; ++k)
           while (!mbar_try_wait(smem_u32(&k_full[k % C::K_STAGES]), (uint32_t)((k / C::K_STAGES) & 1)) &&
                  globaltimer_ns() - t0 < 100000000ull) {
           }
-        for (long long k = max(0LL, n - C::V_STAGES); k < n; ++k)
+        t0 = globaltimer_ns();
+        for (long long k = max(0LL, nv - C::V_STAGES); k < nv; ++k)
           while (!mbar_try_wait(smem_u32(&v_full[k % C::V_STAGES]), (uint32_t)((k / C::V_STAGES) & 1)) &&
                  globaltimer_ns() - t0 < 100000000ull) {
           }
+        t0 = globaltimer_ns();
         if (m > 0)
           while (!mbar_try_wait(smem_u32(q_full), (uint32_t)((m - 1) & 1)) && globaltimer_ns() - t0 < 100000000ull) {
           }
@@ -341,7 +344,8 @@ size_t sa_fwd_tc_scratch_bytes(long long total_q, int Hq, int max_seqlen_k) {
   return sa_fwd_tc_mask_only(total_q, max_seqlen_k) + (size_t)total_q * Hq * 4;
 }
 
-int sa_bwd_mask_build(const int* indices, long long total_q, int k, int max_seqlen_k, uint32_t* mask, cudaStream_t s);
+int sa_bwd_mask_build(const int* indices, const int* cu_q, const int* cu_k, int batch, long long total_q, int k,
+                      int max_seqlen_k, uint32_t* mask, cudaStream_t s);
 
 // O and lse of the selected sets in `indices` by the two masked dense passes; `mask_ws`
 // holds sa_fwd_tc_scratch_bytes.
@@ -360,7 +364,7 @@ int sa_fwd_tc_launch(const void* Q, const void* K, const void* V, const int* ind
   if (total_q <= 0) return DSA_OK;
   uint32_t* mask = static_cast<uint32_t*>(mask_ws);
   float* mx = reinterpret_cast<float*>(static_cast<uint8_t*>(mask_ws) + sa_fwd_tc_mask_only(total_q, max_seqlen_k));
-  int st = sa_bwd_mask_build(indices, total_q, k, max_seqlen_k, mask, s);
+  int st = sa_bwd_mask_build(indices, cu_q, cu_k, batch, total_q, k, max_seqlen_k, mask, s);
   if (st != DSA_OK) return st;
   const float scale_log2 = scale * 1.4426950408889634f;
   st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, total_q, total_k, Hq, Hkv, 0, scale_log2, lse, s, mask,

@@ -1411,17 +1411,10 @@ static int topk_regs_launch(const dsa::TopkParams& p, long long rows, cudaStream
   return last_launch_status();
 }
 
-// One block per row with the streaming kernel, then the exact kernel for rows it marked.
-static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t stream) {
-  static DeviceFlag attr_done, exact_done;
-  if (!attr_done) {
-    const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_stream_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e_ != cudaSuccess) return cuda_fail(e_);
-    attr_done = true;
-  }
-  p.only_marked = 0;
-  dsa::topk_stream_kernel<<<(unsigned)rows, dsa::ST_T, 0, stream>>>(p);
-  if (const int st = last_launch_status(); st != DSA_OK) return st;
+// The exact selection of the rows of [p.row_begin, p.row_begin + rows) whose first index
+// slot holds -2, from the score rows in p.scores; the other rows are left as they are.
+static int topk_marked_rows_launch(dsa::TopkParams p, long long rows, cudaStream_t stream) {
+  static DeviceFlag exact_done;
   p.only_marked = 1;
   if (!exact_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_marked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1432,6 +1425,39 @@ static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t st
   const long long grid = std::max((rows + dsa::TOPK_THREADS - 1) / dsa::TOPK_THREADS, std::min(rows, (long long)sm_count()));
   dsa::topk_marked_kernel<<<(unsigned)grid, dsa::TOPK_THREADS, sizeof(dsa::TopkSmem), stream>>>(p, rows);
   return last_launch_status();
+}
+
+// One block per row with the streaming kernel, then the exact kernel for rows it marked.
+static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t stream) {
+  static DeviceFlag attr_done;
+  if (!attr_done) {
+    const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_stream_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e_ != cudaSuccess) return cuda_fail(e_);
+    attr_done = true;
+  }
+  p.only_marked = 0;
+  dsa::topk_stream_kernel<<<(unsigned)rows, dsa::ST_T, 0, stream>>>(p);
+  if (const int st = last_launch_status(); st != DSA_OK) return st;
+  return topk_marked_rows_launch(p, rows, stream);
+}
+
+// Exact top-k of the rows of [row_begin, row_end) that an earlier pass marked with -2 in
+// their first index slot (indices points at row row_begin's slots).
+int topk_marked_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
+                       long long row_begin, long long row_end, int k, int* indices, cudaStream_t stream) {
+  const long long rows = row_end - row_begin;
+  if (rows <= 0) return DSA_OK;
+  dsa::TopkParams p;
+  p.scores = scores;
+  p.ld = ld;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.batch = batch;
+  p.row_begin = row_begin;
+  p.k = k;
+  p.indices = indices;
+  p.only_marked = 1;
+  return topk_marked_rows_launch(p, rows, stream);
 }
 
 // Workspace of the two-launch path for `rows` rows of up to max_vis positions; 0 where

@@ -69,6 +69,22 @@ def test_host_side_argument_errors():
     assert need > 0
     assert lib.dsa_sparse_attn_decode(fake, fake, fake, fake, fake, 16, 32, 4, 128, 2048, 0.1, fake, None,
                                       fake, need - 1, None) == -3
+    # the allocation-free decode checks its arguments in the same order as the regular one,
+    # and only then its fixed scratch limit
+    big = 64  # batch 64 x 32 heads at d = 128, k = 2048 needs more than the 8 MiB scratch
+    assert lib.dsa_sparse_attn_decode_noalloc(None, fake, fake, fake, fake, big, 32, 4, 128, 2048, 0.1, fake,
+                                              None, None) == -1
+    assert lib.dsa_sparse_attn_decode_noalloc(mis, fake, fake, fake, fake, big, 32, 4, 128, 2048, 0.1, fake,
+                                              None, None) == -1
+    assert lib.dsa_sparse_attn_decode_noalloc(fake, fake, fake, fake, fake, big, 32, 4, 128, 2008, 0.1, fake,
+                                              None, None) == -2  # k not a multiple of 16
+    assert lib.dsa_sparse_attn_decode_noalloc(fake, fake, fake, fake, fake, big, 32, 4, 96, 2048, 0.1, fake,
+                                              None, None) == -2  # head dim without a kernel
+    assert lib.dsa_sparse_attn_decode_noalloc(fake, fake, fake, fake, fake, big, 32, 4, 128, 2048, 0.1, fake,
+                                              None, None) == -3
+    # bounded-wait self-test: limits outside 1 ns .. 1 s are refused before any launch
+    assert lib.dsa_selftest_bounded_wait(0, None) == -1
+    assert lib.dsa_selftest_bounded_wait(2_000_000_000, None) == -1
     assert lib.dsa_prefill_workspace_size(8192, 131072) >= 8192 * 131072 * 4
     # sparse backward: the masked dense path (d = 128, 8 heads per KV head) needs the fp32 dQ
     # accumulator; the gather path the fp32 dK and dV accumulators

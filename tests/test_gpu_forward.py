@@ -231,22 +231,130 @@ def test_sparse_attention_prefill_given_sets(Hq, Hkv, d):
         assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL, r
 
 
+def _fused_vs_separate(wl, k, chunk):
+    """Selected sets by dsa_index_topk on its fused path and on the separate passes."""
+    t = to_device(wl)
+    args = (t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], k)
+    fused = dsa.index_topk(*args, chunk_rows=chunk, path=dsa.PATH_AUTO).cpu().numpy()
+    separate = dsa.index_topk(*args, chunk_rows=chunk, path=dsa.PATH_SEPARATE).cpu().numpy()
+    return fused, separate
+
+
+def test_index_topk_fused_integer_bit_exact():
+    # integer indexer inputs (exact fp32 scores, many ties) at H_I = 64, d_I = 128: the fused
+    # path must return exactly the oracle's sets and exactly the separate path's, in one
+    # chunk and in chunks of 700 rows
+    wl = gen.make_prefill([1500, 700, 1200], 8, 2, 64, 64, 128, 128, seed=36, layout="integer")
+    D = orc.Decoded(wl)
+    ref = _oracle_sets(D, 128)
+    for chunk in (wl.Tq, 700):
+        fused, separate = _fused_vs_separate(wl, 128, chunk)
+        np.testing.assert_array_equal(fused, separate)
+        np.testing.assert_array_equal(fused, ref)
+
+
+def test_index_topk_fused_gaussian_matches_separate_and_oracle():
+    wl = gen.make_prefill([3000, 1000], 8, 2, 64, 64, 128, 64, seed=37, layout="video")
+    fused, separate = _fused_vs_separate(wl, 64, 1024)
+    np.testing.assert_array_equal(fused, separate)
+    D = orc.Decoded(wl)
+    for r in range(0, wl.Tq, 3):
+        o = orc.forward_row(D, r, 64)
+        ok, _ = set_mismatch_ok(fused[r], o["idx"], o["scores"])
+        assert ok, r
+
+
+def test_index_topk_fused_repair_rows():
+    # Rows the sampled bound fails for must still come out exact.  The keys at the sampled
+    # positions (packed rows that are multiples of the stride, 4 here) get the largest
+    # scores and every other key a small one, so a bound taken from the samples lets through
+    # only the sampled positions: fewer than k = 256 for rows that see under 1024 keys (too
+    # few candidates), and rows whose q_idx is zero score 0 everywhere (every position ties,
+    # too many candidates).  Both kinds are recomputed and selected by the exact method.
+    wl = gen.make_prefill([2000, 1500], 8, 2, 64, 64, 128, 256, seed=38, layout="integer")
+    rng = np.random.default_rng(38)
+    k_idx = rng.integers(-1, 2, size=(wl.Tk, 128)).astype(np.float32)
+    k_idx[np.arange(wl.Tk) % 4 == 0] = 8.0
+    q_idx = rng.integers(1, 9, size=(wl.Tq, 64, 128)).astype(np.float32)
+    q_idx[1200:1300] = 0.0  # they see more positions (1201..1300) than a row's 736 candidate slots
+    q_idx[2900:2950] = 0.0
+    wl.k_idx = gen.f32_to_bf16_bits(k_idx)
+    wl.q_idx = gen.f32_to_bf16_bits(q_idx)
+    D = orc.Decoded(wl)
+    ref = _oracle_sets(D, 256)
+    for chunk in (wl.Tq, 1024):
+        fused, separate = _fused_vs_separate(wl, 256, chunk)
+        np.testing.assert_array_equal(fused, ref)
+        np.testing.assert_array_equal(separate, ref)
+
+
+def test_index_topk_fused_repeat_is_bit_identical():
+    # candidate lists arrive in a timing-dependent order; the selected sets must not
+    wl = gen.make_prefill([4000], 8, 2, 64, 64, 128, 128, seed=39, layout="video")
+    t = to_device(wl)
+    args = (t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], 128)
+    first = dsa.index_topk(*args, chunk_rows=1000)
+    for _ in range(3):
+        assert torch.equal(dsa.index_topk(*args, chunk_rows=1000), first)
+
+
 def test_sparse_attention_empty_and_padded_sets():
     wl = gen.make_prefill([40], 8, 2, 64, 4, 32, 32, seed=32)
     D = orc.Decoded(wl)
     idx = np.full((40, 32), -1, np.int32)
-    idx[1, :5] = [0, 1, 7, 20, 39]
-    idx[2, 3] = 11  # a single selected key in the middle of the padding
+    idx[39, :5] = [0, 1, 7, 20, 39]
+    idx[12, 3] = 11  # a single selected key in the middle of the padding
     t = to_device(wl)
     O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"])
     O = O.float().cpu().numpy()
     lse = lse.cpu().numpy()
     assert np.all(O[0] == 0) and np.all(np.isneginf(lse[0]))
-    for r in (1, 2):
+    for r in (39, 12):
         sel = idx[r][idx[r] >= 0]
         Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
         assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL
         assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 4, 128), (8, 2, 64)])
+def test_sparse_attention_ignores_positions_the_row_cannot_see(Hq, Hkv, d):
+    # Two packed sequences [300, 200], k = 64.  In every full set the last slot is replaced
+    # by a position the row cannot see: one past its causal range (inside its sequence),
+    # one in the next sequence of the pack (still inside the K/V tensors), or past the end
+    # of the last sequence (past the end of the tensors).  Such entries must be ignored like
+    # -1, in the forward and in the backward, with no memory read behind them.
+    wl = gen.make_prefill([300, 200], Hq, Hkv, d, 4, 32, 64, seed=35, with_dO=True)
+    D = orc.Decoded(wl)
+    good = _oracle_sets(D, 64)
+    bad = good.copy()
+    kept = good.copy()
+    for r in range(wl.Tq):
+        b, i, Lq, Lk = D.seq_of_row(r)
+        if i < 64:
+            continue
+        bad[r, -1] = (i + 1 + r % 7, Lk + r % 13, 10 * Lk)[r % 3]
+        kept[r, -1] = -1
+    t = to_device(wl)
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(bad.astype(np.int32)).cuda(),
+                                     t["cu_q"], t["cu_k"])
+    Oh, lh = O.float().cpu().numpy(), lse.cpu().numpy()
+    O_ref, lse_ref = [], []
+    for r in range(wl.Tq):
+        b, i, Lq, Lk = D.seq_of_row(r)
+        sel = kept[r][kept[r] >= 0] + int(D.cu_k[b])
+        Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        assert np.max(np.abs(Oh[r] - Or)) <= ATTN_ATOL, r
+        assert np.max(np.abs(lh[r] - lr)) <= LSE_ATOL, r
+        O_ref.append(Or)
+        lse_ref.append(lr)
+    # the backward of the same sets (gather path at d = 64, masked dense path at d = 128)
+    ref = orc.sparse_attention_backward(D, kept, np.stack(O_ref), np.stack(lse_ref), D.full("dO"))
+    dQ, dK, dV = dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse,
+                                             torch.from_numpy(bad.astype(np.int32)).cuda(), t["cu_q"], t["cu_k"],
+                                             max_seqlen_k=t["max_k"])
+    for got, name in ((dQ, "dQ"), (dK, "dK"), (dV, "dV")):
+        g = got.float().cpu().numpy()
+        assert np.max(np.abs(g - ref[name])) <= 1.5e-2 * np.max(np.abs(ref[name])), name
 
 
 def test_sparse_attention_large_rising_logits():
@@ -372,4 +480,21 @@ def test_decode_pipeline():
 
 
 def test_no_device_timeouts_recorded():
+    assert dsa.device_status() == (0, 0)
+
+
+def test_bounded_wait_runs_out_and_reports():
+    # A wait with a 100 us limit on a barrier nothing arrives at (the same wait routine the
+    # pipelined kernels use) gives up, records DSA_ERR_TIMEOUT with its site code, and the
+    # kernel returns; the context stays usable and the status word is cleared on reading.
+    from lightning_indexer_b200 import _lib
+    assert dsa.device_status() == (0, 0)
+    assert _lib.load().dsa_selftest_bounded_wait(100_000, torch.cuda.current_stream().cuda_stream) == 0
+    assert dsa.device_status() == (-5, 900)
+    assert dsa.device_status() == (0, 0)
+    wl = gen.tiny_integer_1k()
+    t = to_device(wl)
+    sc = dsa.index(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"])
+    D = orc.Decoded(wl)
+    np.testing.assert_array_equal(sc[777, :778].cpu().numpy(), _oracle_scores(D, 777).astype(np.float32))
     assert dsa.device_status() == (0, 0)
