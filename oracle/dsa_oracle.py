@@ -288,6 +288,44 @@ def indexer_kl_grad_row(D: Decoded, r: int, T: int):
     return kl, np.maximum(x, 0.0).T @ g, gm.T @ kv
 
 
+def indexer_kl_loss_sparse(D: Decoded, idx: np.ndarray):
+    """Sparse-adaptation KL loss [S1]: the indexer KL of the dense warm-up restricted to each
+    token's selected set, with its gradients w.r.t. q_idx, k_idx and w.
+
+    [S1]'s second stage trains the whole model through sparse attention while the indexer
+    keeps learning from the attention it selects for.  Reading: for row t with selected set
+    S_t (sequence-local positions idx[t] >= 0),
+      p[t,s] = (1/Hq) sum_h softmax_{s in S_t}(scale * Q[t,h] . K[s, g(h)])   (a constant:
+               the head mean of the sparse attention weights)
+      q[t,s] = softmax_{s in S_t}(I[t,s])
+      KL_t   = sum_{s in S_t} p log(p/q);   loss = (1/T) sum_t KL_t
+    and the gradients of indexer_kl_loss with g[t,s] = (q - p)[s] / T on S_t, 0 elsewhere.
+    """
+    T = D.wl.Tq
+    q_idx, k_idx, w, Q, K = (D.full(n) for n in ("q_idx", "k_idx", "w", "Q", "K"))
+    kl = np.zeros(T)
+    dq = np.zeros_like(q_idx)
+    dk = np.zeros_like(k_idx)
+    dw = np.zeros_like(w)
+    for r in range(T):
+        b, i, Lq, Lk = D.seq_of_row(r)
+        k0 = int(D.cu_k[b])
+        sel = idx[r][idx[r] >= 0] + k0
+        if sel.size == 0:
+            continue
+        kv = k_idx[sel]
+        x = kv @ q_idx[r].T  # [n, H_I]
+        I_row = np.maximum(x, 0.0) @ w[r]
+        p_row = dense_target_row(Q[r], K[sel], D.scale)
+        kl[r], gI = kl_row(I_row, p_row)
+        g = gI / T
+        gm = (g[:, None] * (x > 0)) * w[r][None, :]
+        dw[r] = np.maximum(x, 0.0).T @ g
+        dq[r] = gm.T @ kv
+        np.add.at(dk, sel, gm @ q_idx[r])
+    return {"loss": float(kl.mean()), "kl": kl, "dq_idx": dq, "dk_idx": dk, "dw": dw}
+
+
 # ---------------------------------------------------------------------------------------
 # (a6) Sparse-attention backward  [S1] sparse adaptation, [P2] varlen
 # ---------------------------------------------------------------------------------------

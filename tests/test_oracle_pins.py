@@ -290,6 +290,62 @@ def test_kl_gradients_by_finite_differences():
             assert abs(fd - grad[index]) < 1e-7 + 1e-5 * abs(fd), (name, index, fd, grad[index])
 
 
+def test_sparse_kl_with_every_position_selected_is_the_dense_kl():
+    # sets that hold every visible position reduce the sparse-adaptation loss to the dense
+    # warm-up loss (itself pinned above)
+    wl = gen.make_prefill([9, 14], 4, 2, 8, 3, 4, 16, seed=10)
+    D = orc.Decoded(wl)
+    idx = np.stack([orc.forward_row(D, r, 16)["idx"] for r in range(wl.Tq)])
+    sp = orc.indexer_kl_loss_sparse(D, idx)
+    de = orc.indexer_kl_loss(D)
+    assert abs(sp["loss"] - de["loss"]) < 1e-14
+    for n in ("kl", "dq_idx", "dk_idx", "dw"):
+        np.testing.assert_allclose(sp[n], de[n], rtol=1e-12, atol=1e-15)
+
+
+def test_sparse_kl_gradients_by_finite_differences_and_unselected_keys():
+    wl = gen.make_prefill([12, 10], 4, 2, 8, 3, 4, 5, seed=13)
+    D = orc.Decoded(wl)
+    rng = np.random.default_rng(13)
+    idx = np.full((wl.Tq, 5), -1, np.int64)
+    for r in range(wl.Tq):
+        b, i, Lq, Lk = D.seq_of_row(r)
+        n = min(i + 1, 5 if r % 4 else 2)
+        idx[r, :n] = np.sort(rng.choice(i + 1, size=n, replace=False))
+    res = orc.indexer_kl_loss_sparse(D, idx)
+    assert res["loss"] > 0 and np.all(res["kl"] >= -1e-15)
+    # a key no row selected gets no gradient
+    chosen = set()
+    for r in range(wl.Tq):
+        b = D.seq_of_row(r)[0]
+        chosen |= set(int(s) + int(D.cu_k[b]) for s in idx[r] if s >= 0)
+    for s in range(wl.Tk):
+        if s not in chosen:
+            assert np.all(res["dk_idx"][s] == 0)
+    # the order of a row's entries does not matter (a set)
+    perm = idx.copy()
+    for r in range(wl.Tq):
+        perm[r] = perm[r][rng.permutation(5)]
+    res_p = orc.indexer_kl_loss_sparse(D, perm)
+    np.testing.assert_allclose(res_p["dk_idx"], res["dk_idx"], rtol=1e-12, atol=1e-16)
+    assert abs(res_p["loss"] - res["loss"]) < 1e-14
+    base = {n: D.full(n).copy() for n in ("q_idx", "k_idx", "w", "Q", "K")}
+
+    def loss_with(name, index, delta):
+        arrs = {n: v.copy() for n, v in base.items()}
+        arrs[name][index] += delta
+        D2 = orc.Decoded(wl)
+        D2._full.update(arrs)
+        return orc.indexer_kl_loss_sparse(D2, idx)["loss"]
+
+    h = 1e-6
+    for name, grad in (("q_idx", res["dq_idx"]), ("k_idx", res["dk_idx"]), ("w", res["dw"])):
+        for _ in range(6):
+            index = tuple(int(rng.integers(0, n)) for n in base[name].shape)
+            fd = (loss_with(name, index, h) - loss_with(name, index, -h)) / (2 * h)
+            assert abs(fd - grad[index]) <= 1e-6 * max(1.0, abs(fd)), (name, index, fd, grad[index])
+
+
 # ----------------------------------------------------------------------------- backward
 
 def _oracle_bwd(wl, k):
