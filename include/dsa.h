@@ -319,6 +319,32 @@ DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx,
                                 float* loss, float* kl, void* dq_idx, void* dk_idx, void* dw,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------
+ * (9) Indexer KL loss, sparse-adaptation form.  Source: report summary section 1, second
+ * training stage (the whole model trains through sparse attention; the indexer keeps
+ * learning from the attention over the positions it selects).  As (8) with every sum over
+ * the visible positions replaced by a sum over row t's selected set S_t (the entries of
+ * indices[t,:] inside [0, vis(t)), -1 unused):
+ *     p[t,s] = (1/Hq) sum_h softmax_{s in S_t}(scale * Q[t,h].K[s,g(h)])   (a constant)
+ *     q[t,s] = softmax_{s in S_t}(I[t,s]),  kl[t] = sum_{s in S_t} p log(p/q)
+ *     *loss = (1/total_q) sum_t kl[t]
+ * and the gradients of (8) with g[t,s] = (q - p)/total_q on S_t and 0 elsewhere.
+ *   indices device int32 [total_q, k] (as produced by dsa_topk / dsa_index_topk).
+ *   workspace: dsa_indexer_kl_loss_sparse_workspace_size(...) bytes (that of (8) plus the
+ *   selection bits, total_q * ceil(max_seqlen_k / 128) * 16 bytes).
+ * Supported: d = 128 with Hq = 8 Hkv, Hkv <= 4; H_I in {16, 32, 64} with d_I = 128; k <= 4096;
+ * Lq == Lk per sequence.  Deterministic like (8).
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_indexer_kl_loss_sparse_workspace_size(int64_t total_q, int64_t total_k, int max_seqlen_k,
+                                                         int Hq, int H_I, int d_I, int64_t chunk_rows, int batch);
+DSA_API int dsa_indexer_kl_loss_sparse(const void* Q, const void* K, const void* q_idx, const void* k_idx,
+                                       const void* w, const int32_t* indices, int k,
+                                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                                       int64_t total_q, int64_t total_k, int max_seqlen_q, int max_seqlen_k,
+                                       int Hq, int Hkv, int d, int H_I, int d_I, float scale,
+                                       int64_t chunk_rows, float* loss, float* kl, void* dq_idx, void* dk_idx,
+                                       void* dw, void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,7 +14,7 @@ from . import _lib
 from ._lib import DSAError, call
 
 __all__ = ["index", "topk", "topk_workspace_bytes", "index_topk", "index_topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
-           "sparse_attn_prefill_bwd", "indexer_kl_loss", "device_status", "DSAError"]
+           "sparse_attn_prefill_bwd", "indexer_kl_loss", "indexer_kl_loss_sparse", "device_status", "DSAError"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -338,6 +338,33 @@ def indexer_kl_loss(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, max_seqle
          _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Tk, max_seqlen_q, max_seqlen_k, Hq, Hkv, d, H_I, d_I,
          scale, chunk_rows, _ptr(loss), _ptr(kl), _ptr(dq), _ptr(dk), _ptr(dw), _ptr(workspace),
          workspace.numel(), _stream())
+    return loss, kl, dq, dk, dw
+
+
+def indexer_kl_loss_sparse(Q, K, q_idx, k_idx, w, indices, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                           max_seqlen_k: int, scale: Optional[float] = None, chunk_rows: int = 4096,
+                           workspace: Optional[torch.Tensor] = None):
+    """Sparse-adaptation indexer KL loss over each row's selected set, with its gradients.
+
+    Returns (loss [1] fp32, kl [T] fp32, dq_idx, dk_idx, dw) (gradients bf16).
+    """
+    T, Hq, d = Q.shape
+    Tk, Hkv, _ = K.shape
+    H_I, d_I = q_idx.shape[1], q_idx.shape[2]
+    _check(indices, "indices", torch.int32, 2)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    chunk_rows = max(1, min(chunk_rows, T))
+    nbytes = _lib.load().dsa_indexer_kl_loss_sparse_workspace_size(T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows,
+                                                                   cu_seqlens_q.numel() - 1)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=Q.device)
+    loss = torch.empty(1, dtype=torch.float32, device=Q.device)
+    kl = torch.empty(T, dtype=torch.float32, device=Q.device)
+    dq, dk, dw = torch.empty_like(q_idx), torch.empty_like(k_idx), torch.empty_like(w)
+    call("dsa_indexer_kl_loss_sparse", _ptr(Q), _ptr(K), _ptr(q_idx), _ptr(k_idx), _ptr(w), _ptr(indices),
+         indices.shape[1], _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Tk, max_seqlen_q,
+         max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, _ptr(loss), _ptr(kl), _ptr(dq), _ptr(dk), _ptr(dw),
+         _ptr(workspace), workspace.numel(), _stream())
     return loss, kl, dq, dk, dw
 
 

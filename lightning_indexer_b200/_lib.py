@@ -47,6 +47,10 @@ SIGNATURES = {
     "dsa_indexer_kl_loss": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int,
                                     c_int, c_int, c_int, c_int, c_int, c_f32, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp,
                                     c_vp, c_size, c_vp]),
+    "dsa_indexer_kl_loss_sparse_workspace_size": (c_size, [c_i64, c_i64, c_int, c_int, c_int, c_int, c_i64, c_int]),
+    "dsa_indexer_kl_loss_sparse": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_vp, c_int, c_i64, c_i64,
+                                           c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_f32, c_i64, c_vp, c_vp,
+                                           c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
 }
 
 _lib = None

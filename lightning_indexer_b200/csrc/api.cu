@@ -75,12 +75,12 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
 
 struct KLWorkspace;
 size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I, long long chunk_rows,
-                          int batch);
+                          int batch, bool sparse);
 int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
                            const int* cu_q, const int* cu_k, int batch, long long T, long long Tk,
                            int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I,
                            float scale, long long chunk_rows, float* loss, float* kl, void* dq, void* dk, void* dw,
-                           void* ws, cudaStream_t s);
+                           void* ws, cudaStream_t s, const int* indices, int k);
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 static std::once_flag g_encode_once;
@@ -426,14 +426,14 @@ DSA_API size_t dsa_indexer_kl_loss_workspace_size(int64_t total_q, int64_t total
                                                   int H_I, int d_I, int64_t chunk_rows, int batch) {
   if (total_q < 0 || total_k < 0 || max_seqlen_k < 0 || Hq < 1 || H_I < 1 || d_I < 1 || chunk_rows < 1 || batch < 1)
     return 0;
-  return kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch);
+  return kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch, false);
 }
 
-DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
-                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch, int64_t total_q,
-                                int64_t total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I,
-                                int d_I, float scale, int64_t chunk_rows, float* loss, float* kl, void* dq_idx,
-                                void* dk_idx, void* dw, void* workspace, size_t workspace_bytes, void* stream) {
+// Argument checks shared by the dense and the sparse-adaptation KL loss.
+static int kl_args_status(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
+                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                          int64_t total_k, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I, float scale,
+                          int64_t chunk_rows, float* loss, float* kl, void* dq_idx, void* dk_idx, void* dw) {
   if (!Q || !K || !q_idx || !k_idx || !w || !cu_seqlens_q || !cu_seqlens_k || !loss || !kl || !dq_idx || !dk_idx ||
       !dw)
     return DSA_ERR_INVALID_ARG;
@@ -445,12 +445,54 @@ DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx,
   if (!attn_shape_supported(Hq, Hkv, d) || Hkv > 8) return DSA_ERR_UNSUPPORTED;
   if (!((H_I == 64 || H_I == 32 || H_I == 16) && d_I == 128)) return DSA_ERR_UNSUPPORTED;
   if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+DSA_API int dsa_indexer_kl_loss(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                int64_t total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I,
+                                int d_I, float scale, int64_t chunk_rows, float* loss, float* kl, void* dq_idx,
+                                void* dk_idx, void* dw, void* workspace, size_t workspace_bytes, void* stream) {
+  if (const int st = kl_args_status(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                    max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, loss, kl, dq_idx, dk_idx,
+                                    dw);
+      st != DSA_OK)
+    return st;
   if (!workspace || !aligned16(workspace) ||
-      workspace_bytes < kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch))
+      workspace_bytes < kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch, false))
     return DSA_ERR_WORKSPACE;
   return indexer_kl_loss_launch(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
                                 max_seqlen_q, max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, loss, kl, dq_idx,
-                                dk_idx, dw, workspace, static_cast<cudaStream_t>(stream));
+                                dk_idx, dw, workspace, static_cast<cudaStream_t>(stream), nullptr, 0);
+}
+
+DSA_API size_t dsa_indexer_kl_loss_sparse_workspace_size(int64_t total_q, int64_t total_k, int max_seqlen_k, int Hq,
+                                                         int H_I, int d_I, int64_t chunk_rows, int batch) {
+  if (total_q < 0 || total_k < 0 || max_seqlen_k < 0 || Hq < 1 || H_I < 1 || d_I < 1 || chunk_rows < 1 || batch < 1)
+    return 0;
+  return kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch, true);
+}
+
+DSA_API int dsa_indexer_kl_loss_sparse(const void* Q, const void* K, const void* q_idx, const void* k_idx,
+                                       const void* w, const int32_t* indices, int k, const int32_t* cu_seqlens_q,
+                                       const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
+                                       int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I,
+                                       float scale, int64_t chunk_rows, float* loss, float* kl, void* dq_idx,
+                                       void* dk_idx, void* dw, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  if (const int st = kl_args_status(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                    max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, loss, kl, dq_idx, dk_idx,
+                                    dw);
+      st != DSA_OK)
+    return st;
+  if (!indices || k < 1) return DSA_ERR_INVALID_ARG;
+  if (!(d == 128 && Hq == 8 * Hkv && Hkv <= 4) || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < kl_workspace_bytes(total_q, total_k, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch, true))
+    return DSA_ERR_WORKSPACE;
+  return indexer_kl_loss_launch(Q, K, q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                max_seqlen_q, max_seqlen_k, Hq, Hkv, d, H_I, d_I, scale, chunk_rows, loss, kl, dq_idx,
+                                dk_idx, dw, workspace, static_cast<cudaStream_t>(stream), indices, k);
 }
 
 }  // extern "C"

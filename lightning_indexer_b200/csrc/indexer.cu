@@ -45,10 +45,12 @@ struct IndexerParams {
   int mark_ld = 0;
   const int* run_flag = nullptr;
   // Fused top-k candidates (CTA-pair kernel, fused form): scores whose order key is at
-  // least thr[r - row_begin] are appended as (key, position) to cand[(r - row_begin) * cap ..]
-  // with the running count in cnt[r - row_begin]; no score matrix is written.
+  // least thr[(r - row_begin) * state_ld] are appended as (key, position) to
+  // cand[(r - row_begin) * cap ..] with the running count in cnt[(r - row_begin) * state_ld];
+  // no score matrix is written.
   const uint32_t* thr = nullptr;
   uint32_t* cnt = nullptr;
+  long long state_ld = 1;
   uint2* cand = nullptr;
   int cap = 0;
 };

@@ -24,9 +24,10 @@
 //   - fused top-k (FUSED): no score is written; scores whose order key reaches the row's
 //     bound are appended to the row's candidate list as (key, position).  Each epilogue
 //     warp stages its candidates per token in a 64-entry shared-memory ring and moves 32
-//     at a time to global memory behind one atomicAdd on the row's count, so the count's
-//     round trip is paid once per 32 candidates, not once per key tile.  The order of a
-//     row's list depends on timing; the selection made from it does not.
+//     at a time to global memory behind one atomicAdd on the row's count; the add's result
+//     is consumed only at the token's next key tile, so its round trip overlaps a tile of
+//     work instead of stalling the warp.  The order of a row's list depends on timing; the
+//     selection made from it does not.
 #include "common.cuh"
 
 namespace dsa {
@@ -244,37 +245,47 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
         if ((have_next = decode_item<NTOK, TILE_KEYS>(nitem, p, nx))) break;
       if (have_next) prefetch_w(nx, wbuf ^ 1);
       const int dvis = it.Lk - it.Lq + 1;
-      float wr[C::CPT];
+      // this thread's head weights for the whole item, two bf16 per register (a pair never
+      // straddles two tokens: H_I is even); zero for rows past the block's tokens
+      uint32_t wp[C::CPT / 2];
 #pragma unroll
       for (int c = 0; c < C::CPT; c += 2) {
         const uint32_t pr = *reinterpret_cast<const uint32_t*>(w_s + wbuf * C::N + col0 + c);
-        const int tk0 = (col0 + c) / H_I, tk1 = (col0 + c + 1) / H_I;
-        wr[c] = tk0 < it.ntok ? __uint_as_float(pr << 16) : 0.f;
-        wr[c + 1] = tk1 < it.ntok ? __uint_as_float(pr & 0xFFFF0000u) : 0.f;
+        wp[c / 2] = (col0 + c) / H_I < it.ntok ? pr : 0u;
       }
       // visible keys (key-tensor-map rows) of this thread's tokens, 0 past the block's rows;
       // in the fused form also each token's bound and its ring state (warp-uniform)
       int vtok[C::TPW];
-      uint32_t thr_t[C::TPW], rhead[C::TPW], rcount[C::TPW];
+      // fused form, per token slot (warp-uniform): ring head, staged entries not yet
+      // reserved, entries reserved by an atomicAdd whose result (pbase, lane 0) is consumed
+      // only when the slot is next visited, so the add's round trip overlaps a key tile
+      uint32_t thr_t[C::TPW], rhead[C::TPW], rcount[C::TPW], pend[C::TPW], pbase[C::TPW];
 #pragma unroll
       for (int j = 0; j < C::TPW; ++j) {
         const int tok = col0 / H_I + j;
         vtok[j] = tok < it.ntok ? item_visible(p, it, min(max(it.i0 + tok + dvis, 0), it.Lk)) : 0;
-        thr_t[j] = FUSED && tok < it.ntok ? __ldg(p.thr + (it.t0 + tok - p.row_begin)) : 0xFFFFFFFFu;
+        thr_t[j] = FUSED && tok < it.ntok ? __ldg(p.thr + (it.t0 + tok - p.row_begin) * p.state_ld) : 0xFFFFFFFFu;
         rhead[j] = 0;
         rcount[j] = 0;
+        pend[j] = 0;
+        pbase[j] = 0;
       }
-      // moves the oldest n (<= 32) staged candidates of token slot j to the row's list
-      auto flush = [&](int j, uint32_t n) {
-        uint2* ring = reinterpret_cast<uint2*>(smem + C::OFF_RING) + (ep * C::TPW + j) * C::RING;
-        const long long rr = it.t0 + col0 / H_I + j - p.row_begin;
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(p.cnt + rr, n);
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if ((uint32_t)lane < n && base + lane < (uint32_t)p.cap)
-          p.cand[rr * p.cap + base + lane] = ring[(rhead[j] + lane) & (C::RING - 1)];
-        rhead[j] = (rhead[j] + n) & (C::RING - 1);
+      // reserves the oldest n (<= 32) staged candidates of token slot j in the row's list
+      auto reserve = [&](int j, uint32_t n) {
+        if (lane == 0) pbase[j] = atomicAdd(p.cnt + (it.t0 + col0 / H_I + j - p.row_begin) * p.state_ld, n);
+        pend[j] = n;
         rcount[j] -= n;
+      };
+      // stores the reserved entries of token slot j (waits for the reservation's result)
+      auto store_pending = [&](int j) {
+        if (pend[j] == 0) return;
+        const uint2* ring = reinterpret_cast<const uint2*>(smem + C::OFF_RING) + (ep * C::TPW + j) * C::RING;
+        const long long rr = it.t0 + col0 / H_I + j - p.row_begin;
+        const uint32_t base = __shfl_sync(0xffffffffu, pbase[j], 0);
+        if ((uint32_t)lane < pend[j] && base + lane < (uint32_t)p.cap)
+          p.cand[rr * p.cap + base + lane] = ring[(rhead[j] + lane) & (C::RING - 1)];
+        rhead[j] = (rhead[j] + pend[j]) & (C::RING - 1);
+        pend[j] = 0;
         __syncwarp();  // the ring slots just read may be refilled
       };
       for (int tile = it.tile_begin; tile < it.tile_end; ++tile) {
@@ -287,17 +298,27 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
         for (int c = 0; c < C::CPT; c += H_I) {
           const int tok = (col0 + c) / H_I;
           const int j = c / H_I;
-          float acc = 0.f;
+          // four interleaved partial sums over the heads (h mod 4), added pairwise at the
+          // end: a chain of H_I / 4 dependent FMAs instead of H_I
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int h0 = 0; h0 < H_I; h0 += 16) {
             float v[16];
             tmem_ld_x16_sync(tbase + c + h0, v);
 #pragma unroll
-            for (int q = 0; q < 16; ++q) acc = fmaf(wr[c + h0 + q], fmaxf(v[q], 0.f), acc);
+            for (int q = 0; q < 16; q += 2) {
+              const uint32_t pr = wp[(c + h0 + q) / 2];
+              a4[q & 3] = fmaf(__uint_as_float(pr << 16), fmaxf(v[q], 0.f), a4[q & 3]);
+              a4[(q + 1) & 3] = fmaf(__uint_as_float(pr & 0xFFFF0000u), fmaxf(v[q + 1], 0.f), a4[(q + 1) & 3]);
+            }
           }
+          const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
           if constexpr (!FUSED) {
             if (s < vtok[j]) out_row0[(long long)tok * p.ld] = acc;
           } else {
+            // the ring holds at most 31 staged entries here (the reservation of the previous
+            // visit is stored first), so 32 new ones never overrun its 64 slots
+            store_pending(j);
             const uint32_t key = float_order_key(acc);
             const bool pass = s < vtok[j] && key >= thr_t[j];
             const uint32_t m = __ballot_sync(0xffffffffu, pass);
@@ -308,7 +329,7 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
                     make_uint2(key, (uint32_t)s);
               rcount[j] += __popc(m);
               __syncwarp();
-              if (rcount[j] >= 32) flush(j, 32);
+              if (rcount[j] >= 32) reserve(j, 32);
             }
           }
         }
@@ -320,8 +341,13 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
       if constexpr (FUSED) {
         if (ok) {
 #pragma unroll
-          for (int j = 0; j < C::TPW; ++j)
-            if (rcount[j] > 0) flush(j, rcount[j]);
+          for (int j = 0; j < C::TPW; ++j) {
+            store_pending(j);
+            if (rcount[j] > 0) {
+              reserve(j, rcount[j]);
+              store_pending(j);
+            }
+          }
         }
       }
       item = nitem;
@@ -349,8 +375,9 @@ struct Indexer2Pass {
   const int* mark = nullptr;      // repair: rows marked -2 in mark[(r - row_begin) * mark_ld]
   int mark_ld = 0;
   const int* run_flag = nullptr;  // repair: nothing to do while *run_flag == 0
-  const uint32_t* thr = nullptr;  // fused: per-row bound, candidate counts and lists
-  uint32_t* cnt = nullptr;
+  const uint32_t* thr = nullptr;  // fused: per-row bound and candidate count (row stride
+  uint32_t* cnt = nullptr;        // state_ld) and candidate lists
+  long long state_ld = 1;
   uint2* cand = nullptr;
   int cap = 0;
 };
@@ -394,6 +421,7 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
   p.run_flag = pass.run_flag;
   p.thr = pass.thr;
   p.cnt = pass.cnt;
+  p.state_ld = pass.state_ld;
   p.cand = pass.cand;
   p.cap = pass.cap;
   const long long max_keys = S == 1 ? max_seqlen_k : max_seqlen_k / S + 2;

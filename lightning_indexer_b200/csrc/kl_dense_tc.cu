@@ -324,6 +324,10 @@ struct KlTgtParams {
   float* kl_part;        // [T, 4]
   long long n_blocks;    // bound on the 8-row blocks of the chunk
   long long n_slots;     // n_blocks rounded up to whole rounds of gridDim.x
+  // sparse-adaptation form: only the selected (t, s) pairs count (bit s & 31 of
+  // mask[((s >> 7) * mask_rows + t) * 4 + ((s >> 5) & 3)]); the others get g = 0
+  const uint32_t* mask = nullptr;
+  long long mask_rows = 0;
 };
 
 struct KlTgtItem {
@@ -589,10 +593,19 @@ __global__ void __launch_bounds__(KlTgtCfg::THREADS, 1)
 #pragma unroll
         for (int rr = 0; rr < R; ++rr) {
           if (key < vis[rr]) {
-            const float pp = pr[rr] * inv_Hq;
-            const float lq = Iv[rr] - lI[rr];  // log q
-            if (pp > 0.f) kl[rr] += pp * (logf(pp) - lq);
-            Irow[rr][key] = (expf(lq) - pp) * p.inv_T;
+            bool sel = true;
+            if (p.mask) {  // one word per (tile, row, lane quarter): the same for the whole warp
+              const long long t = it.t0 + R * rgrp + rr;
+              sel = (__ldg(p.mask + ((long long)j * p.mask_rows + t) * 4 + quarter) >> lane) & 1u;
+            }
+            if (sel) {
+              const float pp = pr[rr] * inv_Hq;
+              const float lq = Iv[rr] - lI[rr];  // log q
+              if (pp > 0.f) kl[rr] += pp * (logf(pp) - lq);
+              Irow[rr][key] = (expf(lq) - pp) * p.inv_T;
+            } else {
+              Irow[rr][key] = 0.f;
+            }
           }
         }
       }
@@ -682,7 +695,7 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
 int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                         long long Tk, int Hq, int Hkv, long long r0, long long r1, float scale_log2,
                         const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
-                        float* kl_part, cudaStream_t s) {
+                        float* kl_part, const uint32_t* mask, cudaStream_t s) {
   using C = dsa::KlTgtCfg;
   static DeviceFlag attr_done;
   if (!attr_done) {
@@ -721,6 +734,8 @@ int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int
   p.ld = ld;
   p.inv_T = inv_T;
   p.kl_part = kl_part;
+  p.mask = mask;
+  p.mask_rows = T;
   // an upper bound on the 8-row blocks (each sequence piece rounds up once)
   p.n_blocks = (r1 - r0 + 7) / 8 + batch;
   const long long grid = std::min<long long>(p.n_blocks, (long long)sm_count());

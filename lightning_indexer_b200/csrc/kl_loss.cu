@@ -154,8 +154,14 @@ __global__ void __launch_bounds__(KL_WARPS * 32)
 }
 
 // ------------------------------------------------------------------ 3. row LSE of I
+// With a selection mask (the sparse-adaptation form), only the selected positions count:
+// bit s & 31 of mask[((s >> 7) * mask_rows + row) * 4 + ((s >> 5) & 3)].
+__device__ __forceinline__ bool kl_selected(const uint32_t* mask, long long mask_rows, long long row, int s) {
+  return !mask || ((__ldg(mask + ((long long)(s >> 7) * mask_rows + row) * 4 + ((s >> 5) & 3)) >> (s & 31)) & 1u);
+}
+
 __global__ void row_lse_kernel(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
-                               long long row_begin, float* lseI) {
+                               long long row_begin, float* lseI, const uint32_t* mask, long long mask_rows) {
   __shared__ float red[32];
   const long long row = row_begin + blockIdx.x;
   const int b = seq_of_row(cu_q, batch, row);
@@ -164,7 +170,8 @@ __global__ void row_lse_kernel(const float* scores, long long ld, const int* cu_
   const int vis = min(max(i + Lk - Lq + 1, 0), Lk);
   const float* src = scores + (long long)blockIdx.x * ld;
   float m = -INFINITY;
-  for (int s = threadIdx.x; s < vis; s += blockDim.x) m = fmaxf(m, src[s]);
+  for (int s = threadIdx.x; s < vis; s += blockDim.x)
+    if (kl_selected(mask, mask_rows, row, s)) m = fmaxf(m, src[s]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = m;
@@ -174,7 +181,8 @@ __global__ void row_lse_kernel(const float* scores, long long ld, const int* cu_
   __syncthreads();
   const float mu = m == -INFINITY ? 0.f : m;
   float sum = 0.f;
-  for (int s = threadIdx.x; s < vis; s += blockDim.x) sum += expf(src[s] - mu);
+  for (int s = threadIdx.x; s < vis; s += blockDim.x)
+    if (kl_selected(mask, mask_rows, row, s)) sum += expf(src[s] - mu);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = sum;
@@ -620,7 +628,9 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
 int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                         long long Tk, int Hq, int Hkv, long long r0, long long r1, float scale_log2,
                         const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
-                        float* kl_part, cudaStream_t s);
+                        float* kl_part, const uint32_t* mask, cudaStream_t s);
+int sa_bwd_mask_build(const int* indices, const int* cu_q, const int* cu_k, int batch, long long total_q, int k,
+                      int max_seqlen_k, uint32_t* mask, cudaStream_t s);
 int kl_parts_sum_launch(const float* kl_part, long long T, float* kl, cudaStream_t s);
 int kl_dq_tc_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k, int batch,
                     long long total_q, long long total_k, long long r0, long long r1, const float* g, long long ld,
@@ -639,6 +649,7 @@ struct KLWorkspace {
   float* lseI;     // [chunk_rows]
   float* scores;   // [chunk_rows, ld]
   float* kl_part;  // [T, 4] per-key-quarter partials of kl (tensor-core target path)
+  uint32_t* mask;  // sparse-adaptation form: selection bits [ceil(max_seqlen_k / 128), T, 4]
   size_t total;
 };
 
@@ -648,7 +659,7 @@ static size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 static bool kl_tc_backward(int H_I, int d_I) { return H_I == 64 && d_I == 128; }
 
 KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I,
-                                long long chunk_rows, int batch) {
+                                long long chunk_rows, int batch, bool sparse = false) {
   KLWorkspace w{};
   uint8_t* p = static_cast<uint8_t*>(base);
   const size_t ld = ((size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1) + 3) / 4 * 4;
@@ -670,13 +681,15 @@ KLWorkspace kl_workspace_layout(void* base, long long T, long long Tk, int max_s
   off += r256((size_t)chunk_rows * ld * 4);
   w.kl_part = reinterpret_cast<float*>(p + off);
   off += r256((size_t)T * 4 * 4);
+  w.mask = reinterpret_cast<uint32_t*>(p + off);
+  if (sparse) off += r256((size_t)T * (size_t)((max_seqlen_k + 127) / 128) * 16);
   w.total = off;
   return w;
 }
 
 size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I, long long chunk_rows,
-                          int batch) {
-  return kl_workspace_layout(nullptr, T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch).total;
+                          int batch, bool sparse) {
+  return kl_workspace_layout(nullptr, T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch, sparse).total;
 }
 
 template <int H_I, int D_I>
@@ -731,18 +744,32 @@ static int kl_backward_kernels(const void* q_idx, const void* k_idx, const void*
   return DSA_OK;
 }
 
+// The indexer KL loss.  indices == nullptr: the dense warm-up form over every visible
+// position.  Otherwise the sparse-adaptation form over each row's selected set (indices
+// [T, k], sequence-local, -1 unused; tensor-core shapes only): the attention LSE, the row
+// LSE of I, the target and g all count only the selected positions, and g = 0 elsewhere, so
+// the backward kernels are those of the dense form.
 int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, const void* k_idx, const void* w,
                            const int* cu_q, const int* cu_k, int batch, long long T, long long Tk,
                            int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int d, int H_I, int d_I,
                            float scale, long long chunk_rows, float* loss, float* kl, void* dq, void* dk, void* dw,
-                           void* ws, cudaStream_t s) {
-  KLWorkspace W = kl_workspace_layout(ws, T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch);
+                           void* ws, cudaStream_t s, const int* indices, int k) {
+  const bool sparse = indices != nullptr;
+  KLWorkspace W = kl_workspace_layout(ws, T, Tk, max_seqlen_k, Hq, H_I, d_I, chunk_rows, batch, sparse);
   const long long ld = ((long long)(max_seqlen_k > 0 ? max_seqlen_k : 1) + 3) / 4 * 4;
   const float scale_log2 = scale * 1.4426950408889634f;
   if (const cudaError_t e_ = cudaMemsetAsync(W.dk_acc, 0, (size_t)Tk * d_I * 4, s); e_ != cudaSuccess) return cuda_fail(e_);
-  // 1. dense LSE (tensor cores for d = 128 and 8 query heads per KV head)
+  const uint32_t* mask = nullptr;
+  if (sparse) {
+    if (!(d == 128 && Hq == 8 * Hkv && Hkv <= 4)) return DSA_ERR_UNSUPPORTED;
+    const int st = sa_bwd_mask_build(indices, cu_q, cu_k, batch, T, k, max_seqlen_k, W.mask, s);
+    if (st != DSA_OK) return st;
+    mask = W.mask;
+  }
+  // 1. attention LSE over the visible (dense) or selected (sparse) positions (tensor cores
+  //    for d = 128 and 8 query heads per KV head)
   if (d == 128 && Hq == 8 * Hkv) {
-    const int st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, T, Tk, Hq, Hkv, max_seqlen_q, scale_log2, W.lse_att, s, nullptr,
+    const int st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, T, Tk, Hq, Hkv, max_seqlen_q, scale_log2, W.lse_att, s, mask,
                                     1.f, nullptr);
     if (st != DSA_OK) return st;
   } else {
@@ -784,11 +811,11 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
     int st = indexer_launch(q_idx, k_idx, w, cu_q, cu_k, batch, T, Tk, max_seqlen_q, max_seqlen_k, H_I, d_I, r0, r1,
                             W.scores, ld, s);
     if (st != DSA_OK) return st;
-    dsa::row_lse_kernel<<<(unsigned)(r1 - r0), 256, 0, s>>>(W.scores, ld, cu_q, cu_k, batch, r0, W.lseI);
+    dsa::row_lse_kernel<<<(unsigned)(r1 - r0), 256, 0, s>>>(W.scores, ld, cu_q, cu_k, batch, r0, W.lseI, mask, T);
     if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
     if (target_tc) {
       st = kl_target_tc_launch(Q, K, cu_q, cu_k, batch, T, Tk, Hq, Hkv, r0, r1, scale_log2, W.lse_att, W.lseI,
-                               W.scores, ld, inv_T, W.kl_part, s);
+                               W.scores, ld, inv_T, W.kl_part, mask, s);
       if (st != DSA_OK) return st;
     } else {
       const int smem = Hkv * dsa::KL_STAGES * dsa::KL_CHUNK * d * 2;

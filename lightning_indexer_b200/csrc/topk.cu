@@ -45,6 +45,7 @@ struct TopkParams {
   int k;
   int* indices;
   int only_marked;  // exact kernel: process only the rows the fast kernel marked with -2
+  int* flag_reset = nullptr;  // marked-row kernel: cleared (set to 0) by the launch
 };
 
 constexpr int TOPK_THREADS = 1024;
@@ -470,6 +471,7 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_marked_kernel(const TopkPar
     marked[atomicAdd(&nmarked, 1)] = (int)threadIdx.x;
   __syncthreads();
   const int n = nmarked;
+  if (p.flag_reset && blockIdx.x == 0 && threadIdx.x == 0) *p.flag_reset = 0;
   for (int j = 0; j < n; ++j) exact_row_select<1>(p, S, p.row_begin + r0 + marked[j]);
 }
 
@@ -1444,7 +1446,8 @@ static int topk_stream_launch(dsa::TopkParams p, long long rows, cudaStream_t st
 // Exact top-k of the rows of [row_begin, row_end) that an earlier pass marked with -2 in
 // their first index slot (indices points at row row_begin's slots).
 int topk_marked_launch(const float* scores, long long ld, const int* cu_q, const int* cu_k, int batch,
-                       long long row_begin, long long row_end, int k, int* indices, cudaStream_t stream) {
+                       long long row_begin, long long row_end, int k, int* indices, int* flag_reset,
+                       cudaStream_t stream) {
   const long long rows = row_end - row_begin;
   if (rows <= 0) return DSA_OK;
   dsa::TopkParams p;
@@ -1457,6 +1460,7 @@ int topk_marked_launch(const float* scores, long long ld, const int* cu_q, const
   p.k = k;
   p.indices = indices;
   p.only_marked = 1;
+  p.flag_reset = flag_reset;
   return topk_marked_rows_launch(p, rows, stream);
 }
 

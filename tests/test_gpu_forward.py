@@ -276,7 +276,7 @@ def test_index_topk_fused_repair_rows():
     k_idx = rng.integers(-1, 2, size=(wl.Tk, 128)).astype(np.float32)
     k_idx[np.arange(wl.Tk) % 4 == 0] = 8.0
     q_idx = rng.integers(1, 9, size=(wl.Tq, 64, 128)).astype(np.float32)
-    q_idx[1200:1300] = 0.0  # they see more positions (1201..1300) than a row's 736 candidate slots
+    q_idx[1200:1300] = 0.0  # they see more positions (1201..1300) than a row's 992 candidate slots
     q_idx[2900:2950] = 0.0
     wl.k_idx = gen.f32_to_bf16_bits(k_idx)
     wl.q_idx = gen.f32_to_bf16_bits(q_idx)

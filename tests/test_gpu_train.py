@@ -140,3 +140,48 @@ def test_training_medium_varlen_elementwise():
         assert _rel_err(dq.float().cpu().numpy(), ref["dq_idx"]) <= 1.5e-2
         assert _rel_err(dk.float().cpu().numpy(), ref["dk_idx"]) <= 1.5e-2
         assert _rel_err(dw.float().cpu().numpy(), ref["dw"]) <= 1.5e-2
+
+
+@pytest.mark.parametrize("H_I,Hq,Hkv", [(64, 32, 4), (32, 16, 2), (64, 8, 1)])
+def test_indexer_kl_loss_sparse(H_I, Hq, Hkv):
+    # sparse-adaptation KL over the oracle's selected sets (k = 64: rows past 64 select a
+    # strict subset), in one chunk and in chunks of 100 rows
+    wl = gen.make_prefill([260, 1, 129, 75], Hq, Hkv, 128, H_I, 128, 64, seed=56, layout="video")
+    D = orc.Decoded(wl)
+    idx = np.stack([orc.forward_row(D, r, 64)["idx"] for r in range(wl.Tq)])
+    ref = orc.indexer_kl_loss_sparse(D, idx)
+    t = to_device(wl)
+    tidx = torch.from_numpy(idx.astype(np.int32)).cuda()
+    for chunk in (wl.Tq, 100):
+        loss, kl, dq, dk, dw = dsa.indexer_kl_loss_sparse(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], tidx,
+                                                          t["cu_q"], t["cu_k"], t["max_q"], t["max_k"],
+                                                          chunk_rows=chunk)
+        kl = kl.cpu().numpy()
+        assert abs(loss.item() - ref["loss"]) <= 1e-4 * abs(ref["loss"]) + 1e-6
+        assert np.max(np.abs(kl - ref["kl"])) <= 1e-4 * np.max(np.abs(ref["kl"])) + 1e-6
+        assert _rel_err(dq.float().cpu().numpy(), ref["dq_idx"]) <= 1.5e-2
+        assert _rel_err(dk.float().cpu().numpy(), ref["dk_idx"]) <= 1.5e-2
+        assert _rel_err(dw.float().cpu().numpy(), ref["dw"]) <= 1.5e-2
+        # keys no row selected get exactly zero gradient
+        chosen = np.zeros(wl.Tk, bool)
+        for r in range(wl.Tq):
+            b = D.seq_of_row(r)[0]
+            chosen[idx[r][idx[r] >= 0] + int(D.cu_k[b])] = True
+        assert np.all(dk.float().cpu().numpy()[~chosen] == 0)
+
+
+def test_indexer_kl_loss_sparse_with_every_position_selected_matches_dense():
+    # k >= every row's visible count: the sparse-adaptation loss is the dense warm-up loss
+    wl = gen.make_prefill([300, 200], 32, 4, 128, 64, 128, 512, seed=57, layout="video")
+    D = orc.Decoded(wl)
+    idx = np.stack([orc.forward_row(D, r, 512)["idx"] for r in range(wl.Tq)])
+    t = to_device(wl)
+    dense = dsa.indexer_kl_loss(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"],
+                                t["max_k"])
+    sparse = dsa.indexer_kl_loss_sparse(t["Q"], t["K"], t["q_idx"], t["k_idx"], t["w"],
+                                        torch.from_numpy(idx.astype(np.int32)).cuda(), t["cu_q"], t["cu_k"],
+                                        t["max_q"], t["max_k"])
+    assert abs(dense[0].item() - sparse[0].item()) <= 1e-5 * abs(dense[0].item())
+    for a, b in zip(dense[1:], sparse[1:]):
+        a, b = a.float().cpu().numpy(), b.float().cpu().numpy()
+        assert np.max(np.abs(a - b)) <= 1e-2 * max(np.max(np.abs(a)), 1e-30)
