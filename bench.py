@@ -1,8 +1,8 @@
 #!/usr/bin/env python3
 """Throughput of the DSA hot path on B200.
 
-One step = one whole DSA prefill forward (lightning indexer + deterministic top-k, in
-row chunks, then sparse GQA attention) over the 128K-token long-video workload
+One step = one whole DSA prefill forward (lightning indexer + deterministic top-k, fused
+and in row chunks, then sparse GQA attention) over the 128K-token long-video workload
 (L=131072, Hq=32, Hkv=4, d=128, H_I=64, d_I=128, k=2048).  The decode workload (16
 sequences x 262144 cached tokens) is measured in the same run and reported under
 "decode".  Inputs are synthetic and seeded (workloads.generators) and larger than L2.
@@ -30,9 +30,10 @@ sys.path.insert(0, ROOT)
 from workloads import generators as gen  # noqa: E402
 
 PREFILL_CHUNK = 8192
-# DRAM bytes (read + write) per causal (t, s) pair of the indexer kernel, from one ncu
-# capture of this kernel on the last 4096 rows of a 32K video prefill
-IDX_DRAM_BYTES_PER_PAIR = (144.2e6 + 450.5e6) / 125831168
+# DRAM bytes (read + write) per causal (t, s) pair of the fused indexer kernel (candidates
+# instead of scores), from one ncu capture of that kernel on the last 8192 rows of a 32K
+# video prefill (None until such a capture exists for the current kernel)
+IDX_DRAM_BYTES_PER_PAIR = None
 METRIC = "DSA prefill tokens/s at 128K ctx (indexer + top-k + sparse attention)"
 
 
@@ -192,26 +193,21 @@ def run_prefill(args, rank, world, device, dist):
     cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
     t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
     k = wl.topk
-    ld = (L + 3) // 4 * 4
     chunk = PREFILL_CHUNK
-    scores = torch.empty((chunk, ld), dtype=torch.float32, device=device)
+    ws = torch.empty(dsa.index_topk_workspace_bytes(chunk, L), dtype=torch.uint8, device=device)
     idx = torch.empty((L, k), dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
-    chunks = [(r0, min(L, r0 + chunk)) for r0 in range(0, L, chunk)]
 
-    def step(ev=None):
-        for ci, (r0, r1) in enumerate(chunks):
-            if ev is not None:
-                ev[ci][0].record(stream)
-            dsa.index(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, r0, r1, scores=scores[: r1 - r0])
-            if ev is not None:
-                ev[ci][1].record(stream)
-            dsa.topk(scores[: r1 - r0], cu, cu, k, r0, r1, indices=idx[r0:r1])
-            if ev is not None:
-                ev[ci][2].record(stream)
+    def step(ev=None, path=dsa.PATH_AUTO):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, k, chunk_rows=chunk, path=path, indices=idx,
+                       workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
         out = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu)
         if ev is not None:
-            ev[-1][0].record(stream)
+            ev[2].record(stream)
         return out
 
     for _ in range(args.warmup):
@@ -219,7 +215,7 @@ def run_prefill(args, rank, world, device, dist):
     torch.cuda.synchronize(device)
 
     E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    evs = [[[E(), E(), E()] for _ in chunks] + [[E()]] for _ in range(args.steps)]
+    evs = [[E(), E(), E()] for _ in range(args.steps)]
     start, stop = E(), E()
     if dist is not None:
         dist.barrier()
@@ -233,31 +229,34 @@ def run_prefill(args, rank, world, device, dist):
     if dist is not None:
         dist.barrier()
     ms = start.elapsed_time(stop)
-    t_idx = t_topk = t_attn = 0.0
-    for s in range(args.steps):
-        for ci in range(len(chunks)):
-            e0, e1, e2 = evs[s][ci]
-            t_idx += e0.elapsed_time(e1)
-            t_topk += e1.elapsed_time(e2)
-        t_attn += evs[s][len(chunks) - 1][2].elapsed_time(evs[s][-1][0])
+    t_it = sum(e[0].elapsed_time(e[1]) for e in evs)
+    t_attn = sum(e[1].elapsed_time(e[2]) for e in evs)
     ms = max_over_ranks(ms, dist, device)
     ms_step = ms / args.steps
     value = whole_job_rate(L, ms_step, world)
+    # for comparison: the same step with the separate indexer and top-k passes
+    sep = [E(), E()]
+    step(path=dsa.PATH_SEPARATE)
+    sep[0].record(stream)
+    for _ in range(2):
+        step(path=dsa.PATH_SEPARATE)
+    sep[1].record(stream)
+    torch.cuda.synchronize(device)
 
     pairs = wl.causal_pairs()
     sel_pairs = wl.selected_pairs()
     idx_flops = pairs * wl.H_I * wl.d_I * 2
     attn_flops = sel_pairs * wl.Hq * wl.d * 4
-    n_idx_launch = len(chunks) * args.steps
+    n_chunks = (L + chunk - 1) // chunk
     res = {
         "value": value, "ms_per_step": ms_step, "clocks": clk.summary(),
-        "breakdown_ms_per_step": {"indexer": t_idx / args.steps, "topk": t_topk / args.steps,
-                                  "sparse_attn": t_attn / args.steps},
-        "idx_flops_per_launch": idx_flops / len(chunks), "idx_ms_per_launch": t_idx / n_idx_launch,
-        # per chunk: indexer, streaming top-k, exact top-k for the rows it marked; then attention
-        "launches_per_step": 3 * len(chunks) + 1,
-        "flops_per_step": idx_flops + attn_flops, "idx_flops": idx_flops, "attn_flops": attn_flops,
-        "scores_bytes_per_step": pairs * 4,
+        "breakdown_ms_per_step": {"index_topk": t_it / args.steps, "sparse_attn": t_attn / args.steps},
+        "separate_path_ms_per_step": sep[0].elapsed_time(sep[1]) / 2,
+        "idx_flops": idx_flops, "index_topk_ms": t_it / args.steps,
+        # sampled-score indexer and bound kernel, then per chunk: fused indexer, select, and the
+        # repair indexer and exact top-k (which return at once when no row needs them); attention
+        "launches_per_step": 2 + 4 * n_chunks + 1,
+        "flops_per_step": idx_flops + attn_flops, "attn_flops": attn_flops,
         "gather_bytes_per_step": sel_pairs * wl.Hkv * wl.d * 2 * 2,
     }
 
@@ -271,7 +270,7 @@ def run_prefill(args, rank, world, device, dist):
         o_h = torch.empty(tuple(wl.Q.shape), dtype=torch.bfloat16).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host.values()) + 2 * cu_h.numel() * 4
         d2h = o_h.numel() * 2
-        del t, scores, idx
+        del t, ws, idx
         torch.cuda.empty_cache()
         bufs = {}
 
@@ -296,7 +295,7 @@ def run_prefill(args, rank, world, device, dist):
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "api": "lightning_indexer_b200.prefill_from_host"}
         del host, bufs
     else:
-        del t, scores, idx
+        del t, ws, idx
     torch.cuda.empty_cache()
     return wl, res
 
@@ -564,7 +563,9 @@ def main():
         return
 
     peak_tf = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    achieved = res["idx_flops_per_launch"] / (res["idx_ms_per_launch"] / 1e3) / 1e12
+    # the dominant step: the indexer's useful flops over the whole fused index + top-k call
+    # (its sampled pass, bounds, selection and repair checks included)
+    achieved = res["idx_flops"] / (res["index_topk_ms"] / 1e3) / 1e12
     line = {
         "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
@@ -573,15 +574,17 @@ def main():
                    "d": wl.d, "H_I": wl.H_I, "d_I": wl.d_I, "topk": wl.topk, "chunk_rows": PREFILL_CHUNK,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (q_idx 2 GiB, Q 1 GiB), no flush"},
-        "roofline": {"kernel": "indexer (tcgen05)", "bound": "tensor", "achieved": achieved, "peak": peak_tf,
-                     "unit": "TFLOP/s", "frac": achieved / peak_tf,
-                     "traffic": IDX_DRAM_BYTES_PER_PAIR * res["idx_flops_per_launch"] / (2 * wl.H_I * wl.d_I),
-                     "traffic_source": "ncu dram bytes read+write of the indexer on the last 4096 rows of a 32K "
-                                       "video prefill (4.73 B per causal pair), scaled by the pairs of a launch",
+        "roofline": {"kernel": "fused indexer -> top-k (dsa_index_topk, tcgen05 indexer)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                     "traffic": (None if IDX_DRAM_BYTES_PER_PAIR is None
+                                 else IDX_DRAM_BYTES_PER_PAIR * wl.causal_pairs() / ((L + PREFILL_CHUNK - 1) // PREFILL_CHUNK)),
+                     "traffic_source": "ncu dram bytes read+write of the fused indexer kernel on the last 8192 rows of "
+                                       "a 32K video prefill, per causal pair, scaled to an average 128K chunk launch",
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"},
         "clocks": res["clocks"],
         "gpu_launches": res["launches_per_step"] * args.steps,
         "breakdown_ms_per_step": res["breakdown_ms_per_step"],
+        "separate_path_ms_per_step": res["separate_path_ms_per_step"],
         "total_tflops_per_s": res["flops_per_step"] / (res["ms_per_step"] / 1e3) / 1e12,
     }
     if "e2e" in res:

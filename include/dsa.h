@@ -138,12 +138,15 @@ DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_s
                      int k, int32_t* indices, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
- * (2b) Indexer and top-k together: the selected sets of every query row, i.e. (2) applied
- * to the scores of (1), without handing the scores to the caller.  Source: report summary
- * section 1 (the indexer scans every position; each token keeps its k best) and section 8
- * (deterministic top-k).  Rows are processed in chunks of at most `chunk_rows`.
- *   indices device int32 [total_q, k]: as (2), ascending, -1 padded, bit-for-bit the sets
- *           (2) returns on the scores of (1) (the same scores, the same tie rule).
+ * (2b) Indexer and top-k together: the selected sets of the query rows [row_begin,
+ * row_end), i.e. (2) applied to the scores of (1), without handing the scores to the
+ * caller.  Source: report summary section 1 (the indexer scans every position; each token
+ * keeps its k best) and section 8 (deterministic top-k).  Rows are processed in chunks of
+ * at most `chunk_rows`.
+ *   indices device int32 [row_end-row_begin, k]: as (2), ascending, -1 padded, bit-for-bit
+ *           the sets (2) returns on the scores of (1) (the same scores, the same tie rule).
+ *           While the call runs, slots k-2 and k-1 of each row hold that row's working state
+ *           (the fused form's bound and candidate count).
  *   path    DSA_PATH_AUTO: for (H_I, d_I) in {(64,128), (32,128)} with score rows of at
  *           most 524288 positions and room for 2k candidates per row in the scratch, the
  *           fused form: the indexer first scores every S-th key (S a power of two, about
@@ -160,8 +163,9 @@ DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_s
 DSA_API size_t dsa_index_topk_workspace_size(int64_t chunk_rows, int max_seqlen_k);
 DSA_API int dsa_index_topk(const void* q_idx, const void* k_idx, const void* w, const int32_t* cu_seqlens_q,
                            const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
-                           int max_seqlen_q, int max_seqlen_k, int H_I, int d_I, int k, int64_t chunk_rows,
-                           int path, int32_t* indices, void* workspace, size_t workspace_bytes, void* stream);
+                           int max_seqlen_q, int max_seqlen_k, int H_I, int d_I, int k, int64_t row_begin,
+                           int64_t row_end, int64_t chunk_rows, int path, int32_t* indices, void* workspace,
+                           size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * (3) Sparse GQA attention, prefill/varlen.  Source: report summary section 1 (attention
@@ -224,7 +228,7 @@ DSA_API int dsa_sparse_attn_decode_noalloc(const void* Q, const void* K, const v
                                            void* O, float* lse, void* stream);
 
 /* ---------------------------------------------------------------------------------
- * (5) Whole DSA forward for prefill: (2b) with DSA_PATH_SEPARATE over row chunks of at most
+ * (5) Whole DSA forward for prefill: (2b) with DSA_PATH_AUTO over row chunks of at most
  * `chunk_rows` query rows (bounding the fp32 score scratch), then (3).
  *   max_seqlen_q / max_seqlen_k: host ints >= every Lq / Lk.
  *   indices device int32 [total_q, k] receives the selected sets.

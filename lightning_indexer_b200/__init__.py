@@ -94,23 +94,24 @@ def index_topk_workspace_bytes(chunk_rows: int, max_seqlen_k: int) -> int:
 
 def index_topk(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, k: int,
                chunk_rows: int = 8192, path: int = PATH_AUTO, indices: Optional[torch.Tensor] = None,
-               workspace: Optional[torch.Tensor] = None):
-    """Selected sets of every query row (indexer + top-k, fused where it applies):
-    int32 [T, k], ascending, -1 padded (see dsa_index_topk)."""
+               workspace: Optional[torch.Tensor] = None, row_begin: int = 0, row_end: Optional[int] = None):
+    """Selected sets of the query rows [row_begin, row_end) (indexer + top-k, fused where it
+    applies): int32 [rows, k], ascending, -1 padded (see dsa_index_topk)."""
     _check(q_idx, "q_idx", torch.bfloat16, 3)
     _check(k_idx, "k_idx", torch.bfloat16, 2)
     _check(w, "w", torch.bfloat16, 2)
     total_q, H_I, d_I = q_idx.shape
-    chunk_rows = max(1, min(chunk_rows, max(total_q, 1)))
+    row_end = total_q if row_end is None else row_end
+    chunk_rows = max(1, min(chunk_rows, max(row_end - row_begin, 1)))
     if indices is None:
-        indices = torch.empty((total_q, k), dtype=torch.int32, device=q_idx.device)
+        indices = torch.empty((row_end - row_begin, k), dtype=torch.int32, device=q_idx.device)
     _check(indices, "indices", torch.int32, 2)
     if workspace is None:
         workspace = torch.empty(index_topk_workspace_bytes(chunk_rows, max_seqlen_k), dtype=torch.uint8,
                                 device=q_idx.device)
     call("dsa_index_topk", _ptr(q_idx), _ptr(k_idx), _ptr(w), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
-         cu_seqlens_q.numel() - 1, total_q, k_idx.shape[0], max_seqlen_q, max_seqlen_k, H_I, d_I, k, chunk_rows,
-         path, _ptr(indices), _ptr(workspace), workspace.numel(), _stream())
+         cu_seqlens_q.numel() - 1, total_q, k_idx.shape[0], max_seqlen_q, max_seqlen_k, H_I, d_I, k, row_begin,
+         row_end, chunk_rows, path, _ptr(indices), _ptr(workspace), workspace.numel(), _stream())
     return indices
 
 
@@ -203,8 +204,8 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
     """Whole DSA prefill whose inputs and output live in host memory (pin them for overlap).
 
     The key-side tensors (k_idx, K, V) are copied first; then the query rows of each row
-    chunk are copied on a copy stream while the previous chunk runs its indexer, top-k and
-    attention on the current stream, and each chunk's O rows go back on a third stream
+    chunk are copied on a copy stream while the previous chunk runs its (fused) indexer and
+    top-k and its attention on the current stream, and each chunk's O rows go back on a third stream
     while the next chunk runs.  The kernels and their results are those of `prefill`.
     `buffers` (a dict, filled on first use) keeps the device copies between calls.
     Returns O (host, bf16 [T, Hq, d]); the current stream is ordered after every copy.
@@ -225,8 +226,9 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
     cu_chunks = torch.stack([(cq - r0).clamp(0, r1 - r0) for r0, r1 in chunks]).to(torch.int32)
     if "cu_chunks" not in buf or buf["cu_chunks"].shape != cu_chunks.shape:
         buf["cu_chunks"] = torch.empty(cu_chunks.shape, dtype=torch.int32, device=dev)
-    if "scores" not in buf or buf["scores"].shape[0] < chunk_rows or buf["scores"].shape[1] < _ld(L):
-        buf["scores"] = torch.empty((chunk_rows, _ld(L)), dtype=torch.float32, device=dev)
+    ws_bytes = index_topk_workspace_bytes(chunk_rows, L)
+    if "ws" not in buf or buf["ws"].numel() < ws_bytes:
+        buf["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     if "idx" not in buf or buf["idx"].shape != (T, k):
         buf["idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
     if "O" not in buf or buf["O"].shape != Q.shape:
@@ -251,9 +253,8 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
     main.wait_event(ev_keys)
     for c, (r0, r1) in enumerate(chunks):
         main.wait_event(ev_in[c])
-        sc = buf["scores"][: r1 - r0]
-        index(buf["q_idx"], buf["k_idx"], buf["w"], buf["cu_q"], buf["cu_k"], max_seqlen_q, L, r0, r1, scores=sc)
-        topk(sc, buf["cu_q"], buf["cu_k"], k, r0, r1, indices=buf["idx"][r0:r1])
+        index_topk(buf["q_idx"], buf["k_idx"], buf["w"], buf["cu_q"], buf["cu_k"], max_seqlen_q, L, k,
+                   chunk_rows=chunk_rows, indices=buf["idx"][r0:r1], workspace=buf["ws"], row_begin=r0, row_end=r1)
         sparse_attn_prefill(buf["Q"][r0:r1], buf["K"], buf["V"], buf["idx"][r0:r1], buf["cu_chunks"][c],
                             buf["cu_k"], scale, out=(buf["O"][r0:r1], None))
         ev_out = torch.cuda.Event()

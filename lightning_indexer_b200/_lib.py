@@ -24,7 +24,7 @@ SIGNATURES = {
     "dsa_topk": (c_int, [c_vp, c_i64, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "dsa_index_topk_workspace_size": (c_size, [c_i64, c_int]),
     "dsa_index_topk": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_int,
-                               c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
+                               c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "dsa_sparse_attn_prefill": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_int, c_int, c_int,
                                         c_int, c_f32, c_vp, c_vp, c_vp]),
     "dsa_sparse_attn_decode_workspace_size": (c_size, [c_int, c_int, c_int, c_int]),

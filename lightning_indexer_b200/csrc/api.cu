@@ -71,7 +71,8 @@ int sparse_attn_bwd_launch(const void* Q, const void* K, const void* V, const vo
 size_t index_topk_workspace_bytes(long long chunk_rows, int max_seqlen_k);
 int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                       int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k, int H_I,
-                      int d_I, int k, long long chunk_rows, int* indices, void* ws, int fused, cudaStream_t stream);
+                      int d_I, int k, long long row_begin, long long row_end, long long chunk_rows, int* indices,
+                      void* ws, int fused, cudaStream_t stream);
 
 struct KLWorkspace;
 size_t kl_workspace_bytes(long long T, long long Tk, int max_seqlen_k, int Hq, int H_I, int d_I, long long chunk_rows,
@@ -302,21 +303,23 @@ DSA_API size_t dsa_index_topk_workspace_size(int64_t chunk_rows, int max_seqlen_
 
 DSA_API int dsa_index_topk(const void* q_idx, const void* k_idx, const void* w, const int32_t* cu_seqlens_q,
                            const int32_t* cu_seqlens_k, int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
-                           int max_seqlen_k, int H_I, int d_I, int k, int64_t chunk_rows, int path, int32_t* indices,
-                           void* workspace, size_t workspace_bytes, void* stream) {
+                           int max_seqlen_k, int H_I, int d_I, int k, int64_t row_begin, int64_t row_end,
+                           int64_t chunk_rows, int path, int32_t* indices, void* workspace, size_t workspace_bytes,
+                           void* stream) {
   if (!q_idx || !k_idx || !w || !cu_seqlens_q || !cu_seqlens_k || !indices) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
   if (batch < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || chunk_rows < 1 || k < 1)
     return DSA_ERR_INVALID_ARG;
+  if (row_begin < 0 || row_end < row_begin || row_end > total_q) return DSA_ERR_INVALID_ARG;
   if (path != DSA_PATH_AUTO && path != DSA_PATH_SEPARATE) return DSA_ERR_INVALID_ARG;
   if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
   if (!index_shape_supported(H_I, d_I) || k > 4096) return DSA_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace) || workspace_bytes < dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k))
     return DSA_ERR_WORKSPACE;
-  if (total_q == 0) return DSA_OK;
+  if (row_end == row_begin) return DSA_OK;
   return index_topk_launch(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
-                           max_seqlen_k, H_I, d_I, k, chunk_rows, indices, workspace, path == DSA_PATH_AUTO ? 1 : 0,
-                           static_cast<cudaStream_t>(stream));
+                           max_seqlen_k, H_I, d_I, k, row_begin, row_end, chunk_rows, indices, workspace,
+                           path == DSA_PATH_AUTO ? 1 : 0, static_cast<cudaStream_t>(stream));
 }
 
 DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k) {
@@ -334,8 +337,8 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
   if (!workspace || !aligned16(workspace) || workspace_bytes < dsa_prefill_workspace_size(chunk_rows, max_seqlen_k))
     return DSA_ERR_WORKSPACE;
   if (const int st = dsa_index_topk(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
-                                    max_seqlen_q, max_seqlen_k, H_I, d_I, k, chunk_rows, DSA_PATH_SEPARATE, indices,
-                                    workspace, workspace_bytes, stream);
+                                    max_seqlen_q, max_seqlen_k, H_I, d_I, k, 0, total_q, chunk_rows, DSA_PATH_AUTO,
+                                    indices, workspace, workspace_bytes, stream);
       st != DSA_OK)
     return st;
   // dense selected sets: masked dense tensor-core passes, their selection words and row

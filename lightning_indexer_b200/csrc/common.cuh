@@ -312,6 +312,19 @@ __device__ __forceinline__ void cp_async_wait() {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ------------------------------------------------------------------ register reallocation
+// Moves registers between the warpgroups of a block (every warp of a warpgroup executes
+// the same instruction).  The increases of all warpgroups must fit in what the block was
+// launched with (threads x registers per thread) minus what the decreases leave in use.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ misc
 // 2^x by the hardware approximation, subnormal results flushed to zero (ex2.approx.ftz).
 __device__ __forceinline__ float ex2_ftz(float x) {

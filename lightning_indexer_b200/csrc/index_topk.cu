@@ -19,12 +19,13 @@
 //   B. per row chunk:
 //      3. fused indexer: every score whose order key reaches the row's bound is appended to
 //         the row's candidate list as (key, position); no score matrix is written;
-//      4. select: per row, the exact k-th largest key K* over the candidates by radix
-//         levels over (key - bound), then the selected positions through two bitmaps over
-//         the row (keys > K*, ties at K*; the lowest-positioned `remaining` ties are kept)
-//         and a block scan, so the output is ascending whatever order the candidates
-//         arrived in.  A row with fewer than k candidates (an unlucky sample) or more than
-//         `cap` (huge ties) is marked -2 and raises the chunk's repair flag;
+//      4. select: per row, one histogram of the candidates' keys relative to the bound
+//         locates the bin of the k-th largest key; higher bins are selected outright and
+//         the few keys of that bin are ranked exactly by (key descending, position
+//         ascending); a bitmap over the row and a block scan write the positions in
+//         ascending order, whatever order the candidates arrived in.  A row with fewer
+//         than k candidates (an unlucky sample), more than `cap`, or more than 256 keys in
+//         the boundary bin (huge ties) is marked -2 and raises the chunk's repair flag;
 //      5. repair: only if the flag is raised, the indexer writes the full score rows of the
 //         marked rows' blocks to the scratch and the exact top-k selects them (and clears
 //         the flag).
@@ -108,18 +109,27 @@ __global__ void __launch_bounds__(SB_WARPS * 32) topk_sample_bound_kernel(const 
   if (lane == 0) p.thr[rr * p.state_ld] = T;
 }
 
-constexpr int CS_T = 256;  // threads of a select block
+constexpr int CS_T = 256;       // threads of a select block
+constexpr int CS_SMALL = 256;   // keys of the boundary bin resolved one per thread
 
-// Step 4: one block per row.  Dynamic shared memory: the row's candidate keys (cap) and two
-// bitmaps of ceil(vis / 32) words (sized for the longest row of the launch).
+// Step 4: one block per row.  Dynamic shared memory: the row's candidate keys (cap) and a
+// bitmap of the selected positions (ceil(vis / 32) words, sized for the launch's longest
+// row).  With d = key - bound over the candidates and a shift that maps the largest d to
+// 11 bits: one 2048-bin histogram of d >> shift locates the bin b* of the k-th largest key;
+// candidates in higher bins are selected outright; those in b* (normally a handful) go to
+// a small list in which each thread ranks one key against the others by (key descending,
+// position ascending), and the ranks below k - (count above b*) are selected.  A block scan
+// over the bitmap writes the positions in ascending order.  A row whose boundary bin holds
+// more than CS_SMALL keys (massive ties) is marked -2 for the exact path.
 __global__ void __launch_bounds__(CS_T) topk_cand_select_kernel(const FusedTopkParams p, int words) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* ckey = reinterpret_cast<uint32_t*>(smem_raw);
-  uint32_t* selw = ckey + p.cap;  // keys > K*, then the selection
-  uint32_t* tiew = selw + words;  // keys == K*
+  uint32_t* selw = ckey + p.cap;
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t total, bin, above, dmax;
+  __shared__ uint32_t total, bin, above, dmax, nsmall;
+  __shared__ uint32_t skey[CS_SMALL];
+  __shared__ int spos[CS_SMALL];
   const long long rr = blockIdx.x;
   int vis, kg;
   fused_row_geometry(p, p.row_begin + rr, vis, kg);
@@ -140,50 +150,65 @@ __global__ void __launch_bounds__(CS_T) topk_cand_select_kernel(const FusedTopkP
     return;
   }
   const uint2* src = p.cand + rr * p.cap;
-  for (uint32_t j = threadIdx.x; j < n; j += CS_T) ckey[j] = src[j].x;
-  const int W = (vis + 31) / 32;
-  for (int j = threadIdx.x; j < W; j += CS_T) {
-    selw[j] = 0u;
-    tiew[j] = 0u;
-  }
-  __syncthreads();
-  uint32_t kstar, remaining;
-  select_relative<CS_T>(ckey, (int)n, T, (uint32_t)k, hist, warp_sums, &total, &bin, &above, &dmax, kstar,
-                        remaining);
+  uint32_t dm = 0;
   for (uint32_t j = threadIdx.x; j < n; j += CS_T) {
-    const uint32_t key = ckey[j];
-    if (key < kstar) continue;
-    const int s = (int)src[j].y;  // (an L2 hit: the list was just read)
-    if (key > kstar) atomicOr(&selw[s >> 5], 1u << (s & 31));
-    else atomicOr(&tiew[s >> 5], 1u << (s & 31));
+    const uint32_t key = src[j].x;
+    ckey[j] = key;
+    dm = max(dm, key - T);
+  }
+  dm = __reduce_max_sync(0xffffffffu, dm);
+  const int W = (vis + 31) / 32;
+  for (int j = threadIdx.x; j < W; j += CS_T) selw[j] = 0u;
+  for (int j = threadIdx.x; j < 2048; j += CS_T) hist[j] = 0u;
+  if (threadIdx.x == 0) {
+    dmax = 0;
+    nsmall = 0;
   }
   __syncthreads();
-  // a contiguous run of words per thread, so that block scans give position order
+  if ((threadIdx.x & 31) == 0) atomicMax(&dmax, dm);
+  __syncthreads();
+  const int nbits = 32 - __clz((int)dmax);
+  const int shift = max(0, nbits - 11);
+  for (uint32_t j = threadIdx.x; j < n; j += CS_T) atomicAdd(&hist[(ckey[j] - T) >> shift], 1u);
+  __syncthreads();
+  find_bin<CS_T, 2048>(hist, (uint32_t)k, warp_sums, &total, &bin, &above);
+  const uint32_t bstar = bin, rem = (uint32_t)k - above;
+  for (uint32_t j = threadIdx.x; j < n; j += CS_T) {
+    const uint32_t b = (ckey[j] - T) >> shift;
+    if (b < bstar) continue;
+    const int s = (int)src[j].y;  // (an L2 hit: the list was just read)
+    if (b > bstar) {
+      atomicOr(&selw[s >> 5], 1u << (s & 31));
+    } else {
+      const uint32_t slot = atomicAdd(&nsmall, 1u);
+      if (slot < (uint32_t)CS_SMALL) {
+        skey[slot] = ckey[j];
+        spos[slot] = s;
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t m = nsmall;
+  if (m > (uint32_t)CS_SMALL) {  // block-uniform
+    if (threadIdx.x == 0) {
+      out[0] = -2;
+      atomicExch(p.flag, 1);
+    }
+    return;
+  }
+  if (threadIdx.x < m) {
+    const uint32_t key = skey[threadIdx.x];
+    const int s = spos[threadIdx.x];
+    uint32_t rank = 0;
+    for (uint32_t f = 0; f < m; ++f) rank += skey[f] > key || (skey[f] == key && spos[f] < s);
+    if (rank < rem) atomicOr(&selw[s >> 5], 1u << (s & 31));
+  }
+  __syncthreads();
+  // a contiguous run of words per thread, so that a block scan gives position order
   const int wpt = (W + CS_T - 1) / CS_T;
   const int w0 = min(W, (int)threadIdx.x * wpt), w1 = min(W, w0 + wpt);
-  uint32_t ties = 0;
-  for (int w = w0; w < w1; ++w) ties += __popc(tiew[w]);
-  uint32_t before = block_excl_scan<CS_T>(ties, warp_sums, &total);
   uint32_t mine = 0;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t x = tiew[w];
-    const uint32_t c = __popc(x);
-    if (before >= remaining) {
-      x = 0u;
-    } else if (before + c > remaining) {  // keep the lowest (remaining - before) tie positions
-      uint32_t keep = 0u;
-      for (uint32_t t = before; t < remaining; ++t) {
-        const uint32_t low = x & (~x + 1u);
-        keep |= low;
-        x ^= low;
-      }
-      x = keep;
-    }
-    before += c;
-    const uint32_t sel = selw[w] | x;
-    selw[w] = sel;
-    mine += __popc(sel);
-  }
+  for (int w = w0; w < w1; ++w) mine += __popc(selw[w]);
   uint32_t o = block_excl_scan<CS_T>(mine, warp_sums, &total);  // the block selects exactly k
   for (int w = w0; w < w1; ++w) {
     uint32_t x = selw[w];
@@ -244,35 +269,37 @@ int topk_marked_launch(const float* scores, long long ld, const int* cu_q, const
                        long long row_begin, long long row_end, int k, int* indices, int* flag_reset,
                        cudaStream_t stream);
 
-// Selected sets of every query row: the fused path where fused_plan allows it (and `fused`
-// is 1), the separate indexer and top-k passes per chunk otherwise.
+// Selected sets of the query rows [row_begin, row_end) (indices points at row row_begin's
+// slots): the fused path where fused_plan allows it (and `fused` is 1), the separate
+// indexer and top-k passes per chunk otherwise.
 int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                       int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k, int H_I,
-                      int d_I, int k, long long chunk_rows, int* indices, void* ws, int fused, cudaStream_t stream) {
+                      int d_I, int k, long long row_begin, long long row_end, long long chunk_rows, int* indices,
+                      void* ws, int fused, cudaStream_t stream) {
   const long long ld = score_ld(max_seqlen_k);
   const FusedPlan plan = fused_plan(ld, k, H_I, d_I);
   const size_t region = (size_t)chunk_rows * (size_t)ld * 4;  // the chunk's score rows
   float* scores = static_cast<float*>(ws);
   int* flag = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + up256(region));
   if (!(plan.ok && fused != 0)) {
-    for (long long r0 = 0; r0 < total_q; r0 += chunk_rows) {
-      const long long r1 = std::min(total_q, r0 + chunk_rows);
+    for (long long r0 = row_begin; r0 < row_end; r0 += chunk_rows) {
+      const long long r1 = std::min(row_end, r0 + chunk_rows);
       int st = indexer_launch(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k, H_I,
                               d_I, r0, r1, scores, ld, stream);
       if (st != DSA_OK) return st;
-      st = topk_launch(scores, ld, cu_q, cu_k, batch, r0, r1, k, indices + r0 * k,
+      st = topk_launch(scores, ld, cu_q, cu_k, batch, r0, r1, k, indices + (r0 - row_begin) * k,
                        (int)std::min<long long>(ld, 0x7FFFFFFF), nullptr, 0, stream);
       if (st != DSA_OK) return st;
     }
     return DSA_OK;
   }
   static DeviceFlag attr_done;
-  // at most 8192 candidate keys and two bitmaps of 524288 bits: 160 KiB
+  // at most 8192 candidate keys and a bitmap of 524288 bits: 96 KiB
   const int words = (int)((ld + 31) / 32);
-  const int select_smem = plan.cap * 4 + 2 * words * 4;
+  const int select_smem = plan.cap * 4 + words * 4;
   if (!attr_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(dsa::topk_cand_select_kernel,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
     if (e_ != cudaSuccess) return cuda_fail(e_);
     attr_done = true;
   }
@@ -288,8 +315,8 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
   fp.flag = flag;
   // A. sampled scores and bounds of every row, in groups whose sampled rows fit the scratch
   const long long group = std::max<long long>(1, (long long)(region / ((size_t)plan.ld_s * 4)));
-  for (long long g0 = 0; g0 < total_q; g0 += group) {
-    const long long g1 = std::min(total_q, g0 + group);
+  for (long long g0 = row_begin; g0 < row_end; g0 += group) {
+    const long long g1 = std::min(row_end, g0 + group);
     Indexer2Pass ps;
     ps.key_stride = plan.S;
     float* samples = scores;
@@ -299,8 +326,8 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
     fp.samples = samples;
     fp.row_begin = g0;
     fp.rows = g1 - g0;
-    fp.thr = reinterpret_cast<uint32_t*>(indices + g0 * k + (k - 1));
-    fp.cnt = reinterpret_cast<uint32_t*>(indices + g0 * k + (k - 2));
+    fp.thr = reinterpret_cast<uint32_t*>(indices + (g0 - row_begin) * k + (k - 1));
+    fp.cnt = reinterpret_cast<uint32_t*>(indices + (g0 - row_begin) * k + (k - 2));
     dsa::topk_sample_bound_kernel<<<(unsigned)((fp.rows + dsa::SB_WARPS - 1) / dsa::SB_WARPS), dsa::SB_WARPS * 32, 0,
                                     stream>>>(fp);
     if ((st = last_launch_status()) != DSA_OK) return st;
@@ -308,9 +335,9 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
   if (cudaError_t e_ = cudaMemsetAsync(flag, 0, sizeof(int), stream); e_ != cudaSuccess) return cuda_fail(e_);
   // B. per chunk: candidates, selection, repair of the rows the bound failed for
   uint2* cand = reinterpret_cast<uint2*>(ws);
-  for (long long r0 = 0; r0 < total_q; r0 += chunk_rows) {
-    const long long r1 = std::min(total_q, r0 + chunk_rows);
-    int* out = indices + r0 * k;
+  for (long long r0 = row_begin; r0 < row_end; r0 += chunk_rows) {
+    const long long r1 = std::min(row_end, r0 + chunk_rows);
+    int* out = indices + (r0 - row_begin) * k;
     fp.row_begin = r0;
     fp.rows = r1 - r0;
     fp.thr = reinterpret_cast<uint32_t*>(out + (k - 1));

@@ -12,7 +12,11 @@
 // own operand halves with TMA and run their own epilogue over their own 128 keys.
 //   warp 0   TMA producer (both CTAs; completion counted on the even CTA's barriers)
 //   warp 1   MMA issuer (even CTA only) + TMEM allocation (both, cta_group::2)
-//   warps 2+ epilogue (both): tcgen05.ld -> fp32 ReLU/FMA over heads -> stores
+//   warps 2-3 idle (they complete warpgroup 0)
+//   warps 4+ epilogue (both): tcgen05.ld -> fp32 ReLU/FMA over heads -> stores
+// Warpgroup 0 gives registers up (setmaxnreg) to the epilogue warpgroups, whose per-thread
+// state (head weights of two tokens, accumulators, candidate rings) needs more than an even
+// split of the register file allows.
 // Releases go back through multicast commits (stage free, accumulator full) to both CTAs
 // and through remote arrivals (accumulator drained) to the even CTA.
 //
@@ -45,7 +49,13 @@ struct Indexer2Cfg {
   static constexpr int B_BYTES = NH * D_I * 2;
   static constexpr int TMEM_COLS = (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
   static constexpr int EPI_THREADS = NUM_EPI_WARPS * 32;
-  static constexpr int THREADS = 64 + EPI_THREADS;
+  static constexpr int THREADS = 128 + EPI_THREADS;  // warpgroup 0 (roles), then the epilogue
+  // registers per thread after the reallocation: warpgroup 0 / epilogue warpgroups.  With
+  // 384 threads the launch holds 168 per thread (64512); 128 x 80 + 256 x 208 = 63488 fits,
+  // and the 64-head epilogue then runs without spilling.
+  static constexpr int REG_ROLE = 80;
+  static constexpr int REG_EPI = 208;
+  static_assert(NUM_EPI_WARPS % 4 == 0, "whole epilogue warpgroups");
   static constexpr int COL_PARTS = NUM_EPI_WARPS / 4;
   static constexpr int CPT = N / COL_PARTS;
   static_assert(CPT % H_I == 0 && H_I >= 32, "pair kernel epilogue: whole heads of whole tokens per thread");
@@ -126,6 +136,8 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
+  if (warp < 4) {
+  setmaxnreg_dec<C::REG_ROLE>();  // the whole of warpgroup 0, before it splits into roles
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
@@ -202,9 +214,11 @@ __global__ void __launch_bounds__(Indexer2Cfg<H_I, D_I, NTOK, NUM_EPI_WARPS, A_S
       while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
       }
     }
+  }
   } else {
+    setmaxnreg_inc<C::REG_EPI>();
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int ep = warp - 2;
+    const int ep = warp - 4;
     const int lane_grp = warp % 4;
     const int col_part = ep / 4;
     const int ep_tid = ep * 32 + lane;
@@ -394,6 +408,12 @@ static int launch_indexer2(const void* q_idx, const void* k_idx, const void* w, 
   if (!attr_done) {
     const cudaError_t e_ = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e_ != cudaSuccess) return cuda_fail(e_);
+    // the register reallocation must fit what the launch holds, or its increase would wait
+    // for registers that never come: check the compiled register count once
+    cudaFuncAttributes fa;
+    if (const cudaError_t e2 = cudaFuncGetAttributes(&fa, kern); e2 != cudaSuccess) return cuda_fail(e2);
+    if ((long long)fa.numRegs * C::THREADS < 128LL * C::REG_ROLE + (long long)C::EPI_THREADS * C::REG_EPI)
+      return DSA_ERR_UNSUPPORTED;
     attr_done = true;
   }
   const long long S = std::max(1, pass.key_stride);

@@ -257,6 +257,11 @@ def test_index_topk_fused_gaussian_matches_separate_and_oracle():
     wl = gen.make_prefill([3000, 1000], 8, 2, 64, 64, 128, 64, seed=37, layout="video")
     fused, separate = _fused_vs_separate(wl, 64, 1024)
     np.testing.assert_array_equal(fused, separate)
+    # a row range (crossing the sequence boundary) gives the same rows
+    t = to_device(wl)
+    part = dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], 64,
+                          chunk_rows=700, row_begin=2500, row_end=3600).cpu().numpy()
+    np.testing.assert_array_equal(part, fused[2500:3600])
     D = orc.Decoded(wl)
     for r in range(0, wl.Tq, 3):
         o = orc.forward_row(D, r, 64)
