@@ -47,7 +47,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-train", action="store_true")
-    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode", "train", "index_topk"],
+    ap.add_argument("--no-overlap", action="store_true", help="skip the high-overlap attention leg")
+    ap.add_argument("--case", default=None, choices=["indexer", "topk", "sparse_attn", "decode", "train", "index_topk",
+                                                      "overlap", "attn_paths", "reuse"],
                     help="run one kernel on a small case (for profiler captures) instead of the bench")
     ap.add_argument("--case-len", type=int, default=16384, help="sequence length of the --case workload")
     ap.add_argument("--case-chunk", type=int, default=0,
@@ -195,7 +197,11 @@ def run_prefill(args, rank, world, device, dist):
     k = wl.topk
     chunk = PREFILL_CHUNK
     ws = torch.empty(dsa.index_topk_workspace_bytes(chunk, L), dtype=torch.uint8, device=device)
+    rws = torch.empty(dsa.sparse_attn_prefill_reuse_workspace_bytes(L, wl.Hq, 1, L), dtype=torch.uint8, device=device)
     idx = torch.empty((L, k), dtype=torch.int32, device=device)
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((L, wl.Hq), dtype=torch.float32, device=device)
+    bu = torch.empty((L + 15) // 16 + 1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None, path=dsa.PATH_AUTO):
@@ -205,7 +211,8 @@ def run_prefill(args, rank, world, device, dist):
                        workspace=ws)
         if ev is not None:
             ev[1].record(stream)
-        out = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu)
+        out = dsa.sparse_attn_prefill_reuse(t["Q"], t["K"], t["V"], idx, cu, cu, L, out=(O, lse), workspace=rws,
+                                            block_union=bu)
         if ev is not None:
             ev[2].record(stream)
         return out
@@ -234,14 +241,23 @@ def run_prefill(args, rank, world, device, dist):
     ms = max_over_ranks(ms, dist, device)
     ms_step = ms / args.steps
     value = whole_job_rate(L, ms_step, world)
-    # for comparison: the same step with the separate indexer and top-k passes
+    # for comparison: the same step with the separate indexer and top-k passes, and the
+    # attention with every row on the gather kernel
     sep = [E(), E()]
     step(path=dsa.PATH_SEPARATE)
     sep[0].record(stream)
     for _ in range(2):
         step(path=dsa.PATH_SEPARATE)
     sep[1].record(stream)
+    gat = [E(), E()]
+    gat[0].record(stream)
+    for _ in range(2):
+        dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu, out=(O, lse))
+    gat[1].record(stream)
     torch.cuda.synchronize(device)
+    reuse = union_stats(bu[:(L + 15) // 16].cpu().numpy(), wl.topk)
+    reuse["attention_ms"] = t_attn / args.steps
+    reuse["gather_attention_ms"] = gat[0].elapsed_time(gat[1]) / 2
 
     pairs = wl.causal_pairs()
     sel_pairs = wl.selected_pairs()
@@ -251,11 +267,13 @@ def run_prefill(args, rank, world, device, dist):
     res = {
         "value": value, "ms_per_step": ms_step, "clocks": clk.summary(),
         "breakdown_ms_per_step": {"index_topk": t_it / args.steps, "sparse_attn": t_attn / args.steps},
+        "adjacent_query_reuse": reuse,
         "separate_path_ms_per_step": sep[0].elapsed_time(sep[1]) / 2,
         "idx_flops": idx_flops, "index_topk_ms": t_it / args.steps,
         # sampled-score indexer and bound kernel, then per chunk: fused indexer, select, and the
-        # repair indexer and exact top-k (which return at once when no row needs them); attention
-        "launches_per_step": 2 + 4 * n_chunks + 1,
+        # repair indexer and exact top-k (which return at once when no row needs them);
+        # attention: union plan, the two tensor-core passes, the gather kernel
+        "launches_per_step": 2 + 4 * n_chunks + 4,
         "flops_per_step": idx_flops + attn_flops, "attn_flops": attn_flops,
         "gather_bytes_per_step": sel_pairs * wl.Hkv * wl.d * 2 * 2,
     }
@@ -270,7 +288,7 @@ def run_prefill(args, rank, world, device, dist):
         o_h = torch.empty(tuple(wl.Q.shape), dtype=torch.bfloat16).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host.values()) + 2 * cu_h.numel() * 4
         d2h = o_h.numel() * 2
-        del t, ws, idx
+        del t, ws, rws, idx, O, lse
         torch.cuda.empty_cache()
         bufs = {}
 
@@ -295,9 +313,60 @@ def run_prefill(args, rank, world, device, dist):
                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "api": "lightning_indexer_b200.prefill_from_host"}
         del host, bufs
     else:
-        del t, ws, idx
+        del t, ws, rws, idx, O, lse
     torch.cuda.empty_cache()
     return wl, res
+
+
+UNION_CAP = 12288  # union positions per 16-row block that the tensor-core form takes
+
+
+def union_stats(block_union, topk):
+    """Per 16-row block, the number of distinct selected positions (the report's measure of
+    adjacent-query overlap: about 8000 of 16 x 2048 at 128K), over all blocks and over the
+    last 512 (rows with the whole context), and the share of blocks on the tensor-core form."""
+    u = np.asarray(block_union, dtype=np.int64)
+    last = u[-512:]
+    return {"blocks": int(u.size), "selections_per_block": 16 * topk, "mean_union": float(u.mean()),
+            "mean_union_last_512_blocks": float(last.mean()),
+            "tensor_core_block_share": float((u <= UNION_CAP).mean())}
+
+
+def run_high_overlap(args, device):
+    """Attention of the 128K video prefill with the report's adjacent-query overlap
+    (video_prefill_128k_overlap): the union form against the gather kernel on the same sets."""
+    import torch
+    import lightning_indexer_b200 as dsa
+    wl = gen.video_prefill_128k_overlap()
+    L = wl.Tq
+    cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+    idx = dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, wl.topk, chunk_rows=PREFILL_CHUNK)
+    del t["q_idx"]
+    torch.cuda.empty_cache()
+    rws = torch.empty(dsa.sparse_attn_prefill_reuse_workspace_bytes(L, wl.Hq, 1, L), dtype=torch.uint8, device=device)
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((L, wl.Hq), dtype=torch.float32, device=device)
+    bu = torch.empty((L + 15) // 16 + 1, dtype=torch.int32, device=device)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    out = {"workload": wl.name}
+    for name, fn in (("attention_ms", lambda: dsa.sparse_attn_prefill_reuse(t["Q"], t["K"], t["V"], idx, cu, cu, L,
+                                                                           out=(O, lse), workspace=rws,
+                                                                           block_union=bu)),
+                     ("gather_attention_ms", lambda: dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu,
+                                                                            out=(O, lse)))):
+        fn()
+        a, b = E(), E()
+        a.record()
+        for _ in range(3):
+            fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        out[name] = a.elapsed_time(b) / 3
+    out.update(union_stats(bu[:(L + 15) // 16].cpu().numpy(), wl.topk))
+    del t, idx, rws, O, lse
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(args, device, dist):
@@ -393,6 +462,15 @@ def run_case(args):
     if args.case == "index_topk":
         print(json.dumps(run_index_topk_case(args, device)))
         return
+    if args.case == "overlap":
+        print(json.dumps(run_overlap_case(args, device)))
+        return
+    if args.case == "attn_paths":
+        print(json.dumps(run_attn_paths_case(args, device)))
+        return
+    if args.case == "reuse":
+        print(json.dumps(run_reuse_case(args, device)))
+        return
     L = args.case_len
     if args.case == "decode":
         wl = gen.make_decode(16, L, 32, 4, 128, 64, 128, 2048, seed=3, layout="video")
@@ -419,6 +497,9 @@ def run_case(args):
     else:
         scores = dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, r0, Tq)
         idx = dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq)
+    # the decode step's top-k runs with its workspace, as in the timed decode step
+    topk_ws = (torch.empty(max(1, dsa.topk_workspace_bytes(Tq - r0, scores.shape[1], wl.topk)), dtype=torch.uint8,
+                           device=device) if args.case == "decode" else None)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for it in range(args.warmup + args.steps):
@@ -427,7 +508,7 @@ def run_case(args):
         if args.case in ("indexer", "decode"):
             dsa.index(t["q_idx"], t["k_idx"], t["w"], cu_q, cu_k, int(wl.seqlens_q.max()), Lk, r0, Tq, scores=scores)
         if args.case in ("topk", "decode"):
-            dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq, indices=idx)
+            dsa.topk(scores, cu_q, cu_k, wl.topk, r0, Tq, indices=idx, workspace=topk_ws)
         if args.case == "sparse_attn":
             dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu_q, cu_k)
         if args.case == "decode":
@@ -454,7 +535,7 @@ def run_index_topk_case(args, device):
     ws = torch.empty(dsa.index_topk_workspace_bytes(chunk, L), dtype=torch.uint8, device=device)
     out = {}
     res = {"case": "index_topk", "len": L, "chunk_rows": chunk}
-    for name, path in (("fused", dsa.PATH_AUTO), ("separate", dsa.PATH_SEPARATE)):
+    for name, path in (("auto", dsa.PATH_AUTO), ("fused", dsa.PATH_FUSED), ("separate", dsa.PATH_SEPARATE)):
         idx = torch.empty((L, wl.topk), dtype=torch.int32, device=device)
         run = lambda: dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, wl.topk,  # noqa: E731
                                      chunk_rows=chunk, path=path, indices=idx, workspace=ws)
@@ -468,8 +549,108 @@ def run_index_topk_case(args, device):
         torch.cuda.synchronize()
         res[name + "_ms"] = a.elapsed_time(b) / max(1, args.steps)
         out[name] = idx
-    res["identical"] = bool(torch.equal(out["fused"], out["separate"]))
+    res["identical"] = bool(torch.equal(out["fused"], out["separate"]) and torch.equal(out["auto"], out["separate"]))
     return res
+
+
+WORKLOADS_128K = (("video_prefill_128k", gen.video_prefill_128k),
+                  ("video_prefill_128k_coherent", gen.video_prefill_128k_coherent),
+                  ("video_prefill_128k_overlap", gen.video_prefill_128k_overlap))
+
+
+def run_overlap_case(args, device):
+    """How much the selected sets of adjacent query rows overlap on the 128K video prefills:
+    per block of 16 consecutive rows, the number of distinct selected positions (of 16 x k
+    selections), from the reuse attention's per-block union sizes.  (A measurement of the
+    inputs, not a timed step.)"""
+    import torch
+    import lightning_indexer_b200 as dsa
+    out = {"case": "overlap", "block_rows": 16}
+    for name, make in WORKLOADS_128K:
+        wl = make()
+        L = wl.Tq
+        t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+        cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+        idx = dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, wl.topk, chunk_rows=PREFILL_CHUNK)
+        bu = torch.empty((L + 15) // 16 + 1, dtype=torch.int32, device=device)
+        dsa.sparse_attn_prefill_reuse(t["Q"], t["K"], t["V"], idx, cu, cu, L, block_union=bu)
+        out[name] = union_stats(bu[:(L + 15) // 16].cpu().numpy(), wl.topk)
+        del t, idx, bu
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_reuse_case(args, device):
+    """Attention with adjacent-query reuse on a --case-len video prefill with the report's
+    adjacent-query overlap: steps + warmup calls of dsa_sparse_attn_prefill_reuse on the sets
+    from dsa_index_topk (profiling aid), with the per-block union statistics."""
+    import torch
+    import lightning_indexer_b200 as dsa
+    L = args.case_len
+    wl = gen.make_prefill([L], 32, 4, 128, 64, 128, 2048, seed=2, layout="video_overlap", max_frames=480)
+    t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+    cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+    idx = dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], cu, cu, L, L, wl.topk, chunk_rows=min(PREFILL_CHUNK, L))
+    rws = torch.empty(dsa.sparse_attn_prefill_reuse_workspace_bytes(L, wl.Hq, 1, L), dtype=torch.uint8, device=device)
+    O = torch.empty_like(t["Q"])
+    lse = torch.empty((L, wl.Hq), dtype=torch.float32, device=device)
+    bu = torch.empty((L + 15) // 16 + 1, dtype=torch.int32, device=device)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.warmup + args.steps):
+        if i == args.warmup:
+            a.record()
+        dsa.sparse_attn_prefill_reuse(t["Q"], t["K"], t["V"], idx, cu, cu, L, out=(O, lse), workspace=rws,
+                                      block_union=bu)
+    b.record()
+    torch.cuda.synchronize()
+    out = {"case": "reuse", "len": L, "ms_per_iter": a.elapsed_time(b) / max(1, args.steps)}
+    out.update(union_stats(bu[:(L + 15) // 16].cpu().numpy(), wl.topk))
+    return out
+
+
+def run_attn_paths_case(args, device):
+    """Sparse attention of the 128K video prefills, two ways on the same selected sets: with
+    adjacent-query reuse (union form where a block's union is small, gather elsewhere) and
+    with every row on the gather kernel; and the whole prefill pipeline."""
+    import torch
+    import lightning_indexer_b200 as dsa
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    out = {"case": "attn_paths"}
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        a, b = E(), E()
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    for name, make in WORKLOADS_128K:
+        wl = make()
+        L = wl.Tq
+        t = {n: bf16_dev(getattr(wl, n), device) for n in ("q_idx", "k_idx", "w", "Q", "K", "V")}
+        cu = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32)).to(device)
+        ws = torch.empty(dsa.prefill_workspace_bytes(PREFILL_CHUNK, L), dtype=torch.uint8, device=device)
+        idx = torch.empty((L, wl.topk), dtype=torch.int32, device=device)
+        O = torch.empty_like(t["Q"])
+        lse = torch.empty((L, wl.Hq), dtype=torch.float32, device=device)
+        pre = lambda: dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], cu, cu, L, L,  # noqa: E731
+                                  wl.topk, chunk_rows=PREFILL_CHUNK, workspace=ws, out=(idx, O, lse))
+        r = {"prefill_ms": timed(pre, args.steps, args.warmup)}
+        rws = ws[:dsa.sparse_attn_prefill_reuse_workspace_bytes(L, wl.Hq, 1, L)]
+        reu = lambda: dsa.sparse_attn_prefill_reuse(t["Q"], t["K"], t["V"], idx, cu, cu, L,  # noqa: E731
+                                                    out=(O, lse), workspace=rws)
+        gat = lambda: dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu, out=(O, lse))  # noqa: E731
+        r["reuse_attention_ms"] = timed(reu, args.steps, 1)
+        r["gather_attention_ms"] = timed(gat, args.steps, 1)
+        out[name] = r
+        del t, ws, rws, idx, O, lse
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_train(args, device):
@@ -550,6 +731,7 @@ def main():
     wl, res = run_prefill(args, rank, world, device, dist)
     dec = None if args.no_decode else run_decode(args, device, dist)
     train = None if args.no_train else run_train(args, device)
+    overlap = None if args.no_overlap else run_high_overlap(args, device)
     cpu = None
     if rank == 0 and not args.no_cpu:
         v, dt, thr, rows = oracle_rate(wl, 320, seed=7)
@@ -584,6 +766,7 @@ def main():
         "clocks": res["clocks"],
         "gpu_launches": res["launches_per_step"] * args.steps,
         "breakdown_ms_per_step": res["breakdown_ms_per_step"],
+        "adjacent_query_reuse": res["adjacent_query_reuse"],
         "separate_path_ms_per_step": res["separate_path_ms_per_step"],
         "total_tflops_per_s": res["flops_per_step"] / (res["ms_per_step"] / 1e3) / 1e12,
     }
@@ -617,6 +800,8 @@ def main():
                                          "target logits (2*Hq*d per causal pair), sparse attention fwd+bwd "
                                          "(12*Hq*d per selected pair)"}
         line["train"] = train
+    if overlap is not None:
+        line["adjacent_query_reuse"]["high_overlap_input"] = overlap
     print(json.dumps(line), flush=True)
 
 

@@ -64,8 +64,9 @@ typedef enum {
 
 /* How dsa_index_topk finds the selected sets. */
 typedef enum {
-  DSA_PATH_AUTO = 0,     /* the fused indexer -> top-k where it applies, else the separate passes */
-  DSA_PATH_SEPARATE = 1  /* always the separate passes: dsa_index then dsa_topk per row chunk */
+  DSA_PATH_AUTO = 0,      /* the fused indexer -> top-k where it is the faster, else the separate passes */
+  DSA_PATH_SEPARATE = 1,  /* always the separate passes: dsa_index then dsa_topk per row chunk */
+  DSA_PATH_FUSED = 2      /* the fused form wherever its shapes allow (the same sets, whatever the speed) */
 } dsa_path;
 
 /* Human-readable name of a dsa_status value.  Never returns NULL. */
@@ -147,15 +148,18 @@ DSA_API int dsa_topk(const float* scores, int64_t ld_scores, const int32_t* cu_s
  *           the sets (2) returns on the scores of (1) (the same scores, the same tie rule).
  *           While the call runs, slots k-2 and k-1 of each row hold that row's working state
  *           (the fused form's bound and candidate count).
- *   path    DSA_PATH_AUTO: for (H_I, d_I) in {(64,128), (32,128)} with score rows of at
- *           most 524288 positions and room for 2k candidates per row in the scratch, the
- *           fused form: the indexer first scores every S-th key (S a power of two, about
- *           1024 samples per full row) to bound each row's k-th largest score from below,
- *           then scores every key again but keeps only the (score, position) pairs that
- *           reach the bound, and an exact select over those pairs writes the sets; rows the
- *           bound failed for (fewer than k pairs kept, or more than fit) are recomputed
- *           in full and selected by the exact method.  Otherwise, and with
- *           DSA_PATH_SEPARATE, (1) then (2) per chunk.
+ *   path    DSA_PATH_AUTO: for (H_I, d_I) in {(64,128), (32,128)} with score rows of
+ *           65536 to 524288 positions and room for 2k candidates per row in the scratch,
+ *           the fused form: the indexer first scores every S-th key (S a power of two,
+ *           about 1024 samples per full row) to bound each row's k-th largest score from
+ *           below, then scores every key again but keeps only the (score, position) pairs
+ *           that reach the bound, and an exact select over those pairs writes the sets;
+ *           rows the bound failed for (fewer than k pairs kept, or more than fit) are
+ *           recomputed in full and selected by the exact method.  For one self-attention
+ *           sequence (batch 1, total_q == total_k) the leading chunks, whose rows see few
+ *           positions, still take the separate passes.  DSA_PATH_FUSED takes the fused
+ *           form whenever the shapes and scratch allow it, whatever the row lengths.
+ *           Otherwise, and with DSA_PATH_SEPARATE, (1) then (2) per chunk.
  *   workspace  device scratch of dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k)
  *           bytes (16-byte aligned): one chunk of fp32 score rows plus 256 bytes.
  * Supported: the shapes of (1); 1 <= k <= 4096.
@@ -186,6 +190,40 @@ DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
                                     const int32_t* cu_seqlens_k, int batch, int64_t total_q,
                                     int Hq, int Hkv, int d, int k, float scale, void* O,
                                     float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * (3c) Sparse GQA attention, prefill, with adjacent-query reuse.  Source: report summary
+ * section 8 (adjacent queries select highly similar top-k sets; the sets of adjacent
+ * queries are deduplicated and the attention kernel applies a mask laid out for the MMA's
+ * threads: at 128K and k = 2048, 16 adjacent queries touch about 8000 distinct positions
+ * instead of 16 x 2048).  Same inputs, outputs and result as (3).  Per block of 16
+ * consecutive rows of a sequence (rows i0 .. i0+15 of sequence b, i0 a multiple of 16), the
+ * sorted union of the rows' sets S (as defined in (3)) is formed.  A block whose union
+ * holds at most 12288 positions runs on tensor cores over the union, gathered 128 positions
+ * at a time (each K and V row loaded once for the block's 16 rows x 8 query heads), with a
+ * per-(row, position) selection mask on the logits; the rows of the other blocks run the
+ * gather kernel of (3).  O and lse agree with (3) within the same rounding bound.
+ *   max_seqlen_k: host int >= every Lk; total_k: rows of K and V.
+ *   workspace: dsa_sparse_attn_prefill_reuse_workspace_size(total_q, Hq, batch,
+ *     max_seqlen_k) bytes, 16-byte aligned (DSA_ERR_WORKSPACE if NULL or smaller);
+ *     about 75 KiB per block of 16 rows at max_seqlen_k >= 12288.
+ *   lse may be NULL (the workspace holds it then).
+ *   block_union: device int32 [(total_q + 15) / 16 + batch] or NULL: receives per block,
+ *     numbered over the sequences in order (ceil(Lq_b / 16) blocks for sequence b), the
+ *     size of its union (also where it exceeds 12288); the entries past the last block are
+ *     0.  Where no union is formed (see below) every entry is -1.
+ *   The tensor-core form needs d = 128, Hq = 8 Hkv and max_seqlen_k <= 262144; for other
+ *   supported shapes every row runs the gather kernel of (3).
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_sparse_attn_prefill_reuse_workspace_size(int64_t total_q, int Hq, int batch,
+                                                            int max_seqlen_k);
+DSA_API int dsa_sparse_attn_prefill_reuse(const void* Q, const void* K, const void* V,
+                                          const int32_t* indices, const int32_t* cu_seqlens_q,
+                                          const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                          int64_t total_k, int max_seqlen_k, int Hq, int Hkv, int d,
+                                          int k, float scale, void* O, float* lse,
+                                          int32_t* block_union, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
  * (4) Sparse GQA attention, decode.  Source: report summary section 8 (a decode path
@@ -233,11 +271,12 @@ DSA_API int dsa_sparse_attn_decode_noalloc(const void* Q, const void* K, const v
  *   max_seqlen_q / max_seqlen_k: host ints >= every Lq / Lk.
  *   indices device int32 [total_q, k] receives the selected sets.
  *   workspace: dsa_prefill_workspace_size(chunk_rows, max_seqlen_k) bytes.
- *   Step (3) is the gather kernel of (3), except when the selected sets are dense (d = 128,
- *   Hq = 8 Hkv, 8 k >= max_seqlen_k), lse is not NULL and the score scratch also holds
- *   total_q * ceil(max_seqlen_k / 128) * 16 bytes of selection bits plus total_q * Hq * 4
- *   bytes: then masked dense tensor-core passes compute the same O and lse (within the
- *   same rounding bound).
+ *   The attention step, with the same O and lse (within the same rounding bound) whichever
+ *   runs: when the selected sets are dense (d = 128, Hq = 8 Hkv, 8 k >= max_seqlen_k), lse
+ *   is not NULL and the score scratch also holds total_q * ceil(max_seqlen_k / 128) * 16
+ *   bytes of selection bits plus total_q * Hq * 4 bytes, masked dense tensor-core passes;
+ *   else, when the score scratch holds the workspace of (3c), (3c); else the gather kernel
+ *   of (3).
  * ------------------------------------------------------------------------------- */
 DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k);
 DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, const void* Q,

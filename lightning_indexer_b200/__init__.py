@@ -13,7 +13,7 @@ import torch
 from . import _lib
 from ._lib import DSAError, call
 
-__all__ = ["index", "topk", "topk_workspace_bytes", "index_topk", "index_topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_decode", "prefill", "decode",
+__all__ = ["index", "topk", "topk_workspace_bytes", "index_topk", "index_topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_prefill_reuse", "sparse_attn_prefill_reuse_workspace_bytes", "sparse_attn_decode", "prefill", "decode",
            "sparse_attn_prefill_bwd", "indexer_kl_loss", "indexer_kl_loss_sparse", "device_status", "DSAError"]
 
 
@@ -85,7 +85,7 @@ def topk(scores, cu_seqlens_q, cu_seqlens_k, k: int, row_begin: int = 0, row_end
     return indices
 
 
-PATH_AUTO, PATH_SEPARATE = 0, 1
+PATH_AUTO, PATH_SEPARATE, PATH_FUSED = 0, 1, 2
 
 
 def index_topk_workspace_bytes(chunk_rows: int, max_seqlen_k: int) -> int:
@@ -134,6 +134,43 @@ def sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, scale: Opt
     call("dsa_sparse_attn_prefill", _ptr(Q), _ptr(K), _ptr(V), _ptr(indices), _ptr(cu_seqlens_q),
          _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Hq, Hkv, d, indices.shape[1], scale, _ptr(O),
          _ptr(lse), _stream())
+    return O, lse
+
+
+def sparse_attn_prefill_reuse_workspace_bytes(total_q: int, Hq: int, batch: int, max_seqlen_k: int) -> int:
+    return _lib.load().dsa_sparse_attn_prefill_reuse_workspace_size(total_q, Hq, batch, max_seqlen_k)
+
+
+def sparse_attn_prefill_reuse(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, max_seqlen_k: int,
+                              scale: Optional[float] = None, out=None, workspace: Optional[torch.Tensor] = None,
+                              block_union: Optional[torch.Tensor] = None):
+    """Sparse GQA attention with adjacent-query reuse: the same (O, lse) as
+    sparse_attn_prefill, with 16-row blocks whose selections overlap computed on tensor cores
+    over the union of their sets.  `block_union` (int32, (T + 15) // 16 + batch entries) may
+    receive each block's union size."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _check(t, n, torch.bfloat16, 3)
+    _check(indices, "indices", torch.int32, 2)
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    batch = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is not None:
+        O, lse = out
+        _check(O, "O", torch.bfloat16, 3)
+    else:
+        O = torch.empty_like(Q)
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = torch.empty(sparse_attn_prefill_reuse_workspace_bytes(T, Hq, batch, max_seqlen_k),
+                                dtype=torch.uint8, device=Q.device)
+    if block_union is not None:
+        _check(block_union, "block_union", torch.int32, 1)
+        if block_union.numel() < (T + 15) // 16 + batch:
+            raise ValueError("block_union needs (T + 15) // 16 + batch entries")
+    call("dsa_sparse_attn_prefill_reuse", _ptr(Q), _ptr(K), _ptr(V), _ptr(indices), _ptr(cu_seqlens_q),
+         _ptr(cu_seqlens_k), batch, T, K.shape[0], max_seqlen_k, Hq, Hkv, d, indices.shape[1], scale, _ptr(O),
+         _ptr(lse), _ptr(block_union), _ptr(workspace), workspace.numel(), _stream())
     return O, lse
 
 
@@ -205,13 +242,14 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
 
     The key-side tensors (k_idx, K, V) are copied first; then the query rows of each row
     chunk are copied on a copy stream while the previous chunk runs its (fused) indexer and
-    top-k and its attention on the current stream, and each chunk's O rows go back on a third stream
+    top-k and its attention (with adjacent-query reuse) on the current stream, and each chunk's O rows go back on a third stream
     while the next chunk runs.  The kernels and their results are those of `prefill`.
     `buffers` (a dict, filled on first use) keeps the device copies between calls.
     Returns O (host, bf16 [T, Hq, d]); the current stream is ordered after every copy.
     """
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     T, Hq, d = Q.shape
+    B = cu_seqlens_q.numel() - 1
     L = max_seqlen_k
     chunk_rows = max(1, min(chunk_rows, T))
     chunks = [(r0, min(T, r0 + chunk_rows)) for r0 in range(0, T, chunk_rows)]
@@ -220,7 +258,6 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
                     ("cu_q", cu_seqlens_q), ("cu_k", cu_seqlens_k)):
         if name not in buf or buf[name].shape != h.shape:
             buf[name] = torch.empty(h.shape, dtype=h.dtype, device=dev)
-    B = cu_seqlens_q.numel() - 1
     # per chunk: the query offsets shifted to the chunk's first row (attention runs per chunk)
     cq = cu_seqlens_q.to(torch.int64)
     cu_chunks = torch.stack([(cq - r0).clamp(0, r1 - r0) for r0, r1 in chunks]).to(torch.int32)
@@ -229,6 +266,9 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
     ws_bytes = index_topk_workspace_bytes(chunk_rows, L)
     if "ws" not in buf or buf["ws"].numel() < ws_bytes:
         buf["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    rws_bytes = sparse_attn_prefill_reuse_workspace_bytes(chunk_rows, Hq, B, L)
+    if "rws" not in buf or buf["rws"].numel() < rws_bytes:
+        buf["rws"] = torch.empty(rws_bytes, dtype=torch.uint8, device=dev)
     if "idx" not in buf or buf["idx"].shape != (T, k):
         buf["idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
     if "O" not in buf or buf["O"].shape != Q.shape:
@@ -255,8 +295,8 @@ def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_
         main.wait_event(ev_in[c])
         index_topk(buf["q_idx"], buf["k_idx"], buf["w"], buf["cu_q"], buf["cu_k"], max_seqlen_q, L, k,
                    chunk_rows=chunk_rows, indices=buf["idx"][r0:r1], workspace=buf["ws"], row_begin=r0, row_end=r1)
-        sparse_attn_prefill(buf["Q"][r0:r1], buf["K"], buf["V"], buf["idx"][r0:r1], buf["cu_chunks"][c],
-                            buf["cu_k"], scale, out=(buf["O"][r0:r1], None))
+        sparse_attn_prefill_reuse(buf["Q"][r0:r1], buf["K"], buf["V"], buf["idx"][r0:r1], buf["cu_chunks"][c],
+                                  buf["cu_k"], L, scale, out=(buf["O"][r0:r1], None), workspace=buf["rws"])
         ev_out = torch.cuda.Event()
         ev_out.record(main)
         d2h.wait_event(ev_out)

@@ -45,7 +45,17 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
                 size_t ws_bytes, cudaStream_t stream);
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
                                const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
-                               float scale, void* O, float* lse, cudaStream_t stream);
+                               float scale, void* O, float* lse, cudaStream_t stream, const uint8_t* skip_rows);
+size_t sa_block_reuse_scratch_bytes(long long total_q, int Hq, int batch, int max_seqlen_k, int max_chunks);
+bool sa_block_reuse_eligible(int Hq, int Hkv, int d, int max_seqlen_k);
+int sa_block_reuse_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                          const int* cu_k, int batch, long long total_q, long long total_k, int Hq, int Hkv, int k,
+                          int max_seqlen_k, int max_chunks, float scale, void* O, float* lse, void* ws,
+                          int* ucount_out, cudaStream_t s);
+// A 16-row block runs on the tensor-core passes (union form) when the union of its rows'
+// selected positions fits this many chunks of 128 positions: at 128K a block and KV head
+// costs about 1.6 us on the gather kernel and about 13 ns per 128-key chunk on the passes.
+constexpr int kUnionMaxChunks = 96;
 size_t decode_workspace_bytes(int batch, int Hq, int d, int k);
 int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_k,
                               int batch, int Hq, int Hkv, int d, int k, float scale, void* O, float* lse,
@@ -275,7 +285,46 @@ DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
   if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
   if (total_q == 0) return DSA_OK;
   return sparse_attn_prefill_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k,
-                                    scale, O, lse, static_cast<cudaStream_t>(stream));
+                                    scale, O, lse, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+static size_t reuse_lse_bytes(int64_t total_q, int Hq) { return round_up((size_t)total_q * Hq * 4, 256); }
+
+DSA_API size_t dsa_sparse_attn_prefill_reuse_workspace_size(int64_t total_q, int Hq, int batch, int max_seqlen_k) {
+  if (total_q < 0 || Hq < 1 || batch < 1 || max_seqlen_k < 0) return 0;
+  return reuse_lse_bytes(total_q, Hq) +
+         sa_block_reuse_scratch_bytes(total_q, Hq, batch, std::max(max_seqlen_k, 1), kUnionMaxChunks);
+}
+
+DSA_API int dsa_sparse_attn_prefill_reuse(const void* Q, const void* K, const void* V, const int32_t* indices,
+                                          const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                                          int64_t total_q, int64_t total_k, int max_seqlen_k, int Hq, int Hkv, int d,
+                                          int k, float scale, void* O, float* lse, int32_t* block_union,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !indices || !cu_seqlens_q || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(indices))
+    return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || total_k < 0 || max_seqlen_k < 0 || k < 1 || !(scale > 0.f))
+    return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_supported(Hq, Hkv, d) || k % 16 != 0 || k > 4096) return DSA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < dsa_sparse_attn_prefill_reuse_workspace_size(total_q, Hq, batch, max_seqlen_k))
+    return DSA_ERR_WORKSPACE;
+  if (total_q == 0) return DSA_OK;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!sa_block_reuse_eligible(Hq, Hkv, d, max_seqlen_k)) {
+    if (block_union) {
+      const size_t n_blocks = (size_t)((total_q + 15) / 16 + batch);
+      if (const cudaError_t e_ = cudaMemsetAsync(block_union, 0xff, n_blocks * 4, s); e_ != cudaSuccess)
+        return cuda_fail(e_);
+    }
+    return sparse_attn_prefill_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k,
+                                      scale, O, lse, s, nullptr);
+  }
+  float* lse_buf = lse ? lse : static_cast<float*>(workspace);
+  void* ws = static_cast<uint8_t*>(workspace) + reuse_lse_bytes(total_q, Hq);
+  return sa_block_reuse_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, Hq, Hkv, k,
+                               max_seqlen_k, kUnionMaxChunks, scale, O, lse_buf, ws, block_union, s);
 }
 
 DSA_API size_t dsa_sparse_attn_decode_workspace_size(int batch, int Hq, int d, int k) {
@@ -311,7 +360,7 @@ DSA_API int dsa_index_topk(const void* q_idx, const void* k_idx, const void* w, 
   if (batch < 1 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || chunk_rows < 1 || k < 1)
     return DSA_ERR_INVALID_ARG;
   if (row_begin < 0 || row_end < row_begin || row_end > total_q) return DSA_ERR_INVALID_ARG;
-  if (path != DSA_PATH_AUTO && path != DSA_PATH_SEPARATE) return DSA_ERR_INVALID_ARG;
+  if (path != DSA_PATH_AUTO && path != DSA_PATH_SEPARATE && path != DSA_PATH_FUSED) return DSA_ERR_INVALID_ARG;
   if (total_q * (int64_t)H_I > 0x7FFFFFFFLL || total_k > 0x7FFFFFFFLL) return DSA_ERR_UNSUPPORTED;
   if (!index_shape_supported(H_I, d_I) || k > 4096) return DSA_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace) || workspace_bytes < dsa_index_topk_workspace_size(chunk_rows, max_seqlen_k))
@@ -319,7 +368,8 @@ DSA_API int dsa_index_topk(const void* q_idx, const void* k_idx, const void* w, 
   if (row_end == row_begin) return DSA_OK;
   return index_topk_launch(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                            max_seqlen_k, H_I, d_I, k, row_begin, row_end, chunk_rows, indices, workspace,
-                           path == DSA_PATH_AUTO ? 1 : 0, static_cast<cudaStream_t>(stream));
+                           path == DSA_PATH_SEPARATE ? 0 : path == DSA_PATH_AUTO ? 1 : 2,
+                           static_cast<cudaStream_t>(stream));
 }
 
 DSA_API size_t dsa_prefill_workspace_size(int64_t chunk_rows, int max_seqlen_k) {
@@ -350,6 +400,14 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
     return sa_fwd_tc_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, Hq, Hkv, k,
                             max_seqlen_k, scale, O, lse, workspace, static_cast<cudaStream_t>(stream));
   }
+  // sparse sets: blocks of 16 adjacent rows whose selected sets overlap (small union) run on
+  // the tensor cores over the gathered union (each key loaded once for the block), the rest
+  // on the gather kernel, when the score scratch holds the union plans
+  if (sa_block_reuse_eligible(Hq, Hkv, d, max_seqlen_k) &&
+      dsa_sparse_attn_prefill_reuse_workspace_size(total_q, Hq, batch, max_seqlen_k) <= workspace_bytes)
+    return dsa_sparse_attn_prefill_reuse(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                         max_seqlen_k, Hq, Hkv, d, k, scale, O, lse, nullptr, workspace,
+                                         workspace_bytes, stream);
   return dsa_sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k, scale,
                                  O, lse, stream);
 }

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <climits>
+
 #include <atomic>
 #include <utility>
 
@@ -118,6 +120,18 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// TMA row gather: four rows (r0..r3) of a 2-D tensor map whose box is one row high, each
+// box_cols wide from column c0, land one after another at dst (the map's swizzle applies as
+// for a tiled load of those rows); completion counted on `bar`.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0, int r1,
+                                            int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 
@@ -404,6 +418,23 @@ int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 
 int make_tmap_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
                       const uint32_t box[3]);
+
+// Rows of 128 bf16 (256 bytes, e.g. K or V viewed as [Tk * Hkv, 128]) for TMA row gathers:
+// boxes of one row by 64 columns with the 128-byte swizzle.
+inline int make_tmap_rows_gather(CUtensorMap* map, const void* base, long long rows) {
+  return make_tmap_bf16_2d(map, base, (uint64_t)(rows > 0 ? rows : 1), 128, 256, 1, 64, 128);
+}
+
+// The union form of the masked tensor-core attention passes (adjacent-query reuse): per
+// 16-row block the sorted union of its rows' selected positions, its size, the
+// per-(row, union slot) selection words and whether the block takes the form at all.
+struct KlUnion {
+  const int* ukeys;
+  const int* ucount;
+  const uint32_t* umask;
+  const uint8_t* blk_use;
+  int ucap;  // positions per block, a multiple of 128
+};
 
 // A one-time-setup flag kept per GPU: cudaFuncSetAttribute applies to the current device
 // only, and one process may drive several GPUs.  Reads and writes go to the current

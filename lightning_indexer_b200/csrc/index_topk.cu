@@ -114,13 +114,14 @@ constexpr int CS_SMALL = 256;   // keys of the boundary bin resolved one per thr
 
 // Step 4: one block per row.  Dynamic shared memory: the row's candidate keys (cap) and a
 // bitmap of the selected positions (ceil(vis / 32) words, sized for the launch's longest
-// row).  With d = key - bound over the candidates and a shift that maps the largest d to
-// 11 bits: one 2048-bin histogram of d >> shift locates the bin b* of the k-th largest key;
-// candidates in higher bins are selected outright; those in b* (normally a handful) go to
-// a small list in which each thread ranks one key against the others by (key descending,
-// position ascending), and the ranks below k - (count above b*) are selected.  A block scan
-// over the bitmap writes the positions in ascending order.  A row whose boundary bin holds
-// more than CS_SMALL keys (massive ties) is marked -2 for the exact path.
+// row).  With d = key - bound over the candidates: 2048-bin histograms of 11-bit digits of
+// d, from the top of its range, locate the bin of the k-th largest key (one level when
+// that bin holds at most CS_SMALL keys, which is the usual case; up to three otherwise);
+// candidates above that bin are selected outright, and those in it go to a small list in
+// which each thread ranks one key against the others by (key descending, position
+// ascending), the ranks below k - (count above) being selected.  A block scan over the
+// bitmap writes the positions in ascending order.  A row with more than CS_SMALL keys
+// equal to the k-th (massive ties) is marked -2 for the exact path.
 __global__ void __launch_bounds__(CS_T) topk_cand_select_kernel(const FusedTopkParams p, int words) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint32_t* ckey = reinterpret_cast<uint32_t*>(smem_raw);
@@ -151,15 +152,24 @@ __global__ void __launch_bounds__(CS_T) topk_cand_select_kernel(const FusedTopkP
   }
   const uint2* src = p.cand + rr * p.cap;
   uint32_t dm = 0;
-  for (uint32_t j = threadIdx.x; j < n; j += CS_T) {
-    const uint32_t key = src[j].x;
-    ckey[j] = key;
-    dm = max(dm, key - T);
+  // four independent loads in flight per thread
+  for (uint32_t j0 = threadIdx.x; j0 < n; j0 += 4 * CS_T) {
+    uint32_t kk[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = j0 + u * CS_T;
+      kk[u] = j < n ? __ldg(&src[j].x) : T;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = j0 + u * CS_T;
+      if (j < n) ckey[j] = kk[u];
+      dm = max(dm, kk[u] - T);
+    }
   }
   dm = __reduce_max_sync(0xffffffffu, dm);
   const int W = (vis + 31) / 32;
   for (int j = threadIdx.x; j < W; j += CS_T) selw[j] = 0u;
-  for (int j = threadIdx.x; j < 2048; j += CS_T) hist[j] = 0u;
   if (threadIdx.x == 0) {
     dmax = 0;
     nsmall = 0;
@@ -167,35 +177,61 @@ __global__ void __launch_bounds__(CS_T) topk_cand_select_kernel(const FusedTopkP
   __syncthreads();
   if ((threadIdx.x & 31) == 0) atomicMax(&dmax, dm);
   __syncthreads();
+  // radix levels over d = key - bound (11 bits each, from the top of the range): each level
+  // narrows to the bin holding the rem-th largest of the keys that share the prefix so far,
+  // and stops once that bin is small (or the last bits are reached)
   const int nbits = 32 - __clz((int)dmax);
-  const int shift = max(0, nbits - 11);
-  for (uint32_t j = threadIdx.x; j < n; j += CS_T) atomicAdd(&hist[(ckey[j] - T) >> shift], 1u);
-  __syncthreads();
-  find_bin<CS_T, 2048>(hist, (uint32_t)k, warp_sums, &total, &bin, &above);
-  const uint32_t bstar = bin, rem = (uint32_t)k - above;
-  for (uint32_t j = threadIdx.x; j < n; j += CS_T) {
-    const uint32_t b = (ckey[j] - T) >> shift;
-    if (b < bstar) continue;
-    const int s = (int)src[j].y;  // (an L2 hit: the list was just read)
-    if (b > bstar) {
-      atomicOr(&selw[s >> 5], 1u << (s & 31));
-    } else {
-      const uint32_t slot = atomicAdd(&nsmall, 1u);
-      if (slot < (uint32_t)CS_SMALL) {
-        skey[slot] = ckey[j];
-        spos[slot] = s;
-      }
+  int shift = max(0, nbits - 11);
+  uint32_t prefix = 0, pmask = 0, rem = (uint32_t)k, in_bin = 0;
+#pragma unroll 1
+  while (true) {
+    for (int j = threadIdx.x; j < 2048; j += CS_T) hist[j] = 0u;
+    __syncthreads();
+    for (uint32_t j = threadIdx.x; j < n; j += CS_T) {
+      const uint32_t d = ckey[j] - T;
+      if ((d & pmask) == prefix) atomicAdd(&hist[(d >> shift) & 2047u], 1u);
     }
+    __syncthreads();
+    find_bin<CS_T, 2048>(hist, rem, warp_sums, &total, &bin, &above);
+    in_bin = hist[bin];
+    prefix |= bin << shift;
+    pmask |= 2047u << shift;
+    rem -= above;
+    if (in_bin <= (uint32_t)CS_SMALL || shift == 0) break;
+    shift = max(0, shift - 11);
+    __syncthreads();  // every thread has read hist[bin] before the next level clears it
   }
-  __syncthreads();
-  const uint32_t m = nsmall;
-  if (m > (uint32_t)CS_SMALL) {  // block-uniform
+  if (in_bin > (uint32_t)CS_SMALL) {  // block-uniform: more than CS_SMALL equal keys
     if (threadIdx.x == 0) {
       out[0] = -2;
       atomicExch(p.flag, 1);
     }
     return;
   }
+  for (uint32_t j0 = threadIdx.x; j0 < n; j0 += 4 * CS_T) {
+    uint32_t md[4];
+    int sp[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t j = j0 + u * CS_T;
+      md[u] = j < n ? (ckey[j] - T) & pmask : 0u;
+      sp[u] = (j < n && md[u] >= prefix) ? (int)__ldg(&src[j].y) : -1;  // (L2 hits: just read)
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (sp[u] < 0) continue;
+      const int s = sp[u];
+      if (md[u] > prefix) {
+        atomicOr(&selw[s >> 5], 1u << (s & 31));
+      } else {
+        const uint32_t slot = atomicAdd(&nsmall, 1u);
+        skey[slot] = ckey[j0 + u * CS_T];
+        spos[slot] = s;
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t m = nsmall;  // == in_bin <= CS_SMALL
   if (threadIdx.x < m) {
     const uint32_t key = skey[threadIdx.x];
     const int s = spos[threadIdx.x];
@@ -270,8 +306,8 @@ int topk_marked_launch(const float* scores, long long ld, const int* cu_q, const
                        cudaStream_t stream);
 
 // Selected sets of the query rows [row_begin, row_end) (indices points at row row_begin's
-// slots): the fused path where fused_plan allows it (and `fused` is 1), the separate
-// indexer and top-k passes per chunk otherwise.
+// slots): the fused path or the separate indexer and top-k passes per chunk, as `fused`
+// asks (0 separate, 1 automatic, 2 fused where fused_plan allows it).
 int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const int* cu_q, const int* cu_k,
                       int batch, long long total_q, long long total_k, int max_seqlen_q, int max_seqlen_k, int H_I,
                       int d_I, int k, long long row_begin, long long row_end, long long chunk_rows, int* indices,
@@ -281,9 +317,25 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
   const size_t region = (size_t)chunk_rows * (size_t)ld * 4;  // the chunk's score rows
   float* scores = static_cast<float*>(ws);
   int* flag = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + up256(region));
-  if (!(plan.ok && fused != 0)) {
-    for (long long r0 = row_begin; r0 < row_end; r0 += chunk_rows) {
-      const long long r1 = std::min(row_end, r0 + chunk_rows);
+  // Rows [fused_begin, row_end) take the fused path.  It pays where rows see many more
+  // positions than a row keeps candidates (a row of at most `cap` visible positions keeps
+  // them all, as 8-byte pairs, so it is cheaper on the separate passes): not at all for
+  // score rows shorter than 65536 (measured: slower at 16K and 32K, faster at 128K), and for
+  // one self-attention sequence (batch 1, Lq == Lk, row r sees r + 1 positions) not in the
+  // leading chunks whose rows see at most 2 cap positions.
+  // (fused: 0 = separate passes, 1 = that choice, 2 = the fused path wherever the plan allows)
+  long long fused_begin = row_end;
+  if (plan.ok && fused == 2) {
+    fused_begin = row_begin;
+  } else if (plan.ok && fused == 1 && ld >= 65536) {
+    fused_begin = row_begin;
+    if (batch == 1 && total_q == total_k)
+      while (fused_begin < row_end && std::min(row_end, fused_begin + chunk_rows) <= 2LL * plan.cap)
+        fused_begin += chunk_rows;
+  }
+  if (fused_begin > row_begin) {
+    for (long long r0 = row_begin; r0 < fused_begin; r0 += chunk_rows) {
+      const long long r1 = std::min(fused_begin, r0 + chunk_rows);
       int st = indexer_launch(q_idx, k_idx, w, cu_q, cu_k, batch, total_q, total_k, max_seqlen_q, max_seqlen_k, H_I,
                               d_I, r0, r1, scores, ld, stream);
       if (st != DSA_OK) return st;
@@ -291,7 +343,7 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
                        (int)std::min<long long>(ld, 0x7FFFFFFF), nullptr, 0, stream);
       if (st != DSA_OK) return st;
     }
-    return DSA_OK;
+    if (fused_begin == row_end) return DSA_OK;
   }
   static DeviceFlag attr_done;
   // at most 8192 candidate keys and a bitmap of 524288 bits: 96 KiB
@@ -315,7 +367,7 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
   fp.flag = flag;
   // A. sampled scores and bounds of every row, in groups whose sampled rows fit the scratch
   const long long group = std::max<long long>(1, (long long)(region / ((size_t)plan.ld_s * 4)));
-  for (long long g0 = row_begin; g0 < row_end; g0 += group) {
+  for (long long g0 = fused_begin; g0 < row_end; g0 += group) {
     const long long g1 = std::min(row_end, g0 + group);
     Indexer2Pass ps;
     ps.key_stride = plan.S;
@@ -335,7 +387,7 @@ int index_topk_launch(const void* q_idx, const void* k_idx, const void* w, const
   if (cudaError_t e_ = cudaMemsetAsync(flag, 0, sizeof(int), stream); e_ != cudaSuccess) return cuda_fail(e_);
   // B. per chunk: candidates, selection, repair of the rows the bound failed for
   uint2* cand = reinterpret_cast<uint2*>(ws);
-  for (long long r0 = row_begin; r0 < row_end; r0 += chunk_rows) {
+  for (long long r0 = fused_begin; r0 < row_end; r0 += chunk_rows) {
     const long long r1 = std::min(row_end, r0 + chunk_rows);
     int* out = indices + (r0 - row_begin) * k;
     fp.row_begin = r0;

@@ -15,6 +15,11 @@
 // MMA issuer and TMEM owner, warps 2-9 epilogue (two per TMEM lane quarter, one per
 // 64-key half of each tile; their two running (max, sum) pairs merge at the item's end);
 // two accumulator buffers, four key stages.
+//
+// Union form (adjacent-query reuse, report summary section 8): a block visits, instead of
+// its causal key tiles, chunks of 128 positions of the sorted union of its rows' selected
+// sets; the producer warp gathers those K rows with TMA row gathers (one four-row gather per
+// lane and 64-column panel), and the per-(row, union slot) selection bits mask S.
 #include <algorithm>
 
 #include "common.cuh"
@@ -37,17 +42,30 @@ struct KlLseParams {
   const uint32_t* mask;
   long long total_q;
   float* max_out;  // optional [T, Hq]: the row maxima of the scaled logits in base 2
+  // optional union form: only blocks with blk_use[blk] != 0 are items (blk: the block's
+  // number in ascending order over the sequences); block blk visits ceil(ucount[blk] / 128)
+  // chunks of the positions ukeys[blk * ucap ..] (sequence-local, ascending, padded with
+  // position 0 to a whole chunk), with selection words
+  // umask[((blk * (ucap / 128) + chunk) * 16 + row) * 4 + slot / 32] (bit slot % 32) in
+  // place of `mask`; the key tensor map then addresses K as rows (s * Hkv + g) of d values
+  const int* ukeys = nullptr;
+  const int* ucount = nullptr;
+  const uint32_t* umask = nullptr;
+  const uint8_t* blk_use = nullptr;
+  int ucap = 0;
 };
 
 struct KlLseItem {
   long long t0;
   int ntok, i0, Lq, Lk, kbase, g, ntiles;
+  long long blk;
 };
 
 // item -> (block, head); blocks are numbered from the last (usually the longest rows)
 __device__ __forceinline__ bool kl_lse_item(long long item, const KlLseParams& p, KlLseItem& it) {
   it.g = (int)(item % p.Hkv);
   long long r = p.n_blocks - 1 - item / p.Hkv;
+  it.blk = r;
   for (int b = 0; b < p.batch; ++b) {
     const int Lq = p.cu_q[b + 1] - p.cu_q[b];
     const long long nb = (Lq + 15) / 16;
@@ -60,11 +78,47 @@ __device__ __forceinline__ bool kl_lse_item(long long item, const KlLseParams& p
       it.kbase = p.cu_k[b];
       const int vis_last = min(max(it.i0 + it.ntok - 1 + it.Lk - it.Lq + 1, 0), it.Lk);
       it.ntiles = (vis_last + 127) / 128;
+      if (p.ukeys) {
+        if (!p.blk_use[it.blk]) return false;
+        it.ntiles = (__ldg(p.ucount + it.blk) + 127) / 128;
+        return true;
+      }
       return it.ntiles > 0 || p.mask != nullptr;
     }
     r -= nb;
   }
   return false;
+}
+
+// Union form: positions 4 lane .. 4 lane + 3 of a 128-position union chunk (sequence-local,
+// from `chunk_keys`) as rows (s * Hkv + g) of the [Tk * Hkv, 128] view of K or V.  Loaded
+// one chunk ahead of their use, so the load's latency overlaps the wait for a free stage.
+__device__ __forceinline__ int4 union_rows(const int* chunk_keys, int kbase, int Hkv, int g, int lane) {
+  const int4 s = __ldg(reinterpret_cast<const int4*>(chunk_keys) + lane);
+  return make_int4((kbase + s.x) * Hkv + g, (kbase + s.y) * Hkv + g, (kbase + s.z) * Hkv + g, (kbase + s.w) * Hkv + g);
+}
+
+// The chunk's 128 rows gathered into one tile of two 64-column panels (128-byte swizzle, the
+// layout a tiled load gives): every lane of the calling warp gathers its four rows per
+// panel.  The tile's barrier must have been told its bytes before the call.
+__device__ __forceinline__ void union_gather_tile(uint8_t* dst, int panel_bytes, const CUtensorMap* map,
+                                                  uint64_t* bar, int4 rows, int lane) {
+#pragma unroll
+  for (int pn = 0; pn < 2; ++pn)
+    tma_gather4(dst + pn * panel_bytes + lane * 512, map, bar, pn * 64, rows.x, rows.y, rows.z, rows.w);
+}
+
+// The selection words of row u of an item and the distance between its tiles' (or union
+// chunks') words: the union form's per-block words, else the full layout of `mask`, else
+// none.  Rows past the block's tokens read row 0's words (they are masked anyway).
+__device__ __forceinline__ const uint32_t* kl_mask_row(const KlLseParams& p, const KlLseItem& it, int u,
+                                                       long long& stride) {
+  if (p.ukeys) {
+    stride = 64;
+    return p.umask + (it.blk * (p.ucap / 128) * 16 + u) * 4;
+  }
+  stride = p.total_q * 4;
+  return p.mask ? p.mask + (it.t0 + u) * 4 : nullptr;
 }
 
 struct KlLseCfg {
@@ -142,27 +196,49 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
   const int G = p.Hq / p.Hkv;  // 8
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      long long m = 0, n = 0;  // items, key tiles
-      bool ok = true;
-      for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        KlLseItem it;
-        if (!kl_lse_item(item, p, it)) continue;
-        if (!(ok = mbar_wait(a_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 60))) break;
+    // ------------------------------------------------------------ TMA producer (lane 0 waits
+    // and loads; in the union form every lane gathers rows of each key chunk)
+    long long m = 0, n = 0;  // items, key tiles
+    bool ok = true;
+    for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      KlLseItem it;
+      if (!kl_lse_item(item, p, it)) continue;
+      if (lane == 0 && (ok = mbar_wait(a_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 60))) {
         mbar_arrive_expect_tx(a_full, C::TILE_BYTES);
         for (int pn = 0; pn < 2; ++pn)
           tma_load_3d(sA + pn * C::PANEL_BYTES, &tmap_q, a_full, pn * 64, it.g * G, (int)it.t0);
-        ++m;
-        for (int j = 0; j < it.ntiles; ++j, ++n) {
-          const int st = (int)(n % C::B_STAGES);
-          if (!(ok = mbar_wait(&b_empty[st], (uint32_t)((n / C::B_STAGES) & 1) ^ 1u, abort_flag, 61))) break;
+      }
+      if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+      ++m;
+      const int* ukeys = p.ukeys ? p.ukeys + it.blk * p.ucap : nullptr;
+      int4 rows_next = ukeys && it.ntiles > 0 ? union_rows(ukeys, it.kbase, p.Hkv, it.g, lane) : make_int4(0, 0, 0, 0);
+      for (int j = 0; j < it.ntiles; ++j) {
+        const int st = (int)(n % C::B_STAGES);
+        const int4 rows = rows_next;
+        if (ukeys && j + 1 < it.ntiles) rows_next = union_rows(ukeys + (j + 1) * 128, it.kbase, p.Hkv, it.g, lane);
+        if (lane == 0 && (ok = mbar_wait(&b_empty[st], (uint32_t)((n / C::B_STAGES) & 1) ^ 1u, abort_flag, 61)))
           mbar_arrive_expect_tx(&b_full[st], C::TILE_BYTES);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+        if (ukeys)
+          union_gather_tile(sB + st * C::TILE_BYTES, C::PANEL_BYTES, &tmap_k, &b_full[st], rows, lane);
+        else if (lane == 0)
           for (int pn = 0; pn < 2; ++pn)
             tma_load_3d(sB + st * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &b_full[st], pn * 64, it.g,
                         it.kbase + j * 128);
-        }
+        ++n;
       }
+    }
+    if (!ok && lane == 0) {
+      // let the copies issued so far land before the CTA exits (bounded)
+      uint64_t t0 = globaltimer_ns();
+      for (long long q = max(0LL, n - C::B_STAGES); q < n; ++q)
+        while (!mbar_try_wait(smem_u32(&b_full[q % C::B_STAGES]), (uint32_t)((q / C::B_STAGES) & 1)) &&
+               globaltimer_ns() - t0 < 100000000ull) {
+        }
+      t0 = globaltimer_ns();
+      if (m > 0)
+        while (!mbar_try_wait(smem_u32(a_full), (uint32_t)((m - 1) & 1)) && globaltimer_ns() - t0 < 100000000ull) {
+        }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -213,17 +289,21 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
       if (!kl_lse_item(item, p, it)) continue;
       const int u = r / 8;
       const bool valid = u < it.ntok;
-      const int vis = valid ? causal_vis(it.i0 + u, it.Lq, it.Lk) : 0;
+      // (union chunks hold only positions that the rows selecting them can see)
+      const int vis = valid ? (p.ukeys ? INT_MAX : causal_vis(it.i0 + u, it.Lq, it.Lk)) : 0;
       // running max of the raw logits and sum of 2^(scale (x - max)) (scale > 0)
       float mx = -INFINITY, l = 0.f;
-      const uint32_t* mrow = p.mask ? p.mask + (it.t0 + (valid ? u : 0)) * 4 + 2 * half : nullptr;
+      long long mstride;
+      const uint32_t* mrow = kl_mask_row(p, it, valid ? u : 0, mstride);
+      if (mrow) mrow += 2 * half;
       for (int j = 0; j < it.ntiles; ++j, ++n) {
+        const int tile = j;
         const int ab = (int)(n & 1);
         // selection words of this row for the half's 64 keys (all set without a selection)
         uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
         if (mrow) {
-          w0 = mrow[(long long)j * p.total_q * 4];
-          w1 = mrow[(long long)j * p.total_q * 4 + 1];
+          w0 = mrow[(long long)tile * mstride];
+          w1 = mrow[(long long)tile * mstride + 1];
         }
         if (!(ok = mbar_wait(&acc_full[ab], (uint32_t)((n >> 1) & 1), abort_flag, 65))) break;
         tc_fence_after();
@@ -233,7 +313,7 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        const int nvis = vis - (j * 128 + half * 64);  // keys of this half the row sees
+        const int nvis = vis == INT_MAX ? 64 : vis - (tile * 128 + half * 64);  // keys of this half the row sees
         if (nvis < 64) {
 #pragma unroll
           for (int q = 0; q < 64; ++q)
@@ -646,7 +726,8 @@ namespace dsa_host {
 // lse_out = base-2 LSE times out_scale; with `mask`, over the selected keys only.
 int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
-                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out) {
+                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out,
+                     const KlUnion* un) {
   using C = dsa::KlLseCfg;
   static DeviceFlag attr_done;
   if (!attr_done) {
@@ -663,7 +744,9 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
     const uint32_t box[3] = {64, 8, 16};
     if (const int st = make_tmap_bf16_3d(&tq, Q, dims, strides, box); st != DSA_OK) return st;
   }
-  {
+  if (un) {
+    if (const int st = make_tmap_rows_gather(&tk, K, Tk * Hkv); st != DSA_OK) return st;
+  } else {
     const uint64_t dims[3] = {128, (uint64_t)Hkv, (uint64_t)Tk};
     const uint64_t strides[2] = {256, (uint64_t)Hkv * 256};
     const uint32_t box[3] = {64, 1, 128};
@@ -681,6 +764,13 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
   p.mask = mask;
   p.total_q = T;
   p.max_out = max_out;
+  if (un) {
+    p.ukeys = un->ukeys;
+    p.ucount = un->ucount;
+    p.umask = un->umask;
+    p.blk_use = un->blk_use;
+    p.ucap = un->ucap;
+  }
   // an upper bound on the 16-row blocks (each sequence rounds up once)
   p.n_blocks = (T + 15) / 16 + batch;
   p.n_items = p.n_blocks * Hkv;

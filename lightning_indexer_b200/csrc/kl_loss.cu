@@ -624,7 +624,8 @@ int indexer_launch(const void* q_idx, const void* k_idx, const void* w, const in
 int f32_to_bf16_launch(const float* src, void* dst, long long n, cudaStream_t stream);
 int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
-                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out);
+                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out,
+                     const KlUnion* un);
 int kl_target_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                         long long Tk, int Hq, int Hkv, long long r0, long long r1, float scale_log2,
                         const float* lse_att, const float* lseI, float* scores, long long ld, float inv_T,
@@ -770,7 +771,7 @@ int indexer_kl_loss_launch(const void* Q, const void* K, const void* q_idx, cons
   //    for d = 128 and 8 query heads per KV head)
   if (d == 128 && Hq == 8 * Hkv) {
     const int st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, T, Tk, Hq, Hkv, max_seqlen_q, scale_log2, W.lse_att, s, mask,
-                                    1.f, nullptr);
+                                    1.f, nullptr, nullptr);
     if (st != DSA_OK) return st;
   } else {
     const long long tasks = T * Hkv;

@@ -49,6 +49,7 @@ struct SAParams {
   float* lse;   // [rows, Hq] or null
   float* part_o;  // [rows, nsplit, Hq, D] (nsplit > 1)
   float* part_ml; // [rows, nsplit, Hq, 4]: max (log2 domain), exact sum, sum of bf16-rounded weights
+  const uint8_t* skip_rows;  // optional [rows]: rows another kernel computes (left untouched)
 };
 
 // 4-warp CTAs with 2 stages per warp: 3 CTAs, 12 warps per SM.  (Decode launches only a
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
   const long long rem = task - (long long)g * per_head;
   const long long row = rem / p.nsplit;
   const int split = (int)(rem % p.nsplit);
+  if (p.skip_rows && p.skip_rows[row]) return;  // warp-uniform
   int kbase = 0, vis = 0;
   if (p.cu_q) {
     int lo = 0, hi = p.batch;
@@ -408,7 +410,7 @@ static int sa_launch_common(dsa::SAParams& p, int d, cudaStream_t stream) {
 
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
                                const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
-                               float scale, void* O, float* lse, cudaStream_t stream) {
+                               float scale, void* O, float* lse, cudaStream_t stream, const uint8_t* skip_rows) {
   dsa::SAParams p{};
   p.Q = static_cast<const uint16_t*>(Q);
   p.K = static_cast<const uint16_t*>(K);
@@ -426,6 +428,7 @@ int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, cons
   p.scale_log2 = scale * 1.4426950408889634f;
   p.O = static_cast<uint16_t*>(O);
   p.lse = lse;
+  p.skip_rows = skip_rows;
   return sa_launch_common(p, d, stream);
 }
 

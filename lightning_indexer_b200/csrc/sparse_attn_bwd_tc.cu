@@ -503,9 +503,9 @@ __global__ void sa_bwd_mask_kernel(const int* __restrict__ indices, const int* _
                                    int tiles) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * k) return;
+  const long long row = i / k;
   const int s = indices[i];
   if (s < 0 || s >= tiles * 128) return;
-  const long long row = i / k;
   int lo = 0, hi = batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) / 2;

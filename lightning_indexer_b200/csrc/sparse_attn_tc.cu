@@ -12,11 +12,18 @@
 // first is the dense-LSE kernel of kl_dense_tc.cu run with the selection mask (it writes
 // lse and the row maxima m); the second, below, recomputes S = Q_blk . K_tile^T (M = 16
 // tokens x 8 heads on TMEM lanes, N = 128 keys), turns it into P = sel 2^(S scale log2(e) - m)
-// (bf16 in [0, 1], the largest exactly 1; written to shared memory in the 128-byte swizzled
-// K-major layout), accumulates O += P . V_tile in TMEM with V read MN-major, and divides by
-// the row sum 2^(lse - m) in fp32 at the end.  Knowing m first removes the running rescale
-// of O.  Warps: 0 TMA, 1 MMA issuer and TMEM owner, 2-9 epilogue (two per TMEM lane
-// quarter, one per 64-key half of each tile).
+// (in [0, 1], the largest exactly 1; written to shared memory as two bf16 parts, hi + lo, in
+// the 128-byte swizzled K-major layout), accumulates O += P_hi . V_tile + P_lo . V_tile in
+// TMEM with V read MN-major, and divides by the row sum 2^(lse - m) in fp32 at the end.
+// Knowing m first removes the running rescale of O.  Warps: 0 TMA, 1 MMA issuer and TMEM
+// owner, 2-9 epilogue (two per TMEM lane quarter, one per 64-key half of each tile).
+//
+// Adjacent-query reuse (report summary section 8: neighbouring queries select largely the
+// same positions; the pages deduplicate the sets of adjacent queries and mask inside the
+// attention kernel with a mask laid out like the MMA's accumulator): the same two passes in
+// their union form, where a 16-row block visits the 128-position chunks of the sorted union
+// of its rows' selected sets, gathered row by row with TMA (each key loaded once for the 16
+// rows x 8 heads of the block), and the per-(row, union slot) selection bits mask S.
 #include <algorithm>
 
 #include "common.cuh"
@@ -24,9 +31,7 @@
 namespace dsa {
 
 struct SAFwdTcParams {
-  KlLseParams items;      // work items (shared with the LSE pass)
-  const uint32_t* mask;   // selection words, layout of KlLseParams::mask
-  long long total_q;
+  KlLseParams items;      // work items and selection words (shared with the LSE pass)
   const float* lse;       // [T, Hq] natural log (first pass)
   const float* mx;        // [T, Hq] row maxima of the scaled logits, base 2 (first pass)
   uint16_t* O;            // [T, Hq, 128] bf16
@@ -35,14 +40,13 @@ struct SAFwdTcParams {
 struct SAFwdTcCfg {
   static constexpr int TILE_BYTES = 128 * 128 * 2;
   static constexpr int PANEL_BYTES = 128 * 128;
-  // K tiles are free after their S MMA, V tiles only after P.V: separate rings, the K ring
-  // one deeper so the next tiles' keys load while the epilogue works
-  static constexpr int K_STAGES = 3, V_STAGES = 2;
+  // K tiles are free after their S MMA, V tiles only after P.V: separate rings
+  static constexpr int K_STAGES = 2, V_STAGES = 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE_BYTES;
   static constexpr int OFF_V = OFF_K + K_STAGES * TILE_BYTES;
-  static constexpr int OFF_P = OFF_V + V_STAGES * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_P + TILE_BYTES;
+  static constexpr int OFF_P = OFF_V + V_STAGES * TILE_BYTES;  // P as bf16 hi, then bf16 lo parts
+  static constexpr int OFF_BAR = OFF_P + 2 * TILE_BYTES;
   // q_full, q_empty, k_full[K], k_empty[K], v_full[V], v_empty[V], s_full[2], s_empty[2],
   // p_full, p_empty, o_full, o_empty, done
   static constexpr int NUM_BARS = 2 + 2 * K_STAGES + 2 * V_STAGES + 4 + 2 + 2 + 1;
@@ -121,35 +125,50 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
   const int G = ip.Hq / ip.Hkv;  // 8
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      long long m = 0, n = 0;    // items with key tiles, key tiles
-      long long nk = 0, nv = 0;  // K and V tile copies issued (they differ after an abort)
-      bool ok = true;
-      for (long long item = blockIdx.x; item < ip.n_items && ok; item += gridDim.x) {
-        KlLseItem it;
-        if (!kl_lse_item(item, ip, it) || it.ntiles == 0) continue;
-        if (!(ok = mbar_wait(q_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 120))) break;
+    // ------------------------------------------------------------ TMA producer (lane 0 waits
+    // and loads; in the union form every lane gathers rows of each key chunk)
+    long long m = 0, n = 0;    // items with key tiles, key tiles
+    long long nk = 0, nv = 0;  // K and V tile copies issued (they differ after an abort)
+    bool ok = true;
+    for (long long item = blockIdx.x; item < ip.n_items && ok; item += gridDim.x) {
+      KlLseItem it;
+      if (!kl_lse_item(item, ip, it) || it.ntiles == 0) continue;
+      if (lane == 0 && (ok = mbar_wait(q_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 120))) {
         mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
         for (int pn = 0; pn < 2; ++pn)
           tma_load_3d(smem + C::OFF_Q + pn * C::PANEL_BYTES, &tmap_q, q_full, pn * 64, it.g * G, (int)it.t0);
-        ++m;
-        for (int j = 0; j < it.ntiles; ++j, ++n) {
-          const int ks = (int)(n % C::K_STAGES), vs = (int)(n % C::V_STAGES);
-          if (!(ok = mbar_wait(&k_empty[ks], (uint32_t)((n / C::K_STAGES) & 1) ^ 1u, abort_flag, 121))) break;
-          mbar_arrive_expect_tx(&k_full[ks], C::TILE_BYTES);
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_3d(smem + C::OFF_K + ks * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &k_full[ks], pn * 64,
-                        it.g, it.kbase + j * 128);
-          ++nk;
-          if (!(ok = mbar_wait(&v_empty[vs], (uint32_t)((n / C::V_STAGES) & 1) ^ 1u, abort_flag, 130))) break;
-          mbar_arrive_expect_tx(&v_full[vs], C::TILE_BYTES);
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_3d(smem + C::OFF_V + vs * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_v, &v_full[vs], pn * 64,
-                        it.g, it.kbase + j * 128);
-          ++nv;
-        }
       }
+      if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+      ++m;
+      const int* ukeys = ip.ukeys ? ip.ukeys + it.blk * ip.ucap : nullptr;
+      int4 rows_next = ukeys ? union_rows(ukeys, it.kbase, ip.Hkv, it.g, lane) : make_int4(0, 0, 0, 0);
+      for (int j = 0; j < it.ntiles; ++j, ++n) {
+        const int ks = (int)(n % C::K_STAGES), vs = (int)(n % C::V_STAGES);
+        const int4 rows = rows_next;  // the chunk's K and V rows (the same positions)
+        if (ukeys && j + 1 < it.ntiles) rows_next = union_rows(ukeys + (j + 1) * 128, it.kbase, ip.Hkv, it.g, lane);
+        uint8_t* kdst = smem + C::OFF_K + ks * C::TILE_BYTES;
+        uint8_t* vdst = smem + C::OFF_V + vs * C::TILE_BYTES;
+        if (lane == 0 && (ok = mbar_wait(&k_empty[ks], (uint32_t)((n / C::K_STAGES) & 1) ^ 1u, abort_flag, 121)))
+          mbar_arrive_expect_tx(&k_full[ks], C::TILE_BYTES);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+        if (ukeys)
+          union_gather_tile(kdst, C::PANEL_BYTES, &tmap_k, &k_full[ks], rows, lane);
+        else if (lane == 0)
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(kdst + pn * C::PANEL_BYTES, &tmap_k, &k_full[ks], pn * 64, it.g, it.kbase + j * 128);
+        ++nk;
+        if (lane == 0 && (ok = mbar_wait(&v_empty[vs], (uint32_t)((n / C::V_STAGES) & 1) ^ 1u, abort_flag, 130)))
+          mbar_arrive_expect_tx(&v_full[vs], C::TILE_BYTES);
+        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+        if (ukeys)
+          union_gather_tile(vdst, C::PANEL_BYTES, &tmap_v, &v_full[vs], rows, lane);
+        else if (lane == 0)
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(vdst + pn * C::PANEL_BYTES, &tmap_v, &v_full[vs], pn * 64, it.g, it.kbase + j * 128);
+        ++nv;
+      }
+    }
+    if (lane == 0) {
       if (!ok) {
         // let the copies this thread issued land before the CTA exits (bounded; each ring
         // waits only for copies it really issued, each with its own time budget)
@@ -211,10 +230,14 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
           tc_fence_after();
           const uint32_t v_base = smem_u32(smem + C::OFF_V + vs * C::TILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step
-            umma_bf16(tmem_base + 256,
-                      smem_desc_kmajor(p_base + (kk / 4) * C::PANEL_BYTES + (kk % 4) * 32, 128),
-                      smem_desc_mn_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES), C::IDESC_O, (j | kk) != 0);
+          for (int part = 0; part < 2; ++part)  // P = P_hi + P_lo, both bf16
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // K = 128 keys, 16 per step
+              umma_bf16(tmem_base + 256,
+                        smem_desc_kmajor(p_base + part * C::TILE_BYTES + (kk / 4) * C::PANEL_BYTES + (kk % 4) * 32,
+                                         128),
+                        smem_desc_mn_sw128(v_base + kk * 16 * 128, C::PANEL_BYTES), C::IDESC_O,
+                        (j | part | kk) != 0);
           umma_commit(&v_empty[vs]);
           umma_commit(p_empty);
         }
@@ -254,13 +277,14 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
       const float lse2 = valid ? p.lse[row] * 1.4426950408889634f : -INFINITY;
       const float nl = valid ? -p.mx[row] : 0.f;
       const float o_scale = lse2 > -INFINITY ? ex2_ftz(-nl - lse2) : 0.f;
-      const uint32_t* mrow = p.mask + (it.t0 + (valid ? u : 0)) * 4 + 2 * half;
+      long long mstride;
+      const uint32_t* mrow = kl_mask_row(ip, it, valid ? u : 0, mstride) + 2 * half;
       for (int j = 0; j < it.ntiles; ++j, ++n) {
         const int sb = (int)(n & 1);
         uint32_t w0 = 0u, w1 = 0u;
         if (valid) {
-          w0 = mrow[(long long)j * p.total_q * 4];
-          w1 = mrow[(long long)j * p.total_q * 4 + 1];
+          w0 = mrow[(long long)j * mstride];
+          w1 = mrow[(long long)j * mstride + 1];
         }
         if (!(ok = mbar_wait(&s_full[sb], (uint32_t)((n >> 1) & 1), abort_flag, 127))) break;
         tc_fence_after();
@@ -270,21 +294,31 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[sb]);
-        uint32_t pk[32];
+        // P in two bf16 parts, hi = bf16(P) and lo = bf16(P - hi): their sum carries P to about
+        // 2^-17 relative, so the weights entering P.V are not the 2^-9 relative rounding of a
+        // single bf16 (which, on rows with few keys and values of magnitude 2-4, would add
+        // up to the output's own rounding and exceed 1e-2)
+        uint32_t pk[32], pl[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const uint32_t w = c < 32 ? w0 : w1;
           const float p0 = ((w >> (c & 31)) & 1u) ? ex2_ftz(fmaf(x[c], ip.scale_log2, nl)) : 0.f;
           const float p1 = ((w >> ((c + 1) & 31)) & 1u) ? ex2_ftz(fmaf(x[c + 1], ip.scale_log2, nl)) : 0.f;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          pk[c / 2] = *reinterpret_cast<uint32_t*>(&b2);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(p0 - __low2float(hi), p1 - __high2float(hi));
+          pk[c / 2] = *reinterpret_cast<const uint32_t*>(&hi);
+          pl[c / 2] = *reinterpret_cast<const uint32_t*>(&lo);
         }
         if (!(ok = mbar_wait(p_empty, (uint32_t)(n & 1) ^ 1u, abort_flag, 128))) break;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)  // 16-byte chunk q of this row's panel: keys 8q .. 8q+7
+        for (int q = 0; q < 8; ++q) {  // 16-byte chunk q of this row's panel: keys 8q .. 8q+7
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + ((q ^ (r & 7)) * 16)),
                        "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
                        : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + C::TILE_BYTES + ((q ^ (r & 7)) * 16)),
+                       "r"(pl[4 * q]), "r"(pl[4 * q + 1]), "r"(pl[4 * q + 2]), "r"(pl[4 * q + 3])
+                       : "memory");
+        }
         fence_proxy_async_shared();  // the tensor core reads P through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
@@ -323,13 +357,110 @@ __global__ void __launch_bounds__(SAFwdTcCfg::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
+// ---------------------------------------------------------------------------- union plans
+// Per block of 16 consecutive query rows (the work items of the two passes): the sorted union
+// of the rows' selected positions, through a bitmap of the sequence's positions.  A block
+// whose union has at most `ucap` positions takes the union form; the others' rows go to the
+// gather kernel.
+struct SAUnionPlanParams {
+  const int* indices;  // [T, k]
+  int k;
+  const int* cu_q;
+  const int* cu_k;
+  int batch;
+  int ucap;            // union positions per block, a multiple of 128
+  int* ukeys;          // [n_blocks, ucap]: ascending positions, the last chunk padded with 0
+  int* ucount;         // [n_blocks]: union size (also where it exceeds ucap)
+  uint32_t* umask;     // [n_blocks, ucap / 128, 16, 4]: bit slot % 32 of word slot / 32 % 4
+  uint8_t* blk_use;    // [n_blocks]
+  uint8_t* row_tc;     // [T]: 1 for rows of union-form blocks
+};
+
+constexpr int SA_PLAN_T = 256;
+
+// Dynamic shared memory: the position bitmap and its word prefix counts (words each), then
+// the block's selection words (ucap / 128 * 64).
+__global__ void __launch_bounds__(SA_PLAN_T) sa_union_plan_kernel(const SAUnionPlanParams p, int words) {
+  extern __shared__ __align__(16) uint32_t plan_smem[];
+  uint32_t* bits = plan_smem;
+  uint32_t* pre = plan_smem + words;
+  uint32_t* msk = plan_smem + 2 * words;
+  __shared__ uint32_t warp_sums[32];
+  __shared__ uint32_t total;
+  long long r = blockIdx.x;
+  const long long blk = r;
+  int b = 0;
+  for (; b < p.batch; ++b) {
+    const long long nb = (p.cu_q[b + 1] - p.cu_q[b] + 15) / 16;
+    if (r < nb) break;
+    r -= nb;
+  }
+  if (b == p.batch) return;  // past the last block (the bound rounds up per sequence)
+  const int Lq = p.cu_q[b + 1] - p.cu_q[b], Lk = p.cu_k[b + 1] - p.cu_k[b];
+  const int i0 = (int)(r * 16), ntok = min(16, Lq - i0);
+  const long long t0 = p.cu_q[b] + i0;
+  const int W = (Lk + 31) / 32;
+  const int mwords = p.ucap / 128 * 64;
+  for (int w = threadIdx.x; w < W; w += SA_PLAN_T) bits[w] = 0u;
+  for (int w = threadIdx.x; w < mwords; w += SA_PLAN_T) msk[w] = 0u;
+  __syncthreads();
+  for (int e = threadIdx.x; e < ntok * p.k; e += SA_PLAN_T) {
+    const int u = e / p.k;
+    const int s = __ldg(p.indices + (t0 + u) * p.k + (e % p.k));
+    if (s >= 0 && s < causal_vis(i0 + u, Lq, Lk)) atomicOr(&bits[s >> 5], 1u << (s & 31));
+  }
+  __syncthreads();
+  // a contiguous run of words per thread; the block scan numbers the union in position order
+  const int wpt = (W + SA_PLAN_T - 1) / SA_PLAN_T;
+  const int w0 = min(W, (int)threadIdx.x * wpt), w1 = min(W, w0 + wpt);
+  uint32_t mine = 0;
+  for (int w = w0; w < w1; ++w) mine += __popc(bits[w]);
+  uint32_t run = block_excl_scan<SA_PLAN_T>(mine, warp_sums, &total);
+  for (int w = w0; w < w1; ++w) {
+    pre[w] = run;
+    run += __popc(bits[w]);
+  }
+  const uint32_t u_n = total;
+  const bool use = u_n <= (uint32_t)p.ucap;
+  if (threadIdx.x == 0) {
+    p.ucount[blk] = (int)u_n;
+    p.blk_use[blk] = use ? 1 : 0;
+  }
+  if (threadIdx.x < ntok) p.row_tc[t0 + threadIdx.x] = use ? 1 : 0;
+  if (!use) return;  // block-uniform
+  int* keys = p.ukeys + blk * p.ucap;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t x = bits[w];
+    uint32_t o = pre[w];
+    while (x) {
+      keys[o++] = w * 32 + (__ffs(x) - 1);
+      x &= x - 1u;
+    }
+  }
+  const uint32_t u_pad = (u_n + 127) / 128 * 128;
+  for (uint32_t j = u_n + threadIdx.x; j < u_pad; j += SA_PLAN_T) keys[j] = 0;
+  __syncthreads();  // pre[] complete for every word
+  for (int e = threadIdx.x; e < ntok * p.k; e += SA_PLAN_T) {
+    const int u = e / p.k;
+    const int s = __ldg(p.indices + (t0 + u) * p.k + (e % p.k));
+    if (s >= 0 && s < causal_vis(i0 + u, Lq, Lk)) {
+      const uint32_t slot = pre[s >> 5] + __popc(bits[s >> 5] & ((1u << (s & 31)) - 1u));
+      atomicOr(&msk[((slot >> 7) * 16 + u) * 4 + ((slot >> 5) & 3)], 1u << (slot & 31));
+    }
+  }
+  __syncthreads();
+  uint32_t* out = p.umask + blk * (long long)mwords;
+  for (uint32_t w = threadIdx.x; w < u_pad / 128 * 64; w += SA_PLAN_T) out[w] = msk[w];
+}
+
 }  // namespace dsa
 
 namespace dsa_host {
 
 int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* cu_k, int batch, long long T,
                      long long Tk, int Hq, int Hkv, int max_seqlen_q, float scale_log2, float* lse_out,
-                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out);
+                     cudaStream_t s, const uint32_t* mask, float out_scale, float* max_out,
+                     const KlUnion* un);
 
 bool sa_fwd_tc_eligible(int Hq, int Hkv, int d, int k, int max_seqlen_k) {
   return d == 128 && Hq == 8 * Hkv && max_seqlen_k > 0 && 8LL * k >= (long long)max_seqlen_k;
@@ -368,7 +499,7 @@ int sa_fwd_tc_launch(const void* Q, const void* K, const void* V, const int* ind
   if (st != DSA_OK) return st;
   const float scale_log2 = scale * 1.4426950408889634f;
   st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, total_q, total_k, Hq, Hkv, 0, scale_log2, lse, s, mask,
-                        0.69314718055994531f, mx);
+                        0.69314718055994531f, mx, nullptr);
   if (st != DSA_OK) return st;
   CUtensorMap tq, tk, tv;
   {
@@ -398,14 +529,159 @@ int sa_fwd_tc_launch(const void* Q, const void* K, const void* V, const int* ind
   p.items.mask = mask;
   p.items.total_q = total_q;
   p.items.max_out = nullptr;
-  p.mask = mask;
-  p.total_q = total_q;
   p.lse = lse;
   p.mx = mx;
   p.O = static_cast<uint16_t*>(O);
   const long long grid = std::min<long long>(p.items.n_items, (long long)sm_count());
   dsa::sa_fwd_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, tv, p);
   return last_launch_status();
+}
+
+// ---------------------------------------------------------------------------- union path
+// Scratch of sa_block_reuse_launch: the row maxima, the per-block unions, their sizes,
+// selection words and flags, and the per-row flags.
+struct SAUnionWs {
+  float* mx;
+  int* ukeys;
+  int* ucount;
+  uint32_t* umask;
+  uint8_t* blk_use;
+  uint8_t* row_tc;
+  int ucap;
+  size_t total;
+};
+
+// Union positions per block: at most `max_chunks` chunks of 128, and no more than the
+// longest sequence holds.
+static int sa_union_cap(int max_seqlen_k, int max_chunks) {
+  return std::max(1, std::min(max_chunks, (max_seqlen_k + 127) / 128)) * 128;
+}
+
+static SAUnionWs sa_union_layout(void* base, long long total_q, int Hq, int batch, int max_seqlen_k, int max_chunks) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  SAUnionWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  const long long n_blocks = (total_q + 15) / 16 + batch;
+  w.ucap = sa_union_cap(max_seqlen_k, max_chunks);
+  w.mx = reinterpret_cast<float*>(p + off);
+  off += up((size_t)total_q * Hq * 4);
+  w.ukeys = reinterpret_cast<int*>(p + off);
+  off += up((size_t)n_blocks * w.ucap * 4);
+  w.ucount = reinterpret_cast<int*>(p + off);
+  off += up((size_t)n_blocks * 4);
+  w.umask = reinterpret_cast<uint32_t*>(p + off);
+  off += up((size_t)n_blocks * (w.ucap / 128) * 256);
+  w.blk_use = p + off;
+  off += up((size_t)n_blocks);
+  w.row_tc = p + off;
+  off += up((size_t)total_q);
+  w.total = off;
+  return w;
+}
+
+size_t sa_block_reuse_scratch_bytes(long long total_q, int Hq, int batch, int max_seqlen_k, int max_chunks) {
+  return sa_union_layout(nullptr, total_q, Hq, batch, max_seqlen_k, max_chunks).total;
+}
+
+// The union plan holds a bitmap of a sequence's positions and its prefix counts in shared
+// memory: 2 x 32 KiB at 262144 positions.
+bool sa_block_reuse_eligible(int Hq, int Hkv, int d, int max_seqlen_k) {
+  return d == 128 && Hq == 8 * Hkv && max_seqlen_k > 0 && max_seqlen_k <= 262144;
+}
+
+int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                               const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
+                               float scale, void* O, float* lse, cudaStream_t stream, const uint8_t* skip_rows);
+
+// Sparse attention of the selected sets with adjacent-query reuse: the union plan per 16-row
+// block, the two masked tensor-core passes in their union form over the blocks whose union
+// has at most max_chunks x 128 positions, and the gather kernel for the other rows.  Same O
+// and lse as the gather kernel (within the same rounding bound).
+int sa_block_reuse_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                          const int* cu_k, int batch, long long total_q, long long total_k, int Hq, int Hkv, int k,
+                          int max_seqlen_k, int max_chunks, float scale, void* O, float* lse, void* ws,
+                          int* ucount_out, cudaStream_t s) {
+  using C = dsa::SAFwdTcCfg;
+  const SAUnionWs W = sa_union_layout(ws, total_q, Hq, batch, max_seqlen_k, max_chunks);
+  const int words = (max_seqlen_k + 31) / 32;
+  const int plan_smem = (2 * words + W.ucap / 128 * 64) * 4;
+  static DeviceFlag attr_done;
+  if (!attr_done) {
+    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sa_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    C::SMEM_BYTES);
+        e_ != cudaSuccess)
+      return cuda_fail(e_);
+    if (const cudaError_t e_ = cudaFuncSetAttribute(dsa::sa_union_plan_kernel,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        e_ != cudaSuccess)
+      return cuda_fail(e_);
+    attr_done = true;
+  }
+  if (total_q <= 0) return DSA_OK;
+  if (plan_smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
+  int* ucount = ucount_out ? ucount_out : W.ucount;
+  dsa::SAUnionPlanParams pp;
+  pp.indices = indices;
+  pp.k = k;
+  pp.cu_q = cu_q;
+  pp.cu_k = cu_k;
+  pp.batch = batch;
+  pp.ucap = W.ucap;
+  pp.ukeys = W.ukeys;
+  pp.ucount = ucount;
+  pp.umask = W.umask;
+  pp.blk_use = W.blk_use;
+  pp.row_tc = W.row_tc;
+  const long long n_blocks = (total_q + 15) / 16 + batch;
+  // blocks past the last sequence's end keep these zero: no union-form item, no count
+  if (const cudaError_t e_ = cudaMemsetAsync(W.blk_use, 0, (size_t)n_blocks, s); e_ != cudaSuccess) return cuda_fail(e_);
+  if (const cudaError_t e_ = cudaMemsetAsync(ucount, 0, (size_t)n_blocks * 4, s); e_ != cudaSuccess)
+    return cuda_fail(e_);
+  dsa::sa_union_plan_kernel<<<(unsigned)n_blocks, dsa::SA_PLAN_T, plan_smem, s>>>(pp, words);
+  if (const int st = last_launch_status(); st != DSA_OK) return st;
+  KlUnion un{W.ukeys, ucount, W.umask, W.blk_use, W.ucap};
+  const float scale_log2 = scale * 1.4426950408889634f;
+  int st = kl_lse_tc_launch(Q, K, cu_q, cu_k, batch, total_q, total_k, Hq, Hkv, 0, scale_log2, lse, s, nullptr,
+                            0.69314718055994531f, W.mx, &un);
+  if (st != DSA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t dims[3] = {128, (uint64_t)Hq, (uint64_t)total_q};
+    const uint64_t strides[2] = {256, (uint64_t)Hq * 256};
+    const uint32_t box[3] = {64, 8, 16};
+    if (const int e = make_tmap_bf16_3d(&tq, Q, dims, strides, box); e != DSA_OK) return e;
+  }
+  if (const int e = make_tmap_rows_gather(&tk, K, total_k * Hkv); e != DSA_OK) return e;
+  if (const int e = make_tmap_rows_gather(&tv, V, total_k * Hkv); e != DSA_OK) return e;
+  dsa::SAFwdTcParams p;
+  p.items.cu_q = cu_q;
+  p.items.cu_k = cu_k;
+  p.items.batch = batch;
+  p.items.Hq = Hq;
+  p.items.Hkv = Hkv;
+  p.items.scale_log2 = scale_log2;
+  p.items.lse_out = lse;
+  p.items.out_scale = 1.f;
+  p.items.n_blocks = n_blocks;
+  p.items.n_items = n_blocks * Hkv;
+  p.items.mask = nullptr;
+  p.items.total_q = total_q;
+  p.items.max_out = nullptr;
+  p.items.ukeys = W.ukeys;
+  p.items.ucount = ucount;
+  p.items.umask = W.umask;
+  p.items.blk_use = W.blk_use;
+  p.items.ucap = W.ucap;
+  p.lse = lse;
+  p.mx = W.mx;
+  p.O = static_cast<uint16_t*>(O);
+  const long long grid = std::min<long long>(p.items.n_items, (long long)sm_count());
+  dsa::sa_fwd_tc_kernel<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, tv, p);
+  if (last_launch_status() != DSA_OK) return DSA_ERR_CUDA;
+  // the rows of the other blocks on the gather kernel
+  return sparse_attn_prefill_launch(Q, K, V, indices, cu_q, cu_k, batch, total_q, Hq, Hkv, 128, k, scale, O, lse, s,
+                                    W.row_tc);
 }
 
 }  // namespace dsa_host

@@ -64,6 +64,21 @@ def test_host_side_argument_errors():
                                        None, None) == -2
     assert lib.dsa_sparse_attn_prefill(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 128, 64, -1.0, fake,
                                        None, None) == -1
+    # attention with adjacent-query reuse: shape and scale checks as (3), then the workspace
+    wsz = lib.dsa_sparse_attn_prefill_reuse_workspace_size(131072, 32, 1, 131072)
+    assert 620e6 < wsz < 680e6  # per 16-row block: 12288 union positions, their selection words, lse and maxima
+    assert lib.dsa_sparse_attn_prefill_reuse_workspace_size(-1, 32, 1, 4096) == 0
+    assert lib.dsa_sparse_attn_prefill_reuse(fake, fake, fake, fake, fake, fake, 1, 8, 8, 8, 32, 4, 96, 64, 0.1,
+                                             fake, None, None, fake, wsz, None) == -2
+    assert lib.dsa_sparse_attn_prefill_reuse(fake, fake, fake, fake, fake, fake, 1, 8, 8, 8, 32, 4, 128, 64, 0.0,
+                                             fake, None, None, fake, wsz, None) == -1
+    small = lib.dsa_sparse_attn_prefill_reuse_workspace_size(8, 32, 1, 8)
+    assert lib.dsa_sparse_attn_prefill_reuse(fake, fake, fake, fake, fake, fake, 1, 8, 8, 8, 32, 4, 128, 64, 0.1,
+                                             fake, None, None, fake, small - 16, None) == -3
+    assert lib.dsa_sparse_attn_prefill_reuse(fake, fake, fake, fake, fake, fake, 1, 8, 8, 8, 32, 4, 128, 64, 0.1,
+                                             fake, None, None, None, small, None) == -3
+    assert lib.dsa_sparse_attn_prefill_reuse(fake, fake, fake, fake, fake, fake, 1, 0, 0, 8, 32, 4, 128, 64, 0.1,
+                                             fake, None, None, fake, wsz, None) == 0  # nothing to do
     # workspace too small
     need = lib.dsa_sparse_attn_decode_workspace_size(16, 32, 128, 2048)
     assert need > 0

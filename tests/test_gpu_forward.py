@@ -231,11 +231,68 @@ def test_sparse_attention_prefill_given_sets(Hq, Hkv, d):
         assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL, r
 
 
+def _reuse_sets(cu, k, seed):
+    """Selected sets with a known union structure, for the adjacent-query reuse path: in
+    every other 16-row block the rows draw from one pool of 1.5 k positions that all of the
+    block's rows can see (small union: the tensor-core form), in the others each row draws
+    from its whole visible range (a union that outgrows 12288 positions late in a long
+    sequence: the gather kernel).  A few -1 slots end each row, and a row that has room also
+    lists the position just past its causal limit, which every path must ignore."""
+    rng = np.random.default_rng(seed)
+    idx = np.full((int(cu[-1]), k), -1, np.int32)
+    for b in range(len(cu) - 1):
+        L = int(cu[b + 1] - cu[b])
+        for i0 in range(0, L, 16):
+            pool = rng.choice(i0 + 1, size=min(i0 + 1, 3 * k // 2), replace=False) if (i0 // 16) % 2 == 0 else None
+            for i in range(i0, min(L, i0 + 16)):
+                src = pool if pool is not None else np.arange(i + 1)
+                n = min(len(src), k - int(rng.integers(1, 8)))
+                row = idx[cu[b] + i]
+                row[:n] = np.sort(rng.choice(src, size=n, replace=False))
+                if i + 1 < L:
+                    row[n] = i + 1
+    return idx
+
+
+def test_sparse_attention_reuse_given_sets():
+    wl = gen.make_prefill([14000, 1000], 32, 4, 128, 4, 32, 2048, seed=33)
+    cu = wl.cu_seqlens_q.astype(np.int64)
+    idx = _reuse_sets(cu, 2048, seed=33)
+    t = to_device(wl)
+    idx_d = torch.from_numpy(idx).cuda()
+    nb = (wl.Tq + 15) // 16 + wl.B
+    bu = torch.full((nb,), -7, dtype=torch.int32, device="cuda")
+    O, lse = dsa.sparse_attn_prefill_reuse(t["Q"], t["K"], t["V"], idx_d, t["cu_q"], t["cu_k"], t["max_k"],
+                                           block_union=bu)
+    Og, lg = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx_d, t["cu_q"], t["cu_k"])
+    # per-block union sizes, exactly (entries past the last block are 0)
+    want = []
+    for b in range(wl.B):
+        L = int(cu[b + 1] - cu[b])
+        for i0 in range(0, L, 16):
+            rows = idx[cu[b] + i0:cu[b] + min(L, i0 + 16)]
+            vis = np.arange(i0, min(L, i0 + 16))[:, None] + 1
+            want.append(np.unique(rows[(rows >= 0) & (rows < vis)]).size)
+    got = bu.cpu().numpy()
+    assert np.array_equal(got[:len(want)], np.array(want)) and (got[len(want):] == 0).all()
+    assert (np.array(want) <= 12288).sum() > 100 and (np.array(want) > 12288).sum() > 10  # both paths ran
+    O, lse, Og, lg = O.float().cpu().numpy(), lse.cpu().numpy(), Og.float().cpu().numpy(), lg.cpu().numpy()
+    assert np.max(np.abs(O - Og)) <= 2 * ATTN_ATOL and np.max(np.abs(lse - lg)) <= 2 * LSE_ATOL
+    D = orc.Decoded(wl)
+    for r in orc.sample_rows(wl.Tq, seed=33, n_first=40, n_last=40, n_mid=120) + [14000 + 37, 14999]:
+        b, i, Lq, Lk = D.seq_of_row(r)
+        row = idx[r]
+        sel = row[(row >= 0) & (row <= i)] + int(D.cu_k[b])
+        Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
+        assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL, r
+        assert np.max(np.abs(lse[r] - lr)) <= LSE_ATOL, r
+
+
 def _fused_vs_separate(wl, k, chunk):
     """Selected sets by dsa_index_topk on its fused path and on the separate passes."""
     t = to_device(wl)
     args = (t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], k)
-    fused = dsa.index_topk(*args, chunk_rows=chunk, path=dsa.PATH_AUTO).cpu().numpy()
+    fused = dsa.index_topk(*args, chunk_rows=chunk, path=dsa.PATH_FUSED).cpu().numpy()
     separate = dsa.index_topk(*args, chunk_rows=chunk, path=dsa.PATH_SEPARATE).cpu().numpy()
     return fused, separate
 
@@ -260,7 +317,7 @@ def test_index_topk_fused_gaussian_matches_separate_and_oracle():
     # a row range (crossing the sequence boundary) gives the same rows
     t = to_device(wl)
     part = dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], 64,
-                          chunk_rows=700, row_begin=2500, row_end=3600).cpu().numpy()
+                          chunk_rows=700, row_begin=2500, row_end=3600, path=dsa.PATH_FUSED).cpu().numpy()
     np.testing.assert_array_equal(part, fused[2500:3600])
     D = orc.Decoded(wl)
     for r in range(0, wl.Tq, 3):
@@ -298,9 +355,9 @@ def test_index_topk_fused_repeat_is_bit_identical():
     wl = gen.make_prefill([4000], 8, 2, 64, 64, 128, 128, seed=39, layout="video")
     t = to_device(wl)
     args = (t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], 128)
-    first = dsa.index_topk(*args, chunk_rows=1000)
+    first = dsa.index_topk(*args, chunk_rows=1000, path=dsa.PATH_FUSED)
     for _ in range(3):
-        assert torch.equal(dsa.index_topk(*args, chunk_rows=1000), first)
+        assert torch.equal(dsa.index_topk(*args, chunk_rows=1000, path=dsa.PATH_FUSED), first)
 
 
 def test_sparse_attention_empty_and_padded_sets():
@@ -446,6 +503,57 @@ def test_prefill_pipeline_gaussian_varlen():
             assert np.array_equal(idx[r], ref["idx"])
             assert np.max(np.abs(O[r] - ref["O"])) <= ATTN_ATOL, r
             assert np.max(np.abs(lse[r] - ref["lse"])) <= LSE_ATOL, r
+
+
+def _check_prefill_rows(wl, rows, chunk):
+    """dsa.prefill against the oracle on the given rows (sets by the swap rule; O and lse
+    where the sets are identical), and against the gather kernel on the same sets."""
+    t = to_device(wl)
+    idx, O, lse = dsa.prefill(t["q_idx"], t["k_idx"], t["w"], t["Q"], t["K"], t["V"], t["cu_q"], t["cu_k"],
+                              t["max_q"], t["max_k"], wl.topk, chunk_rows=chunk)
+    Og, lg = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, t["cu_q"], t["cu_k"])
+    idx_h, O_h, lse_h = idx.cpu().numpy(), O.float().cpu().numpy(), lse.cpu().numpy()
+    # two kernels, each within the tolerance of the exact result, so within twice it of each
+    # other (two bf16 roundings of one value of magnitude 2..4 can differ by 2^-6 > 1e-2)
+    assert np.max(np.abs(O_h - Og.float().cpu().numpy())) <= 2 * ATTN_ATOL
+    assert np.max(np.abs(lse_h - lg.cpu().numpy())) <= 2 * LSE_ATOL
+    D = orc.Decoded(wl)
+    exact = 0
+    for r in rows:
+        ref = orc.forward_row(D, r)
+        ok, nsw = set_mismatch_ok(idx_h[r], ref["idx"], ref["scores"])
+        assert ok, r
+        if nsw == 0:
+            exact += 1
+            assert np.max(np.abs(O_h[r] - ref["O"])) <= ATTN_ATOL, r
+            assert np.max(np.abs(lse_h[r] - ref["lse"])) <= LSE_ATOL, r
+    assert exact >= 0.8 * len(rows)
+
+
+def test_prefill_union_coherent_video():
+    # frame-coherent indexer queries, k = 64 over 3000 and 1000 positions (sparse sets: 8 k
+    # < L): every 16-row block's union of selections fits the union form, so attention runs
+    # on the tensor-core passes over the gathered union of each block
+    wl = gen.make_prefill([3000, 1000], 32, 4, 128, 64, 128, 64, seed=40, layout="video_coherent")
+    _check_prefill_rows(wl, list(range(0, wl.Tq, 5)), 1024)
+
+
+def test_prefill_union_mixed_blocks():
+    # i.i.d. queries, k = 2048 over 20480 positions: blocks of rows that see at most 12288
+    # positions take the union form, the later blocks' unions (about 16 x 2048 positions with
+    # little overlap) exceed it and their rows run on the gather kernel
+    wl = gen.make_prefill([20480], 8, 1, 128, 64, 128, 2048, seed=41, layout="gaussian")
+    rows = orc.sample_rows(wl.Tq, seed=41, n_first=32, n_last=48, n_mid=64)
+    _check_prefill_rows(wl, rows, 4096)
+
+
+def test_prefill_union_high_overlap_video():
+    # the high-overlap video layout at the 128K heads, 20480 positions, k = 2048: most blocks'
+    # unions (the report's regime: a few thousand distinct positions per 16 queries) take the
+    # union form
+    wl = gen.make_prefill([20480], 32, 4, 128, 64, 128, 2048, seed=42, layout="video_overlap", max_frames=80)
+    rows = orc.sample_rows(wl.Tq, seed=42, n_first=16, n_last=32, n_mid=48)
+    _check_prefill_rows(wl, rows, 4096)
 
 
 def test_prefill_from_host_matches_device_prefill():

@@ -34,6 +34,7 @@ VIDEO_TEXT_PER_FRAME = 8
 
 # stream ids: one independent random stream per tensor role
 _S_QIDX, _S_KIDX, _S_W, _S_Q, _S_K, _S_V, _S_DO, _S_MEANK, _S_MEANKI, _S_LENS = range(1, 11)
+_S_MEANQI, _S_MEANW = 11, 12
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -85,9 +86,14 @@ def _normal_bf16(seed: int, stream: int, shape, row_mean: Optional[np.ndarray] =
     return out.reshape(shape)
 
 
-def _softmax_weights_bf16(seed: int, rows: int, H_I: int) -> np.ndarray:
-    """Indexer head weights: per token, a softmax over H_I of N(0, 1) logits, stored bf16."""
+def _softmax_weights_bf16(seed: int, rows: int, H_I: int, row_mean: Optional[np.ndarray] = None,
+                          mean_rows: Optional[np.ndarray] = None, noise_std: float = 1.0) -> np.ndarray:
+    """Indexer head weights: per token, a softmax over H_I of N(0, 1) logits, stored bf16;
+    where a row has a mean (as in ``_normal_bf16``) the logits are mean + noise_std * N(0, 1)."""
     z = _rng(seed, _S_W, 0).standard_normal((rows, H_I), dtype=np.float32)
+    if mean_rows is not None:
+        clustered = mean_rows >= 0
+        z[clustered] = row_mean[mean_rows[clustered]] + np.float32(noise_std) * z[clustered]
     z = z - z.max(axis=1, keepdims=True)
     e = np.exp(z)
     return f32_to_bf16_bits(e / e.sum(axis=1, keepdims=True))
@@ -188,6 +194,14 @@ def make_prefill(seqlens, Hq: int, Hkv: int, d: int, H_I: int, d_I: int, topk: i
                   {1/2, 1/4, 1/8}; Q/K/V N(0,1).  Indexer scores are exact in fp32.
       "video":    per sequence, the timestamped-frame layout; K (per KV head) and k_idx of
                   frame tokens are frame-mean N(0,1) + N(0, 0.25) noise; the rest N(0,1).
+      "video_coherent": "video", and the indexer queries q_idx of a frame's tokens also
+                  share a frame mean N(0,1) (per head) plus N(0, 0.25) noise, so adjacent
+                  tokens of a frame select partly the same positions.
+      "video_overlap": "video_coherent" with N(0, 0.01) query noise around the frame mean and
+                  head-weight logits that are a frame mean N(0,1) plus N(0, 0.01) noise, so the
+                  16 adjacent tokens of a block select mostly the same positions (the overlap
+                  the report summary gives for 128K video: about 8000 distinct positions for
+                  16 queries at k = 2048).
     """
     seqlens = [int(x) for x in seqlens]
     T = sum(seqlens)
@@ -201,9 +215,9 @@ def make_prefill(seqlens, Hq: int, Hkv: int, d: int, H_I: int, d_I: int, topk: i
         w = f32_to_bf16_bits(np.array([0.5, 0.25, 0.125], np.float32)[g.integers(0, 3, size=(T, H_I))])
         mean_rows_k = None
     else:
-        q_idx = _normal_bf16(seed, _S_QIDX, (T, H_I, d_I))
-        w = _softmax_weights_bf16(seed, T, H_I)
-        if layout == "video":
+        q_idx = None
+        w = None
+        if layout in ("video", "video_coherent", "video_overlap"):
             fids = np.concatenate([video_frame_ids(L, max_frames) for L in seqlens])
             # frame ids are made unique across sequences
             offs = np.concatenate([[0], np.cumsum([L // VIDEO_PERIOD + 1 for L in seqlens])[:-1]])
@@ -213,13 +227,24 @@ def make_prefill(seqlens, Hq: int, Hkv: int, d: int, H_I: int, d_I: int, topk: i
             mean_ki = _normal_bf16_f32(seed, _S_MEANKI, (n_means, d_I))
             k_idx = _normal_bf16(seed, _S_KIDX, (T, d_I), row_mean=mean_ki, mean_rows=mean_rows_k,
                                  noise_std=0.5)
+            if layout in ("video_coherent", "video_overlap"):
+                mean_qi = _normal_bf16_f32(seed, _S_MEANQI, (n_means, H_I, d_I))
+                q_idx = _normal_bf16(seed, _S_QIDX, (T, H_I, d_I), row_mean=mean_qi, mean_rows=mean_rows_k,
+                                     noise_std=0.5 if layout == "video_coherent" else 0.1)
+            if layout == "video_overlap":
+                mean_w = _normal_bf16_f32(seed, _S_MEANW, (n_means, H_I))
+                w = _softmax_weights_bf16(seed, T, H_I, row_mean=mean_w, mean_rows=mean_rows_k, noise_std=0.1)
         elif layout == "gaussian":
             mean_rows_k = None
             k_idx = _normal_bf16(seed, _S_KIDX, (T, d_I))
         else:
             raise ValueError(f"unknown layout {layout!r}")
+        if q_idx is None:
+            q_idx = _normal_bf16(seed, _S_QIDX, (T, H_I, d_I))
+        if w is None:
+            w = _softmax_weights_bf16(seed, T, H_I)
     Q = _normal_bf16(seed, _S_Q, (T, Hq, d))
-    if layout == "video":
+    if layout in ("video", "video_coherent", "video_overlap"):
         mean_k = _normal_bf16_f32(seed, _S_MEANK, (int(mean_rows_k.max()) + 1, Hkv, d))
         K = _normal_bf16(seed, _S_K, (T, Hkv, d), row_mean=mean_k, mean_rows=mean_rows_k, noise_std=0.5)
     else:
@@ -305,6 +330,18 @@ def video_prefill_128k() -> Workload:
     """L=131072 long-video prefill: 480 x (8 timestamp + 256 frame tokens) + 4352 text tokens."""
     return make_prefill([131072], 32, 4, 128, 64, 128, 2048, seed=2, layout="video",
                         name="video_prefill_128k", max_frames=480)
+
+
+def video_prefill_128k_coherent() -> Workload:
+    """The 128K long-video prefill with frame-coherent indexer queries (high set overlap)."""
+    return make_prefill([131072], 32, 4, 128, 64, 128, 2048, seed=2, layout="video_coherent",
+                        name="video_prefill_128k_coherent", max_frames=480)
+
+
+def video_prefill_128k_overlap() -> Workload:
+    """The 128K long-video prefill with the report's adjacent-query overlap (high set overlap)."""
+    return make_prefill([131072], 32, 4, 128, 64, 128, 2048, seed=2, layout="video_overlap",
+                        name="video_prefill_128k_overlap", max_frames=480)
 
 
 def decode_256k() -> Workload:
