@@ -123,18 +123,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// TMA row gather: four rows (r0..r3) of a 2-D tensor map whose box is one row high, each
-// box_cols wide from column c0, land one after another at dst (the map's swizzle applies as
-// for a tiled load of those rows); completion counted on `bar`.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
-      "%5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -165,6 +153,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D (+)= A . B with A read from tensor memory at a_tmem (lane m = row m of A; along K, two
+// bf16 per 32-bit column, so K = 16 spans 8 columns) and B from shared memory (descriptor).
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -188,6 +188,19 @@ __device__ __forceinline__ void tmem_ld_x32_sync(uint32_t taddr, float* v) {
         "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns stored from registers (thread i of the warp to
+// lane base + i), and the wait for the stores to complete, in one statement.
+__device__ __forceinline__ void tmem_st_x32_sync(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
 
@@ -313,6 +326,11 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Arrive on `bar` once every cp.async this thread issued so far has landed (the arrival
+// counts toward the barrier's expected count; nothing else arrives for this thread).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // ------------------------------------------------------------------ programmatic dependent launch
 // A kernel launched with the programmatic-serialization attribute may be scheduled before
@@ -419,12 +437,6 @@ int make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_
 int make_tmap_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides[2],
                       const uint32_t box[3]);
 
-// Rows of 128 bf16 (256 bytes, e.g. K or V viewed as [Tk * Hkv, 128]) for TMA row gathers:
-// boxes of one row by 64 columns with the 128-byte swizzle.
-inline int make_tmap_rows_gather(CUtensorMap* map, const void* base, long long rows) {
-  return make_tmap_bf16_2d(map, base, (uint64_t)(rows > 0 ? rows : 1), 128, 256, 1, 64, 128);
-}
-
 // The union form of the masked tensor-core attention passes (adjacent-query reuse): per
 // 16-row block the sorted union of its rows' selected positions, its size, the
 // per-(row, union slot) selection words and whether the block takes the form at all.
@@ -434,6 +446,8 @@ struct KlUnion {
   const uint32_t* umask;
   const uint8_t* blk_use;
   int ucap;  // positions per block, a multiple of 128
+  const int* blk_list;  // the blocks that take the form, and their number (device)
+  const int* n_used;
 };
 
 // A one-time-setup flag kept per GPU: cudaFuncSetAttribute applies to the current device

@@ -14,12 +14,13 @@
 // is thread-local in the epilogue.  Persistent CTAs, warp-specialised: warp 0 TMA, warp 1
 // MMA issuer and TMEM owner, warps 2-9 epilogue (two per TMEM lane quarter, one per
 // 64-key half of each tile; their two running (max, sum) pairs merge at the item's end);
-// two accumulator buffers, four key stages.
+// two accumulator buffers, six key stages.
 //
 // Union form (adjacent-query reuse, report summary section 8): a block visits, instead of
 // its causal key tiles, chunks of 128 positions of the sorted union of its rows' selected
-// sets; the producer warp gathers those K rows with TMA row gathers (one four-row gather per
-// lane and 64-column panel), and the per-(row, union slot) selection bits mask S.
+// sets; two gather warps copy those K rows into the swizzled tile with 16-byte cp.async
+// (each warp instruction reads two whole 256-byte rows), and the per-(row, union slot)
+// selection bits mask S.
 #include <algorithm>
 
 #include "common.cuh"
@@ -53,6 +54,11 @@ struct KlLseParams {
   const uint32_t* umask = nullptr;
   const uint8_t* blk_use = nullptr;
   int ucap = 0;
+  const uint16_t* K = nullptr;  // union form: K [Tk, Hkv, 128] bf16, read by the gather warps
+  // union form: the union-form blocks (item i is block blk_list[i / Hkv], head i % Hkv) and
+  // their number, so that the passes visit no other block
+  const int* blk_list = nullptr;
+  const int* n_used = nullptr;
 };
 
 struct KlLseItem {
@@ -62,9 +68,14 @@ struct KlLseItem {
 };
 
 // item -> (block, head); blocks are numbered from the last (usually the longest rows)
+// The number of items of a launch: every (block, KV head), or the union form's listed ones.
+__device__ __forceinline__ long long kl_item_count(const KlLseParams& p) {
+  return p.blk_list ? (long long)__ldg(p.n_used) * p.Hkv : p.n_items;
+}
+
 __device__ __forceinline__ bool kl_lse_item(long long item, const KlLseParams& p, KlLseItem& it) {
   it.g = (int)(item % p.Hkv);
-  long long r = p.n_blocks - 1 - item / p.Hkv;
+  long long r = p.blk_list ? __ldg(p.blk_list + item / p.Hkv) : p.n_blocks - 1 - item / p.Hkv;
   it.blk = r;
   for (int b = 0; b < p.batch; ++b) {
     const int Lq = p.cu_q[b + 1] - p.cu_q[b];
@@ -90,23 +101,56 @@ __device__ __forceinline__ bool kl_lse_item(long long item, const KlLseParams& p
   return false;
 }
 
-// Union form: positions 4 lane .. 4 lane + 3 of a 128-position union chunk (sequence-local,
-// from `chunk_keys`) as rows (s * Hkv + g) of the [Tk * Hkv, 128] view of K or V.  Loaded
-// one chunk ahead of their use, so the load's latency overlaps the wait for a free stage.
-__device__ __forceinline__ int4 union_rows(const int* chunk_keys, int kbase, int Hkv, int g, int lane) {
-  const int4 s = __ldg(reinterpret_cast<const int4*>(chunk_keys) + lane);
-  return make_int4((kbase + s.x) * Hkv + g, (kbase + s.y) * Hkv + g, (kbase + s.z) * Hkv + g, (kbase + s.w) * Hkv + g);
+// Union form: the 128 rows (positions chunk_keys[0..127], sequence-local; head g of a
+// [Tk, Hkv, 128] bf16 tensor) of one union chunk copied into a K-major tile with the
+// 128-byte swizzle (two 64-column panels of 128-byte rows, 16-byte chunk c of row r at
+// ((c ^ (r % 8)) * 16)), the layout a tiled TMA load gives.  Called by `nw` gather warps
+// (wg = 0 .. nw-1); each warp instruction copies two whole rows (16 lanes x 16 bytes each),
+// and every lane then arrives on `bar` when its copies have landed (nw * 32 arrivals).
+__device__ __forceinline__ void union_copy_tile(uint8_t* dst, int panel_bytes, const uint16_t* src,
+                                                const int* chunk_keys, int kbase, int Hkv, int g, int nw, int wg,
+                                                int lane, uint64_t* bar) {
+  const int4 k4 = __ldg(reinterpret_cast<const int4*>(chunk_keys) + lane);  // positions 4 lane .. 4 lane + 3
+  const int half = lane >> 4, c = lane & 15;
+  const uint32_t dbase = smem_u32(dst) + (c >> 3) * panel_bytes;
+#pragma unroll 4
+  for (int m = wg; m < 64; m += nw) {
+    // rows 2 m and 2 m + 1; their positions sit in lane m / 2 (warp-uniform)
+    const int r = 2 * m + half;
+    const int xa = __shfl_sync(0xffffffffu, (m & 1) ? k4.z : k4.x, m >> 1);
+    const int xb = __shfl_sync(0xffffffffu, (m & 1) ? k4.w : k4.y, m >> 1);
+    const int s = half ? xb : xa;
+    const uint16_t* row = src + ((long long)(kbase + s) * Hkv + g) * 128;
+    cp_async_16(dbase + r * 128 + (((c & 7) ^ (r & 7)) * 16), row + c * 8, true);
+  }
+  cp_async_mbar_arrive(bar);
 }
 
-// The chunk's 128 rows gathered into one tile of two 64-column panels (128-byte swizzle, the
-// layout a tiled load gives): every lane of the calling warp gathers its four rows per
-// panel.  The tile's barrier must have been told its bytes before the call.
-__device__ __forceinline__ void union_gather_tile(uint8_t* dst, int panel_bytes, const CUtensorMap* map,
-                                                  uint64_t* bar, int4 rows, int lane) {
-#pragma unroll
-  for (int pn = 0; pn < 2; ++pn)
-    tma_gather4(dst + pn * panel_bytes + lane * 512, map, bar, pn * 64, rows.x, rows.y, rows.z, rows.w);
-}
+// One row's two selection words (a 64-key half) per tile, loaded two tiles ahead of their use:
+// their global-memory latency would otherwise stall the epilogue at every tile.  Without a
+// row (no selection, or a row past the block's tokens) every word is `fill`.
+struct MaskWords {
+  const uint32_t* row;
+  long long stride;
+  int n;
+  uint32_t fill;
+  uint2 a, b;  // the words of tiles j and j + 1
+  __device__ __forceinline__ MaskWords(const uint32_t* r, long long s, int ntiles, uint32_t f)
+      : row(r), stride(s), n(ntiles), fill(f) {
+    a = load(0);
+    b = load(1);
+  }
+  __device__ __forceinline__ uint2 load(int j) const {
+    return (row && j < n) ? make_uint2(row[(long long)j * stride], row[(long long)j * stride + 1]) : make_uint2(fill, fill);
+  }
+  // the words of tile j (called with j = 0, 1, 2, ... in order)
+  __device__ __forceinline__ uint2 next(int j) {
+    const uint2 w = a;
+    a = b;
+    b = load(j + 2);
+    return w;
+  }
+};
 
 // The selection words of row u of an item and the distance between its tiles' (or union
 // chunks') words: the union form's per-block words, else the full layout of `mask`, else
@@ -124,7 +168,7 @@ __device__ __forceinline__ const uint32_t* kl_mask_row(const KlLseParams& p, con
 struct KlLseCfg {
   static constexpr int TILE_BYTES = 128 * 128 * 2;
   static constexpr int PANEL_BYTES = 128 * 128;
-  static constexpr int B_STAGES = 4;
+  static constexpr int B_STAGES = 6;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + TILE_BYTES;
   static constexpr int OFF_BAR = OFF_B + B_STAGES * TILE_BYTES;
@@ -133,8 +177,15 @@ struct KlLseCfg {
   static constexpr int OFF_ML = OFF_BAR + NUM_BARS * 8;  // 128 (max, sum) pairs of the second half
   static constexpr int OFF_MISC = OFF_ML + 128 * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // Warps: 0 TMA, 1 MMA and TMEM, 2-3 gather (warpgroup 0); 4-11 epilogue (warpgroups 1-2);
+  // 12-15 gather (warpgroup 3).  The six gather warps copy the union form's key chunks with
+  // cp.async and idle otherwise.  Registers after the reallocation: 80 for warpgroup 0, 152
+  // for the epilogue, 64 for warpgroup 3 (128 x (80 + 64) + 256 x 152 = 57344 of the 65536
+  // that 512 threads at 128 registers hold).
   static constexpr int EPI_WARPS = 8;
-  static constexpr int THREADS = 64 + EPI_WARPS * 32;
+  static constexpr int GATHER_WARPS = 6;
+  static constexpr int THREADS = 512;
+  static constexpr int REG_WG0 = 80, REG_EPI = 152, REG_WG3 = 64;
   static constexpr int TMEM_COLS = 256;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, 128);
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -168,7 +219,9 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
     mbar_init(a_full, 1);
     mbar_init(a_empty, 1);
     for (int i = 0; i < C::B_STAGES; ++i) {
-      mbar_init(&b_full[i], 1);
+      // a key tile lands by TMA (one arrival with its bytes), or in the union form by the
+      // gather warps' cp.async (one arrival per gather thread)
+      mbar_init(&b_full[i], p.ukeys ? C::GATHER_WARPS * 32 : 1);
       mbar_init(&b_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -194,97 +247,119 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int G = p.Hq / p.Hkv;  // 8
+  const long long n_items = kl_item_count(p);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (lane 0 waits
-    // and loads; in the union form every lane gathers rows of each key chunk)
-    long long m = 0, n = 0;  // items, key tiles
-    bool ok = true;
-    for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-      KlLseItem it;
-      if (!kl_lse_item(item, p, it)) continue;
-      if (lane == 0 && (ok = mbar_wait(a_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 60))) {
-        mbar_arrive_expect_tx(a_full, C::TILE_BYTES);
-        for (int pn = 0; pn < 2; ++pn)
-          tma_load_3d(sA + pn * C::PANEL_BYTES, &tmap_q, a_full, pn * 64, it.g * G, (int)it.t0);
-      }
-      if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
-      ++m;
-      const int* ukeys = p.ukeys ? p.ukeys + it.blk * p.ucap : nullptr;
-      int4 rows_next = ukeys && it.ntiles > 0 ? union_rows(ukeys, it.kbase, p.Hkv, it.g, lane) : make_int4(0, 0, 0, 0);
-      for (int j = 0; j < it.ntiles; ++j) {
-        const int st = (int)(n % C::B_STAGES);
-        const int4 rows = rows_next;
-        if (ukeys && j + 1 < it.ntiles) rows_next = union_rows(ukeys + (j + 1) * 128, it.kbase, p.Hkv, it.g, lane);
-        if (lane == 0 && (ok = mbar_wait(&b_empty[st], (uint32_t)((n / C::B_STAGES) & 1) ^ 1u, abort_flag, 61)))
-          mbar_arrive_expect_tx(&b_full[st], C::TILE_BYTES);
-        if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
-        if (ukeys)
-          union_gather_tile(sB + st * C::TILE_BYTES, C::PANEL_BYTES, &tmap_k, &b_full[st], rows, lane);
-        else if (lane == 0)
-          for (int pn = 0; pn < 2; ++pn)
-            tma_load_3d(sB + st * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &b_full[st], pn * 64, it.g,
-                        it.kbase + j * 128);
-        ++n;
-      }
-    }
-    if (!ok && lane == 0) {
-      // let the copies issued so far land before the CTA exits (bounded)
-      uint64_t t0 = globaltimer_ns();
-      for (long long q = max(0LL, n - C::B_STAGES); q < n; ++q)
-        while (!mbar_try_wait(smem_u32(&b_full[q % C::B_STAGES]), (uint32_t)((q / C::B_STAGES) & 1)) &&
-               globaltimer_ns() - t0 < 100000000ull) {
-        }
-      t0 = globaltimer_ns();
-      if (m > 0)
-        while (!mbar_try_wait(smem_u32(a_full), (uint32_t)((m - 1) & 1)) && globaltimer_ns() - t0 < 100000000ull) {
-        }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      long long m = 0, n = 0;
+  // ------------------------------------------------------------ gather warps (union form),
+  // in warpgroups 0 and 3: warps 2-3 and 12-15
+  auto gather_role = [&]() {
+    if (p.ukeys) {
+      const int wg = warp < 4 ? warp - 2 : warp - 10;
+      long long n = 0;
       bool ok = true;
-      const uint32_t a_base = smem_u32(sA);
-      for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (long long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
         KlLseItem it;
         if (!kl_lse_item(item, p, it)) continue;
-        if (!(ok = mbar_wait(a_full, (uint32_t)(m & 1), abort_flag, 62))) break;
-        tc_fence_after();
+        const int* keys = p.ukeys + it.blk * p.ucap;
         for (int j = 0; j < it.ntiles; ++j, ++n) {
           const int st = (int)(n % C::B_STAGES);
-          const int ab = (int)(n & 1);
-          if (!(ok = mbar_wait(&acc_empty[ab], (uint32_t)((n >> 1) & 1) ^ 1u, abort_flag, 63))) break;
-          if (!(ok = mbar_wait(&b_full[st], (uint32_t)((n / C::B_STAGES) & 1), abort_flag, 64))) break;
-          tc_fence_after();
-          const uint32_t b_base = smem_u32(sB + st * C::TILE_BYTES);
-#pragma unroll
-          for (int pn = 0; pn < 2; ++pn)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(tmem_base + ab * 128, smem_desc_kmajor(a_base + pn * C::PANEL_BYTES + kk * 32, 128),
-                        smem_desc_kmajor(b_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC, (pn | kk) != 0);
-          umma_commit(&b_empty[st]);
-          umma_commit(&acc_full[ab]);
+          if (lane == 0) ok = mbar_wait(&b_empty[st], (uint32_t)((n / C::B_STAGES) & 1) ^ 1u, abort_flag, 68);
+          if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+          union_copy_tile(sB + st * C::TILE_BYTES, C::PANEL_BYTES, p.K, keys + j * 128, it.kbase, p.Hkv, it.g,
+                          C::GATHER_WARPS, wg, lane, &b_full[st]);
         }
-        if (!ok) break;
-        umma_commit(a_empty);
-        ++m;
       }
-      umma_commit(mma_done);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
-      }
+      cp_async_wait<0>();  // nothing of this thread's in flight when the CTA leaves
     }
-  } else {
+  };
+  if (warp < 4) {
+    setmaxnreg_dec<C::REG_WG0>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer (the query
+      // block of each item; the key tiles too, except in the union form)
+      if (lane == 0) {
+        long long m = 0, n = 0;  // items, key tiles
+        bool ok = true;
+        for (long long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+          KlLseItem it;
+          if (!kl_lse_item(item, p, it)) continue;
+          if (!(ok = mbar_wait(a_empty, (uint32_t)(m & 1) ^ 1u, abort_flag, 60))) break;
+          mbar_arrive_expect_tx(a_full, C::TILE_BYTES);
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(sA + pn * C::PANEL_BYTES, &tmap_q, a_full, pn * 64, it.g * G, (int)it.t0);
+          ++m;
+          if (p.ukeys) continue;  // the gather warps copy the union chunks
+          for (int j = 0; j < it.ntiles; ++j) {
+            const int st = (int)(n % C::B_STAGES);
+            if (!(ok = mbar_wait(&b_empty[st], (uint32_t)((n / C::B_STAGES) & 1) ^ 1u, abort_flag, 61))) break;
+            mbar_arrive_expect_tx(&b_full[st], C::TILE_BYTES);
+            for (int pn = 0; pn < 2; ++pn)
+              tma_load_3d(sB + st * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmap_k, &b_full[st], pn * 64, it.g,
+                          it.kbase + j * 128);
+            ++n;
+          }
+        }
+        if (!ok) {
+          // let the copies issued so far land before the CTA exits (bounded)
+          uint64_t t0 = globaltimer_ns();
+          for (long long q = max(0LL, n - C::B_STAGES); q < n; ++q)
+            while (!mbar_try_wait(smem_u32(&b_full[q % C::B_STAGES]), (uint32_t)((q / C::B_STAGES) & 1)) &&
+                   globaltimer_ns() - t0 < 100000000ull) {
+            }
+          t0 = globaltimer_ns();
+          if (m > 0)
+            while (!mbar_try_wait(smem_u32(a_full), (uint32_t)((m - 1) & 1)) && globaltimer_ns() - t0 < 100000000ull) {
+            }
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        long long m = 0, n = 0;
+        bool ok = true;
+        const uint32_t a_base = smem_u32(sA);
+        for (long long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+          KlLseItem it;
+          if (!kl_lse_item(item, p, it)) continue;
+          if (!(ok = mbar_wait(a_full, (uint32_t)(m & 1), abort_flag, 62))) break;
+          tc_fence_after();
+          for (int j = 0; j < it.ntiles; ++j, ++n) {
+            const int st = (int)(n % C::B_STAGES);
+            const int ab = (int)(n & 1);
+            if (!(ok = mbar_wait(&acc_empty[ab], (uint32_t)((n >> 1) & 1) ^ 1u, abort_flag, 63))) break;
+            if (!(ok = mbar_wait(&b_full[st], (uint32_t)((n / C::B_STAGES) & 1), abort_flag, 64))) break;
+            tc_fence_after();
+            const uint32_t b_base = smem_u32(sB + st * C::TILE_BYTES);
+  #pragma unroll
+            for (int pn = 0; pn < 2; ++pn)
+  #pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(tmem_base + ab * 128, smem_desc_kmajor(a_base + pn * C::PANEL_BYTES + kk * 32, 128),
+                          smem_desc_kmajor(b_base + pn * C::PANEL_BYTES + kk * 32, 128), C::IDESC, (pn | kk) != 0);
+            umma_commit(&b_empty[st]);
+            umma_commit(&acc_full[ab]);
+          }
+          if (!ok) break;
+          umma_commit(a_empty);
+          ++m;
+        }
+        umma_commit(mma_done);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(smem_u32(mma_done), 0) && globaltimer_ns() - t0 < 200000000ull) {
+        }
+      }
+    } else {
+      gather_role();
+    }
+  } else if (warp < 4 + C::EPI_WARPS) {
+    setmaxnreg_inc<C::REG_EPI>();
     // ------------------------------------------------------------ epilogue (8 warps)
     const int lane_grp = warp % 4;
-    const int half = (warp - 2) / 4;     // keys 64 half .. 64 half + 63 of each tile
+    const int half = (warp - 4) / 4;     // keys 64 half .. 64 half + 63 of each tile
     const int r = lane_grp * 32 + lane;  // (row, head) of this thread: row r / 8, head r % 8
     const uint32_t lane_off = (uint32_t)(lane_grp * 32) << 16;
     long long n = 0, m = 0;
     bool ok = true;
-    for (long long item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (long long item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       KlLseItem it;
       if (!kl_lse_item(item, p, it)) continue;
       const int u = r / 8;
@@ -296,15 +371,13 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
       long long mstride;
       const uint32_t* mrow = kl_mask_row(p, it, valid ? u : 0, mstride);
       if (mrow) mrow += 2 * half;
+      // selection words of this row for the half's 64 keys (all set without a selection)
+      MaskWords mw(mrow, mstride, it.ntiles, 0xffffffffu);
       for (int j = 0; j < it.ntiles; ++j, ++n) {
         const int tile = j;
         const int ab = (int)(n & 1);
-        // selection words of this row for the half's 64 keys (all set without a selection)
-        uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
-        if (mrow) {
-          w0 = mrow[(long long)tile * mstride];
-          w1 = mrow[(long long)tile * mstride + 1];
-        }
+        const uint2 wj = mw.next(j);
+        const uint32_t w0 = wj.x, w1 = wj.y;
         if (!(ok = mbar_wait(&acc_full[ab], (uint32_t)((n >> 1) & 1), abort_flag, 65))) break;
         tc_fence_after();
         float v[64];
@@ -367,8 +440,10 @@ __global__ void __launch_bounds__(KlLseCfg::THREADS, 1)
       }
       ++m;
     }
+  } else {
+    setmaxnreg_dec<C::REG_WG3>();
+    gather_role();
   }
-
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -735,6 +810,12 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
                                                     C::SMEM_BYTES);
         e_ != cudaSuccess)
       return cuda_fail(e_);
+    // the register reallocation must fit what a launch holds, or its increase would wait for
+    // registers that never come
+    cudaFuncAttributes fa;
+    if (const cudaError_t e_ = cudaFuncGetAttributes(&fa, dsa::kl_lse_tc_kernel); e_ != cudaSuccess) return cuda_fail(e_);
+    if ((long long)fa.numRegs * C::THREADS < 128LL * (C::REG_WG0 + C::REG_WG3) + 256LL * C::REG_EPI)
+      return DSA_ERR_UNSUPPORTED;
     attr_done = true;
   }
   CUtensorMap tq, tk;
@@ -744,10 +825,8 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
     const uint32_t box[3] = {64, 8, 16};
     if (const int st = make_tmap_bf16_3d(&tq, Q, dims, strides, box); st != DSA_OK) return st;
   }
-  if (un) {
-    if (const int st = make_tmap_rows_gather(&tk, K, Tk * Hkv); st != DSA_OK) return st;
-  } else {
-    const uint64_t dims[3] = {128, (uint64_t)Hkv, (uint64_t)Tk};
+  {
+    const uint64_t dims[3] = {128, (uint64_t)Hkv, (uint64_t)std::max<long long>(Tk, 1)};
     const uint64_t strides[2] = {256, (uint64_t)Hkv * 256};
     const uint32_t box[3] = {64, 1, 128};
     if (const int st = make_tmap_bf16_3d(&tk, K, dims, strides, box); st != DSA_OK) return st;
@@ -765,11 +844,14 @@ int kl_lse_tc_launch(const void* Q, const void* K, const int* cu_q, const int* c
   p.total_q = T;
   p.max_out = max_out;
   if (un) {
+    p.blk_list = un->blk_list;
+    p.n_used = un->n_used;
     p.ukeys = un->ukeys;
     p.ucount = un->ucount;
     p.umask = un->umask;
     p.blk_use = un->blk_use;
     p.ucap = un->ucap;
+    p.K = static_cast<const uint16_t*>(K);
   }
   // an upper bound on the 16-row blocks (each sequence rounds up once)
   p.n_blocks = (T + 15) / 16 + batch;
