@@ -32,8 +32,8 @@ from workloads import generators as gen  # noqa: E402
 PREFILL_CHUNK = 8192
 # DRAM bytes (read + write) per causal (t, s) pair of the fused indexer kernel (candidates
 # instead of scores), from one ncu capture of that kernel on the last 8192 rows of a 32K
-# video prefill (None until such a capture exists for the current kernel)
-IDX_DRAM_BYTES_PER_PAIR = None
+# video prefill: (282.7 + 176.3) MB over 234.9 M pairs (profiles/indexer2_fused_prefill_32k_late_chunk.md)
+IDX_DRAM_BYTES_PER_PAIR = 1.954
 METRIC = "DSA prefill tokens/s at 128K ctx (indexer + top-k + sparse attention)"
 
 
@@ -759,7 +759,7 @@ def main():
         "roofline": {"kernel": "fused indexer -> top-k (dsa_index_topk, tcgen05 indexer)", "bound": "tensor",
                      "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                      "traffic": (None if IDX_DRAM_BYTES_PER_PAIR is None
-                                 else IDX_DRAM_BYTES_PER_PAIR * wl.causal_pairs() / ((L + PREFILL_CHUNK - 1) // PREFILL_CHUNK)),
+                                 else IDX_DRAM_BYTES_PER_PAIR * wl.causal_pairs() / ((wl.Tq + PREFILL_CHUNK - 1) // PREFILL_CHUNK)),
                      "traffic_source": "ncu dram bytes read+write of the fused indexer kernel on the last 8192 rows of "
                                        "a 32K video prefill, per causal pair, scaled to an average 128K chunk launch",
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"},

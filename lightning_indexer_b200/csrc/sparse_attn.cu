@@ -331,21 +331,28 @@ __global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAPara
   }
 }
 
-// Merges the per-split partial softmax states of decode: one warp per (row, head), lane s
-// holding split s (nsplit <= 32), so every load of the merge is issued at once.
+// Merges the per-split partial softmax states of decode: one warp per (row, head, 32 of the
+// D output dims), lane s holding split s's (max, sum, weight sum) (nsplit <= 32).  Every
+// load of the warp (its splits' 32 dims of O, and the states) is issued before any of the
+// merge arithmetic, so the kernel costs about one memory round trip.
 template <int D>
 __global__ void decode_combine_kernel(const float* part_o, const float* part_ml, int rows, int Hq, int nsplit,
                                       uint16_t* O, float* lse) {
   pdl_wait();
   pdl_trigger();
+  constexpr int PARTS = D / 32;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
-  if (gw >= rows * Hq) return;
-  const int row = gw / Hq, h = gw % Hq;
-  const size_t mine = ((size_t)row * nsplit + lane) * Hq + h;  // this lane's split
+  if (gw >= rows * Hq * PARTS) return;
+  const int part = gw % PARTS, rh = gw / PARTS;
+  const int row = rh / Hq, h = rh % Hq;
+  float v[32];
+#pragma unroll
+  for (int s = 0; s < 32; ++s)
+    v[s] = s < nsplit ? part_o[(((size_t)row * nsplit + s) * Hq + h) * D + part * 32 + lane] : 0.f;
   float m = -INFINITY, l = 0.f, rr = 0.f;
   if (lane < nsplit) {
-    const float4 ml = *reinterpret_cast<const float4*>(part_ml + mine * 4);
+    const float4 ml = *reinterpret_cast<const float4*>(part_ml + (((size_t)row * nsplit + lane) * Hq + h) * 4);
     m = ml.x;
     l = ml.y;
     rr = ml.z;
@@ -361,21 +368,12 @@ __global__ void decode_combine_kernel(const float* part_o, const float* part_ml,
     L += __shfl_xor_sync(0xffffffffu, L, o);
     R += __shfl_xor_sync(0xffffffffu, R, o);
   }
-  float o_[D / 32];
+  float acc = 0.f;
 #pragma unroll
-  for (int j = 0; j < D / 32; ++j) o_[j] = 0.f;
-#pragma unroll 4
-  for (int s = 0; s < nsplit; ++s) {
-    const float fs = __shfl_sync(0xffffffffu, f, s);
-    const float* po = part_o + (((size_t)row * nsplit + s) * Hq + h) * D;
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) o_[j] += fs * po[j * 32 + lane];
-  }
+  for (int s = 0; s < 32; ++s) acc += __shfl_sync(0xffffffffu, f, s) * v[s];
   const float inv = R > 0.f ? 1.f / R : 0.f;
-#pragma unroll
-  for (int j = 0; j < D / 32; ++j)
-    O[((size_t)row * Hq + h) * D + j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o_[j] * inv));
-  if (lse && lane == 0) lse[(size_t)row * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  O[((size_t)row * Hq + h) * D + part * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(acc * inv));
+  if (lse && part == 0 && lane == 0) lse[(size_t)row * Hq + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace dsa
@@ -469,7 +467,7 @@ int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const
   p.part_ml = p.part_o + (size_t)batch * p.nsplit * Hq * d;
   int st = sa_launch_common(p, d, stream);
   if (st != DSA_OK) return st;
-  const int warps = batch * Hq;
+  const int warps = batch * Hq * (d / 32);
   const int threads = 256;
   const int blocks = (warps * 32 + threads - 1) / threads;
   const float* part_o = p.part_o;
