@@ -288,6 +288,34 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * (5b) Whole DSA forward for prefill from HOST buffers.  Same computation as (5): per row
+ * chunk of at most `chunk_rows` rows, (2b) with DSA_PATH_AUTO, then (3c) on the chunk's rows
+ * (its query offsets shifted to the chunk); the O rows agree with (5)'s sparse path bit for
+ * bit.  The inputs are copied in and O copied out inside the call's stream order: the key
+ * side first, then each chunk's q_idx, w and Q rows, so that a chunk's copies overlap its
+ * neighbours' kernels; each chunk's O rows are copied back as soon as they are ready.
+ *   q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k: HOST memory, layouts as in (5)
+ *     (pinned memory for the copies to overlap the kernels);
+ *   O: HOST bf16 [total_q, Hq, d], written when the work enqueued on `stream` completes;
+ *   workspace: DEVICE memory of dsa_prefill_host_workspace_size() bytes, 16-byte aligned
+ *     (DSA_ERR_WORKSPACE if NULL or smaller): it holds the device copies of the inputs, the
+ *     selected sets, O, and the scratch of (2b) and (3c).
+ * The copies run on two copy streams the library creates on first use on each device (and
+ * keeps); `stream` is made to wait for them, so synchronising `stream` covers the whole
+ * call, including the copy of O.  Host pointers must stay valid until then.  Devices
+ * numbered 64 or more return DSA_ERR_UNSUPPORTED.
+ * ------------------------------------------------------------------------------- */
+DSA_API size_t dsa_prefill_host_workspace_size(int batch, int64_t total_q, int64_t total_k,
+                                               int max_seqlen_k, int Hq, int Hkv, int d, int H_I,
+                                               int d_I, int k, int64_t chunk_rows);
+DSA_API int dsa_prefill_host(const void* q_idx, const void* k_idx, const void* w, const void* Q,
+                             const void* K, const void* V, const int32_t* cu_seqlens_q,
+                             const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                             int64_t total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv,
+                             int d, int H_I, int d_I, int k, float scale, int64_t chunk_rows,
+                             void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * (6) Whole DSA decode step: (1) with one query row per sequence over its cache, (2),
  * then (4).  q_idx device bf16 [batch, H_I, d_I]; w device bf16 [batch, H_I]; k_idx
  * device bf16 [total_k, d_I]; Q/K/V/O as in (4); indices device int32 [batch, k].

@@ -13,7 +13,7 @@ import torch
 from . import _lib
 from ._lib import DSAError, call
 
-__all__ = ["index", "topk", "topk_workspace_bytes", "index_topk", "index_topk_workspace_bytes", "prefill_from_host", "sparse_attn_prefill", "sparse_attn_prefill_reuse", "sparse_attn_prefill_reuse_workspace_bytes", "sparse_attn_decode", "prefill", "decode",
+__all__ = ["index", "topk", "topk_workspace_bytes", "index_topk", "index_topk_workspace_bytes", "prefill_from_host", "prefill_host_workspace_bytes", "sparse_attn_prefill", "sparse_attn_prefill_reuse", "sparse_attn_prefill_reuse_workspace_bytes", "sparse_attn_decode", "prefill", "decode",
            "sparse_attn_prefill_bwd", "indexer_kl_loss", "indexer_kl_loss_sparse", "device_status", "DSAError"]
 
 
@@ -225,85 +225,44 @@ def prefill(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: 
     return indices, O, lse
 
 
-_aux_streams = {}
-
-
-def _streams(device: torch.device):
-    key = device.index
-    if key not in _aux_streams:
-        _aux_streams[key] = (torch.cuda.Stream(device), torch.cuda.Stream(device))
-    return _aux_streams[key]
+def prefill_host_workspace_bytes(batch: int, total_q: int, total_k: int, max_seqlen_k: int, Hq: int, Hkv: int, d: int,
+                                 H_I: int, d_I: int, k: int, chunk_rows: int) -> int:
+    return _lib.load().dsa_prefill_host_workspace_size(batch, total_q, total_k, max_seqlen_k, Hq, Hkv, d, H_I, d_I, k,
+                                                       chunk_rows)
 
 
 def prefill_from_host(q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                       k: int, chunk_rows: int = 8192, scale: Optional[float] = None, O=None,
                       device: Optional[torch.device] = None, buffers: Optional[dict] = None):
-    """Whole DSA prefill whose inputs and output live in host memory (pin them for overlap).
-
-    The key-side tensors (k_idx, K, V) are copied first; then the query rows of each row
-    chunk are copied on a copy stream while the previous chunk runs its (fused) indexer and
-    top-k and its attention (with adjacent-query reuse) on the current stream, and each chunk's O rows go back on a third stream
-    while the next chunk runs.  The kernels and their results are those of `prefill`.
-    `buffers` (a dict, filled on first use) keeps the device copies between calls.
-    Returns O (host, bf16 [T, Hq, d]); the current stream is ordered after every copy.
-    """
+    """Whole DSA prefill whose inputs and output live in host memory (pin them for overlap),
+    through the library's dsa_prefill_host: the key side is copied first, each row chunk's
+    query rows are copied while its neighbours run their indexer + top-k and attention, and
+    each chunk's O rows are copied back as soon as they are ready.  `buffers` (a dict,
+    filled on first use) keeps the device workspace between calls.  Returns O (host, bf16
+    [T, Hq, d]); the current stream is ordered after every copy."""
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    for t, n in ((q_idx, "q_idx"), (k_idx, "k_idx"), (w, "w"), (Q, "Q"), (K, "K"), (V, "V")):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous bfloat16 host tensor")
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k")):
+        if t.dtype != torch.int32 or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous int32 host tensor")
     T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    H_I, d_I = q_idx.shape[1], q_idx.shape[2]
     B = cu_seqlens_q.numel() - 1
-    L = max_seqlen_k
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
     chunk_rows = max(1, min(chunk_rows, T))
-    chunks = [(r0, min(T, r0 + chunk_rows)) for r0 in range(0, T, chunk_rows)]
     buf = {} if buffers is None else buffers
-    for name, h in (("q_idx", q_idx), ("k_idx", k_idx), ("w", w), ("Q", Q), ("K", K), ("V", V),
-                    ("cu_q", cu_seqlens_q), ("cu_k", cu_seqlens_k)):
-        if name not in buf or buf[name].shape != h.shape:
-            buf[name] = torch.empty(h.shape, dtype=h.dtype, device=dev)
-    # per chunk: the query offsets shifted to the chunk's first row (attention runs per chunk)
-    cq = cu_seqlens_q.to(torch.int64)
-    cu_chunks = torch.stack([(cq - r0).clamp(0, r1 - r0) for r0, r1 in chunks]).to(torch.int32)
-    if "cu_chunks" not in buf or buf["cu_chunks"].shape != cu_chunks.shape:
-        buf["cu_chunks"] = torch.empty(cu_chunks.shape, dtype=torch.int32, device=dev)
-    ws_bytes = index_topk_workspace_bytes(chunk_rows, L)
-    if "ws" not in buf or buf["ws"].numel() < ws_bytes:
-        buf["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    rws_bytes = sparse_attn_prefill_reuse_workspace_bytes(chunk_rows, Hq, B, L)
-    if "rws" not in buf or buf["rws"].numel() < rws_bytes:
-        buf["rws"] = torch.empty(rws_bytes, dtype=torch.uint8, device=dev)
-    if "idx" not in buf or buf["idx"].shape != (T, k):
-        buf["idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
-    if "O" not in buf or buf["O"].shape != Q.shape:
-        buf["O"] = torch.empty(Q.shape, dtype=torch.bfloat16, device=dev)
+    nbytes = prefill_host_workspace_bytes(B, T, K.shape[0], max_seqlen_k, Hq, Hkv, d, H_I, d_I, k, chunk_rows)
+    if "ws" not in buf or buf["ws"].numel() < nbytes or buf["ws"].device != dev:
+        buf["ws"] = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     if O is None:
         O = torch.empty(Q.shape, dtype=torch.bfloat16, pin_memory=True)
-    main = torch.cuda.current_stream(dev)
-    h2d, d2h = _streams(dev)
-    h2d.wait_stream(main)  # the buffers are free once earlier work on this stream is done
-    d2h.wait_stream(main)
-    ev_keys = torch.cuda.Event()
-    ev_in = [torch.cuda.Event() for _ in chunks]
-    with torch.cuda.stream(h2d):
-        for name, h in (("cu_q", cu_seqlens_q), ("cu_k", cu_seqlens_k), ("k_idx", k_idx), ("K", K), ("V", V)):
-            buf[name].copy_(h, non_blocking=True)
-        buf["cu_chunks"].copy_(cu_chunks, non_blocking=True)
-        ev_keys.record(h2d)
-        for (r0, r1), ev in zip(chunks, ev_in):
-            for name, h in (("q_idx", q_idx), ("w", w), ("Q", Q)):
-                buf[name][r0:r1].copy_(h[r0:r1], non_blocking=True)
-            ev.record(h2d)
-    main.wait_event(ev_keys)
-    for c, (r0, r1) in enumerate(chunks):
-        main.wait_event(ev_in[c])
-        index_topk(buf["q_idx"], buf["k_idx"], buf["w"], buf["cu_q"], buf["cu_k"], max_seqlen_q, L, k,
-                   chunk_rows=chunk_rows, indices=buf["idx"][r0:r1], workspace=buf["ws"], row_begin=r0, row_end=r1)
-        sparse_attn_prefill_reuse(buf["Q"][r0:r1], buf["K"], buf["V"], buf["idx"][r0:r1], buf["cu_chunks"][c],
-                                  buf["cu_k"], L, scale, out=(buf["O"][r0:r1], None), workspace=buf["rws"])
-        ev_out = torch.cuda.Event()
-        ev_out.record(main)
-        d2h.wait_event(ev_out)
-        with torch.cuda.stream(d2h):
-            O[r0:r1].copy_(buf["O"][r0:r1], non_blocking=True)
-    main.wait_stream(d2h)
-    main.wait_stream(h2d)
+    with torch.cuda.device(dev):
+        call("dsa_prefill_host", _ptr(q_idx), _ptr(k_idx), _ptr(w), _ptr(Q), _ptr(K), _ptr(V), _ptr(cu_seqlens_q),
+             _ptr(cu_seqlens_k), B, T, K.shape[0], max_seqlen_q, max_seqlen_k, Hq, Hkv, d, H_I, d_I, k, scale,
+             chunk_rows, _ptr(O), _ptr(buf["ws"]), buf["ws"].numel(), _stream())
     return O
 
 

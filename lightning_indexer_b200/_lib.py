@@ -39,6 +39,10 @@ SIGNATURES = {
     "dsa_prefill": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int,
                             c_int, c_int, c_int, c_int, c_int, c_int, c_f32, c_i64, c_vp, c_vp, c_vp, c_vp,
                             c_size, c_vp]),
+    "dsa_prefill_host_workspace_size": (c_size, [c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                 c_i64]),
+    "dsa_prefill_host": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int,
+                                 c_int, c_int, c_int, c_int, c_int, c_int, c_f32, c_i64, c_vp, c_vp, c_size, c_vp]),
     "dsa_decode_workspace_size": (c_size, [c_int, c_int, c_int, c_int, c_int]),
     "dsa_decode": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_int, c_int, c_int, c_int,
                            c_int, c_int, c_int, c_f32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),

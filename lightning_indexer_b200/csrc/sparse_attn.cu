@@ -54,7 +54,7 @@ struct SAParams {
 
 // 4-warp CTAs with 2 stages per warp: 3 CTAs, 12 warps per SM.  (Decode launches only a
 // thousand warps; 1-warp CTAs with 4 stages each, all resident at once, measured slower.)
-constexpr int SA_WARPS = 4;   // warps per CTA
+constexpr int SA_WARPS = 7;   // warps per CTA (two CTAs per SM: 14 warps, 224 KB of K/V rings at d = 128)
 constexpr int SA_STAGES = 2;  // chunks in flight per warp, the one in use included
 constexpr int SA_CHUNK = 16;
 
@@ -99,7 +99,7 @@ __device__ __forceinline__ uint32_t tile_off(int row, int seg) {
 }
 
 template <int D, int SA_STAGES, int SA_WARPS>
-__global__ void __launch_bounds__(SA_WARPS * 32) sparse_attn_kernel(const SAParams p) {
+__global__ void __launch_bounds__(SA_WARPS * 32, 2) sparse_attn_kernel(const SAParams p) {
   constexpr int SEGS = D / 8;                   // 16-byte segments per row
   constexpr int TILE_BYTES = SA_CHUNK * D * 2;  // one K or V chunk
   constexpr int STAGE_BYTES = 2 * TILE_BYTES;

@@ -79,6 +79,23 @@ def test_host_side_argument_errors():
                                              fake, None, None, None, small, None) == -3
     assert lib.dsa_sparse_attn_prefill_reuse(fake, fake, fake, fake, fake, fake, 1, 0, 0, 8, 32, 4, 128, 64, 0.1,
                                              fake, None, None, fake, wsz, None) == 0  # nothing to do
+    # host-input prefill: argument checks before anything is enqueued
+    hw = lib.dsa_prefill_host_workspace_size(1, 131072, 131072, 131072, 32, 4, 128, 64, 128, 2048, 8192)
+    assert hw > 131072 * (64 * 128 * 2 + 32 * 128 * 2 * 2 + 2048 * 4)  # device copies of the inputs, O, indices
+    assert lib.dsa_prefill_host_workspace_size(0, 8, 8, 8, 32, 4, 128, 64, 128, 64, 8) == 0
+    args = [fake] * 8 + [1, 8, 8, 8, 8, 32, 4, 128, 64, 128, 64, 0.1, 8, fake]
+    bad = list(args)
+    bad[15] = 96  # d
+    assert lib.dsa_prefill_host(*bad, fake, hw, None) == -2
+    bad = list(args)
+    bad[18] = 40  # k not a multiple of 16
+    assert lib.dsa_prefill_host(*bad, fake, hw, None) == -2
+    bad = list(args)
+    bad[19] = 0.0  # scale
+    assert lib.dsa_prefill_host(*bad, fake, hw, None) == -1
+    need_small = lib.dsa_prefill_host_workspace_size(1, 8, 8, 8, 32, 4, 128, 64, 128, 64, 8)
+    assert lib.dsa_prefill_host(*args, fake, need_small - 16, None) == -3
+    assert lib.dsa_prefill_host(*args, None, need_small, None) == -3
     # workspace too small
     need = lib.dsa_sparse_attn_decode_workspace_size(16, 32, 128, 2048)
     assert need > 0

@@ -577,6 +577,47 @@ def test_prefill_from_host_matches_device_prefill():
         assert torch.equal(O.view(torch.int16), O_ref.cpu().view(torch.int16))
 
 
+def test_prefill_from_host_tensor_core_shape():
+    # the native host-input pipeline at the 128K heads (d = 128, 8 query heads per KV head),
+    # two sequences, row chunks of 2048 crossing the sequence boundary: sets by the swap rule
+    # and O against the oracle on sampled rows, and the same O as the device-side calls
+    # (index + top-k, then the reuse attention) chunk by chunk
+    wl = gen.make_prefill([3000, 1500], 32, 4, 128, 64, 128, 256, seed=44)
+    t = to_device(wl)
+
+    def host(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    cu_q = torch.from_numpy(wl.cu_seqlens_q.astype(np.int32))
+    cu_k = torch.from_numpy(wl.cu_seqlens_k.astype(np.int32))
+    O = dsa.prefill_from_host(host(wl.q_idx), host(wl.k_idx), host(wl.w), host(wl.Q), host(wl.K), host(wl.V), cu_q,
+                              cu_k, t["max_q"], t["max_k"], wl.topk, chunk_rows=2048)
+    torch.cuda.current_stream().synchronize()
+    idx = torch.empty((wl.Tq, wl.topk), dtype=torch.int32, device="cuda")
+    O_dev = torch.empty_like(t["Q"])
+    for r0 in range(0, wl.Tq, 2048):
+        r1 = min(wl.Tq, r0 + 2048)
+        dsa.index_topk(t["q_idx"], t["k_idx"], t["w"], t["cu_q"], t["cu_k"], t["max_q"], t["max_k"], wl.topk,
+                       chunk_rows=2048, indices=idx[r0:r1], row_begin=r0, row_end=r1)
+        cq = torch.from_numpy(np.clip(wl.cu_seqlens_q.astype(np.int64) - r0, 0, r1 - r0).astype(np.int32)).cuda()
+        dsa.sparse_attn_prefill_reuse(t["Q"][r0:r1], t["K"], t["V"], idx[r0:r1], cq, t["cu_k"], t["max_k"],
+                                      out=(O_dev[r0:r1], None))
+    torch.cuda.synchronize()
+    assert torch.equal(O.view(torch.int16), O_dev.cpu().view(torch.int16))
+    D = orc.Decoded(wl)
+    Oh, idx_h = O.float().numpy(), idx.cpu().numpy()
+    exact = 0
+    rows = list(range(0, wl.Tq, 75))
+    for r in rows:
+        ref = orc.forward_row(D, r)
+        ok, nsw = set_mismatch_ok(idx_h[r], ref["idx"], ref["scores"])
+        assert ok, r
+        if nsw == 0:
+            exact += 1
+            assert np.max(np.abs(Oh[r] - ref["O"])) <= ATTN_ATOL, r
+    assert exact >= 0.8 * len(rows)
+
+
 def test_decode_pipeline():
     wl = gen.make_decode(4, 20000, 32, 4, 128, 64, 128, 2048, seed=42, layout="video")
     t = to_device(wl)
