@@ -291,9 +291,10 @@ DSA_API int dsa_prefill(const void* q_idx, const void* k_idx, const void* w, con
  * (5b) Whole DSA forward for prefill from HOST buffers.  Same computation as (5): per row
  * chunk of at most `chunk_rows` rows, (2b) with DSA_PATH_AUTO, then (3c) on the chunk's rows
  * (its query offsets shifted to the chunk); the O rows agree with (5)'s sparse path bit for
- * bit.  The inputs are copied in and O copied out inside the call's stream order: the key
- * side first, then each chunk's q_idx, w and Q rows, so that a chunk's copies overlap its
- * neighbours' kernels; each chunk's O rows are copied back as soon as they are ready.
+ * bit.  The inputs are copied in and O copied out inside the call's stream order: per
+ * chunk, the key-side rows (k_idx, K, V) its rows can see that earlier chunks did not need,
+ * then its q_idx, w and Q rows, so that a chunk's copies overlap its neighbours' kernels;
+ * each chunk's O rows are copied back as soon as they are ready.
  *   q_idx, k_idx, w, Q, K, V, cu_seqlens_q, cu_seqlens_k: HOST memory, layouts as in (5)
  *     (pinned memory for the copies to overlap the kernels);
  *   O: HOST bf16 [total_q, Hq, d], written when the work enqueued on `stream` completes;

@@ -114,7 +114,7 @@ DSA_API int dsa_prefill_host(const void* q_idx, const void* k_idx, const void* w
   cudaStream_t h2d, d2h;
   if (const int st = copy_streams(h2d, d2h); st != DSA_OK) return st;
   const int nchunks = (int)((total_q + chunk_rows - 1) / chunk_rows);
-  // events: start, keys landed, per chunk inputs landed and outputs ready, copies out done
+  // events: start, offsets landed, per chunk inputs landed and outputs ready, copies out done
   std::vector<cudaEvent_t> ev(3 + 2 * (size_t)nchunks, nullptr);
   int status = DSA_OK;
   auto check = [&](cudaError_t e_) {
@@ -139,15 +139,39 @@ DSA_API int dsa_prefill_host(const void* q_idx, const void* k_idx, const void* w
     check(cudaEventRecord(e_start, main)) && check(cudaStreamWaitEvent(h2d, e_start, 0)) &&
         check(cudaStreamWaitEvent(d2h, e_start, 0));
   }
-  // key side first, then the query rows chunk by chunk
+  // the offsets first; then per chunk, the key-side rows its rows can see that earlier
+  // chunks did not need (whole 256-key tiles ahead, since the indexer loads keys by tile),
+  // then the chunk's query rows: the first chunk starts after its own keys, not all of them
+  const auto* ki = static_cast<const uint8_t*>(k_idx);
+  const auto* Ki = static_cast<const uint8_t*>(K);
+  const auto* Vi = static_cast<const uint8_t*>(V);
+  const size_t ki_row = (size_t)d_I * 2, kv_row = (size_t)Hkv * d * 2;
+  int64_t keys_done = 0;
+  auto copy_keys_to = [&](int64_t kend) {
+    kend = std::min<int64_t>(total_k, kend);
+    if (kend <= keys_done) return true;
+    const int64_t k0 = keys_done, nk = kend - keys_done;
+    keys_done = kend;
+    return h2d_copy(L.k_idx + k0 * ki_row, ki + k0 * ki_row, nk * ki_row) &&
+           h2d_copy(L.K + k0 * kv_row, Ki + k0 * kv_row, nk * kv_row) &&
+           h2d_copy(L.V + k0 * kv_row, Vi + k0 * kv_row, nk * kv_row);
+  };
+  // the end of the keys that rows below r1 see (bottom-right causal alignment per sequence)
+  auto key_end = [&](int64_t r1) {
+    int b = 0;
+    while (b + 1 < batch && cu_seqlens_q[b + 1] <= r1 - 1) ++b;
+    const int64_t Lq = cu_seqlens_q[b + 1] - cu_seqlens_q[b], Lk = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+    const int64_t vis = std::min(Lk, std::max<int64_t>(0, (r1 - 1 - cu_seqlens_q[b]) + (Lk - Lq) + 1));
+    return cu_seqlens_k[b] + (vis + 511) / 256 * 256;
+  };
   if (status == DSA_OK && h2d_copy(L.cu_q, cu_seqlens_q, (size_t)(batch + 1) * 4) &&
-      h2d_copy(L.cu_k, cu_seqlens_k, (size_t)(batch + 1) * 4) && h2d_copy(L.k_idx, k_idx, (size_t)total_k * d_I * 2) &&
-      h2d_copy(L.K, K, (size_t)total_k * Hkv * d * 2) && h2d_copy(L.V, V, (size_t)total_k * Hkv * d * 2) &&
-      check(cudaEventRecord(e_keys, h2d))) {
+      h2d_copy(L.cu_k, cu_seqlens_k, (size_t)(batch + 1) * 4) && check(cudaEventRecord(e_keys, h2d))) {
     for (int c = 0; c < nchunks && status == DSA_OK; ++c) {
       const int64_t r0 = (int64_t)c * chunk_rows, n = std::min(total_q, r0 + chunk_rows) - r0;
-      h2d_copy(L.q_idx + r0 * qi_row, qi + r0 * qi_row, n * qi_row) && h2d_copy(L.w + r0 * w_row, wi + r0 * w_row, n * w_row) &&
-          h2d_copy(L.Q + r0 * q_row, Qi + r0 * q_row, n * q_row) && check(cudaEventRecord(e_in[c], h2d));
+      copy_keys_to(c + 1 == nchunks ? total_k : key_end(r0 + n)) &&
+          h2d_copy(L.q_idx + r0 * qi_row, qi + r0 * qi_row, n * qi_row) &&
+          h2d_copy(L.w + r0 * w_row, wi + r0 * w_row, n * w_row) && h2d_copy(L.Q + r0 * q_row, Qi + r0 * q_row, n * q_row) &&
+          check(cudaEventRecord(e_in[c], h2d));
     }
   }
   if (status == DSA_OK && check(cudaStreamWaitEvent(main, e_keys, 0))) {
