@@ -52,9 +52,8 @@ int sa_block_reuse_launch(const void* Q, const void* K, const void* V, const int
                           const int* cu_k, int batch, long long total_q, long long total_k, int Hq, int Hkv, int k,
                           int max_seqlen_k, int max_chunks, float scale, void* O, float* lse, void* ws,
                           int* ucount_out, cudaStream_t s);
-// A 16-row block runs on the tensor-core passes (union form) when the union of its rows'
-// selected positions fits this many chunks of 128 positions: at 128K a block and KV head
-// costs about 1.6 us on the gather kernel and about 13 ns per 128-key chunk on the passes.
+// At most this many chunks of 128 positions in a 16-row block's union for the tensor-core
+// passes (union form); the cost rule in sparse_attn_tc.cu decides below that.
 constexpr int kUnionMaxChunks = 96;
 size_t decode_workspace_bytes(int batch, int Hq, int d, int k);
 int sparse_attn_decode_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_k,
