@@ -20,8 +20,10 @@
 //   dV += P^T . dO_blk,  dK += dS^T . Q_blk                         (B read MN-major)
 //   dQ^T[d x rows] = K_tile^T . dS^T                                (A and B read MN-major)
 // dQ^T goes to an fp32 accumulator with 16-byte float reductions after a 4 x 4 lane
-// transpose (their order can vary between runs; dK and dV are deterministic).  Items are taken from a global counter, tile-
-// major, so the long early tiles start first.  Warps: 0 TMA, 1 MMA issuer and TMEM owner,
+// transpose (their order can vary between runs; dK and dV are deterministic).  Items are
+// taken from a global counter with the KV head slowest, then the sequence, then the key tile
+// (long early tiles first), so that the dQ rows the items in flight reduce into (one or two
+// sequences of one KV head) stay in L2.  Warps: 0 TMA, 1 MMA issuer and TMEM owner,
 // 2-9 epilogue (warp w: keys 32 (w % 4) .., rows 32 ((w - 2) / 4) .. of each block).
 #include <algorithm>
 
@@ -53,9 +55,12 @@ struct SABwdItem {
 };
 
 __device__ __forceinline__ bool sa_bwd_item(int id, const SABwdTcParams& p, SABwdItem& it) {
-  it.g = id % p.Hkv;
-  it.b = (id / p.Hkv) % p.batch;
-  it.j = id / (p.Hkv * p.batch);
+  // KV head slowest, then sequence, then key tile (the long early tiles first): the items
+  // in flight at a time reduce dQ into the rows of one or two sequences of one KV head,
+  // which stay in L2
+  it.g = (int)(id / (p.tiles_max * p.batch));
+  it.b = (id / p.tiles_max) % p.batch;
+  it.j = id % p.tiles_max;
   it.qbase = p.cu_q[it.b];
   it.kbase = p.cu_k[it.b];
   it.Lq = p.cu_q[it.b + 1] - it.qbase;
