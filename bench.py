@@ -254,6 +254,12 @@ def run_prefill(args, rank, world, device, dist):
     for _ in range(2):
         dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu, out=(O, lse))
     gat[1].record(stream)
+    # the tensor-core entry point of the same operation (tcgen05, 128 selected slots per tile)
+    gtc = [E(), E()]
+    gtc[0].record(stream)
+    for _ in range(2):
+        dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], idx, cu, cu, out=(O, lse), kernel="tensor_core")
+    gtc[1].record(stream)
     # and the gather kernel inside the step (after the index + top-k call, as the reuse
     # attention runs in the timed step; back to back it finds more of K and V in L2)
     gin = []
@@ -269,6 +275,7 @@ def run_prefill(args, rank, world, device, dist):
     reuse = union_stats(bu[:(L + 15) // 16].cpu().numpy(), wl.topk)
     reuse["attention_ms"] = t_attn / args.steps
     reuse["gather_attention_ms"] = gat[0].elapsed_time(gat[1]) / 2
+    reuse["gather_tc_attention_ms"] = gtc[0].elapsed_time(gtc[1]) / 2
     reuse["gather_attention_in_step_ms"] = sum(e[0].elapsed_time(e[1]) for e in gin) / len(gin)
 
     pairs = wl.causal_pairs()

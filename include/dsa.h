@@ -192,6 +192,25 @@ DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
                                     float* lse, void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * (3b) The operation of (3) on the tensor cores, tile by tile over the selected slots.
+ * Source: report summary section 1 (attention over the selected positions, one set per
+ * token shared by the query heads of its KV group).  Same inputs, outputs, validity rule
+ * and rounding bound as (3); a separate entry point because (3)'s warp-level kernel is the
+ * faster one on B200 at the shapes measured (the selected K/V rows come from L2 at a
+ * latency of microseconds, and its per-warp rings keep more bytes in flight than this
+ * kernel's shared tile rings).  Per (row, KV head), 128 selected slots at a time: K and V
+ * rows are gathered into shared memory, S^T = K.Q^T and O^T += V^T.P^T run as tcgen05 MMAs
+ * with M = 128 slots and the accumulators in tensor memory.
+ * Supported: d = 128, Hq = 8 Hkv, k a multiple of 16 and <= 2048, indices 16-byte aligned
+ * (DSA_ERR_UNSUPPORTED otherwise).
+ * ------------------------------------------------------------------------------- */
+DSA_API int dsa_sparse_attn_prefill_tc(const void* Q, const void* K, const void* V,
+                                       const int32_t* indices, const int32_t* cu_seqlens_q,
+                                       const int32_t* cu_seqlens_k, int batch, int64_t total_q,
+                                       int Hq, int Hkv, int d, int k, float scale, void* O,
+                                       float* lse, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * (3c) Sparse GQA attention, prefill, with adjacent-query reuse.  Source: report summary
  * section 8 (adjacent queries select highly similar top-k sets; the sets of adjacent
  * queries are deduplicated and the attention kernel applies a mask laid out for the MMA's

@@ -116,9 +116,11 @@ def index_topk(q_idx, k_idx, w, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, m
 
 
 def sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, scale: Optional[float] = None,
-                        with_lse: bool = True, out=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                        with_lse: bool = True, out=None, kernel: str = "gather") -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Sparse GQA attention of every packed query row over its selected keys.  `out` may
-    give (O, lse) tensors to write (lse may be None)."""
+    give (O, lse) tensors to write (lse may be None).  kernel="tensor_core" calls the
+    tcgen05 entry point (d = 128, Hq = 8 Hkv, k <= 2048) instead of the default one."""
+    entry = {"gather": "dsa_sparse_attn_prefill", "tensor_core": "dsa_sparse_attn_prefill_tc"}[kernel]
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _check(t, n, torch.bfloat16, 3)
     _check(indices, "indices", torch.int32, 2)
@@ -131,7 +133,7 @@ def sparse_attn_prefill(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, scale: Opt
     else:
         O = torch.empty_like(Q)
         lse = torch.empty((T, Hq), dtype=torch.float32, device=Q.device) if with_lse else None
-    call("dsa_sparse_attn_prefill", _ptr(Q), _ptr(K), _ptr(V), _ptr(indices), _ptr(cu_seqlens_q),
+    call(entry, _ptr(Q), _ptr(K), _ptr(V), _ptr(indices), _ptr(cu_seqlens_q),
          _ptr(cu_seqlens_k), cu_seqlens_q.numel() - 1, T, Hq, Hkv, d, indices.shape[1], scale, _ptr(O),
          _ptr(lse), _stream())
     return O, lse

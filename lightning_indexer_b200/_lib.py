@@ -27,6 +27,8 @@ SIGNATURES = {
                                c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "dsa_sparse_attn_prefill": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_int, c_int, c_int,
                                         c_int, c_f32, c_vp, c_vp, c_vp]),
+    "dsa_sparse_attn_prefill_tc": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_int, c_int, c_int,
+                                           c_int, c_f32, c_vp, c_vp, c_vp]),
     "dsa_sparse_attn_prefill_reuse_workspace_size": (c_size, [c_i64, c_int, c_int, c_int]),
     "dsa_sparse_attn_prefill_reuse": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_i64, c_i64, c_int, c_int,
                                               c_int, c_int, c_int, c_f32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),

@@ -46,6 +46,10 @@ int topk_launch(const float* scores, long long ld, const int* cu_q, const int* c
 int sparse_attn_prefill_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
                                const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int d, int k,
                                float scale, void* O, float* lse, cudaStream_t stream, const uint8_t* skip_rows);
+bool sa_gather_tc_eligible(int Hq, int Hkv, int d, int k, const void* indices);
+int sa_gather_tc_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
+                        const int* cu_k, int batch, long long total_q, int Hq, int Hkv, int k, float scale, void* O,
+                        float* lse, cudaStream_t stream, const uint8_t* skip_rows);
 size_t sa_block_reuse_scratch_bytes(long long total_q, int Hq, int batch, int max_seqlen_k, int max_chunks);
 bool sa_block_reuse_eligible(int Hq, int Hkv, int d, int max_seqlen_k);
 int sa_block_reuse_launch(const void* Q, const void* K, const void* V, const int* indices, const int* cu_q,
@@ -285,6 +289,20 @@ DSA_API int dsa_sparse_attn_prefill(const void* Q, const void* K, const void* V,
   if (total_q == 0) return DSA_OK;
   return sparse_attn_prefill_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, d, k,
                                     scale, O, lse, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+DSA_API int dsa_sparse_attn_prefill_tc(const void* Q, const void* K, const void* V, const int32_t* indices,
+                                       const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                                       int64_t total_q, int Hq, int Hkv, int d, int k, float scale, void* O,
+                                       float* lse, void* stream) {
+  if (!Q || !K || !V || !indices || !cu_seqlens_q || !cu_seqlens_k || !O) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(indices))
+    return DSA_ERR_INVALID_ARG;
+  if (batch < 1 || total_q < 0 || k < 1 || !(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (!sa_gather_tc_eligible(Hq, Hkv, d, k, indices)) return DSA_ERR_UNSUPPORTED;
+  if (total_q == 0) return DSA_OK;
+  return sa_gather_tc_launch(Q, K, V, indices, cu_seqlens_q, cu_seqlens_k, batch, total_q, Hq, Hkv, k, scale, O, lse,
+                             static_cast<cudaStream_t>(stream), nullptr);
 }
 
 static size_t reuse_lse_bytes(int64_t total_q, int Hq) { return round_up((size_t)total_q * Hq * 4, 256); }

@@ -217,6 +217,27 @@ __device__ __forceinline__ void tmem_ld_x16_sync(uint32_t taddr, float* v) {
       : "memory");
 }
 
+// 32 lanes x 8 consecutive 32-bit columns, load and wait in one statement.
+__device__ __forceinline__ void tmem_ld_x8_sync(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns stored from registers, and the wait for them.
+__device__ __forceinline__ void tmem_st_x8_sync(uint32_t taddr, const float* v) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored as rows of
 // `swizzle_bytes` (128 or 64) bytes with the matching TMA swizzle; 8-row groups are
 // 8*swizzle_bytes apart.  Fields: start address >> 4 (bits 0-13), leading byte offset
@@ -371,6 +392,20 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over `nthreads` threads that also returns whether `pred` held in any of them.
+__device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0u;
 }
 
 // Query rows [row_begin, row_end) of a varlen batch split, per sequence, into blocks of R

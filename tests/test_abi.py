@@ -64,6 +64,14 @@ def test_host_side_argument_errors():
                                        None, None) == -2
     assert lib.dsa_sparse_attn_prefill(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 128, 64, -1.0, fake,
                                        None, None) == -1
+    # the tensor-core entry: d = 128, Hq = 8 Hkv, k a multiple of 16 up to 2048, aligned indices
+    for Hq, Hkv, d, k in ((32, 4, 64, 64), (16, 4, 128, 64), (32, 4, 128, 40), (32, 4, 128, 4096)):
+        assert lib.dsa_sparse_attn_prefill_tc(fake, fake, fake, fake, fake, fake, 1, 8, Hq, Hkv, d, k, 0.1, fake,
+                                              None, None) == -2, (Hq, Hkv, d, k)
+    assert lib.dsa_sparse_attn_prefill_tc(fake, fake, fake, mis, fake, fake, 1, 8, 32, 4, 128, 64, 0.1, fake,
+                                          None, None) == -1  # misaligned indices
+    assert lib.dsa_sparse_attn_prefill_tc(fake, fake, fake, fake, fake, fake, 1, 8, 32, 4, 128, 64, 0.0, fake,
+                                          None, None) == -1
     # attention with adjacent-query reuse: shape and scale checks as (3), then the workspace
     wsz = lib.dsa_sparse_attn_prefill_reuse_workspace_size(131072, 32, 1, 131072)
     assert 620e6 < wsz < 680e6  # per 16-row block: 12288 union positions, their selection words, lse and maxima

@@ -213,14 +213,16 @@ def _oracle_sets(D, k):
     return np.stack([orc.forward_row(D, r, k)["idx"] for r in range(wl.Tq)])
 
 
-@pytest.mark.parametrize("Hq,Hkv,d", [(32, 4, 128), (8, 2, 64), (16, 4, 64)])
-def test_sparse_attention_prefill_given_sets(Hq, Hkv, d):
+# "tensor_core": the tcgen05 entry point (d = 128, 8 query heads per KV head)
+@pytest.mark.parametrize("Hq,Hkv,d,kernel", [(32, 4, 128, "gather"), (32, 4, 128, "tensor_core"), (8, 2, 64, "gather"),
+                                             (16, 4, 64, "gather"), (16, 4, 128, "gather")])
+def test_sparse_attention_prefill_given_sets(Hq, Hkv, d, kernel):
     wl = gen.make_prefill([200, 57, 400], Hq, Hkv, d, 4, 32, 64, seed=31)
     D = orc.Decoded(wl)
     idx = _oracle_sets(D, 64)
     t = to_device(wl)
     O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx.astype(np.int32)).cuda(),
-                                     t["cu_q"], t["cu_k"])
+                                     t["cu_q"], t["cu_k"], kernel=kernel)
     O = O.float().cpu().numpy()
     lse = lse.cpu().numpy()
     for r in range(wl.Tq):
@@ -360,18 +362,24 @@ def test_index_topk_fused_repeat_is_bit_identical():
         assert torch.equal(dsa.index_topk(*args, chunk_rows=1000, path=dsa.PATH_FUSED), first)
 
 
-def test_sparse_attention_empty_and_padded_sets():
-    wl = gen.make_prefill([40], 8, 2, 64, 4, 32, 32, seed=32)
+@pytest.mark.parametrize("Hq,Hkv,d,k,kernel", [(8, 2, 64, 32, "gather"), (16, 2, 128, 48, "gather"),
+                                               (16, 2, 128, 48, "tensor_core"), (16, 2, 128, 176, "tensor_core")])
+def test_sparse_attention_empty_and_padded_sets(Hq, Hkv, d, k, kernel):
+    # on the tensor-core kernel k = 48 is one partial tile of 128 slots, k = 176 a full tile
+    # and a ragged one
+    wl = gen.make_prefill([40], Hq, Hkv, d, 4, 32, 32, seed=32)
     D = orc.Decoded(wl)
-    idx = np.full((40, 32), -1, np.int32)
+    idx = np.full((40, k), -1, np.int32)
     idx[39, :5] = [0, 1, 7, 20, 39]
     idx[12, 3] = 11  # a single selected key in the middle of the padding
+    idx[20, k - 1] = 4  # a key in the last slot of the last tile
     t = to_device(wl)
-    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"])
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"],
+                                     kernel=kernel)
     O = O.float().cpu().numpy()
     lse = lse.cpu().numpy()
     assert np.all(O[0] == 0) and np.all(np.isneginf(lse[0]))
-    for r in (39, 12):
+    for r in (39, 12, 20):
         sel = idx[r][idx[r] >= 0]
         Or, lr = orc.sparse_attention_row(D.rows("Q", r), D.rows("K", sel), D.rows("V", sel), D.scale)
         assert np.max(np.abs(O[r] - Or)) <= ATTN_ATOL
@@ -409,6 +417,13 @@ def test_sparse_attention_ignores_positions_the_row_cannot_see(Hq, Hkv, d):
         assert np.max(np.abs(lh[r] - lr)) <= LSE_ATOL, r
         O_ref.append(Or)
         lse_ref.append(lr)
+    if d == 128 and Hq == 8 * Hkv:  # the tensor-core entry point applies the same rule
+        O2, l2 = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(bad.astype(np.int32)).cuda(),
+                                         t["cu_q"], t["cu_k"], kernel="tensor_core")
+        O2, l2 = O2.float().cpu().numpy(), l2.cpu().numpy()
+        for r in range(wl.Tq):
+            assert np.max(np.abs(O2[r] - O_ref[r])) <= ATTN_ATOL, r
+            assert np.max(np.abs(l2[r] - lse_ref[r])) <= LSE_ATOL, r
     # the backward of the same sets (gather path at d = 64, masked dense path at d = 128)
     ref = orc.sparse_attention_backward(D, kept, np.stack(O_ref), np.stack(lse_ref), D.full("dO"))
     dQ, dK, dV = dsa.sparse_attn_prefill_bwd(t["Q"], t["K"], t["V"], O, t["dO"], lse,
@@ -419,7 +434,8 @@ def test_sparse_attention_ignores_positions_the_row_cannot_see(Hq, Hkv, d):
         assert np.max(np.abs(g - ref[name])) <= 1.5e-2 * np.max(np.abs(ref[name])), name
 
 
-def test_sparse_attention_large_rising_logits():
+@pytest.mark.parametrize("kernel", ["gather", "tensor_core"])
+def test_sparse_attention_large_rising_logits(kernel):
     """Logits of tens of units that grow along the key order: the running max moves in
     most chunks, by more than the rescale threshold, and the weights span many octaves."""
     wl = gen.make_prefill([300], 32, 4, 128, 4, 32, 128, seed=34)
@@ -437,7 +453,8 @@ def test_sparse_attention_large_rising_logits():
         n = min(r + 1, 128)
         idx[r, :n] = np.linspace(0, r, n).astype(np.int64)  # step >= 1: distinct, ascending
     t = to_device(wl)
-    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"])
+    O, lse = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"],
+                                     kernel=kernel)
     O = O.float().cpu().numpy()
     lse = lse.cpu().numpy()
     for r in range(0, 300, 7):

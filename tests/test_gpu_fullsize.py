@@ -66,7 +66,13 @@ def _check_prefill(wl, chunk=8192, seed=0):
 
 
 def test_prefill_32k_sampled_rows():
-    _check_prefill(gen.prefill_32k(), seed=1)
+    t, idx, O, lse = _check_prefill(gen.prefill_32k(), seed=1)
+    # the tensor-core entry point on the same selections: every row against the gather
+    # kernel's, each within its own bound of the oracle, so within twice that of each other
+    O2, l2 = dsa.sparse_attn_prefill(t["Q"], t["K"], t["V"], torch.from_numpy(idx).cuda(), t["cu_q"], t["cu_k"],
+                                     kernel="tensor_core")
+    assert np.max(np.abs(O2.float().cpu().numpy() - O)) <= 2 * ATTN_ATOL
+    assert np.max(np.abs(l2.cpu().numpy() - lse)) <= 2 * 2e-3
 
 
 def test_video_prefill_128k_sampled_rows():
