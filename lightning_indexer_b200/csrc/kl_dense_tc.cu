@@ -105,23 +105,25 @@ __device__ __forceinline__ bool kl_lse_item(long long item, const KlLseParams& p
 // [Tk, Hkv, 128] bf16 tensor) of one union chunk copied into a K-major tile with the
 // 128-byte swizzle (two 64-column panels of 128-byte rows, 16-byte chunk c of row r at
 // ((c ^ (r % 8)) * 16)), the layout a tiled TMA load gives.  Called by `nw` gather warps
-// (wg = 0 .. nw-1); each warp instruction copies two whole rows (16 lanes x 16 bytes each),
-// and every lane then arrives on `bar` when its copies have landed (nw * 32 arrivals).
+// (wg = 0 .. nw-1).  Eight lanes per row: each warp instruction moves the 128-byte halves of
+// four rows (whole lines, as coalesced as two full rows per instruction), and a row's
+// position and address are worked out once for both halves.  Every lane then arrives on
+// `bar` when its copies have landed (nw * 32 arrivals).
 __device__ __forceinline__ void union_copy_tile(uint8_t* dst, int panel_bytes, const uint16_t* src,
                                                 const int* chunk_keys, int kbase, int Hkv, int g, int nw, int wg,
                                                 int lane, uint64_t* bar) {
-  const int4 k4 = __ldg(reinterpret_cast<const int4*>(chunk_keys) + lane);  // positions 4 lane .. 4 lane + 3
-  const int half = lane >> 4, c = lane & 15;
-  const uint32_t dbase = smem_u32(dst) + (c >> 3) * panel_bytes;
-#pragma unroll 4
-  for (int m = wg; m < 64; m += nw) {
-    // rows 2 m and 2 m + 1; their positions sit in lane m / 2 (warp-uniform)
-    const int r = 2 * m + half;
-    const int xa = __shfl_sync(0xffffffffu, (m & 1) ? k4.z : k4.x, m >> 1);
-    const int xb = __shfl_sync(0xffffffffu, (m & 1) ? k4.w : k4.y, m >> 1);
-    const int s = half ? xb : xa;
-    const uint16_t* row = src + ((long long)(kbase + s) * Hkv + g) * 128;
-    cp_async_16(dbase + r * 128 + (((c & 7) ^ (r & 7)) * 16), row + c * 8, true);
+  const int sub = lane >> 3, c = lane & 7;
+  const uint32_t dbase = smem_u32(dst);
+  const uint16_t* base = src + (long long)g * 128 + c * 8;
+  const long long stride = (long long)Hkv * 128;
+#pragma unroll 2
+  for (int q = wg; q < 32; q += nw) {
+    const int r = 4 * q + sub;
+    const int s = __ldg(chunk_keys + r);  // eight lanes read each position (one L1 line per chunk)
+    const uint16_t* row = base + (long long)(kbase + s) * stride;
+    const uint32_t d0 = dbase + r * 128 + ((c ^ (r & 7)) * 16);
+    cp_async_16(d0, row, true);                     // columns 8c .. 8c + 7 (panel 0)
+    cp_async_16(d0 + panel_bytes, row + 64, true);  // columns 64 + 8c .. (panel 1)
   }
   cp_async_mbar_arrive(bar);
 }
