@@ -4,7 +4,7 @@
 // the selected rows arrive from L2 at a latency of microseconds under this load, so the
 // gather needs about 200 KB in flight per SM; that kernel's per-warp rings keep nearly all
 // of their 224 KB in flight, while here each 32 KB stage is also held through S, the
-// softmax and P.V (measured at 128K: 89 against 46 ms).
+// softmax and P.V (measured at 128K: 89.5 against 39.1 ms).
 //
 // Source: Keye-VL-2.0 report summary (mqxn.cn/news/1966), section 1: attention runs only
 // over the positions the indexer selected, and DSA is adapted to GQA with one selected set
