@@ -125,15 +125,21 @@ __global__ void __launch_bounds__(BWD_WARPS * 32, 3) sparse_attn_bwd_kernel(cons
     const int my_idx = __ldg(idx + c * BWD_CHUNK + (lane & 15));
     const uint32_t kdst = my_s + st * STAGE_BYTES;
     const uint32_t vdst = kdst + TILE_BYTES;
+    // eight lanes per row: each copy instruction moves 128-byte pieces (whole lines) of four
+    // rows, and a row's slot, validity and address are worked out once for all its pieces
+    const int sub = lane >> 3, cc = lane & 7;
 #pragma unroll
-    for (int j = 0; j < BWD_CHUNK * SEGS / 32; ++j) {
-      const int e = j * 32 + lane;
-      const int r = e / SEGS, seg = e % SEGS;
+    for (int j = 0; j < BWD_CHUNK / 4; ++j) {
+      const int r = 4 * j + sub;
       const int s = __shfl_sync(0xffffffffu, my_idx, r);
       const bool valid = (unsigned)s < (unsigned)vis;  // -1 and positions the row cannot see
-      const size_t off = valid ? (size_t)(kbase + s) * kv_row_stride + seg * 8 : 0;
-      cp_async_16(kdst + tile_off<D>(r, seg), Kg + off, valid);
-      cp_async_16(vdst + tile_off<D>(r, seg), Vg + off, valid);
+      const size_t off = valid ? (size_t)(kbase + s) * kv_row_stride + cc * 8 : 0;
+      const uint32_t o = tile_off<D>(r, cc);
+#pragma unroll
+      for (int h = 0; h < SEGS / 8; ++h) {  // segment cc + 8h lands 128 h bytes after segment cc
+        cp_async_16(kdst + o + h * 128, Kg + off + h * 64, valid);
+        cp_async_16(vdst + o + h * 128, Vg + off + h * 64, valid);
+      }
     }
   };
 
