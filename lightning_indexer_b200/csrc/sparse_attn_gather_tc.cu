@@ -20,13 +20,14 @@
 //   S^T [128 slots x 16]  = K_tile [128 x d] . Q_g^T [d x 16]        (columns 0-7: the heads)
 //   O^T [d x 16]         += V_tile^T [d x 128 slots] . P^T [128 x 16]
 // N = 16 is the smallest N of the M = 128 shape; columns 8-15 are never read.  Roles of the
-// 16 warps of a persistent CTA (one per SM, ~210 KB of shared memory):
-//   warp 0        the item's Q_g (8 rows of 256 B) into a 2-stage buffer (cp.async);
+// 16 warps of a persistent CTA (one per SM, 226 KB of shared memory):
+//   warp 0        the item's slot list (one bulk copy into shared memory, read there by
+//                 the copy and epilogue warps) and Q_g (8 rows of 256 B, cp.async), 2 stages;
 //   warp 1        TMEM owner and MMA issuer (S of tile n + 1 is issued before P.V of tile n);
 //   warps 4-7     epilogue: thread i owns slot i of S^T (TMEM lane i) and dimension i of O^T;
 //   warps 2-3, 8-10  copy K rows, warps 11-15 V rows, 16-byte cp.async into 3-stage rings in
-//                 the 128-byte-swizzled layout (zero-filled for invalid slots), completion
-//                 signalled with cp.async.mbarrier.arrive.noinc.
+//                 the 128-byte-swizzled layout (zero-filled for invalid slots; eight lanes
+//                 per row), completion signalled with cp.async.mbarrier.arrive.noinc.
 // Online softmax in the log2 domain: the running max of a head moves only when a tile
 // exceeds it by more than 8, decided for all 128 epilogue threads at once by one barrier
 // reduction per tile; in that case the tile's maxima are reduced through shared memory and
