@@ -283,16 +283,22 @@ def run_prefill(args, rank, world, device, dist):
     idx_flops = pairs * wl.H_I * wl.d_I * 2
     attn_flops = sel_pairs * wl.Hq * wl.d * 4
     n_chunks = (L + chunk - 1) // chunk
+    # leading chunks whose rows see at most 2 x cap positions (cap: the fused path's candidate
+    # list per row, min(8192, (4 ld - 64) / 8) rounded to 4) run the separate passes
+    ld = (L + 3) // 4 * 4
+    cap = min(8192, (4 * ld - 64) // 8) // 4 * 4
+    n_sep = sum(1 for c in range(n_chunks) if min(L, (c + 1) * chunk) <= 2 * cap)
     res = {
         "value": value, "ms_per_step": ms_step, "clocks": clk.summary(),
         "breakdown_ms_per_step": {"index_topk": t_it / args.steps, "sparse_attn": t_attn / args.steps},
         "adjacent_query_reuse": reuse,
         "separate_path_ms_per_step": sep[0].elapsed_time(sep[1]) / 2,
         "idx_flops": idx_flops, "index_topk_ms": t_it / args.steps,
-        # sampled-score indexer and bound kernel, then per chunk: fused indexer, select, and the
-        # repair indexer and exact top-k (which return at once when no row needs them);
-        # attention: union plan, the two tensor-core passes, the gather kernel
-        "launches_per_step": 2 + 4 * n_chunks + 4,
+        # sampled-score indexer and bound kernel, then per fused chunk: fused indexer, select, and
+        # the repair indexer and exact top-k (which return at once when no row needs them); per
+        # separate chunk: indexer, top-k, exact top-k of marked rows; attention: union plan, the
+        # two tensor-core passes, the gather kernel (68 per 128K step, as the ncu launch list)
+        "launches_per_step": 2 + 4 * (n_chunks - n_sep) + 3 * n_sep + 4,
         "flops_per_step": idx_flops + attn_flops, "attn_flops": attn_flops,
         "gather_bytes_per_step": sel_pairs * wl.Hkv * wl.d * 2 * 2,
     }
