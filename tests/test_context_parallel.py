@@ -1,7 +1,7 @@
 """Context-parallel prefill of one sequence over ranks: the partition, the key all-gather
 and the per-block bottom-right alignment.
 
-CPU tests run two gloo ranks whose per-block computation is the fp64 oracle: the
+CPU tests run two or three gloo ranks whose per-block computation is the fp64 oracle: the
 concatenated result of the ranks must equal the oracle's whole-sequence forward at the
 same positions (an integer-valued indexer input makes every score exact, so the sets are
 compared bit for bit).  The GPU test runs the library's prefill on each zig-zag block of
@@ -89,14 +89,13 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("L", [203, 96])
-def test_two_gloo_ranks_match_whole_sequence_oracle(L):
+@pytest.mark.parametrize("L,world", [(203, 2), (96, 2), (203, 3)])
+def test_gloo_ranks_match_whole_sequence_oracle(L, world):
     import torch.multiprocessing as mp
     from oracle import dsa_oracle as orc
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    world = 2
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, L, q)) for r in range(world)]
     for p in procs:
         p.start()
